@@ -1,0 +1,362 @@
+#!/usr/bin/env python
+"""Throughput of the full MoE layer forward on B200 (one JSON line on rank 0).
+
+Workload (full_layer_bf16): T=16384 tokens, hidden 2048, 256 routed SwiGLU
+experts (intermediate 512), top-8, capacity factor 1.25 (C=640), one always-on
+shared SwiGLU expert (intermediate 512), router bias skew, aux coefficient 0.001.
+One step = router GEMM, softmax/top-k/gates, slot scan, gather, routed experts,
+shared expert, combine and load statistics over one batch.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one rank per GPU, each rank on its own batch
+(weak scaling; no collective on the data path).  Timing: CUDA events on the
+launch stream around every step, an L2 flush (a 256 MiB write) between steps,
+a barrier + synchronize on both sides of the timed loop, max over ranks.
+``--impl reference`` times the fp64 CPU oracle on a bounded token sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/sec fwd(+bwd) on 1 B200; % of HBM and bf16 tensor-core roofline"
+UNIT = "tokens/s"
+WORKLOAD = dict(workload="full_layer_bf16", T=16384, hidden=2048, experts=256, top_k=8, expert_intermediate=512,
+                shared_experts=1, shared_intermediate=512, capacity_factor=1.25, capacity=640, aux_coef=0.001)
+KERNELS_PER_STEP = 11  # router GEMM, top-k, reduce, scan, gather, 2 routed GEMMs, 2 shared GEMMs, combine, aux
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, max clock, power, clock-event reasons) in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            uuid = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                pass
+            h = None
+            if uuid:
+                for i in range(pynvml.nvmlDeviceGetCount()):
+                    hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+                    u = pynvml.nvmlDeviceGetUUID(hh)
+                    u = u.decode() if isinstance(u, bytes) else u
+                    if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                        h = hh
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append(mhz)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------------
+def oracle_step(cfg64, S: int):
+    """The fp64 CPU oracle over the first S tokens of the batch (route .. combine, aux)."""
+    from oracle import oracle as O
+
+    xs = cfg64["x"][:S]
+    s = O.router_logits(xs, cfg64["w_router_de"], cfg64["bias"])
+    _, sel, gates, counts, psum = O.route(s, WORKLOAD["top_k"])
+    C = O.capacity(S, WORKLOAD["top_k"], WORKLOAD["experts"], WORKLOAD["capacity_factor"])
+    disp = O.dispatch(sel, WORKLOAD["experts"], C)
+    shared = O.expert_rows("swiglu", xs, np.arange(S), np.zeros(S, np.int64), cfg64["shared"])
+    y = O.layer_rows("swiglu", xs, sel, disp["kept"], gates, cfg64["experts"], base_kind="tensor", base=shared)
+    O.aux(counts, psum, S, WORKLOAD["top_k"])
+    return y
+
+
+def oracle_inputs(cfg):
+    from sparse_mixture_experts_stable_b200.inputs import pages_layout
+
+    return dict(
+        x=cfg["x"].double().numpy(), w_router_de=cfg["w_router"].double().numpy().T.copy(),
+        bias=cfg["router_bias"].double().numpy(),
+        experts=dict(w1=pages_layout(cfg["w_gate"]), w3=pages_layout(cfg["w_up"]), w2=pages_layout(cfg["w_down"])),
+        shared=dict(w1=pages_layout(cfg["s_gate"]), w3=pages_layout(cfg["s_up"]), w2=pages_layout(cfg["s_down"])),
+    )
+
+
+def time_oracle(cfg64, budget_s: float):
+    """Pick a token sample that takes about budget_s, then time it.  Returns (tokens/s, S, seconds)."""
+    t0 = time.perf_counter()
+    oracle_step(cfg64, 16)
+    per_tok = (time.perf_counter() - t0) / 16
+    S = int(max(16, min(WORKLOAD["T"], budget_s / max(per_tok, 1e-6))))
+    t0 = time.perf_counter()
+    oracle_step(cfg64, S)
+    dt = time.perf_counter() - t0
+    return S / dt, S, dt
+
+
+def run_reference(args, world, rank):
+    from sparse_mixture_experts_stable_b200 import inputs as I
+
+    if rank != 0:
+        return
+    cfg = I.full_layer_bf16(seed=0)
+    cfg64 = oracle_inputs(cfg)
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    t0 = time.perf_counter()
+    oracle_step(cfg64, 16)
+    per_tok = (time.perf_counter() - t0) / 16
+    S = int(max(16, min(WORKLOAD["T"], budget / max(per_tok, 1e-6))))
+    for _ in range(args.warmup):
+        oracle_step(cfg64, S)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(cfg64, S)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = S * args.steps / total
+    line = dict(impl="reference", metric=METRIC, value=value, unit=UNIT, n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=1e3 * total / args.steps, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype="f64", data="synthetic",
+                config=dict(WORKLOAD, sample_tokens_per_step=S, l2="n/a (CPU)"),
+                cpu_baseline=dict(value=value, unit=UNIT, cores=os.cpu_count(), kind="oracle",
+                                  sample=f"first {S} tokens of the batch per step, capacity from the sample's T"),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    import sparse_mixture_experts_stable_b200 as moe
+    from sparse_mixture_experts_stable_b200 import inputs as I
+    from sparse_mixture_experts_stable_b200.layer import SwiGLUMoE
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    moe.lib()  # fail loudly if the CUDA library is missing
+    cfg = I.full_layer_bf16(seed=rank)
+    T, H, E, F, k = cfg["T"], cfg["H"], cfg["E"], cfg["F"], cfg["k"]
+    names = ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")
+    dv = {n: cfg[n].to(dev) for n in names}
+    layer = SwiGLUMoE(T, H, E, F, k, cfg["capacity_factor"], F_shared=cfg["F_shared"], aux_coef=cfg["aux_coef"],
+                      device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    ffn_ev = []
+
+    def step(x):
+        r = moe.moe_route(x, k, w_router=dv["w_router"], layout="ED", logit_bias=dv["router_bias"],
+                          out=layer.route_out, dev_status=layer.status, workspace=layer.ws_route)
+        d = moe.moe_dispatch(r["selected"], E, layer.C, x=x, out=layer.disp_out, dev_status=layer.status,
+                             workspace=layer.ws_disp)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        moe.moe_expert_ffn("swiglu", d["xbuf"], d["used"], dv["w_gate"], w2=dv["w_down"], w3=dv["w_up"],
+                           ybuf=layer.ybuf, dev_status=layer.status, workspace=layer.ws_ffn)
+        e1.record(stream)
+        ffn_ev.append((e0, e1))
+        moe.moe_expert_ffn("swiglu", x.view(1, T, H), None, dv["s_gate"], w2=dv["s_down"], w3=dv["s_up"],
+                           ybuf=layer.shared.view(1, T, H), dev_status=layer.status, workspace=layer.ws_shared)
+        y = moe.moe_combine(layer.ybuf, r["selected"], d["slot"], r["gates_f32"], base_kind="tensor",
+                            base=layer.shared, y=layer.y, dev_status=layer.status)
+        f, P, aux = moe.moe_aux_stats(r["counts"], r["prob_sum"], T, k, True, cfg["aux_coef"],
+                                      out_dtype=torch.bfloat16)
+        return y, aux
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(dv["x"])
+    torch.cuda.synchronize()
+    assert moe.moe_read_status(layer.status) == 0, "device status reported an error"
+    ffn_ev.clear()
+
+    # ---- device-timed loop ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step(dv["x"])
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ffn_ms = [a.elapsed_time(b) for a, b in ffn_ev]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    value = T * args.steps * world / (total_ms / 1e3)
+
+    # ---- end to end: host input -> device -> layer -> host output ----
+    x_host = cfg["x"].pin_memory()
+    y_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    aux_host = torch.empty(2, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(dv["x"])
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        y, aux = step(x_dev)
+        y_host.copy_(y, non_blocking=True)
+        aux_host.copy_(aux, non_blocking=True)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), world)
+    e2e_value = T * args.steps * world / (e2e_ms / 1e3)
+    assert moe.moe_read_status(layer.status) == 0
+
+    # ---- roofline of the dominant kernel (routed SwiGLU grouped GEMMs) ----
+    kept = int(layer.disp_out["used"].sum().item())
+    flops = 2.0 * kept * (2 * H * F) + 2.0 * kept * F * H
+    ffn_avg_s = statistics.mean(ffn_ms) / 1e3
+    pk = measured_peaks()
+    achieved = flops / ffn_avg_s / 1e12
+    roof = dict(bound="tensor", kernel="tc_gemm_kernel: routed SwiGLU gate/up + down launches", achieved=achieved,
+                peak=pk["bf16_sustained"], unit="TFLOP/s", frac=achieved / pk["bf16_sustained"], traffic=None,
+                peak_source=f"{pk['source']} bf16 sustained", frac_of_burst=achieved / pk["bf16"],
+                flops_per_launch=flops, kept_rows=kept, avg_launch_ms=1e3 * ffn_avg_s)
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cfg64 = oracle_inputs(cfg)
+        tps, S, dt = time_oracle(cfg64, args.cpu_seconds)
+        cpu = dict(value=tps, unit=UNIT, cores=os.cpu_count(), kind="oracle",
+                   sample=f"first {S} tokens of the batch ({dt:.1f} s), capacity from the sample's T")
+    line = dict(
+        metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+        ms_per_step=total_ms / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+        data="synthetic",
+        config=dict(WORKLOAD, parallelism=f"replicas{world}", global_batch=T * world,
+                    l2="flushed between steps (256 MiB write)", tokens_kept=kept),
+        e2e=dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=T * H * 2, d2h_bytes_per_step=T * H * 2 + 8),
+        gpu_launches=KERNELS_PER_STEP * args.steps,
+        roofline=roof, cpu_baseline=cpu, clocks=clocks.summary(),
+    )
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,315 @@
+/*
+ * moe.h -- C ABI of libmoe.so: a capacity-limited top-k sparse
+ * mixture-of-experts layer for NVIDIA B200 (sm_100a).
+ *
+ * Sources of the operations (page title, then section):
+ *   [P1] "Sparse MoE Layer in NumPy -- Token Drop, Exact Dispatch/Combine,
+ *        Aux Loss & Backward": sections 1 (root causes), 2 (implementation),
+ *        4 (usage).
+ *   [P2] "Top-k MoE Router with Load Statistics": problem statement,
+ *        Requirements, Constraints.
+ *   [P3] "Module 7. Mixture of Experts": route_logits, expert_capacity,
+ *        dispatch_with_capacity, switch_auxiliary_loss, swiglu_expert,
+ *        EducationalMoE.
+ *   [P4] "32. Sparse MoE Token Dispatch & Combine (Capacity-Limited)":
+ *        Problem, Step-by-Step Approach.
+ *   [P5] "mixture-of-experts/3": Expert, TopKMoE, _load_balancing_loss.
+ *
+ * General conventions (apply to every entry point):
+ *   - Pointers marked "device" must point to memory of the current CUDA
+ *     device; pointers marked "host" to host memory.  The caller owns every
+ *     buffer.  The library never allocates device memory: scratch space is
+ *     a caller-provided device workspace whose minimum size is returned by
+ *     the matching *_workspace_size function.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL
+ *     is the legacy default stream).  No entry point synchronises, except
+ *     moe_read_status.
+ *   - Matrices are row-major.  "Row stride" arguments (ld*) count elements.
+ *     bf16 operands that feed the tensor-core path need 16-byte aligned
+ *     base pointers and row strides that are multiples of 8 elements.
+ *   - Inputs are never modified ([P2] Requirements).
+ *   - Return value: MOE_OK, or an error from moe_status for a problem
+ *     detected on the host before anything was enqueued (nothing is
+ *     enqueued then).  Problems that depend on device data (an expert index
+ *     outside [0,E), a non-finite logit, a wait that exceeded its time
+ *     limit) are written by the kernels into the device status word
+ *     `dev_status` (may be NULL to ignore them): the first error wins, the
+ *     word is never reset by a kernel.  Clear it with moe_clear_status and
+ *     read it with moe_read_status.
+ *   - Expert weights use the (out, in) layout of nn.Linear ([P5] Expert):
+ *     a matrix that maps K_in features to N_out features is stored
+ *     (N_out, K_in), one such matrix per expert, experts outermost.  The
+ *     pages' x @ W matrices (E, K_in, N_out) ([P1] section 2, [P3]
+ *     EducationalMoE, [P4]) are the transposes; moe_transpose_weights
+ *     converts them once.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* bad size, NULL pointer, k outside [1,E], capacity_factor <= 0 */
+    MOE_ERR_UNSUPPORTED = 2, /* valid per the pages but outside this build's limits */
+    MOE_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed */
+    MOE_ERR_BAD_INDEX = 4,   /* device: an expert index outside [0, E) */
+    MOE_ERR_NONFINITE = 5,   /* device: a non-finite router logit */
+    MOE_ERR_TIMEOUT = 6,     /* device: a bounded wait gave up */
+    MOE_ERR_WORKSPACE = 7    /* workspace NULL or smaller than required */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* What the combine adds the gated expert outputs to ([P1] section 1 item 4:
+ * the input row; [P2]: the shared output; [P4]/[P5]: nothing). */
+typedef enum { MOE_BASE_ZERO = 0, MOE_BASE_INPUT = 1, MOE_BASE_TENSOR = 2 } moe_base;
+
+/* Expert function: [P1]/[P4] linear x @ W; [P5] fc2(gelu(fc1 x)) with
+ * biases and exact (erf) GELU; [P3] swiglu_expert (silu(x Wg) * x Wu) Wd. */
+typedef enum { MOE_FFN_LINEAR = 0, MOE_FFN_GELU_MLP = 1, MOE_FFN_SWIGLU = 2 } moe_ffn_kind;
+
+/* Router weight layout: (D, E) as on [P2]; (E, D) as nn.Linear in [P5]. */
+typedef enum { MOE_ROUTER_DE = 0, MOE_ROUTER_ED = 1 } moe_router_layout;
+
+/* Static string for a moe_status value. */
+MOE_API const char* moe_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+MOE_API int moe_version(void);
+
+/*
+ * moe_capacity -- per-expert capacity C = ceil(capacity_factor * T * k / E),
+ * at least 1 ([P3] expert_capacity; [P1] section 1 item 2).  Evaluated in
+ * IEEE double in the order capacity_factor * T * k / E.
+ *   T, k, E  : tokens, experts per token, experts; T >= 1, 1 <= k <= E.
+ *   capacity_factor : finite and > 0, else MOE_ERR_INVALID_ARG ([P3]
+ *              rejects a zero factor).
+ *   C_out    : host; receives C.
+ * A caller that wants C = 0 (every assignment dropped, [P1] section 3 edge
+ * checks) passes C = 0 directly to moe_dispatch.
+ */
+MOE_API int moe_capacity(int64_t T, int32_t k, int32_t E, double capacity_factor, int64_t* C_out);
+
+/*
+ * moe_route -- router scores, softmax, stable top-k, renormalised gates,
+ * pre-drop counts and probability sums for T tokens.
+ *
+ * Computes, per token t ([P2] problem statement; [P1] section 2
+ * top_k_gating; [P3] route_logits, stable_softmax, _deterministic_top_k;
+ * [P5] TopKMoE.forward):
+ *   s[t,e]   = x_t . w_e (+ logit_bias[e])    (fp32 accumulation)
+ *   p[t,:]   = softmax(s[t,:]) in fp32, maximum subtracted first
+ *   selected = the k experts with the largest s, in descending order, an
+ *              exact tie going to the lower expert index
+ *   gate_j   = exp(s_j - s_max) / sum_r exp(s_r - s_max) over the selected
+ *              experts (= p_j / sum_r p_r)
+ *   counts[e]   = #{(t,j) : selected[t,j] = e}      (before any drop)
+ *   prob_sum[e] = sum_t p[t,e]                      (fixed-order reduction)
+ *
+ * Arguments:
+ *   x          device; (T, D) activations with row stride ldx, dtype `dtype`.
+ *              If w_router is NULL, x instead holds the (T, E) router logits
+ *              (row stride ldx, dtype `dtype`) and D is ignored.
+ *   w_router   device or NULL; router weight in `layout`, dtype `dtype`.
+ *              bf16 scores are computed on the tensor cores (fp32
+ *              accumulate); fp32 scores with fp32 FFMA.
+ *   logit_bias device fp32 (E) or NULL.
+ *   k          1 <= k <= E; this build requires k <= 64 and E <= 1024.
+ *   logits_out device fp32 (T, E) or NULL; receives s.
+ *   selected   device int64 (T, k).
+ *   gates      device (T, k) in `dtype` or NULL ([P2]: results in x's dtype).
+ *   gates_f32  device fp32 (T, k) or NULL.
+ *   counts     device int32 (E).
+ *   prob_sum   device fp32 (E).
+ *   dev_status device int32 or NULL: MOE_ERR_NONFINITE if a logit is not
+ *              finite (that token's outputs are then unspecified, [P3]
+ *              rejects such input).
+ *   workspace  device, >= moe_route_workspace_size(...) bytes.
+ */
+MOE_API size_t moe_route_workspace_size(int64_t T, int64_t D, int32_t E, moe_dtype dtype,
+                                int has_router_weight, moe_router_layout layout);
+MOE_API int moe_route(const void* x, moe_dtype dtype, int64_t T, int64_t D, int64_t ldx,
+              const void* w_router, moe_router_layout layout, int32_t E, const float* logit_bias,
+              int32_t k, float* logits_out, int64_t* selected, void* gates, float* gates_f32,
+              int32_t* counts, float* prob_sum, int32_t* dev_status, void* workspace,
+              size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * moe_dispatch -- greedy position-priority slot assignment and the gather
+ * into expert-major buffers.
+ *
+ * Over the assignment stream ordered by token t ascending, then route slot
+ * j ascending (selection order = descending gate), an assignment (t,j) to
+ * expert e is kept iff fewer than C earlier assignments to e were kept
+ * ([P1] section 2 position_priority_dispatch; [P3] dispatch_with_capacity;
+ * [P4] step 2, the exclusive running count).  Computed as a single-pass
+ * per-expert prefix count with decoupled look-back; the result is unique.
+ *   slot[t,j]          rank of (t,j) among e's kept rows, -1 if dropped
+ *   kept[t,j]          1 kept / 0 dropped
+ *   used[e]            min(count_e, C)
+ *   overflow[e]        count_e - used[e] ([P1] section 1 item 3)
+ *   drops_per_token[t] dropped assignments of token t ([P1] section 4)
+ *   token_of_slot[e,c] token in slot c of expert e, -1 for c >= used[e]
+ *   xbuf[e,c,:]        = x[token_of_slot[e,c], :] for c < used[e]
+ *                      ([P4] step 5 gather); rows c >= used[e] untouched.
+ *
+ * Arguments:
+ *   selected  device int64 (T, k) expert indices (from moe_route, or given
+ *             as in [P4]); an index outside [0, E) sets MOE_ERR_BAD_INDEX
+ *             in dev_status and is treated as dropped.
+ *   T, k, E, C : T >= 1, 1 <= k <= 64, 1 <= E <= 2048, C >= 0; T * k < 2^30.
+ *   x         device (T, D) row stride ldx, dtype `dtype`, or NULL to skip
+ *             the gather (then xbuf is ignored).
+ *   xbuf      device (E, C, D) contiguous, dtype `dtype`.
+ *   slot, kept, used, overflow, drops_per_token, token_of_slot : device
+ *             outputs as above (int64, uint8, int32, int32, int32, int32).
+ *   workspace device, >= moe_dispatch_workspace_size(T, k, E) bytes.
+ */
+MOE_API size_t moe_dispatch_workspace_size(int64_t T, int32_t k, int32_t E);
+MOE_API int moe_dispatch(const int64_t* selected, int64_t T, int32_t k, int32_t E, int64_t C,
+                 const void* x, moe_dtype dtype, int64_t D, int64_t ldx, int64_t* slot,
+                 uint8_t* kept, int32_t* used, int32_t* overflow, int32_t* drops_per_token,
+                 int32_t* token_of_slot, void* xbuf, int32_t* dev_status, void* workspace,
+                 size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * moe_expert_ffn -- every expert applied to its own rows of an expert-major
+ * buffer (grouped GEMM over variable-occupancy experts).
+ *
+ * For each expert e and row c < rows(e) (rows(e) = used[e], or C when used
+ * is NULL):  ybuf[e,c,:] = Expert_e(xbuf[e,c,:]) with
+ *   LINEAR   : x W1_e^T                      W1 (E, Dout, D)       [P1], [P4]
+ *   GELU_MLP : gelu(x W1_e^T + b1_e) W2_e^T + b2_e                  [P5]
+ *              W1 (E, F, D), b1 (E, F), W2 (E, Dout, F), b2 (E, Dout)
+ *   SWIGLU   : (silu(x W1_e^T) * (x W3_e^T)) W2_e^T                 [P3]
+ *              W1 = gate (E, F, D), W3 = up (E, F, D), W2 = down (E, Dout, F)
+ * bf16: tcgen05 tensor cores, fp32 accumulation, the intermediate
+ * activation rounded to bf16, outputs bf16.  fp32: fp32 FFMA throughout.
+ * Rows c >= rows(e) of ybuf are not written.  An always-on shared expert
+ * ([P3] EducationalMoE) is this call with E = 1, C = T, used = NULL and the
+ * token matrix as xbuf.
+ *
+ * Arguments:
+ *   xbuf      device (E, C, D) contiguous, dtype `dtype`.
+ *   used      device int32 (E) or NULL.
+ *   w1,b1,w2,b2,w3 device, layouts above, dtype `dtype` (biases too);
+ *             unused ones may be NULL.
+ *   ybuf      device (E, C, Dout) contiguous, dtype `dtype`.
+ *   workspace device, >= moe_expert_ffn_workspace_size(...) bytes.
+ */
+MOE_API size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dtype, int32_t E, int64_t C,
+                                     int64_t F);
+MOE_API int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32_t* used,
+                   int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout, const void* w1,
+                   const void* b1, const void* w2, const void* b2, const void* w3, void* ybuf,
+                   int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                   moe_stream_t stream);
+
+/*
+ * moe_combine -- gate-weighted combine back to token order.
+ *   y[t,:] = base[t,:] + sum_{j : slot[t,j] >= 0} gate[t,j] * ybuf[e_{t,j}, slot[t,j], :]
+ * ([P1] section 1 item 4: y = x + sum over kept; [P2] y = shared + sum;
+ * [P4] step 6 and [P5]: no base, a dropped token gives a zero row).  The
+ * sum runs over j in ascending order in fp32 for every element, with no
+ * atomics, so the result is deterministic.
+ *
+ * Arguments:
+ *   ybuf      device (E, C, N) contiguous, dtype `dtype`.
+ *   selected, slot : device int64 (T, k), as produced by moe_route / moe_dispatch.
+ *   gates     device (T, k) of dtype `gate_dtype`, or NULL for all-ones.
+ *   base_kind MOE_BASE_ZERO (base ignored), MOE_BASE_INPUT or MOE_BASE_TENSOR
+ *             (base = device (T, N), row stride ldbase, dtype `dtype`).
+ *   y         device (T, N) row stride ldy, dtype `dtype`.
+ *   dev_status: MOE_ERR_BAD_INDEX for a kept assignment whose expert or slot
+ *             lies outside (E, C); such a term is skipped.
+ */
+MOE_API int moe_combine(const void* ybuf, const int64_t* selected, const int64_t* slot, const void* gates,
+                moe_dtype gate_dtype, int64_t T, int32_t k, int32_t E, int64_t C, int64_t N,
+                moe_base base_kind, const void* base, int64_t ldbase, void* y, int64_t ldy,
+                moe_dtype dtype, int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * moe_aux_stats -- load statistics and the Switch auxiliary loss.
+ *   f[e] = counts[e] / T                         ([P2] token_fraction, sums to k)
+ *   P[e] = prob_sum[e] / T                       ([P2] probability_mass, sums to 1)
+ *   aux[0] = E * sum_e (counts[e] / (T * kn)) * P[e]
+ *            kn = k if normalize_by_k ([P1] section 1 item 6, [P3]
+ *            switch_auxiliary_loss: 1 at uniform routing), else kn = 1 ([P5])
+ *   aux[1] = aux_coef * aux[0]
+ * f and P are written in `out_dtype`; aux in fp32.  Fixed-order reduction.
+ * All pointers device: counts int32 (E), prob_sum fp32 (E), f (E), P (E),
+ * aux fp32 (2).
+ */
+MOE_API int moe_aux_stats(const int32_t* counts, const float* prob_sum, int64_t T, int32_t E, int32_t k,
+                  int normalize_by_k, float aux_coef, void* f, void* P, moe_dtype out_dtype,
+                  float* aux, moe_stream_t stream);
+
+/*
+ * moe_backward -- backward of the linear-expert layer, the kept mask and the
+ * drops held constant ([P1] section 1 item 7 and section 2 moe_backward).
+ * fp32 only in this build (kind must be MOE_FFN_LINEAR, dtype MOE_F32).
+ *
+ * With out_{t,j} = x_t W_e^T (e = selected[t,j], kept) and the loss
+ * L = sum_t dy_t . y_t + aux_coef * aux:
+ *   dgate[t,j]    = kept ? dy_t . out_{t,j} : 0
+ *   dlogits[t,i]  = gate_i (dgate_i - sum_j gate_j dgate_j) on the selected
+ *                   experts, 0 elsewhere (gate = softmax of the selected
+ *                   logits), plus, when aux_coef != 0,
+ *                   aux_coef * E / (T*T*kn) * p[t,e] * (counts[e] - sum_e' counts[e'] p[t,e'])
+ *   dW[e]         = sum_{kept (t,j) -> e} gate * dy_t^T x_t      (E, Dout, D)
+ *   dx[t]         = [dy_t] + sum_{kept j} gate_j dy_t W_e        (T, D)
+ * The residual term [dy_t] needs Dout == D.
+ *
+ * Arguments (device unless noted):
+ *   dy (T, Dout), x (T, D), logits fp32 (T, E), selected int64 (T, k),
+ *   gates fp32 (T, k), slot int64 (T, k), used int32 (E),
+ *   token_of_slot int32 (E, C), xbuf (E, C, D) and ybuf (E, C, Dout) from
+ *   the forward (ybuf = ungated expert outputs), W (E, Dout, D),
+ *   counts int32 (E) (read only when aux_coef != 0).
+ *   Outputs dx (T, D), dW (E, Dout, D), dlogits fp32 (T, E), dgate fp32 (T, k).
+ *   workspace >= moe_backward_workspace_size(...) bytes.
+ */
+MOE_API size_t moe_backward_workspace_size(int32_t E, int64_t C, int64_t D, int64_t Dout);
+MOE_API int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, const void* x,
+                 const float* logits, const int64_t* selected, const float* gates,
+                 const int64_t* slot, const int32_t* used, const int32_t* token_of_slot,
+                 const void* xbuf, const void* ybuf, const void* W, int64_t T, int32_t k,
+                 int32_t E, int64_t C, int64_t D, int64_t Dout, int use_residual, float aux_coef,
+                 int normalize_by_k, const int32_t* counts, void* dx, void* dW, float* dlogits,
+                 float* dgate, int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                 moe_stream_t stream);
+
+/*
+ * moe_transpose_weights -- convert expert matrices from the pages' x @ W
+ * layout (E, K_in, N_out) to this library's (E, N_out, K_in), on device.
+ * src and dst must not overlap.  dtype f32 or bf16.
+ */
+MOE_API int moe_transpose_weights(const void* src, void* dst, int32_t E, int64_t K_in, int64_t N_out,
+                          moe_dtype dtype, moe_stream_t stream);
+
+/* Set the device status word to MOE_OK (stream-ordered). */
+MOE_API int moe_clear_status(int32_t* dev_status, moe_stream_t stream);
+
+/* Synchronise `stream`, then copy the device status word into *host_status
+ * (host pointer).  Returns MOE_ERR_CUDA if the synchronisation failed. */
+MOE_API int moe_read_status(const int32_t* dev_status, moe_stream_t stream, int32_t* host_status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

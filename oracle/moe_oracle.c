@@ -60,13 +60,18 @@ int64_t oracle_capacity(int64_t T, int32_t k, int32_t E, double capacity_factor)
 /* ------------------------------------------------------------------------ */
 void oracle_router_logits(const double* x, const double* w_router, const double* bias,
                           int64_t T, int64_t D, int32_t E, double* s) {
+    /* Each s[t,e] accumulates its D products in ascending d; the loop nest
+     * only walks w_router row by row. */
     OMP_FOR
     for (int64_t t = 0; t < T; ++t) {
-        for (int32_t e = 0; e < E; ++e) {
-            double acc = 0.0;
-            for (int64_t d = 0; d < D; ++d) acc += x[t * D + d] * w_router[d * E + e];
-            s[t * E + e] = acc + (bias ? bias[e] : 0.0);
+        double* acc = s + t * E;
+        for (int32_t e = 0; e < E; ++e) acc[e] = 0.0;
+        for (int64_t d = 0; d < D; ++d) {
+            const double xv = x[t * D + d];
+            const double* wr = w_router + d * E;
+            for (int32_t e = 0; e < E; ++e) acc[e] += xv * wr[e];
         }
+        for (int32_t e = 0; e < E; ++e) acc[e] += bias ? bias[e] : 0.0;
     }
 }
 
@@ -188,11 +193,9 @@ static double gelu_erf(double z) { return 0.5 * z * (1.0 + erf(z / sqrt(2.0))); 
 void oracle_expert_linear_row(const double* xrow, const double* W, int32_t e,
                               int64_t D, int64_t N, double* out) {
     const double* We = W + (int64_t)e * D * N;
-    for (int64_t n = 0; n < N; ++n) {
-        double acc = 0.0;
-        for (int64_t d = 0; d < D; ++d) acc += xrow[d] * We[d * N + n];
-        out[n] = acc;
-    }
+    for (int64_t n = 0; n < N; ++n) out[n] = 0.0;
+    for (int64_t d = 0; d < D; ++d)        /* out[n] sums over d ascending */
+        for (int64_t n = 0; n < N; ++n) out[n] += xrow[d] * We[d * N + n];
 }
 
 /* Two-layer GELU MLP with biases ([P5] Expert: fc2(gelu(fc1(x)))).
@@ -203,16 +206,14 @@ void oracle_expert_gelu_row(const double* xrow, const double* W1, const double* 
     double* h = (double*)malloc((size_t)F * sizeof(double));
     const double* W1e = W1 + (int64_t)e * D * F;
     const double* W2e = W2 + (int64_t)e * F * N;
-    for (int64_t f = 0; f < F; ++f) {
-        double acc = 0.0;
-        for (int64_t d = 0; d < D; ++d) acc += xrow[d] * W1e[d * F + f];
-        h[f] = gelu_erf(acc + b1[(int64_t)e * F + f]);
-    }
-    for (int64_t n = 0; n < N; ++n) {
-        double acc = 0.0;
-        for (int64_t f = 0; f < F; ++f) acc += h[f] * W2e[f * N + n];
-        out[n] = acc + b2[(int64_t)e * N + n];
-    }
+    for (int64_t f = 0; f < F; ++f) h[f] = 0.0;
+    for (int64_t d = 0; d < D; ++d)
+        for (int64_t f = 0; f < F; ++f) h[f] += xrow[d] * W1e[d * F + f];
+    for (int64_t f = 0; f < F; ++f) h[f] = gelu_erf(h[f] + b1[(int64_t)e * F + f]);
+    for (int64_t n = 0; n < N; ++n) out[n] = 0.0;
+    for (int64_t f = 0; f < F; ++f)
+        for (int64_t n = 0; n < N; ++n) out[n] += h[f] * W2e[f * N + n];
+    for (int64_t n = 0; n < N; ++n) out[n] += b2[(int64_t)e * N + n];
     free(h);
 }
 
@@ -225,16 +226,15 @@ void oracle_expert_swiglu_row(const double* xrow, const double* Wg, const double
     const double* Wge = Wg + (int64_t)e * D * F;
     const double* Wue = Wu + (int64_t)e * D * F;
     const double* Wde = Wd + (int64_t)e * F * N;
-    for (int64_t f = 0; f < F; ++f) {
-        double g = 0.0, u = 0.0;
-        for (int64_t d = 0; d < D; ++d) { g += xrow[d] * Wge[d * F + f]; u += xrow[d] * Wue[d * F + f]; }
-        h[f] = g * sigmoid_stable(g) * u;
-    }
-    for (int64_t n = 0; n < N; ++n) {
-        double acc = 0.0;
-        for (int64_t f = 0; f < F; ++f) acc += h[f] * Wde[f * N + n];
-        out[n] = acc;
-    }
+    double* u = (double*)malloc((size_t)F * sizeof(double));
+    for (int64_t f = 0; f < F; ++f) { h[f] = 0.0; u[f] = 0.0; }
+    for (int64_t d = 0; d < D; ++d)
+        for (int64_t f = 0; f < F; ++f) { h[f] += xrow[d] * Wge[d * F + f]; u[f] += xrow[d] * Wue[d * F + f]; }
+    for (int64_t f = 0; f < F; ++f) h[f] = h[f] * sigmoid_stable(h[f]) * u[f];
+    for (int64_t n = 0; n < N; ++n) out[n] = 0.0;
+    for (int64_t f = 0; f < F; ++f)
+        for (int64_t n = 0; n < N; ++n) out[n] += h[f] * Wde[f * N + n];
+    free(u);
     free(h);
 }
 

@@ -1,0 +1,12 @@
+"""Capacity-limited top-k sparse mixture-of-experts layer for NVIDIA B200 (sm_100a).
+
+The computation lives in ``libmoe.so`` (C ABI, ``include/moe.h``); this package
+holds the CUDA sources (``csrc/``), the build step (``build.py``), the ctypes
+binding (``binding.py``), a layer helper that chains the entry points with
+preallocated buffers (``layer.py``) and the seeded synthetic workloads
+(``inputs.py``).
+"""
+from .binding import (  # noqa: F401
+    EXPORTED, LIB_PATH, MoeError, lib, moe_aux_stats, moe_backward, moe_capacity, moe_clear_status, moe_combine,
+    moe_dispatch, moe_expert_ffn, moe_read_status, moe_route, moe_transpose_weights, new_status, status_string,
+)

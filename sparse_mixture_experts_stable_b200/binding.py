@@ -1,0 +1,339 @@
+"""Thin ctypes binding of ``libmoe.so`` (declared in ``include/moe.h``).
+
+Every function here has the name of the C entry point it calls and does only
+argument marshalling: it checks shapes and dtypes, allocates missing output and
+workspace tensors with PyTorch on the current CUDA device, and passes raw
+pointers plus the current stream.  All arithmetic runs in the CUDA library.
+There is no fallback: if ``libmoe.so`` is missing or fails to load, importing
+this module's functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_CUDA = 3
+MOE_ERR_BAD_INDEX = 4
+MOE_ERR_NONFINITE = 5
+MOE_ERR_TIMEOUT = 6
+MOE_ERR_WORKSPACE = 7
+
+MOE_F32, MOE_BF16 = 0, 1
+BASE = {"zero": 0, "input": 1, "tensor": 2}
+FFN = {"linear": 0, "gelu_mlp": 1, "swiglu": 2}
+ROUTER_LAYOUT = {"DE": 0, "ED": 1}
+
+EXPORTED = [
+    "moe_status_string", "moe_version", "moe_capacity", "moe_route_workspace_size", "moe_route",
+    "moe_dispatch_workspace_size", "moe_dispatch", "moe_expert_ffn_workspace_size", "moe_expert_ffn",
+    "moe_combine", "moe_aux_stats", "moe_backward_workspace_size", "moe_backward", "moe_transpose_weights",
+    "moe_clear_status", "moe_read_status",
+]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+
+
+_lib = None
+_vp, _i64, _i32, _sz, _f32, _f64 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t,
+                                     ctypes.c_float, ctypes.c_double)
+
+
+def lib():
+    """Load ``libmoe.so`` (raises OSError/FileNotFoundError when it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise FileNotFoundError(
+                f"{LIB_PATH} is not built; run `python -m sparse_mixture_experts_stable_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_version.restype = ctypes.c_int
+        L.moe_capacity.argtypes = [_i64, _i32, _i32, _f64, ctypes.POINTER(_i64)]
+        L.moe_route_workspace_size.restype = _sz
+        L.moe_route_workspace_size.argtypes = [_i64, _i64, _i32, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.moe_route.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, ctypes.c_int, _i32, _vp, _i32, _vp, _vp,
+                                _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_dispatch_workspace_size.restype = _sz
+        L.moe_dispatch_workspace_size.argtypes = [_i64, _i32, _i32]
+        L.moe_dispatch.argtypes = [_vp, _i64, _i32, _i32, _i64, _vp, ctypes.c_int, _i64, _i64, _vp, _vp, _vp, _vp,
+                                   _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_expert_ffn_workspace_size.restype = _sz
+        L.moe_expert_ffn_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, _i32, _i64, _i64]
+        L.moe_expert_ffn.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _vp,
+                                     _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_combine.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i64, _i32, _i32, _i64, _i64, ctypes.c_int,
+                                  _vp, _i64, _vp, _i64, ctypes.c_int, _vp, _vp]
+        L.moe_aux_stats.argtypes = [_vp, _vp, _i64, _i32, _i32, ctypes.c_int, _f32, _vp, _vp, ctypes.c_int, _vp,
+                                    _vp]
+        L.moe_backward_workspace_size.restype = _sz
+        L.moe_backward_workspace_size.argtypes = [_i32, _i64, _i64, _i64]
+        L.moe_backward.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, _i64, _i32, _i32, _i64, _i64, _i64, ctypes.c_int, _f32, ctypes.c_int, _vp,
+                                   _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_transpose_weights.argtypes = [_vp, _vp, _i32, _i64, _i64, ctypes.c_int, _vp]
+        L.moe_clear_status.argtypes = [_vp, _vp]
+        L.moe_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_i32)]
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().moe_status_string(int(code)).decode()
+
+
+def _check(fn: str, rc: int):
+    if rc != MOE_OK:
+        raise MoeError(fn, rc)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MOE_F32
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected float32 or bfloat16")
+
+
+def _tdt(code: int):
+    return torch.float32 if code == MOE_F32 else torch.bfloat16
+
+
+def _dev(t: torch.Tensor):
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    return t.device
+
+
+def _rowstride(t: torch.Tensor) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit column stride")
+    return t.stride(0)
+
+
+def _workspace(nbytes: int, device, ws: Optional[torch.Tensor]):
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise ValueError(f"workspace holds {ws.numel() * ws.element_size()} bytes, needs {nbytes}")
+        return ws
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def new_status(device=None) -> torch.Tensor:
+    """A zeroed device status word."""
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+# ------------------------------------------------------------------------------
+def moe_capacity(T: int, k: int, E: int, capacity_factor: float) -> int:
+    c = _i64(0)
+    _check("moe_capacity", lib().moe_capacity(T, k, E, float(capacity_factor), ctypes.byref(c)))
+    return int(c.value)
+
+
+def moe_route_workspace_size(T, D, E, dtype: int, has_router_weight: bool, layout: str = "ED") -> int:
+    return int(lib().moe_route_workspace_size(T, D, E, dtype, int(has_router_weight), ROUTER_LAYOUT[layout]))
+
+
+def moe_route(x: torch.Tensor, k: int, w_router: Optional[torch.Tensor] = None, layout: str = "ED",
+              E: Optional[int] = None, logit_bias: Optional[torch.Tensor] = None, want_logits: bool = False,
+              out: Optional[dict] = None, dev_status: Optional[torch.Tensor] = None,
+              workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Router scores, softmax, stable top-k, gates, counts and probability sums.
+
+    ``x`` is (T, D) activations with ``w_router`` given in ``layout`` ("ED" =
+    nn.Linear (E, D), "DE" = (D, E)), or (T, E) logits when ``w_router`` is None.
+    Returns a dict of device tensors: selected, gates (x dtype), gates_f32,
+    counts, prob_sum (and logits when requested).
+    """
+    dev = _dev(x)
+    dt = _dt(x)
+    T = x.shape[0]
+    if w_router is not None:
+        if w_router.dtype != x.dtype:
+            raise TypeError("w_router must have x's dtype")
+        D = x.shape[1]
+        E = w_router.shape[0] if layout == "ED" else w_router.shape[1]
+        w_router = w_router.contiguous()
+    else:
+        D = 0
+        E = x.shape[1]
+    o = dict(out or {})
+    o.setdefault("selected", torch.empty(T, k, dtype=torch.int64, device=dev))
+    o.setdefault("gates", torch.empty(T, k, dtype=x.dtype, device=dev))
+    o.setdefault("gates_f32", torch.empty(T, k, dtype=torch.float32, device=dev))
+    o.setdefault("counts", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("prob_sum", torch.empty(E, dtype=torch.float32, device=dev))
+    if want_logits:
+        o.setdefault("logits", torch.empty(T, E, dtype=torch.float32, device=dev))
+    ws = _workspace(moe_route_workspace_size(T, D, E, dt, w_router is not None, layout), dev, workspace)
+    bias = None if logit_bias is None else logit_bias.to(torch.float32).contiguous()
+    rc = lib().moe_route(_p(x), dt, T, D, _rowstride(x), _p(w_router), ROUTER_LAYOUT[layout], E, _p(bias), k,
+                         _p(o.get("logits")), _p(o["selected"]), _p(o["gates"]), _p(o["gates_f32"]),
+                         _p(o["counts"]), _p(o["prob_sum"]), _p(dev_status), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_route", rc)
+    return o
+
+
+def moe_dispatch_workspace_size(T: int, k: int, E: int) -> int:
+    return int(lib().moe_dispatch_workspace_size(T, k, E))
+
+
+def moe_dispatch(selected: torch.Tensor, E: int, C: int, x: Optional[torch.Tensor] = None,
+                 out: Optional[dict] = None, dev_status: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Greedy position-priority slots (+ gather of x into xbuf (E, C, D) when x is given)."""
+    dev = _dev(selected)
+    if selected.dtype != torch.int64:
+        raise TypeError("selected must be int64")
+    sel = selected.reshape(selected.shape[0], -1).contiguous()
+    T, k = sel.shape
+    o = dict(out or {})
+    o.setdefault("slot", torch.empty(T, k, dtype=torch.int64, device=dev))
+    o.setdefault("kept", torch.empty(T, k, dtype=torch.uint8, device=dev))
+    o.setdefault("used", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("overflow", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("drops", torch.empty(T, dtype=torch.int32, device=dev))
+    o.setdefault("token_of_slot", torch.empty(E, max(C, 0), dtype=torch.int32, device=dev))
+    dt, D, ldx = MOE_F32, 0, 0
+    if x is not None:
+        dt, D, ldx = _dt(x), x.shape[1], _rowstride(x)
+        o.setdefault("xbuf", torch.empty(E, C, D, dtype=x.dtype, device=dev))
+    ws = _workspace(moe_dispatch_workspace_size(T, k, E), dev, workspace)
+    rc = lib().moe_dispatch(_p(sel), T, k, E, C, _p(x), dt, D, ldx, _p(o["slot"]), _p(o["kept"]), _p(o["used"]),
+                            _p(o["overflow"]), _p(o["drops"]), _p(o["token_of_slot"]), _p(o.get("xbuf")),
+                            _p(dev_status), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_dispatch", rc)
+    return o
+
+
+def moe_expert_ffn_workspace_size(kind: str, dtype: int, E: int, C: int, F: int) -> int:
+    return int(lib().moe_expert_ffn_workspace_size(FFN[kind], dtype, E, C, F))
+
+
+def moe_expert_ffn(kind: str, xbuf: torch.Tensor, used: Optional[torch.Tensor], w1: torch.Tensor,
+                   b1: Optional[torch.Tensor] = None, w2: Optional[torch.Tensor] = None,
+                   b2: Optional[torch.Tensor] = None, w3: Optional[torch.Tensor] = None,
+                   ybuf: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Grouped expert FFN over an expert-major buffer xbuf (E, C, D); weights in (out, in) layout."""
+    dev = _dev(xbuf)
+    dt = _dt(xbuf)
+    E, C, D = xbuf.shape
+    if kind == "linear":
+        F, Dout = 0, w1.shape[1]
+    else:
+        F, Dout = w1.shape[1], w2.shape[1]
+    for w in (w1, b1, w2, b2, w3):
+        if w is not None and (w.dtype != xbuf.dtype or not w.is_contiguous()):
+            raise TypeError("weights must be contiguous and share xbuf's dtype")
+    if not xbuf.is_contiguous():
+        raise ValueError("xbuf must be contiguous")
+    if ybuf is None:
+        ybuf = torch.empty(E, C, Dout, dtype=xbuf.dtype, device=dev)
+    ws = _workspace(moe_expert_ffn_workspace_size(kind, dt, E, C, max(F, 1)), dev, workspace)
+    rc = lib().moe_expert_ffn(FFN[kind], dt, _p(xbuf), _p(used), E, C, D, F, Dout, _p(w1), _p(b1), _p(w2), _p(b2),
+                              _p(w3), _p(ybuf), _p(dev_status), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_expert_ffn", rc)
+    return ybuf
+
+
+def moe_combine(ybuf: torch.Tensor, selected: torch.Tensor, slot: torch.Tensor, gates: Optional[torch.Tensor],
+                base_kind: str = "zero", base: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                dev_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y = base + sum over kept assignments of gate * ybuf[e, slot] (fixed j order, fp32 accumulation)."""
+    dev = _dev(ybuf)
+    dt = _dt(ybuf)
+    E, C, N = ybuf.shape
+    sel = selected.reshape(selected.shape[0], -1).contiguous()
+    T, k = sel.shape
+    sl = slot.reshape(T, k).contiguous()
+    g = None if gates is None else gates.reshape(T, k).contiguous()
+    gdt = MOE_F32 if g is None else _dt(g)
+    if y is None:
+        y = torch.empty(T, N, dtype=ybuf.dtype, device=dev)
+    ldb = _rowstride(base) if base is not None else 0
+    rc = lib().moe_combine(_p(ybuf), _p(sel), _p(sl), _p(g), gdt, T, k, E, C, N, BASE[base_kind], _p(base), ldb,
+                           _p(y), _rowstride(y), dt, _p(dev_status), _stream(stream))
+    _check("moe_combine", rc)
+    return y
+
+
+def moe_aux_stats(counts: torch.Tensor, prob_sum: torch.Tensor, T: int, k: int, normalize_by_k: bool = True,
+                  aux_coef: float = 0.0, out_dtype=torch.float32, stream=None):
+    """(f, P, aux) with aux = tensor([aux, aux_coef * aux])."""
+    dev = _dev(counts)
+    E = counts.shape[0]
+    f = torch.empty(E, dtype=out_dtype, device=dev)
+    P = torch.empty(E, dtype=out_dtype, device=dev)
+    aux = torch.empty(2, dtype=torch.float32, device=dev)
+    rc = lib().moe_aux_stats(_p(counts), _p(prob_sum), T, E, k, int(bool(normalize_by_k)), float(aux_coef), _p(f),
+                             _p(P), MOE_BF16 if out_dtype == torch.bfloat16 else MOE_F32, _p(aux), _stream(stream))
+    _check("moe_aux_stats", rc)
+    return f, P, aux
+
+
+def moe_backward_workspace_size(E: int, C: int, D: int, Dout: int) -> int:
+    return int(lib().moe_backward_workspace_size(E, C, D, Dout))
+
+
+def moe_backward(dy, x, logits, selected, gates_f32, slot, used, token_of_slot, xbuf, ybuf, W, C: int,
+                 use_residual: bool = True, aux_coef: float = 0.0, normalize_by_k: bool = True, counts=None,
+                 dev_status=None, workspace=None, stream=None):
+    """Backward of the fp32 linear-expert layer.  Returns (dx, dW, dlogits, dgate)."""
+    dev = _dev(dy)
+    T, Dout = dy.shape
+    E, _, D = xbuf.shape
+    k = selected.shape[1]
+    dx = torch.empty(T, D, dtype=dy.dtype, device=dev)
+    dW = torch.empty(E, Dout, D, dtype=dy.dtype, device=dev)
+    dl = torch.empty(T, E, dtype=torch.float32, device=dev)
+    dg = torch.empty(T, k, dtype=torch.float32, device=dev)
+    ws = _workspace(moe_backward_workspace_size(E, C, D, Dout), dev, workspace)
+    rc = lib().moe_backward(FFN["linear"], _dt(dy), _p(dy), _p(x), _p(logits), _p(selected), _p(gates_f32), _p(slot),
+                            _p(used), _p(token_of_slot), _p(xbuf), _p(ybuf), _p(W), T, k, E, C, D, Dout,
+                            int(bool(use_residual)), float(aux_coef), int(bool(normalize_by_k)), _p(counts), _p(dx),
+                            _p(dW), _p(dl), _p(dg), _p(dev_status), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_backward", rc)
+    return dx, dW, dl, dg
+
+
+def moe_transpose_weights(src: torch.Tensor, stream=None) -> torch.Tensor:
+    """(E, K_in, N_out) x@W matrices -> (E, N_out, K_in) (out, in) layout."""
+    E, K, N = src.shape
+    dst = torch.empty(E, N, K, dtype=src.dtype, device=src.device)
+    rc = lib().moe_transpose_weights(_p(src.contiguous()), _p(dst), E, K, N, _dt(src), _stream(stream))
+    _check("moe_transpose_weights", rc)
+    return dst
+
+
+def moe_clear_status(dev_status: torch.Tensor, stream=None):
+    _check("moe_clear_status", lib().moe_clear_status(_p(dev_status), _stream(stream)))
+
+
+def moe_read_status(dev_status: torch.Tensor, stream=None) -> int:
+    h = _i32(0)
+    _check("moe_read_status", lib().moe_read_status(_p(dev_status), _stream(stream), ctypes.byref(h)))
+    return int(h.value)

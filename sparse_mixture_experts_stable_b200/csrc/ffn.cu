@@ -1,0 +1,173 @@
+// moe_expert_ffn: the expert FFNs as grouped GEMMs over variable-occupancy
+// experts.  bf16 runs on the tcgen05 tensor cores (tc_gemm), fp32 on FFMA.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "simt_gemm.cuh"
+#include "tc_gemm.cuh"
+
+using namespace moe;
+
+extern "C" size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dtype, int32_t E, int64_t C,
+                                                int64_t F) {
+    if (kind == MOE_FFN_LINEAR || E < 1 || C < 1 || F < 1) return 0;
+    return align_up((size_t)E * C * F * dtype_size(dtype), 1024);
+}
+
+extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32_t* used, int32_t E,
+                              int64_t C, int64_t D, int64_t F, int64_t Dout, const void* w1, const void* b1,
+                              const void* w2, const void* b2, const void* w3, void* ybuf, int32_t* dev_status,
+                              void* workspace, size_t workspace_bytes, moe_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    MOE_REQUIRE(valid_dtype(dtype), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(kind == MOE_FFN_LINEAR || kind == MOE_FFN_GELU_MLP || kind == MOE_FFN_SWIGLU, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(xbuf && ybuf && w1 && E >= 1 && C >= 0 && D >= 1 && Dout >= 1, MOE_ERR_INVALID_ARG);
+    if (C == 0) return MOE_OK;
+    if (kind == MOE_FFN_GELU_MLP) MOE_REQUIRE(b1 && w2 && b2 && F >= 1, MOE_ERR_INVALID_ARG);
+    if (kind == MOE_FFN_SWIGLU) MOE_REQUIRE(w2 && w3 && F >= 1, MOE_ERR_INVALID_ARG);
+    void* h = nullptr;
+    if (kind != MOE_FFN_LINEAR) {
+        MOE_REQUIRE(workspace && workspace_bytes >= moe_expert_ffn_workspace_size(kind, dtype, E, C, F),
+                    MOE_ERR_WORKSPACE);
+        h = workspace;
+    }
+
+    if (dtype == MOE_BF16) {
+        // first GEMM: xbuf (E*C, D) x W^T
+        TcGemmProblem p{};
+        p.a = xbuf;
+        p.lda = D;
+        p.a_rows_total = (int64_t)E * C;
+        p.a_rows_per_group = C;
+        p.G = E;
+        p.M = C;
+        p.K = D;
+        p.rows = used;
+        p.out_rows_per_group = C;
+        p.status = dev_status;
+        if (kind == MOE_FFN_LINEAR) {
+            p.b = w1;
+            p.ldb = D;
+            p.b_rows_total = (int64_t)E * Dout;
+            p.b_rows_per_group = Dout;
+            p.N = Dout;
+            p.out = ybuf;
+            p.ldo = Dout;
+            p.epilogue = TC_EPI_BF16;
+            return tc_gemm_run(p, stream);
+        }
+        p.ldb = D;
+        p.b_rows_total = (int64_t)E * F;
+        p.b_rows_per_group = F;
+        p.N = F;
+        p.out = h;
+        p.ldo = F;
+        if (kind == MOE_FFN_SWIGLU) {
+            p.b = w1;   // gate
+            p.b2 = w3;  // up
+            p.epilogue = TC_EPI_SWIGLU;
+        } else {
+            p.b = w1;
+            p.bias = b1;
+            p.bias_group_stride = F;
+            p.epilogue = TC_EPI_GELU_BIAS;
+        }
+        int rc = tc_gemm_run(p, stream);
+        if (rc != MOE_OK) return rc;
+        // second GEMM: h (E*C, F) x W2^T
+        TcGemmProblem q{};
+        q.a = h;
+        q.lda = F;
+        q.a_rows_total = (int64_t)E * C;
+        q.a_rows_per_group = C;
+        q.b = w2;
+        q.ldb = F;
+        q.b_rows_total = (int64_t)E * Dout;
+        q.b_rows_per_group = Dout;
+        q.G = E;
+        q.M = C;
+        q.N = Dout;
+        q.K = F;
+        q.rows = used;
+        q.out = ybuf;
+        q.ldo = Dout;
+        q.out_rows_per_group = C;
+        q.status = dev_status;
+        if (kind == MOE_FFN_GELU_MLP) {
+            q.bias = b2;
+            q.bias_group_stride = Dout;
+            q.epilogue = TC_EPI_BF16_BIAS;
+        } else {
+            q.epilogue = TC_EPI_BF16;
+        }
+        return tc_gemm_run(q, stream);
+    }
+
+    // fp32: FFMA GEMMs, B = weights in (out, in) layout -> transposed operand
+    SimtGemm g{};
+    g.A = static_cast<const float*>(xbuf);
+    g.lda = D;
+    g.a_group_stride = C * D;
+    g.b_trans = true;
+    g.M = C;
+    g.K = D;
+    g.groups = E;
+    g.rows = used;
+    g.rows_mode = used ? 1 : 0;
+    if (kind == MOE_FFN_LINEAR) {
+        g.B = static_cast<const float*>(w1);
+        g.ldb = D;
+        g.b_group_stride = Dout * D;
+        g.C = static_cast<float*>(ybuf);
+        g.ldc = Dout;
+        g.c_group_stride = C * Dout;
+        g.N = Dout;
+        return simt_gemm_run(g, stream);
+    }
+    float* hf = static_cast<float*>(h);
+    g.ldb = D;
+    g.b_group_stride = F * D;
+    g.C = hf;
+    g.ldc = F;
+    g.c_group_stride = C * F;
+    g.N = F;
+    int rc;
+    if (kind == MOE_FFN_GELU_MLP) {
+        g.B = static_cast<const float*>(w1);
+        g.bias = static_cast<const float*>(b1);
+        g.bias_group_stride = F;
+        g.epilogue = SIMT_EPI_BIAS_GELU;
+        rc = simt_gemm_run(g, stream);
+    } else {
+        g.B = static_cast<const float*>(w3);  // up -> h
+        rc = simt_gemm_run(g, stream);
+        if (rc != MOE_OK) return rc;
+        g.B = static_cast<const float*>(w1);  // gate: h = silu(gate) * up
+        g.epilogue = SIMT_EPI_SILU_MUL;
+        rc = simt_gemm_run(g, stream);
+    }
+    if (rc != MOE_OK) return rc;
+    SimtGemm d{};
+    d.A = hf;
+    d.lda = F;
+    d.a_group_stride = C * F;
+    d.B = static_cast<const float*>(w2);
+    d.ldb = F;
+    d.b_trans = true;
+    d.b_group_stride = Dout * F;
+    d.C = static_cast<float*>(ybuf);
+    d.ldc = Dout;
+    d.c_group_stride = C * Dout;
+    d.M = C;
+    d.N = Dout;
+    d.K = F;
+    d.groups = E;
+    d.rows = used;
+    d.rows_mode = used ? 1 : 0;
+    if (kind == MOE_FFN_GELU_MLP) {
+        d.bias = static_cast<const float*>(b2);
+        d.bias_group_stride = Dout;
+        d.epilogue = SIMT_EPI_BIAS;
+    }
+    return simt_gemm_run(d, stream);
+}

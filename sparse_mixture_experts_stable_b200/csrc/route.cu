@@ -1,0 +1,385 @@
+// moe_route and moe_aux_stats.
+//
+// Router scores come from the tensor-core GEMM (bf16) or the FFMA GEMM (fp32),
+// written as fp32 logits; then one warp per token does softmax, top-k and the
+// renormalised gates entirely in registers, and each block leaves per-expert
+// partial counts and probability sums that a second kernel adds up in a fixed
+// order (so prob_sum is bitwise reproducible).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "simt_gemm.cuh"
+#include "tc_gemm.cuh"
+#include "util_kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kRouteWarps = 8;
+constexpr int kRouteThreads = kRouteWarps * 32;
+constexpr int kMaxRouteBlocks = 1024;
+constexpr int kMaxK = 64;
+constexpr int kMaxE = 1024;
+
+int route_blocks(int64_t T) {
+    int64_t b = (T + kRouteWarps - 1) / kRouteWarps;
+    return (int)(b < kMaxRouteBlocks ? b : kMaxRouteBlocks);
+}
+
+// Is (v, i) ranked ahead of (bv, bi)?  Larger score first, then lower index.
+__device__ __forceinline__ bool ahead(float v, int i, float bv, int bi) {
+    return v > bv || (v == bv && i < bi);
+}
+
+// Each lane holds experts e = m*32 + lane, m < EPL.
+template <int EPL, typename InT>
+__global__ void __launch_bounds__(kRouteThreads)
+    route_topk_kernel(const InT* __restrict__ logits, int64_t ld, int64_t T, int E, int k,
+                      const float* __restrict__ bias, float* __restrict__ logits_out,
+                      int64_t* __restrict__ selected, void* __restrict__ gates_out, int gates_bf16,
+                      float* __restrict__ gates_f32, int32_t* __restrict__ part_counts,
+                      float* __restrict__ part_psum, int32_t* status) {
+    extern __shared__ float s_dyn[];
+    float* s_psum = s_dyn;                                            // [kRouteWarps][E]
+    int* s_counts = reinterpret_cast<int*>(s_psum + kRouteWarps * E);  // [E]
+    float* s_selv = reinterpret_cast<float*>(s_counts + E);            // [kRouteWarps][k]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_counts[e] = 0;
+    __syncthreads();
+
+    float bias_r[EPL];
+    float psum[EPL];
+#pragma unroll
+    for (int m = 0; m < EPL; ++m) {
+        const int e = m * 32 + lane;
+        bias_r[m] = (bias && e < E) ? bias[e] : 0.f;
+        psum[m] = 0.f;
+    }
+    float* selv = s_selv + warp * k;
+
+    const int64_t stride = (int64_t)gridDim.x * kRouteWarps;
+    for (int64_t t = (int64_t)blockIdx.x * kRouteWarps + warp; t < T; t += stride) {
+        const InT* row = logits + t * ld;
+        float v[EPL];
+        uint32_t taken = 0;
+        bool finite = true;
+#pragma unroll
+        for (int m = 0; m < EPL; ++m) {
+            const int e = m * 32 + lane;
+            if (e < E) {
+                float x = to_f32(row[e]) + bias_r[m];
+                if (!isfinite(x)) {
+                    finite = false;
+                    x = -INFINITY;
+                }
+                v[m] = x;
+                if (logits_out) logits_out[t * E + e] = x;
+            } else {
+                v[m] = -INFINITY;
+                taken |= 1u << m;
+            }
+        }
+        if (!__all_sync(0xffffffffu, finite) && lane == 0) set_status(status, MOE_ERR_NONFINITE);
+
+        // top-k: k rounds of (local best, warp arg-max with index tie-break)
+        float vmax = 0.f;
+        for (int j = 0; j < k; ++j) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int m = 0; m < EPL; ++m) {
+                const int e = m * 32 + lane;
+                if (!((taken >> m) & 1u) && ahead(v[m], e, bv, bi)) {
+                    bv = v[m];
+                    bi = e;
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (ahead(ov, oi, bv, bi)) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if (j == 0) vmax = bv;
+            if (lane == 0) {
+                selv[j] = bv;
+                selected[t * k + j] = bi;
+                atomicAdd(&s_counts[bi], 1);
+            }
+        }
+        __syncwarp();
+
+        // softmax over all experts (max-subtracted), accumulated per expert
+        float part = 0.f;
+        float ex[EPL];
+#pragma unroll
+        for (int m = 0; m < EPL; ++m) {
+            const int e = m * 32 + lane;
+            ex[m] = e < E ? expf(v[m] - vmax) : 0.f;
+            part += ex[m];
+        }
+        const float inv = 1.0f / warp_sum(part);
+#pragma unroll
+        for (int m = 0; m < EPL; ++m) psum[m] += ex[m] * inv;
+
+        // renormalised gates = softmax over the selected scores
+        float gp = 0.f;
+        for (int j = lane; j < k; j += 32) gp += expf(selv[j] - vmax);
+        const float ginv = 1.0f / warp_sum(gp);
+        for (int j = lane; j < k; j += 32) {
+            const float g = expf(selv[j] - vmax) * ginv;
+            if (gates_f32) gates_f32[t * k + j] = g;
+            if (gates_out) {
+                if (gates_bf16) reinterpret_cast<__nv_bfloat16*>(gates_out)[t * k + j] = __float2bfloat16_rn(g);
+                else reinterpret_cast<float*>(gates_out)[t * k + j] = g;
+            }
+        }
+        __syncwarp();
+    }
+
+    // block partials in a fixed order: warps 0..7, then per block slot
+#pragma unroll
+    for (int m = 0; m < EPL; ++m) {
+        const int e = m * 32 + lane;
+        if (e < E) s_psum[warp * E + e] = psum[m];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float s = 0.f;
+        for (int w = 0; w < kRouteWarps; ++w) s += s_psum[w * E + e];
+        part_psum[(int64_t)blockIdx.x * E + e] = s;
+        part_counts[(int64_t)blockIdx.x * E + e] = s_counts[e];
+    }
+}
+
+// counts[e] and prob_sum[e] = fixed-order sums of the block partials.
+__global__ void route_reduce_kernel(const int32_t* __restrict__ part_counts, const float* __restrict__ part_psum,
+                                    int nblocks, int E, int32_t* __restrict__ counts, float* __restrict__ prob_sum) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= E) return;
+    int c = 0;
+    float s = 0.f;
+    for (int b = 0; b < nblocks; ++b) {
+        c += part_counts[(int64_t)b * E + e];
+        s += part_psum[(int64_t)b * E + e];
+    }
+    counts[e] = c;
+    prob_sum[e] = s;
+}
+
+template <typename InT>
+int launch_topk(int epl, const InT* logits, int64_t ld, int64_t T, int E, int k, const float* bias,
+                float* logits_out, int64_t* selected, void* gates, int gates_bf16, float* gates_f32,
+                int32_t* part_counts, float* part_psum, int32_t* status, cudaStream_t stream) {
+    const int nb = route_blocks(T);
+    const size_t smem = sizeof(float) * (size_t)kRouteWarps * E + sizeof(int) * (size_t)E +
+                        sizeof(float) * (size_t)kRouteWarps * k;
+#define MOE_TOPK_CASE(N)                                                                                      \
+    case N: {                                                                                                 \
+        auto kern = route_topk_kernel<N, InT>;                                                                \
+        if (smem > 48 * 1024)                                                                                 \
+            MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); \
+        kern<<<nb, kRouteThreads, smem, stream>>>(logits, ld, T, E, k, bias, logits_out, selected, gates,     \
+                                                  gates_bf16, gates_f32, part_counts, part_psum, status);     \
+        break;                                                                                                \
+    }
+    switch (epl) {
+        MOE_TOPK_CASE(1)
+        MOE_TOPK_CASE(2)
+        MOE_TOPK_CASE(4)
+        MOE_TOPK_CASE(8)
+        MOE_TOPK_CASE(16)
+        MOE_TOPK_CASE(32)
+        default: return MOE_ERR_UNSUPPORTED;
+    }
+#undef MOE_TOPK_CASE
+    return launch_status();
+}
+
+int epl_for(int E) {
+    int epl = 1;
+    while (epl * 32 < E) epl *= 2;
+    return epl;
+}
+
+struct RouteWs {
+    size_t logits_off, wt_off, pc_off, pp_off, total;
+};
+
+RouteWs route_ws_layout(int64_t T, int64_t D, int32_t E, moe_dtype dtype, int has_w, moe_router_layout layout) {
+    RouteWs w{};
+    size_t off = 0;
+    w.logits_off = off;
+    if (has_w) off += align_up((size_t)T * E * sizeof(float), 256);
+    w.wt_off = off;
+    if (has_w && dtype == MOE_BF16 && layout == MOE_ROUTER_DE) off += align_up((size_t)E * D * 2, 256);
+    const int nb = route_blocks(T);
+    w.pc_off = off;
+    off += align_up((size_t)nb * E * sizeof(int32_t), 256);
+    w.pp_off = off;
+    off += align_up((size_t)nb * E * sizeof(float), 256);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" size_t moe_route_workspace_size(int64_t T, int64_t D, int32_t E, moe_dtype dtype, int has_router_weight,
+                                           moe_router_layout layout) {
+    if (T < 1 || E < 1) return 0;
+    return route_ws_layout(T, D, E, dtype, has_router_weight, layout).total;
+}
+
+extern "C" int moe_route(const void* x, moe_dtype dtype, int64_t T, int64_t D, int64_t ldx, const void* w_router,
+                         moe_router_layout layout, int32_t E, const float* logit_bias, int32_t k, float* logits_out,
+                         int64_t* selected, void* gates, float* gates_f32, int32_t* counts, float* prob_sum,
+                         int32_t* dev_status, void* workspace, size_t workspace_bytes, moe_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    MOE_REQUIRE(valid_dtype(dtype), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(x && selected && counts && prob_sum, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(T >= 1 && E >= 1 && k >= 1 && k <= E, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(E <= kMaxE && k <= kMaxK, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(layout == MOE_ROUTER_DE || layout == MOE_ROUTER_ED, MOE_ERR_INVALID_ARG);
+    const int has_w = w_router != nullptr;
+    if (has_w) MOE_REQUIRE(D >= 1 && ldx >= D, MOE_ERR_INVALID_ARG);
+    else MOE_REQUIRE(ldx >= E, MOE_ERR_INVALID_ARG);
+    const RouteWs wl = route_ws_layout(T, D, E, dtype, has_w, layout);
+    MOE_REQUIRE(workspace != nullptr && workspace_bytes >= wl.total, MOE_ERR_WORKSPACE);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* part_counts = reinterpret_cast<int32_t*>(ws + wl.pc_off);
+    float* part_psum = reinterpret_cast<float*>(ws + wl.pp_off);
+    const int epl = epl_for(E);
+    const int gates_bf16 = dtype == MOE_BF16;
+    int rc = MOE_OK;
+
+    if (has_w) {
+        // scores s = x . W (+ bias) into fp32 logits
+        float* lg = logits_out ? logits_out : reinterpret_cast<float*>(ws + wl.logits_off);
+        if (dtype == MOE_BF16) {
+            const void* w_ed = w_router;
+            if (layout == MOE_ROUTER_DE) {
+                void* wt = ws + wl.wt_off;
+                rc = transpose_matrices(w_router, wt, 1, D, E, MOE_BF16, stream);
+                if (rc != MOE_OK) return rc;
+                w_ed = wt;
+            }
+            TcGemmProblem p{};
+            p.a = x;
+            p.lda = ldx;
+            p.a_rows_total = T;
+            p.a_rows_per_group = 0;
+            p.b = w_ed;
+            p.b2 = nullptr;
+            p.ldb = D;
+            p.b_rows_total = E;
+            p.b_rows_per_group = 0;
+            p.G = 1;
+            p.M = T;
+            p.N = E;
+            p.K = D;
+            p.rows = nullptr;
+            p.out = lg;
+            p.ldo = E;
+            p.out_rows_per_group = 0;
+            p.bias = logit_bias;
+            p.bias_group_stride = 0;
+            p.epilogue = TC_EPI_F32;
+            p.status = dev_status;
+            rc = tc_gemm_run(p, stream);
+        } else {
+            SimtGemm g{};
+            g.A = static_cast<const float*>(x);
+            g.lda = ldx;
+            g.a_trans = false;
+            g.B = static_cast<const float*>(w_router);
+            // B(k=d, n=e): (D,E) row-major is "not transposed"; (E,D) is transposed.
+            g.b_trans = layout == MOE_ROUTER_ED;
+            g.ldb = layout == MOE_ROUTER_ED ? D : E;
+            g.C = lg;
+            g.ldc = E;
+            g.M = T;
+            g.N = E;
+            g.K = D;
+            g.groups = 1;
+            g.bias = logit_bias;
+            g.epilogue = SIMT_EPI_BIAS;
+            rc = simt_gemm_run(g, stream);
+        }
+        if (rc != MOE_OK) return rc;
+        rc = launch_topk<float>(epl, lg, E, T, E, k, nullptr, nullptr, selected, gates, gates_bf16, gates_f32,
+                                part_counts, part_psum, dev_status, stream);
+    } else if (dtype == MOE_BF16) {
+        rc = launch_topk<__nv_bfloat16>(epl, static_cast<const __nv_bfloat16*>(x), ldx, T, E, k, logit_bias,
+                                        logits_out, selected, gates, gates_bf16, gates_f32, part_counts, part_psum,
+                                        dev_status, stream);
+    } else {
+        rc = launch_topk<float>(epl, static_cast<const float*>(x), ldx, T, E, k, logit_bias, logits_out, selected,
+                                gates, gates_bf16, gates_f32, part_counts, part_psum, dev_status, stream);
+    }
+    if (rc != MOE_OK) return rc;
+    const int nb = route_blocks(T);
+    route_reduce_kernel<<<(E + 255) / 256, 256, 0, stream>>>(part_counts, part_psum, nb, E, counts, prob_sum);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// moe_aux_stats
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+__global__ void aux_stats_kernel(const int32_t* __restrict__ counts, const float* __restrict__ prob_sum, int64_t T,
+                                 int E, float kn, float aux_coef, void* f_out, void* P_out, int out_bf16,
+                                 float* aux) {
+    __shared__ float s_red[1024];
+    float acc = 0.f;
+    const float invT = 1.0f / (float)T;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const float c = (float)counts[e];
+        const float f = c * invT;
+        const float P = prob_sum[e] * invT;
+        if (out_bf16) {
+            reinterpret_cast<__nv_bfloat16*>(f_out)[e] = __float2bfloat16_rn(f);
+            reinterpret_cast<__nv_bfloat16*>(P_out)[e] = __float2bfloat16_rn(P);
+        } else {
+            reinterpret_cast<float*>(f_out)[e] = f;
+            reinterpret_cast<float*>(P_out)[e] = P;
+        }
+        acc += (c / ((float)T * kn)) * P;
+    }
+    s_red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+        if (threadIdx.x < s) s_red[threadIdx.x] += s_red[threadIdx.x + s];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const float a = (float)E * s_red[0];
+        aux[0] = a;
+        aux[1] = aux_coef * a;
+    }
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_aux_stats(const int32_t* counts, const float* prob_sum, int64_t T, int32_t E, int32_t k,
+                             int normalize_by_k, float aux_coef, void* f, void* P, moe_dtype out_dtype, float* aux,
+                             moe_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    MOE_REQUIRE(counts && prob_sum && f && P && aux, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(T >= 1 && E >= 1 && k >= 1 && valid_dtype(out_dtype), MOE_ERR_INVALID_ARG);
+    aux_stats_kernel<<<1, 1024, 0, stream>>>(counts, prob_sum, T, E, normalize_by_k ? (float)k : 1.0f, aux_coef, f, P,
+                                             out_dtype == MOE_BF16, aux);
+    return launch_status();
+}

@@ -1,0 +1,579 @@
+// Grouped bf16 GEMM on sm_100a: TMA (128B swizzle) -> shared memory ->
+// tcgen05.mma (kind::f16, fp32 accumulate in TMEM) -> tcgen05.ld -> epilogue.
+//
+// Warp roles in a 192-thread persistent CTA (one per SM):
+//   warp 0      : TMA producer (one lane), 4-stage smem ring
+//   warp 1      : TMEM allocator and MMA issuer (one lane)
+//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4) .. 32*(w%4)+31
+// The accumulator is double-buffered in TMEM (2 x 256 fp32 columns), so the
+// epilogue of one tile overlaps the main loop of the next.
+//
+// Every wait on an mbarrier is bounded (kWaitLimitNs); on expiry the kernel
+// records MOE_ERR_TIMEOUT, every role leaves its loop, and TMEM is freed.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "tc_gemm.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;      // UMMA M (one CTA)
+constexpr int kBK = 64;       // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int kBN = 256;      // TMEM columns per accumulator buffer / max UMMA N
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kMaxGroups = 1024;
+constexpr int kABytes = kBM * kBK * 2;  // 16 KB
+constexpr int kBBytes = kBN * kBK * 2;  // 32 KB
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * (kABytes + kBBytes) + 256;
+
+struct KParams {
+    int G;
+    int64_t a_rows_per_group;
+    int64_t b_rows_per_group;
+    int64_t M;
+    int64_t N;
+    int n_tiles;
+    int n_mma;        // UMMA N (multiple of 32, <= 256)
+    int tile_n_out;   // output columns produced per tile
+    int b_box_rows;   // rows per B TMA box (n_mma, or n_mma/2 for the dual form)
+    int k_blocks;
+    uint32_t tx_bytes;
+    const int32_t* rows;
+    void* out;
+    int64_t ldo;
+    int64_t out_rows_per_group;
+    const void* bias;
+    int64_t bias_group_stride;
+    int vec_ok;
+    int32_t* status;
+};
+
+// ------------------------------- PTX wrappers -------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(a, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            set_status(status, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand tile written by TMA with
+// 128-byte swizzle; rows of 128 bytes, 8-row core groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address (16-byte units)
+    d |= (uint64_t)1 << 16;                    // leading byte offset (unused with this swizzle)
+    d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: next 8-row group
+    d |= (uint64_t)1 << 46;                    // descriptor version for tcgen05
+    d |= (uint64_t)2 << 61;                    // layout: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major.
+__device__ __forceinline__ uint32_t make_idesc(int m, int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+// Wait for outstanding tcgen05.ld; the registers are tied in so that no use of
+// them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+          "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+          "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
+          "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+          "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+        :
+        : "memory");
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+__device__ __forceinline__ float gelu_f(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Map a linear tile index to (group, m-tile, n-tile).  prefix[g] is the first
+// tile of group g; tiles of a group run m fastest so that concurrently active
+// CTAs share the group's weight tile.
+__device__ __forceinline__ void decode_tile(int tile, const int* prefix, int G, int n_tiles, int& g,
+                                            int& mt, int& nt) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= tile) lo = mid;
+        else hi = mid - 1;
+    }
+    g = lo;
+    const int local = tile - prefix[g];
+    const int mtiles = (prefix[g + 1] - prefix[g]) / n_tiles;
+    nt = local / mtiles;
+    mt = local - nt * mtiles;
+}
+
+// Store 32 bf16 values (already packed in pairs) for columns n0..n0+31 of one row.
+__device__ __forceinline__ void store_bf16_32(__nv_bfloat16* row, int64_t n0, int64_t N, const uint32_t (&pk)[16],
+                                              bool vec) {
+    if (vec && n0 + 32 <= N) {
+        uint4* dst = reinterpret_cast<uint4*>(row + n0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (n0 + i < N) {
+                const uint32_t w = pk[i >> 1];
+                const uint16_t h = (i & 1) ? (uint16_t)(w >> 16) : (uint16_t)(w & 0xFFFFu);
+                row[n0 + i] = __ushort_as_bfloat16(h);
+            }
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB2, const KParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ int s_prefix[kMaxGroups + 1];
+    __shared__ uint32_t s_tmem;
+    __shared__ volatile int s_abort;
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smA = smem;
+    uint8_t* smB = smem + kStages * kABytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smB + kStages * kBBytes);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + kStages;
+    uint64_t* tfull = bars + 2 * kStages;
+    uint64_t* tempty = bars + 2 * kStages + 2;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- setup: barriers, TMEM, tile table ----
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                     "r"(2 * kBN)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    for (int g = threadIdx.x; g < p.G; g += blockDim.x) {
+        int64_t r = p.rows ? (int64_t)p.rows[g] : p.M;
+        r = r < 0 ? 0 : (r > p.M ? p.M : r);
+        s_prefix[g + 1] = (int)((r + kBM - 1) / kBM);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0) {
+        s_prefix[0] = 0;
+        for (int g = 0; g < p.G; ++g) s_prefix[g + 1] = s_prefix[g] + s_prefix[g + 1] * p.n_tiles;
+    }
+    __syncthreads();
+    const int total = s_prefix[p.G];
+    const uint32_t tmem_base = s_tmem;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
+                int g, mt, nt;
+                decode_tile(tile, s_prefix, p.G, p.n_tiles, g, mt, nt);
+                const int32_t a_y = (int32_t)(g * p.a_rows_per_group + (int64_t)mt * kBM);
+                const int32_t b_y = (int32_t)(g * p.b_rows_per_group + (int64_t)nt * p.b_box_rows);
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) {
+                        s_abort = 1;
+                        break;
+                    }
+                    mbar_expect_tx(&full[stage], p.tx_bytes);
+                    uint8_t* a_dst = smA + stage * kABytes;
+                    uint8_t* b_dst = smB + stage * kBBytes;
+                    tma_load_2d(a_dst, &tmA, kb * kBK, a_y, &full[stage]);
+                    tma_load_2d(b_dst, &tmB, kb * kBK, b_y, &full[stage]);
+                    if (EPI == TC_EPI_SWIGLU)
+                        tma_load_2d(b_dst + p.b_box_rows * (kBK * 2), &tmB2, kb * kBK, b_y, &full[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer -------------------------------
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc(kBM, p.n_mma);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t it = 0;
+            for (int tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x, ++it) {
+                const uint32_t acc = it & 1u;
+                const uint32_t acc_phase = (it >> 1) & 1u;
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status)) {
+                    s_abort = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * kBN;
+                bool ok = true;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, p.status)) {
+                        s_abort = 1;
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(smem_u32(smA + stage * kABytes));
+                    const uint64_t bd = sw128_desc(smem_u32(smB + stage * kBBytes));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        tc_mma(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&empty[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&tfull[acc]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // -------------------------------- epilogue --------------------------------
+        const int q = warp & 3;
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+            int g, mt, nt;
+            decode_tile(tile, s_prefix, p.G, p.n_tiles, g, mt, nt);
+            const uint32_t acc = it & 1u;
+            const uint32_t acc_phase = (it >> 1) & 1u;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&tfull[acc], acc_phase, p.status) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                s_abort = 1;
+                break;
+            }
+            tc_fence_after();
+            const int row = q * 32 + lane;
+            const int64_t m = (int64_t)mt * kBM + row;
+            int64_t rows_g = p.rows ? (int64_t)p.rows[g] : p.M;
+            rows_g = rows_g > p.M ? p.M : rows_g;
+            const bool row_ok = m < rows_g;
+            const int64_t out_row = (int64_t)g * p.out_rows_per_group + m;
+            const uint32_t t_row = tmem_base + acc * kBN + ((uint32_t)(q * 32) << 16);
+
+            if (EPI == TC_EPI_SWIGLU) {
+                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * p.ldo;
+                const int half = p.n_mma / 2;
+                for (int c = 0; c < half / 32; ++c) {
+                    uint32_t rg[32], ru[32];
+                    tmem_ld32(t_row + c * 32, rg);
+                    tmem_ld_wait(rg);
+                    tmem_ld32(t_row + half + c * 32, ru);
+                    tmem_ld_wait(ru);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float h0 = silu_f(__uint_as_float(rg[2 * i])) * __uint_as_float(ru[2 * i]);
+                        const float h1 = silu_f(__uint_as_float(rg[2 * i + 1])) * __uint_as_float(ru[2 * i + 1]);
+                        pk[i] = pack_bf16x2(h0, h1);
+                    }
+                    const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
+                    if (row_ok) store_bf16_32(orow, n0, p.N, pk, p.vec_ok);
+                }
+            } else if (EPI == TC_EPI_F32) {
+                float* orow = reinterpret_cast<float*>(p.out) + out_row * p.ldo;
+                const float* bias = reinterpret_cast<const float*>(p.bias);
+                for (int c = 0; c < p.n_mma / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(t_row + c * 32, r);
+                    tmem_ld_wait(r);
+                    const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
+                    if (row_ok) {
+                        if (p.vec_ok && n0 + 32 <= p.N) {
+                            float4* dst = reinterpret_cast<float4*>(orow + n0);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                float4 v;
+                                v.x = __uint_as_float(r[4 * i + 0]) + (bias ? bias[n0 + 4 * i + 0] : 0.f);
+                                v.y = __uint_as_float(r[4 * i + 1]) + (bias ? bias[n0 + 4 * i + 1] : 0.f);
+                                v.z = __uint_as_float(r[4 * i + 2]) + (bias ? bias[n0 + 4 * i + 2] : 0.f);
+                                v.w = __uint_as_float(r[4 * i + 3]) + (bias ? bias[n0 + 4 * i + 3] : 0.f);
+                                dst[i] = v;
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (n0 + i < p.N) orow[n0 + i] = __uint_as_float(r[i]) + (bias ? bias[n0 + i] : 0.f);
+                        }
+                    }
+                }
+            } else {
+                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * p.ldo;
+                const __nv_bfloat16* bias =
+                    reinterpret_cast<const __nv_bfloat16*>(p.bias) + (p.bias ? g * p.bias_group_stride : 0);
+                for (int c = 0; c < p.n_mma / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(t_row + c * 32, r);
+                    tmem_ld_wait(r);
+                    const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float v0 = __uint_as_float(r[2 * i]);
+                        float v1 = __uint_as_float(r[2 * i + 1]);
+                        if (EPI == TC_EPI_BF16_BIAS || EPI == TC_EPI_GELU_BIAS) {
+                            const int64_t na = n0 + 2 * i, nb = n0 + 2 * i + 1;
+                            v0 += na < p.N ? __bfloat162float(bias[na]) : 0.f;
+                            v1 += nb < p.N ? __bfloat162float(bias[nb]) : 0.f;
+                        }
+                        if (EPI == TC_EPI_GELU_BIAS) {
+                            v0 = gelu_f(v0);
+                            v1 = gelu_f(v1);
+                        }
+                        pk[i] = pack_bf16x2(v0, v1);
+                    }
+                    if (row_ok) store_bf16_32(orow, n0, p.N, pk, p.vec_ok);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (s_abort) break;
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(2 * kBN)
+                     : "memory");
+    }
+}
+
+// ------------------------------- host side ---------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D bf16 map over a (rows, inner) row-major matrix, box = (box_rows, 64),
+// 128-byte swizzle, zero fill outside the matrix.
+bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld_elems, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld_elems * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int EPI>
+int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const KParams& kp, int grid,
+           cudaStream_t stream) {
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 64 && !attr_set[dev]) {
+        MOE_CUDA_TRY(cudaFuncSetAttribute(tc_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)kSmemBytes));
+        attr_set[dev] = true;
+    }
+    tc_gemm_kernel<EPI><<<grid, kThreads, kSmemBytes, stream>>>(a, b, b2, kp);
+    return launch_status();
+}
+
+}  // namespace
+
+int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
+    MOE_REQUIRE(p.a && p.b && p.out, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(p.G >= 1 && p.M >= 1 && p.N >= 1 && p.K >= 1, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(p.G <= kMaxGroups, MOE_ERR_UNSUPPORTED);
+    // TMA: 16-byte aligned bases, row strides a multiple of 16 bytes.
+    MOE_REQUIRE(aligned16(p.a) && aligned16(p.b) && (p.lda * 2) % 16 == 0 && (p.ldb * 2) % 16 == 0,
+                MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(p.lda >= p.K && p.ldb >= p.K, MOE_ERR_INVALID_ARG);
+    const bool dual = p.epilogue == TC_EPI_SWIGLU;
+    if (dual) MOE_REQUIRE(p.b2 && aligned16(p.b2), MOE_ERR_INVALID_ARG);
+    // TMA coordinates are 32-bit.
+    MOE_REQUIRE(p.a_rows_total < (int64_t(1) << 31) && p.b_rows_total < (int64_t(1) << 31), MOE_ERR_UNSUPPORTED);
+
+    KParams kp{};
+    kp.G = p.G;
+    kp.a_rows_per_group = p.a_rows_per_group;
+    kp.b_rows_per_group = p.b_rows_per_group;
+    kp.M = p.M;
+    kp.N = p.N;
+    if (dual) {
+        kp.n_mma = kBN;
+        kp.tile_n_out = kBN / 2;
+        kp.b_box_rows = kBN / 2;
+    } else {
+        int64_t n = (p.N + 31) / 32 * 32;
+        kp.n_mma = (int)(n < kBN ? n : kBN);
+        kp.tile_n_out = kp.n_mma;
+        kp.b_box_rows = kp.n_mma;
+    }
+    kp.n_tiles = (int)((p.N + kp.tile_n_out - 1) / kp.tile_n_out);
+    kp.k_blocks = (int)((p.K + kBK - 1) / kBK);
+    kp.tx_bytes = (uint32_t)(kABytes + kp.n_mma * kBK * 2);
+    kp.rows = p.rows;
+    kp.out = p.out;
+    kp.ldo = p.ldo;
+    kp.out_rows_per_group = p.out_rows_per_group;
+    kp.bias = p.bias;
+    kp.bias_group_stride = p.bias_group_stride;
+    const size_t esz = p.epilogue == TC_EPI_F32 ? 4 : 2;
+    kp.vec_ok = aligned16(p.out) && (p.ldo * (int64_t)esz) % 16 == 0;
+    kp.status = p.status;
+
+    CUtensorMap ma, mb, mb2;
+    MOE_REQUIRE(make_map(&ma, p.a, p.K, p.a_rows_total, p.lda, kBM), MOE_ERR_CUDA);
+    MOE_REQUIRE(make_map(&mb, p.b, p.K, p.b_rows_total, p.ldb, kp.b_box_rows), MOE_ERR_CUDA);
+    if (dual) MOE_REQUIRE(make_map(&mb2, p.b2, p.K, p.b_rows_total, p.ldb, kp.b_box_rows), MOE_ERR_CUDA);
+    else mb2 = mb;
+
+    const int64_t max_tiles = (int64_t)p.G * ((p.M + kBM - 1) / kBM) * kp.n_tiles;
+    MOE_REQUIRE(max_tiles < (int64_t(1) << 30), MOE_ERR_UNSUPPORTED);
+    int grid = device_sm_count();
+    if (max_tiles < grid) grid = (int)max_tiles;
+    if (grid < 1) grid = 1;
+
+    switch (p.epilogue) {
+        case TC_EPI_F32: return launch<TC_EPI_F32>(ma, mb, mb2, kp, grid, stream);
+        case TC_EPI_BF16: return launch<TC_EPI_BF16>(ma, mb, mb2, kp, grid, stream);
+        case TC_EPI_BF16_BIAS: return launch<TC_EPI_BF16_BIAS>(ma, mb, mb2, kp, grid, stream);
+        case TC_EPI_GELU_BIAS: return launch<TC_EPI_GELU_BIAS>(ma, mb, mb2, kp, grid, stream);
+        case TC_EPI_SWIGLU: return launch<TC_EPI_SWIGLU>(ma, mb, mb2, kp, grid, stream);
+        default: return MOE_ERR_INVALID_ARG;
+    }
+}
+
+}  // namespace moe

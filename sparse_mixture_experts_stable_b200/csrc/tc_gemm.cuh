@@ -1,0 +1,53 @@
+// Grouped bf16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// out[g, m, n] = epilogue( sum_k A[g, m, k] * B[g, n, k] )     for m < rows[g]
+//
+// Both operands are K-major bf16 (A: activations (rows, K); B: weights in the
+// (out, in) layout), fp32 accumulation in tensor memory.  One persistent CTA per
+// SM walks a static list of (group, m-tile, n-tile) tiles whose length depends on
+// the per-group row counts read on the device.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+enum TcEpilogue : int {
+    TC_EPI_F32 = 0,        // fp32 out (+ optional fp32 column bias)      -- router scores
+    TC_EPI_BF16 = 1,       // bf16 out                                    -- linear / down
+    TC_EPI_BF16_BIAS = 2,  // bf16 out, + bf16 bias                       -- GELU MLP fc2
+    TC_EPI_GELU_BIAS = 3,  // bf16 gelu(acc + bias)                       -- GELU MLP fc1
+    TC_EPI_SWIGLU = 4      // dual B: bf16 silu(acc_gate) * acc_up        -- SwiGLU gate/up
+};
+
+struct TcGemmProblem {
+    const void* a;            // bf16, row-major (a_rows_total, K), row stride lda
+    int64_t lda;
+    int64_t a_rows_total;
+    int64_t a_rows_per_group; // row offset of group g in A
+    const void* b;            // bf16 (b_rows_total, K), row stride ldb
+    const void* b2;           // second B for TC_EPI_SWIGLU (same shape), else NULL
+    int64_t ldb;
+    int64_t b_rows_total;
+    int64_t b_rows_per_group; // row offset of group g in B
+    int G;                    // groups
+    int64_t M;                // max rows per group
+    int64_t N;                // output columns per group
+    int64_t K;
+    const int32_t* rows;      // device (G) valid rows per group, or NULL (= M)
+    void* out;                // fp32 or bf16 per epilogue
+    int64_t ldo;
+    int64_t out_rows_per_group;
+    const void* bias;         // fp32 (TC_EPI_F32) or bf16, per output column
+    int64_t bias_group_stride;
+    int epilogue;
+    int32_t* status;
+};
+
+// Validates alignment, encodes the tensor maps and launches.  Returns a moe_status.
+int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream);
+
+}  // namespace moe

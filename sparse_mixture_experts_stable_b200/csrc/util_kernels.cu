@@ -1,0 +1,257 @@
+// Row movement kernels: batched transpose, token-major gather into expert-major
+// buffers, and the deterministic gate-weighted combine.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "util_kernels.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+
+// ------------------------------- transpose ----------------------------------
+template <typename T>
+__global__ void transpose_kernel(const T* __restrict__ src, T* __restrict__ dst, int64_t rows, int64_t cols) {
+    __shared__ T tile[32][33];
+    const int64_t b = blockIdx.z;
+    const T* s = src + b * rows * cols;
+    T* d = dst + b * rows * cols;
+    const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int64_t r = r0 + i, c = c0 + threadIdx.x;
+        if (r < rows && c < cols) tile[i][threadIdx.x] = s[r * cols + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int64_t c = c0 + i, r = r0 + threadIdx.x;
+        if (r < rows && c < cols) d[c * rows + r] = tile[threadIdx.x][i];
+    }
+}
+
+// Per-token assignment table held in two registers per lane (j < 64).
+struct Assign {
+    int64_t e0, e1, s0, s1;
+    float g0, g1;
+};
+
+__device__ __forceinline__ void load_assign(Assign& a, int lane, int64_t t, int k, const int64_t* selected,
+                                            const int64_t* slot) {
+    a.e0 = lane < k ? selected[t * k + lane] : -1;
+    a.s0 = lane < k ? slot[t * k + lane] : -1;
+    a.e1 = lane + 32 < k ? selected[t * k + lane + 32] : -1;
+    a.s1 = lane + 32 < k ? slot[t * k + lane + 32] : -1;
+}
+
+__device__ __forceinline__ void get_assign(const Assign& a, int j, int64_t& e, int64_t& s) {
+    const int src = j & 31;
+    const int64_t e0 = __shfl_sync(0xffffffffu, a.e0, src), e1 = __shfl_sync(0xffffffffu, a.e1, src);
+    const int64_t s0 = __shfl_sync(0xffffffffu, a.s0, src), s1 = __shfl_sync(0xffffffffu, a.s1, src);
+    e = j < 32 ? e0 : e1;
+    s = j < 32 ? s0 : s1;
+}
+
+__device__ __forceinline__ float get_gate(const Assign& a, int j) {
+    const int src = j & 31;
+    const float g0 = __shfl_sync(0xffffffffu, a.g0, src), g1 = __shfl_sync(0xffffffffu, a.g1, src);
+    return j < 32 ? g0 : g1;
+}
+
+// ------------------------------- gather -------------------------------------
+// One warp per token; 16-byte vectors when every row start is 16-byte aligned.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    gather_kernel(const T* __restrict__ src, int64_t lds, int64_t Ttok, int k, const int64_t* __restrict__ selected,
+                  const int64_t* __restrict__ slot, int E, int64_t C, const float* __restrict__ scale,
+                  T* __restrict__ dst, int64_t D, int32_t* status) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
+    if (t >= Ttok) return;
+    Assign a;
+    load_assign(a, lane, t, k, selected, slot);
+    a.g0 = (scale && lane < k) ? scale[t * k + lane] : 1.f;
+    a.g1 = (scale && lane + 32 < k) ? scale[t * k + lane + 32] : 1.f;
+    const T* srow = src + t * lds;
+    constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte vector
+    for (int j = 0; j < k; ++j) {
+        int64_t e, s;
+        get_assign(a, j, e, s);
+        if (s < 0) continue;
+        if (e < 0 || e >= E || s >= C) {
+            if (lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
+            continue;
+        }
+        const float g = get_gate(a, j);
+        T* drow = dst + (e * C + s) * D;
+        if (VEC) {
+            const int64_t nv = D / EPV;
+            for (int64_t v = lane; v < nv; v += 32) {
+                uint4 x = reinterpret_cast<const uint4*>(srow)[v];
+                if (scale) {
+                    float4 f = *reinterpret_cast<float4*>(&x);
+                    f.x *= g; f.y *= g; f.z *= g; f.w *= g;
+                    x = *reinterpret_cast<uint4*>(&f);
+                }
+                reinterpret_cast<uint4*>(drow)[v] = x;
+            }
+        } else {
+            for (int64_t d = lane; d < D; d += 32) {
+                const float v = to_f32(srow[d]) * (scale ? g : 1.f);
+                drow[d] = scale ? from_f32<T>(v) : srow[d];
+            }
+        }
+    }
+}
+
+// ------------------------------- combine ------------------------------------
+template <typename T, typename G, bool VEC>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+    combine_kernel(const T* __restrict__ ybuf, const int64_t* __restrict__ selected, const int64_t* __restrict__ slot,
+                   const G* __restrict__ gates, int64_t Ttok, int k, int E, int64_t C, int64_t N,
+                   const T* __restrict__ base, int64_t ldbase, T* __restrict__ y, int64_t ldy, int32_t* status) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
+    if (t >= Ttok) return;
+    Assign a;
+    load_assign(a, lane, t, k, selected, slot);
+    a.g0 = (gates && lane < k) ? to_f32(gates[t * k + lane]) : 1.f;
+    a.g1 = (gates && lane + 32 < k) ? to_f32(gates[t * k + lane + 32]) : 1.f;
+    // validate once per token
+    bool bad = false;
+    for (int j = 0; j < k; ++j) {
+        int64_t e, s;
+        get_assign(a, j, e, s);
+        if (s >= 0 && (e < 0 || e >= E || s >= C)) bad = true;
+    }
+    if (bad && lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
+    T* yrow = y + t * ldy;
+    const T* brow = base ? base + t * ldbase : nullptr;
+    if (VEC) {
+        constexpr int EPV = 16 / sizeof(T);
+        const int64_t nv = N / EPV;
+        for (int64_t v = lane; v < nv; v += 32) {
+            float acc[EPV];
+            if (brow) {
+                const uint4 b = reinterpret_cast<const uint4*>(brow)[v];
+                const T* bv = reinterpret_cast<const T*>(&b);
+#pragma unroll
+                for (int i = 0; i < EPV; ++i) acc[i] = to_f32(bv[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
+            }
+            for (int j = 0; j < k; ++j) {
+                int64_t e, s;
+                get_assign(a, j, e, s);
+                if (s < 0 || e < 0 || e >= E || s >= C) continue;
+                const float g = get_gate(a, j);
+                const uint4 r = reinterpret_cast<const uint4*>(ybuf + (e * C + s) * N)[v];
+                const T* rv = reinterpret_cast<const T*>(&r);
+#pragma unroll
+                for (int i = 0; i < EPV; ++i) acc[i] = fmaf(g, to_f32(rv[i]), acc[i]);
+            }
+            uint4 o;
+            T* ov = reinterpret_cast<T*>(&o);
+#pragma unroll
+            for (int i = 0; i < EPV; ++i) ov[i] = from_f32<T>(acc[i]);
+            reinterpret_cast<uint4*>(yrow)[v] = o;
+        }
+    } else {
+        for (int64_t n = lane; n < N; n += 32) {
+            float acc = brow ? to_f32(brow[n]) : 0.f;
+            for (int j = 0; j < k; ++j) {
+                int64_t e, s;
+                get_assign(a, j, e, s);
+                if (s < 0 || e < 0 || e >= E || s >= C) continue;
+                acc = fmaf(get_gate(a, j), to_f32(ybuf[(e * C + s) * N + n]), acc);
+            }
+            yrow[n] = from_f32<T>(acc);
+        }
+    }
+}
+
+}  // namespace
+
+int transpose_matrices(const void* src, void* dst, int64_t batches, int64_t rows, int64_t cols, moe_dtype dtype,
+                       cudaStream_t stream) {
+    MOE_REQUIRE(src && dst && batches >= 1 && rows >= 1 && cols >= 1, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(batches <= 65535 && (rows + 31) / 32 <= 65535, MOE_ERR_UNSUPPORTED);
+    dim3 grid((unsigned)((cols + 31) / 32), (unsigned)((rows + 31) / 32), (unsigned)batches);
+    dim3 block(32, 8);
+    if (dtype == MOE_BF16)
+        transpose_kernel<uint16_t><<<grid, block, 0, stream>>>(static_cast<const uint16_t*>(src),
+                                                               static_cast<uint16_t*>(dst), rows, cols);
+    else
+        transpose_kernel<float><<<grid, block, 0, stream>>>(static_cast<const float*>(src), static_cast<float*>(dst),
+                                                            rows, cols);
+    return launch_status();
+}
+
+int gather_rows(const void* src, int64_t lds, int64_t T, int32_t k, const int64_t* selected, const int64_t* slot,
+                int32_t E, int64_t C, const float* scale, void* dst, int64_t D, moe_dtype dtype, int32_t* status,
+                cudaStream_t stream) {
+    MOE_REQUIRE(k >= 1 && k <= 64, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(!(scale && dtype != MOE_F32), MOE_ERR_UNSUPPORTED);
+    if (T == 0 || C == 0 || D == 0) return MOE_OK;
+    const size_t es = dtype_size(dtype);
+    const bool vec = aligned16(src) && aligned16(dst) && ((size_t)lds * es) % 16 == 0 && ((size_t)D * es) % 16 == 0;
+    const unsigned grid = (unsigned)((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
+    const int threads = kWarpsPerBlock * 32;
+    if (dtype == MOE_BF16) {
+        auto s = static_cast<const __nv_bfloat16*>(src);
+        auto d = static_cast<__nv_bfloat16*>(dst);
+        if (vec) gather_kernel<__nv_bfloat16, true><<<grid, threads, 0, stream>>>(s, lds, T, k, selected, slot, E, C, scale, d, D, status);
+        else gather_kernel<__nv_bfloat16, false><<<grid, threads, 0, stream>>>(s, lds, T, k, selected, slot, E, C, scale, d, D, status);
+    } else {
+        auto s = static_cast<const float*>(src);
+        auto d = static_cast<float*>(dst);
+        if (vec) gather_kernel<float, true><<<grid, threads, 0, stream>>>(s, lds, T, k, selected, slot, E, C, scale, d, D, status);
+        else gather_kernel<float, false><<<grid, threads, 0, stream>>>(s, lds, T, k, selected, slot, E, C, scale, d, D, status);
+    }
+    return launch_status();
+}
+
+template <typename T, typename G>
+static void launch_combine(bool vec, unsigned grid, const void* ybuf, const int64_t* selected, const int64_t* slot,
+                           const void* gates, int64_t T_, int k, int E, int64_t C, int64_t N, const void* base,
+                           int64_t ldbase, void* y, int64_t ldy, int32_t* status, cudaStream_t stream) {
+    const int threads = kWarpsPerBlock * 32;
+    if (vec)
+        combine_kernel<T, G, true><<<grid, threads, 0, stream>>>(
+            static_cast<const T*>(ybuf), selected, slot, static_cast<const G*>(gates), T_, k, E, C, N,
+            static_cast<const T*>(base), ldbase, static_cast<T*>(y), ldy, status);
+    else
+        combine_kernel<T, G, false><<<grid, threads, 0, stream>>>(
+            static_cast<const T*>(ybuf), selected, slot, static_cast<const G*>(gates), T_, k, E, C, N,
+            static_cast<const T*>(base), ldbase, static_cast<T*>(y), ldy, status);
+}
+
+int combine_rows(const void* ybuf, const int64_t* selected, const int64_t* slot, const void* gates,
+                 moe_dtype gate_dtype, int64_t T, int32_t k, int32_t E, int64_t C, int64_t N, const void* base,
+                 int64_t ldbase, void* y, int64_t ldy, moe_dtype dtype, int32_t* status, cudaStream_t stream) {
+    MOE_REQUIRE(k >= 1 && k <= 64, MOE_ERR_UNSUPPORTED);
+    if (T == 0 || N == 0) return MOE_OK;
+    const size_t es = dtype_size(dtype);
+    const bool vec = aligned16(ybuf) && aligned16(y) && (!base || aligned16(base)) && ((size_t)N * es) % 16 == 0 &&
+                     ((size_t)ldy * es) % 16 == 0 && (!base || ((size_t)ldbase * es) % 16 == 0);
+    const unsigned grid = (unsigned)((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
+    if (dtype == MOE_BF16) {
+        if (gate_dtype == MOE_BF16)
+            launch_combine<__nv_bfloat16, __nv_bfloat16>(vec, grid, ybuf, selected, slot, gates, T, k, E, C, N, base,
+                                                         ldbase, y, ldy, status, stream);
+        else
+            launch_combine<__nv_bfloat16, float>(vec, grid, ybuf, selected, slot, gates, T, k, E, C, N, base, ldbase,
+                                                 y, ldy, status, stream);
+    } else {
+        if (gate_dtype == MOE_BF16)
+            launch_combine<float, __nv_bfloat16>(vec, grid, ybuf, selected, slot, gates, T, k, E, C, N, base, ldbase,
+                                                 y, ldy, status, stream);
+        else
+            launch_combine<float, float>(vec, grid, ybuf, selected, slot, gates, T, k, E, C, N, base, ldbase, y, ldy,
+                                         status, stream);
+    }
+    return launch_status();
+}
+
+}  // namespace moe

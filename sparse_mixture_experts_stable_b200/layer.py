@@ -1,0 +1,74 @@
+"""Whole-layer forward passes built from the C-ABI calls, buffers allocated once.
+
+Each ``forward`` enqueues the layer's kernels on the current stream in the order
+route -> dispatch -> expert FFN -> combine -> load statistics and returns device
+tensors; nothing is synchronised.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+
+class SwiGLUMoE:
+    """Router GEMM + SwiGLU routed experts + optional always-on shared SwiGLU expert.
+
+    y = shared(x) + sum_{kept j} gate_j * Expert_{e_j}(x)   (or no shared term)
+    """
+
+    def __init__(self, T: int, H: int, E: int, F: int, k: int, capacity_factor: float, F_shared: int = 0,
+                 aux_coef: float = 0.0, dtype=torch.bfloat16, device="cuda"):
+        self.T, self.H, self.E, self.F, self.k = T, H, E, F, k
+        self.F_shared, self.aux_coef, self.dtype = F_shared, aux_coef, dtype
+        self.C = B.moe_capacity(T, k, E, capacity_factor)
+        dev = torch.device(device)
+        dt = B.MOE_BF16 if dtype == torch.bfloat16 else B.MOE_F32
+        C = self.C
+        self.route_out = dict(
+            selected=torch.empty(T, k, dtype=torch.int64, device=dev),
+            gates=torch.empty(T, k, dtype=dtype, device=dev),
+            gates_f32=torch.empty(T, k, dtype=torch.float32, device=dev),
+            counts=torch.empty(E, dtype=torch.int32, device=dev),
+            prob_sum=torch.empty(E, dtype=torch.float32, device=dev),
+        )
+        self.disp_out = dict(
+            slot=torch.empty(T, k, dtype=torch.int64, device=dev),
+            kept=torch.empty(T, k, dtype=torch.uint8, device=dev),
+            used=torch.empty(E, dtype=torch.int32, device=dev),
+            overflow=torch.empty(E, dtype=torch.int32, device=dev),
+            drops=torch.empty(T, dtype=torch.int32, device=dev),
+            token_of_slot=torch.empty(E, C, dtype=torch.int32, device=dev),
+            xbuf=torch.empty(E, C, H, dtype=dtype, device=dev),
+        )
+        self.ybuf = torch.empty(E, C, H, dtype=dtype, device=dev)
+        self.y = torch.empty(T, H, dtype=dtype, device=dev)
+        self.shared = torch.empty(T, H, dtype=dtype, device=dev) if F_shared else None
+        self.status = B.new_status(dev)
+        self.ws_route = torch.empty(max(B.moe_route_workspace_size(T, H, E, dt, True, "ED"), 256),
+                                    dtype=torch.uint8, device=dev)
+        self.ws_disp = torch.empty(max(B.moe_dispatch_workspace_size(T, k, E), 256), dtype=torch.uint8, device=dev)
+        self.ws_ffn = torch.empty(max(B.moe_expert_ffn_workspace_size("swiglu", dt, E, C, F), 256),
+                                  dtype=torch.uint8, device=dev)
+        self.ws_shared = (torch.empty(max(B.moe_expert_ffn_workspace_size("swiglu", dt, 1, T, F_shared), 256),
+                                      dtype=torch.uint8, device=dev) if F_shared else None)
+
+    def forward(self, x, w_router, router_bias, w_gate, w_up, w_down, s_gate=None, s_up=None, s_down=None):
+        """x (T,H); w_router (E,H); w_gate/w_up (E,F,H); w_down (E,H,F); shared (1,F_s,H)/(1,H,F_s)."""
+        r = B.moe_route(x, self.k, w_router=w_router, layout="ED", logit_bias=router_bias, out=self.route_out,
+                        dev_status=self.status, workspace=self.ws_route)
+        d = B.moe_dispatch(r["selected"], self.E, self.C, x=x, out=self.disp_out, dev_status=self.status,
+                           workspace=self.ws_disp)
+        B.moe_expert_ffn("swiglu", d["xbuf"], d["used"], w_gate, w2=w_down, w3=w_up, ybuf=self.ybuf,
+                         dev_status=self.status, workspace=self.ws_ffn)
+        base_kind, base = "zero", None
+        if self.F_shared:
+            B.moe_expert_ffn("swiglu", x.view(1, self.T, self.H), None, s_gate, w2=s_down, w3=s_up,
+                             ybuf=self.shared.view(1, self.T, self.H), dev_status=self.status,
+                             workspace=self.ws_shared)
+            base_kind, base = "tensor", self.shared
+        B.moe_combine(self.ybuf, r["selected"], d["slot"], r["gates_f32"], base_kind=base_kind, base=base, y=self.y,
+                      dev_status=self.status)
+        f, P, aux = B.moe_aux_stats(r["counts"], r["prob_sum"], self.T, self.k, True, self.aux_coef,
+                                    out_dtype=self.dtype)
+        return dict(y=self.y, f=f, P=P, aux=aux, **r, **d)
