@@ -138,14 +138,25 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device="cuda") -> float:
+    """Largest per-rank value (the slowest rank's time decides the job time)."""
     if world == 1:
         return v
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's device time."""
+    return tokens_per_rank_step * steps * world / (max_ms / 1e3)
+
+
+def rank_seed(rank: int) -> int:
+    """Weak scaling: each rank draws its own batch (and its own random-init weights) from its seed."""
+    return rank
 
 
 # ------------------------------------------------------------------------------------------------
@@ -227,7 +238,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     moe.lib()  # fail loudly if the CUDA library is missing
-    cfg = I.full_layer_bf16(seed=rank)
+    cfg = I.full_layer_bf16(seed=rank_seed(rank), T=args.tokens, E=args.experts)
     T, H, E, F, k = cfg["T"], cfg["H"], cfg["E"], cfg["F"], cfg["k"]
     names = ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down")
     dv = {n: cfg[n].to(dev) for n in names}
@@ -279,29 +290,12 @@ def run_ours(args, world, rank, local):
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ffn_ms = [a.elapsed_time(b) for a, b in ffn_ev]
     total_ms = max_over_ranks(sum(step_ms), world)
-    value = T * args.steps * world / (total_ms / 1e3)
+    value = job_throughput(T, args.steps, world, total_ms)
 
-    # ---- end to end: host input -> device -> layer -> host output ----
-    x_host = cfg["x"].pin_memory()
-    y_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
-    aux_host = torch.empty(2, dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(dv["x"])
-    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        flush.zero_()
-        e_starts[i].record(stream)
-        x_dev.copy_(x_host, non_blocking=True)
-        y, aux = step(x_dev)
-        y_host.copy_(y, non_blocking=True)
-        aux_host.copy_(aux, non_blocking=True)
-        e_ends[i].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), world)
-    e2e_value = T * args.steps * world / (e2e_ms / 1e3)
+    if args.no_e2e:
+        e2e_value = None
+    else:
+        e2e_value = run_e2e(args, world, cfg, dv, step, flush, stream)
     assert moe.moe_read_status(layer.status) == 0
 
     # ---- roofline of the dominant kernel (routed SwiGLU grouped GEMMs) ----
@@ -323,17 +317,45 @@ def run_ours(args, world, rank, local):
         tps, S, dt = time_oracle(cfg64, args.cpu_seconds)
         cpu = dict(value=tps, unit=UNIT, cores=os.cpu_count(), kind="oracle",
                    sample=f"first {S} tokens of the batch ({dt:.1f} s), capacity from the sample's T")
+    wl = dict(WORKLOAD, T=T, experts=E, capacity=layer.C)
     line = dict(
         metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
         ms_per_step=total_ms / args.steps, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
         data="synthetic",
-        config=dict(WORKLOAD, parallelism=f"replicas{world}", global_batch=T * world,
+        config=dict(wl, parallelism=f"replicas{world}", global_batch=T * world,
                     l2="flushed between steps (256 MiB write)", tokens_kept=kept),
-        e2e=dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=T * H * 2, d2h_bytes_per_step=T * H * 2 + 8),
+        e2e=None if e2e_value is None else dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=T * H * 2,
+                                                d2h_bytes_per_step=T * H * 2 + 8),
         gpu_launches=KERNELS_PER_STEP * args.steps,
         roofline=roof, cpu_baseline=cpu, clocks=clocks.summary(),
     )
     print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, world, cfg, dv, step, flush, stream):
+    """Same steps, with the step's input copied from pinned host memory and the
+    output and aux loss copied back inside the timed region."""
+    T, H = cfg["T"], cfg["H"]
+    x_host = cfg["x"].pin_memory()
+    y_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    aux_host = torch.empty(2, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(dv["x"])
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        y, aux = step(x_dev)
+        y_host.copy_(y, non_blocking=True)
+        aux_host.copy_(aux, non_blocking=True)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), world)
+    return job_throughput(T, args.steps, world, e2e_ms)
 
 
 def main():
@@ -344,6 +366,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--tokens", type=int, default=WORKLOAD["T"], help="tokens per rank (smaller for profiling)")
+    ap.add_argument("--experts", type=int, default=WORKLOAD["experts"], help="routed experts (smaller for profiling)")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:

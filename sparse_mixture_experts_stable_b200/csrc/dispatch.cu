@@ -181,12 +181,13 @@ int dispatch_check_args(const int64_t* selected, int64_t T, int32_t k, int32_t E
                         moe_dtype dtype, int64_t D, int64_t ldx, const int64_t* slot, const uint8_t* kept,
                         const int32_t* used, const int32_t* overflow, const int32_t* drops,
                         const int32_t* token_of_slot, const void* xbuf) {
-    MOE_REQUIRE(selected && slot && kept && used && overflow && drops && token_of_slot, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(selected && slot && kept && used && overflow && drops, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(C == 0 || token_of_slot != nullptr, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(T >= 1 && k >= 1 && E >= 1 && C >= 0, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(T * (int64_t)k < (int64_t(1) << 30) && C < (int64_t(1) << 30), MOE_ERR_UNSUPPORTED);
     MOE_REQUIRE(E <= 2048 && k <= 64, MOE_ERR_UNSUPPORTED);  // scan smem: (16 E + 512) * 4 bytes
     if (x) {
-        MOE_REQUIRE(valid_dtype(dtype) && xbuf && D >= 1 && ldx >= D, MOE_ERR_INVALID_ARG);
+        MOE_REQUIRE(valid_dtype(dtype) && (xbuf || C == 0) && D >= 1 && ldx >= D, MOE_ERR_INVALID_ARG);
     }
     return MOE_OK;
 }

@@ -105,26 +105,45 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 }
 
 // ------------------------------- combine ------------------------------------
+// One warp per token.  The token's (row offset, gate) table for j < k is staged
+// in shared memory first, so the row loops below contain no warp shuffles and
+// may diverge freely over ragged row lengths.
+constexpr int kMaxKCombine = 64;
+
 template <typename T, typename G, bool VEC>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     combine_kernel(const T* __restrict__ ybuf, const int64_t* __restrict__ selected, const int64_t* __restrict__ slot,
                    const G* __restrict__ gates, int64_t Ttok, int k, int E, int64_t C, int64_t N,
                    const T* __restrict__ base, int64_t ldbase, T* __restrict__ y, int64_t ldy, int32_t* status) {
+    __shared__ int64_t s_row[kWarpsPerBlock][kMaxKCombine];
+    __shared__ float s_gate[kWarpsPerBlock][kMaxKCombine];
+    __shared__ int s_n[kWarpsPerBlock];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
     if (t >= Ttok) return;
-    Assign a;
-    load_assign(a, lane, t, k, selected, slot);
-    a.g0 = (gates && lane < k) ? to_f32(gates[t * k + lane]) : 1.f;
-    a.g1 = (gates && lane + 32 < k) ? to_f32(gates[t * k + lane + 32]) : 1.f;
-    // validate once per token
-    bool bad = false;
-    for (int j = 0; j < k; ++j) {
-        int64_t e, s;
-        get_assign(a, j, e, s);
-        if (s >= 0 && (e < 0 || e >= E || s >= C)) bad = true;
+    // compact the kept, in-range assignments in ascending j (lane 0 keeps the order)
+    if (lane == 0) {
+        int n = 0;
+        bool bad = false;
+        for (int j = 0; j < k; ++j) {
+            const int64_t s = slot[t * k + j];
+            if (s < 0) continue;
+            const int64_t e = selected[t * k + j];
+            if (e < 0 || e >= E || s >= C) {
+                bad = true;
+                continue;
+            }
+            s_row[warp][n] = (e * C + s) * N;
+            s_gate[warp][n] = gates ? to_f32(gates[t * k + j]) : 1.f;
+            ++n;
+        }
+        s_n[warp] = n;
+        if (bad) set_status(status, MOE_ERR_BAD_INDEX);
     }
-    if (bad && lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
+    __syncwarp();
+    const int n_terms = s_n[warp];
+    const int64_t* rows = s_row[warp];
+    const float* gs = s_gate[warp];
     T* yrow = y + t * ldy;
     const T* brow = base ? base + t * ldbase : nullptr;
     if (VEC) {
@@ -141,12 +160,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 #pragma unroll
                 for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
             }
-            for (int j = 0; j < k; ++j) {
-                int64_t e, s;
-                get_assign(a, j, e, s);
-                if (s < 0 || e < 0 || e >= E || s >= C) continue;
-                const float g = get_gate(a, j);
-                const uint4 r = reinterpret_cast<const uint4*>(ybuf + (e * C + s) * N)[v];
+            for (int j = 0; j < n_terms; ++j) {
+                const float g = gs[j];
+                const uint4 r = reinterpret_cast<const uint4*>(ybuf + rows[j])[v];
                 const T* rv = reinterpret_cast<const T*>(&r);
 #pragma unroll
                 for (int i = 0; i < EPV; ++i) acc[i] = fmaf(g, to_f32(rv[i]), acc[i]);
@@ -160,12 +176,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     } else {
         for (int64_t n = lane; n < N; n += 32) {
             float acc = brow ? to_f32(brow[n]) : 0.f;
-            for (int j = 0; j < k; ++j) {
-                int64_t e, s;
-                get_assign(a, j, e, s);
-                if (s < 0 || e < 0 || e >= E || s >= C) continue;
-                acc = fmaf(get_gate(a, j), to_f32(ybuf[(e * C + s) * N + n]), acc);
-            }
+            for (int j = 0; j < n_terms; ++j) acc = fmaf(gs[j], to_f32(ybuf[rows[j] + n]), acc);
             yrow[n] = from_f32<T>(acc);
         }
     }
@@ -230,7 +241,7 @@ static void launch_combine(bool vec, unsigned grid, const void* ybuf, const int6
 int combine_rows(const void* ybuf, const int64_t* selected, const int64_t* slot, const void* gates,
                  moe_dtype gate_dtype, int64_t T, int32_t k, int32_t E, int64_t C, int64_t N, const void* base,
                  int64_t ldbase, void* y, int64_t ldy, moe_dtype dtype, int32_t* status, cudaStream_t stream) {
-    MOE_REQUIRE(k >= 1 && k <= 64, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(k >= 1 && k <= kMaxKCombine, MOE_ERR_UNSUPPORTED);
     if (T == 0 || N == 0) return MOE_OK;
     const size_t es = dtype_size(dtype);
     const bool vec = aligned16(ybuf) && aligned16(y) && (!base || aligned16(base)) && ((size_t)N * es) % 16 == 0 &&

@@ -5,7 +5,7 @@ import torch
 
 import sparse_mixture_experts_stable_b200 as moe
 from oracle import oracle as O
-from tests.gpu_util import BF16_ATOL, BF16_RTOL, DEV, F32_ATOL, F32_RTOL, assert_close, cpu64
+from tests.gpu_util import BF16_ATOL, BF16_RTOL, DEV, F32_ATOL, F32_RTOL, assert_close, assert_close_mag, cpu64
 
 pytestmark = pytest.mark.gpu
 
@@ -27,8 +27,12 @@ def test_combine_matches_oracle(dtype, base_kind, N):
                         base=None if base is None else base.to(DEV))
     want = O.combine_slots(cpu64(ybuf), sel, d["slot"], d["kept"], gates,
                            base=None if base is None else cpu64(base))
-    rtol, atol = (F32_RTOL, F32_ATOL) if dtype == torch.float32 else (BF16_RTOL, BF16_ATOL)
-    assert_close(cpu64(y), want, rtol, atol, f"combine {dtype} {base_kind}")
+    if dtype == torch.float32:
+        mag = O.combine_slots(np.abs(cpu64(ybuf)), sel, d["slot"], d["kept"], gates,
+                              base=None if base is None else np.abs(cpu64(base)))
+        assert_close_mag(cpu64(y), want, mag, F32_RTOL, F32_ATOL, f"combine {dtype} {base_kind}")
+    else:
+        assert_close(cpu64(y), want, BF16_RTOL, BF16_ATOL, f"combine {dtype} {base_kind}")
     # fully dropped tokens give exactly the base row
     full = np.flatnonzero(d["drops"] == k)
     if len(full):

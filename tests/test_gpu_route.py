@@ -15,7 +15,7 @@ import sparse_mixture_experts_stable_b200 as moe
 from oracle import oracle as O
 from sparse_mixture_experts_stable_b200 import inputs as I
 from tests.conftest import GOLDEN
-from tests.gpu_util import DEV, F32_ATOL, F32_RTOL, assert_close, bf16_round, cpu, cpu64
+from tests.gpu_util import DEV, F32_ATOL, F32_RTOL, assert_close, assert_within_bf16_ulp, cpu, cpu64
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +28,7 @@ def _check_route(r, s64, k, what, logits_exact=True):
     np.testing.assert_array_equal(cpu(r["counts"]), counts, err_msg=what + " counts")
     assert_close(cpu64(r["gates_f32"]), gates, F32_RTOL, F32_ATOL, what + " gates_f32")
     if r["gates"].dtype == torch.bfloat16:
-        assert_close(cpu64(r["gates"]), bf16_round(gates), 2 ** -8, 0, what + " gates bf16")
+        assert_within_bf16_ulp(cpu64(r["gates"]), gates, what + " gates bf16")
     assert_close(cpu64(r["prob_sum"]), psum, F32_RTOL, F32_ATOL * s64.shape[0], what + " prob_sum")
     return probs, sel, gates, counts, psum
 
@@ -79,8 +79,8 @@ def test_router_bf16_full_size():
     probs, sel, gates, counts, psum = _check_route(r, s64, 8, "router bf16 full")
     f, P, aux = moe.moe_aux_stats(r["counts"], r["prob_sum"], cfg["T"], 8, out_dtype=torch.bfloat16)
     fo, Po, auxo = O.aux(counts, psum, cfg["T"], 8)
-    assert_close(cpu64(f), bf16_round(fo), 2 ** -8, 0, "f")
-    assert_close(cpu64(P), bf16_round(Po), 2 ** -8, 1e-9, "P")
+    assert_within_bf16_ulp(cpu64(f), fo, "f")
+    assert_within_bf16_ulp(cpu64(P), Po, "P")
     assert math.isclose(float(aux[0]), auxo, rel_tol=1e-5)
     assert math.isclose(float(cpu64(f).sum()), 8.0, rel_tol=1e-2)
 
