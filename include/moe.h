@@ -187,6 +187,42 @@ MOE_API int moe_dispatch(const int64_t* selected, int64_t T, int32_t k, int32_t 
                  size_t workspace_bytes, moe_stream_t stream);
 
 /*
+ * moe_dispatch_static -- moe_dispatch for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this is an interface variant of
+ * moe_dispatch with the same results, not a different computation.
+ *
+ * Who needs it: code that a host framework calls with nothing but input and
+ * output pointers (a plugin or custom-operator interface that manages the
+ * device memory budget itself) may not call cudaMalloc or cudaFree, which
+ * would synchronise the device and bypass that budget, so it cannot provide
+ * the workspace that moe_dispatch asks for.
+ *
+ * This entry point takes no workspace.  The slot scan's look-back state lives
+ * in one fixed file-scope device array of moe_dispatch_static_max_state_bytes()
+ * bytes (1 MiB) that every GPU which loads the library holds until the process
+ * exits.  The call allocates nothing: no cudaMalloc, cudaFree or allocating
+ * library routine.
+ *
+ * Arguments and outputs: as moe_dispatch, without workspace/workspace_bytes.
+ * Limit: ceil(T/512) * E * 4 + 4 bytes of state, rounded up to 256, must fit in
+ * the array (E = 256 allows T <= 523776); a larger problem returns
+ * MOE_ERR_UNSUPPORTED and enqueues nothing.
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.
+ * Sharing: all calls on a device use the same array; each call clears, in
+ * stream order, the part it uses before the scan, so a later call never sees
+ * an earlier call's state.  Calls that can overlap on the GPU (different
+ * streams not ordered by events) race on the array and must not be issued.
+ */
+MOE_API size_t moe_dispatch_static_max_state_bytes(void);
+MOE_API int moe_dispatch_static(const int64_t* selected, int64_t T, int32_t k, int32_t E, int64_t C,
+                                const void* x, moe_dtype dtype, int64_t D, int64_t ldx, int64_t* slot,
+                                uint8_t* kept, int32_t* used, int32_t* overflow, int32_t* drops_per_token,
+                                int32_t* token_of_slot, void* xbuf, int32_t* dev_status,
+                                moe_stream_t stream);
+
+/*
  * moe_expert_ffn -- every expert applied to its own rows of an expert-major
  * buffer (grouped GEMM over variable-occupancy experts).
  *

@@ -36,7 +36,7 @@ EXPORTED = [
     "moe_status_string", "moe_version", "moe_capacity", "moe_route_workspace_size", "moe_route",
     "moe_dispatch_workspace_size", "moe_dispatch", "moe_expert_ffn_workspace_size", "moe_expert_ffn",
     "moe_combine", "moe_aux_stats", "moe_backward_workspace_size", "moe_backward", "moe_transpose_weights",
-    "moe_clear_status", "moe_read_status",
+    "moe_clear_status", "moe_read_status", "moe_dispatch_static_max_state_bytes", "moe_dispatch_static",
 ]
 
 
@@ -71,6 +71,10 @@ def lib():
         L.moe_dispatch_workspace_size.argtypes = [_i64, _i32, _i32]
         L.moe_dispatch.argtypes = [_vp, _i64, _i32, _i32, _i64, _vp, ctypes.c_int, _i64, _i64, _vp, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_dispatch_static_max_state_bytes.restype = _sz
+        L.moe_dispatch_static_max_state_bytes.argtypes = []
+        L.moe_dispatch_static.argtypes = [_vp, _i64, _i32, _i32, _i64, _vp, ctypes.c_int, _i64, _i64, _vp, _vp, _vp,
+                                          _vp, _vp, _vp, _vp, _vp, _vp]
         L.moe_expert_ffn_workspace_size.restype = _sz
         L.moe_expert_ffn_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, _i32, _i64, _i64]
         L.moe_expert_ffn.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _vp,
@@ -226,6 +230,36 @@ def moe_dispatch(selected: torch.Tensor, E: int, C: int, x: Optional[torch.Tenso
                             _p(o["overflow"]), _p(o["drops"]), _p(o["token_of_slot"]), _p(o.get("xbuf")),
                             _p(dev_status), _p(ws), ws.numel(), _stream(stream))
     _check("moe_dispatch", rc)
+    return o
+
+
+def moe_dispatch_static(selected: torch.Tensor, E: int, C: int, x: Optional[torch.Tensor] = None,
+                        out: Optional[dict] = None, dev_status: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """moe_dispatch without a workspace: the scan state is a fixed device array in the library.
+
+    For callers that may not allocate device memory; the outputs here are still
+    allocated by PyTorch when ``out`` does not provide them.
+    """
+    dev = _dev(selected)
+    if selected.dtype != torch.int64:
+        raise TypeError("selected must be int64")
+    sel = selected.reshape(selected.shape[0], -1).contiguous()
+    T, k = sel.shape
+    o = dict(out or {})
+    o.setdefault("slot", torch.empty(T, k, dtype=torch.int64, device=dev))
+    o.setdefault("kept", torch.empty(T, k, dtype=torch.uint8, device=dev))
+    o.setdefault("used", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("overflow", torch.empty(E, dtype=torch.int32, device=dev))
+    o.setdefault("drops", torch.empty(T, dtype=torch.int32, device=dev))
+    o.setdefault("token_of_slot", torch.empty(E, max(C, 0), dtype=torch.int32, device=dev))
+    dt, D, ldx = MOE_F32, 0, 0
+    if x is not None:
+        dt, D, ldx = _dt(x), x.shape[1], _rowstride(x)
+        o.setdefault("xbuf", torch.empty(E, C, D, dtype=x.dtype, device=dev))
+    rc = lib().moe_dispatch_static(_p(sel), T, k, E, C, _p(x), dt, D, ldx, _p(o["slot"]), _p(o["kept"]),
+                                   _p(o["used"]), _p(o["overflow"]), _p(o["drops"]), _p(o["token_of_slot"]),
+                                   _p(o.get("xbuf")), _p(dev_status), _stream(stream))
+    _check("moe_dispatch_static", rc)
     return o
 
 
