@@ -490,3 +490,84 @@ void oracle_combine_slots(const double* ybuf, int64_t T, int32_t E, int64_t C, i
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Router variants of [P3] route_logits.                                       */
+/*   scoring 0: softmax clean scores; 1: logistic sigmoid clean scores         */
+/*   ([P3] stable_softmax / stable_sigmoid, element-wise for the sigmoid).     */
+/*   Selection key: the raw logits when no selection bias is given, else the   */
+/*   clean score plus the per-expert selection bias ([P3]: the bias moves the  */
+/*   selection only).  Ties go to the lower expert index.                      */
+/*   Gates: softmax of the selected logits (softmax scoring), or the selected  */
+/*   sigmoids normalised to sum one, computed as a softmax of log-sigmoids so  */
+/*   that it stays finite when every sigmoid underflows ([P3] sigmoid branch). */
+/*   clean (T,E) receives the clean scores.                                    */
+/* ------------------------------------------------------------------------ */
+static double log_sigmoid(double z) {
+    /* log(sigmoid(z)) = -log(1 + exp(-z)), split by sign to avoid overflow */
+    if (z >= 0.0) return -log1p(exp(-z));
+    return z - log1p(exp(z));
+}
+
+void oracle_route_variant(const double* s, int64_t T, int32_t E, int32_t k, int scoring,
+                          const double* selection_bias, double* clean, int64_t* selected,
+                          double* gates, int64_t* counts) {
+    OMP_FOR
+    for (int64_t t = 0; t < T; ++t) {
+        const double* st = s + t * E;
+        double* ct = clean + t * E;
+        if (scoring == 0) {
+            double mx = st[0];
+            for (int32_t e = 1; e < E; ++e) if (st[e] > mx) mx = st[e];
+            double den = 0.0;
+            for (int32_t e = 0; e < E; ++e) den += exp(st[e] - mx);
+            for (int32_t e = 0; e < E; ++e) ct[e] = exp(st[e] - mx) / den;
+        } else {
+            for (int32_t e = 0; e < E; ++e) ct[e] = sigmoid_stable(st[e]);
+        }
+        double* key = (double*)malloc((size_t)E * sizeof(double));
+        for (int32_t e = 0; e < E; ++e) key[e] = selection_bias ? ct[e] + selection_bias[e] : st[e];
+        char* taken = (char*)calloc((size_t)E, 1);
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || key[e] > key[best]) best = e;
+            }
+            taken[best] = 1;
+            selected[t * k + j] = best;
+        }
+        free(taken);
+        free(key);
+        /* gates: softmax over the selected logits, or over their log-sigmoids */
+        double* w = (double*)malloc((size_t)k * sizeof(double));
+        for (int32_t j = 0; j < k; ++j) {
+            double z = st[selected[t * k + j]];
+            w[j] = scoring == 0 ? z : log_sigmoid(z);
+        }
+        double wmax = w[0];
+        for (int32_t j = 1; j < k; ++j) if (w[j] > wmax) wmax = w[j];
+        double den = 0.0;
+        for (int32_t j = 0; j < k; ++j) den += exp(w[j] - wmax);
+        for (int32_t j = 0; j < k; ++j) gates[t * k + j] = exp(w[j] - wmax) / den;
+        free(w);
+    }
+    for (int32_t e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t i = 0; i < T * k; ++i) counts[selected[i]] += 1;
+}
+
+/* Survivor renormalisation ([P3] dispatch_with_capacity with                  */
+/* renormalize_kept_gates): dropped assignments get weight 0 and the kept      */
+/* weights of a token are divided by their sum; a token with nothing kept      */
+/* keeps all-zero weights.                                                     */
+void oracle_renormalize_kept(const double* gates, const uint8_t* kept, int64_t T, int32_t k,
+                             double* out) {
+    for (int64_t t = 0; t < T; ++t) {
+        double mass = 0.0;
+        for (int32_t j = 0; j < k; ++j) mass += kept[t * k + j] ? gates[t * k + j] : 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            double g = kept[t * k + j] ? gates[t * k + j] : 0.0;
+            out[t * k + j] = mass > 0.0 ? g / mass : 0.0;
+        }
+    }
+}

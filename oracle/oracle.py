@@ -67,6 +67,8 @@ def _load():
                                                    _D, _D]
         lib.oracle_combine_slots.argtypes = [_D, i64, i32, i64, i64, _I64, _I64, _U8, _D, i32,
                                              ctypes.c_int, _D, _D]
+        lib.oracle_route_variant.argtypes = [_D, i64, i32, i32, ctypes.c_int, _D, _D, _I64, _D, _I64]
+        lib.oracle_renormalize_kept.argtypes = [_D, _U8, i64, i32, _D]
         lib.oracle_dense_linear.argtypes = [_D, _I64, _I64, _U8, _D, _D, i64, i32, i32, i64, i64, i64,
                                             ctypes.c_int, _U8, _D, _D]
         _lib = lib
@@ -135,6 +137,42 @@ def route(s, k: int):
     _load().oracle_route(_p(s, _D), T, E, k, _p(probs, _D), _p(sel, _I64), _p(gates, _D),
                          _p(counts, _I64), _p(psum, _D))
     return probs, sel, gates, counts, psum
+
+
+SCORING = {"softmax": 0, "sigmoid": 1}
+
+
+def route_variant(s, k: int, scoring: str = "sigmoid", selection_bias=None):
+    """Module-7 router: softmax or sigmoid clean scores, optional selection-only bias.
+
+    Returns ``(clean (T,E), selected (T,k), gates (T,k), counts (E))``.
+    """
+    s = _f64(s)
+    if s.ndim == 1:
+        s = s[None, :]
+    T, E = s.shape
+    if not (1 <= k <= E):
+        raise ValueError("k must lie in [1, E]")
+    if not np.all(np.isfinite(s)):
+        raise ValueError("logits must be finite")
+    b = None if selection_bias is None else _f64(selection_bias)
+    clean = np.empty((T, E), np.float64)
+    sel = np.empty((T, k), np.int64)
+    gates = np.empty((T, k), np.float64)
+    counts = np.empty(E, np.int64)
+    _load().oracle_route_variant(_p(s, _D), T, E, k, SCORING[scoring], _p(b, _D), _p(clean, _D), _p(sel, _I64),
+                                 _p(gates, _D), _p(counts, _I64))
+    return clean, sel, gates, counts
+
+
+def renormalize_kept(gates, kept):
+    """Kept gates of each token divided by their sum; dropped (and fully dropped) rows are 0."""
+    g = _f64(gates)
+    T, k = g.shape
+    kp = _u8(kept).reshape(T, k)
+    out = np.empty((T, k), np.float64)
+    _load().oracle_renormalize_kept(_p(g, _D), _p(kp, _U8), T, k, _p(out, _D))
+    return out
 
 
 def dispatch(selected, E: int, C: int):

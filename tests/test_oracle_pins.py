@@ -438,3 +438,65 @@ def test_golden_files_cite_their_source():
     for name in os.listdir(GOLDEN):
         if name.endswith(".json"):
             assert "source" in _golden(name), name
+
+
+# --------------------------------------------------------------------------
+# module-7 router variants: sigmoid scoring, selection-only bias, survivor renormalisation
+# --------------------------------------------------------------------------
+def test_module7_sigmoid_router_pins():
+    g = _golden("module7_router_variants.json")
+    tol = g["check_tolerance"]
+    s = np.array([g["logits"]])
+    clean, sel, gates, counts = O.route_variant(s, g["top_k"], "sigmoid")
+    np.testing.assert_allclose(clean[0], g["scores"], rtol=0, atol=1e-15)
+    assert sel[0].tolist() == g["selected"]
+    np.testing.assert_allclose(gates[0], g["gates"], rtol=0, atol=tol)
+    _, selb, gatesb, _ = O.route_variant(s, g["top_k"], "sigmoid", selection_bias=g["bias"])
+    assert selb[0].tolist() == g["selected_with_bias"]
+    np.testing.assert_allclose(gatesb[0], g["gates_with_bias"], rtol=0, atol=tol)
+    # the bias moves the selection only: gates are the selected clean sigmoids, renormalised
+    sig = np.array(g["scores"])[selb[0]]
+    np.testing.assert_allclose(gatesb[0], sig / sig.sum(), rtol=1e-14)
+
+
+def test_module7_sigmoid_extreme_logits_and_softmax_variant():
+    # sigmoid gates stay finite where every sigmoid underflows; two logits 1 apart -> [sigma(1), sigma(-1)]
+    _, sel, gates, _ = O.route_variant(np.array([[-1002.0, -1000.0, -1001.0]]), 2, "sigmoid")
+    assert sel[0].tolist() == [1, 2]
+    np.testing.assert_allclose(gates[0], [1 / (1 + math.exp(-1)), 1 / (1 + math.exp(1))], rtol=1e-12)
+    # softmax scoring without a bias is the plain router
+    rng = np.random.default_rng(21)
+    s = rng.integers(-3, 4, size=(30, 6)).astype(float)
+    clean, sel, gates, counts = O.route_variant(s, 3, "softmax")
+    probs, sel0, gates0, counts0, _ = O.route(s, 3)
+    np.testing.assert_array_equal(sel, sel0)
+    np.testing.assert_allclose(gates, gates0, rtol=1e-15)
+    np.testing.assert_allclose(clean, probs, rtol=1e-15)
+    assert (counts == counts0).all()
+    # softmax scoring with a selection bias ranks p + b, gates still come from the logits
+    b = np.linspace(0.0, 0.5, 6)
+    _, selb, gatesb, _ = O.route_variant(s, 3, "softmax", selection_bias=b)
+    for t in range(30):
+        key = probs[t] + b
+        assert selb[t].tolist() == sorted(range(6), key=lambda e: (-key[e], e))[:3]
+        z = s[t, selb[t]]
+        np.testing.assert_allclose(gatesb[t], np.exp(z - z.max()) / np.exp(z - z.max()).sum(), rtol=1e-14)
+
+
+def test_module7_survivor_renormalisation():
+    g = _golden("module7_capacity_fifo.json")
+    s = np.array(g["logits"])
+    T, E = s.shape
+    _, sel, gates, _, _ = O.route(s, g["top_k"])
+    d = O.dispatch(sel, E, O.capacity(T, g["top_k"], E, g["capacity_factor"]))
+    r = O.renormalize_kept(gates, d["kept"])
+    # the capacity cell checks that the surviving weights of every token sum to one
+    np.testing.assert_allclose(r.sum(1), 1.0, rtol=1e-15)
+    assert (r[~d["kept"]] == 0).all()
+    # all-same case: fully dropped tokens keep all-zero weights, no division by zero
+    a = _golden("module7_capacity_fifo.json")["all_same_case"]
+    s2 = np.array(a["logits"])
+    _, sel2, gates2, _, _ = O.route(s2, a["top_k"])
+    d2 = O.dispatch(sel2, 2, O.capacity(4, a["top_k"], 2, a["capacity_factor"]))
+    r2 = O.renormalize_kept(gates2, d2["kept"])
+    assert (r2[1:] == 0).all() and r2[0, 0] == 1.0
