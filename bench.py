@@ -304,7 +304,7 @@ def run_ours(args, world, rank, local):
     ffn_avg_s = statistics.mean(ffn_ms) / 1e3
     pk = measured_peaks()
     achieved = flops / ffn_avg_s / 1e12
-    roof = dict(bound="tensor", kernel="tc_gemm_kernel: routed SwiGLU gate/up + down launches", achieved=achieved,
+    roof = dict(bound="tensor", kernel="tcx_kernel: routed SwiGLU gate/up + down launches", achieved=achieved,
                 peak=pk["bf16_sustained"], unit="TFLOP/s", frac=achieved / pk["bf16_sustained"], traffic=None,
                 peak_source=f"{pk['source']} bf16 sustained", frac_of_burst=achieved / pk["bf16"],
                 flops_per_launch=flops, kept_rows=kept, avg_launch_ms=1e3 * ffn_avg_s)
@@ -317,6 +317,9 @@ def run_ours(args, world, rank, local):
         tps, S, dt = time_oracle(cfg64, args.cpu_seconds)
         cpu = dict(value=tps, unit=UNIT, cores=os.cpu_count(), kind="oracle",
                    sample=f"first {S} tokens of the batch ({dt:.1f} s), capacity from the sample's T")
+    others = None
+    if world == 1 and not args.no_other_workloads:
+        others = run_other_workloads(min(args.steps, 20), max(3, min(args.warmup, 5)), flush, stream, dev)
     wl = dict(WORKLOAD, T=T, experts=E, capacity=layer.C)
     line = dict(
         metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
@@ -327,7 +330,7 @@ def run_ours(args, world, rank, local):
         e2e=None if e2e_value is None else dict(value=e2e_value, unit=UNIT, h2d_bytes_per_step=T * H * 2,
                                                 d2h_bytes_per_step=T * H * 2 + 8),
         gpu_launches=KERNELS_PER_STEP * args.steps,
-        roofline=roof, cpu_baseline=cpu, clocks=clocks.summary(),
+        roofline=roof, cpu_baseline=cpu, clocks=clocks.summary(), workloads=others,
     )
     print(json.dumps(line), flush=True)
 
@@ -358,6 +361,179 @@ def run_e2e(args, world, cfg, dv, step, flush, stream):
     return job_throughput(T, args.steps, world, e2e_ms)
 
 
+# ------------------------------------------------------------------------------------------------
+# The other workloads of the pages, timed the same way (events around every step, L2 flush between
+# steps) and reported in the "workloads" field.  Each names its dominant kernel call and roofline.
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # FFMA lanes x 2 flops x max SM clock
+
+
+def _time_steps(step, steps, warmup, flush, stream, inner=None):
+    """Device time of `steps` calls of step() (ms each) and of the inner event pair step() records."""
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if inner is not None:
+        inner.clear()
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        st[i].record(stream)
+        step()
+        en[i].record(stream)
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in zip(st, en)]
+    inner_ms = [a.elapsed_time(b) for a, b in inner] if inner is not None else []
+    return step_ms, inner_ms
+
+
+def run_other_workloads(steps, warmup, flush, stream, dev):
+    import sparse_mixture_experts_stable_b200 as moe
+    from sparse_mixture_experts_stable_b200 import binding as B
+    from sparse_mixture_experts_stable_b200 import inputs as I
+
+    pk = measured_peaks()
+    out = {}
+
+    def events(lst):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        lst.append((e0, e1))
+        return e0, e1
+
+    # router-only with load statistics (router GEMM + softmax/top-k/gates + statistics)
+    c = I.router_bf16(seed=0)
+    T, D, E, k = c["T"], c["D"], c["E"], c["k"]
+    x, w = c["x"].to(dev), c["w_router"].to(dev)
+    ro = dict(selected=torch.empty(T, k, dtype=torch.int64, device=dev),
+              gates=torch.empty(T, k, dtype=torch.bfloat16, device=dev),
+              gates_f32=torch.empty(T, k, dtype=torch.float32, device=dev),
+              counts=torch.empty(E, dtype=torch.int32, device=dev), prob_sum=torch.empty(E, device=dev))
+    ws = torch.empty(B.moe_route_workspace_size(T, D, E, B.MOE_BF16, True, "ED"), dtype=torch.uint8, device=dev)
+    inner = []
+
+    def step_router():
+        e0, e1 = events(inner)
+        e0.record(stream)
+        moe.moe_route(x, k, w_router=w, out=ro, workspace=ws)
+        e1.record(stream)
+        moe.moe_aux_stats(ro["counts"], ro["prob_sum"], T, k, out_dtype=torch.bfloat16)
+
+    sm, im = _time_steps(step_router, steps, warmup, flush, stream, inner)
+    r_s = statistics.mean(im) / 1e3
+    bytes_alg = T * D * 2 + E * D * 2 + T * k * (8 + 2 + 4) + E * 8
+    flops = 2.0 * T * D * E
+    out["router_bf16"] = dict(
+        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+        config=dict(T=T, D=D, E=E, k=k),
+        roofline=dict(bound="hbm/tensor ridge", kernel="moe_route (tcx router GEMM + top-k + reduce)",
+                      achieved=bytes_alg / r_s / 1e9, peak=pk["hbm"], unit="GB/s", frac=bytes_alg / r_s / 1e9 / pk["hbm"],
+                      tflops=flops / r_s / 1e12, frac_tensor=flops / r_s / 1e12 / pk["bf16"], traffic=None,
+                      bytes_per_launch=bytes_alg, flops_per_launch=flops, avg_launch_ms=1e3 * r_s))
+    del x, w, ws, ro
+
+    # capacity-limited top-1 dispatch/combine with linear experts
+    c = I.dispatch_top1_bf16(seed=0)
+    T, D, E = c["T"], c["D"], c["E"]
+    C = moe.moe_capacity(T, 1, E, c["capacity_factor"])
+    idx = c["expert_idx"].view(T, 1).to(dev)
+    x, w, gate = c["x"].to(dev), c["w"].to(dev), c["gate"].view(T, 1).to(dev)
+    do = dict(slot=torch.empty(T, 1, dtype=torch.int64, device=dev), kept=torch.empty(T, 1, dtype=torch.uint8, device=dev),
+              used=torch.empty(E, dtype=torch.int32, device=dev), overflow=torch.empty(E, dtype=torch.int32, device=dev),
+              drops=torch.empty(T, dtype=torch.int32, device=dev),
+              token_of_slot=torch.empty(E, C, dtype=torch.int32, device=dev),
+              xbuf=torch.empty(E, C, D, dtype=torch.bfloat16, device=dev))
+    ybuf = torch.empty(E, C, D, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
+    wsd = torch.empty(B.moe_dispatch_workspace_size(T, 1, E), dtype=torch.uint8, device=dev)
+    inner = []
+
+    def step_top1():
+        moe.moe_dispatch(idx, E, C, x=x, out=do, workspace=wsd)
+        e0, e1 = events(inner)
+        e0.record(stream)
+        moe.moe_expert_ffn("linear", do["xbuf"], do["used"], w, ybuf=ybuf)
+        e1.record(stream)
+        moe.moe_combine(ybuf, idx, do["slot"], gate, y=y)
+
+    sm, im = _time_steps(step_top1, steps, warmup, flush, stream, inner)
+    used = do["used"].cpu()
+    kept = int(used.sum())
+    active = int((used > 0).sum())
+    f_s = statistics.mean(im) / 1e3
+    bytes_alg = kept * D * 2 + active * D * D * 2 + kept * D * 2
+    out["dispatch_top1_bf16"] = dict(
+        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+        config=dict(T=T, D=D, E=E, k=1, capacity=C, kept=kept),
+        roofline=dict(bound="hbm", kernel="tcx_kernel: linear experts (moe_expert_ffn)", achieved=bytes_alg / f_s / 1e9,
+                      peak=pk["hbm"], unit="GB/s", frac=bytes_alg / f_s / 1e9 / pk["hbm"], traffic=None,
+                      tflops=2.0 * kept * D * D / f_s / 1e12, bytes_per_launch=bytes_alg, avg_launch_ms=1e3 * f_s))
+    del x, w, gate, do, ybuf, y
+
+    # tiny top-2 GELU layer, fp32
+    c = I.tiny_gelu_fp32(seed=0)
+    T, D, E, F, k = c["T"], c["D"], c["E"], c["F"], c["k"]
+    C = moe.moe_capacity(T, k, E, c["capacity_factor"])
+    dv = {n: c[n].to(dev) for n in ("x", "w_router", "w1", "b1", "w2", "b2")}
+    inner = []
+
+    def step_tiny():
+        r = moe.moe_route(dv["x"], k, w_router=dv["w_router"])
+        d = moe.moe_dispatch(r["selected"], E, C, x=dv["x"])
+        e0, e1 = events(inner)
+        e0.record(stream)
+        yb = moe.moe_expert_ffn("gelu_mlp", d["xbuf"], d["used"], dv["w1"], b1=dv["b1"], w2=dv["w2"], b2=dv["b2"])
+        e1.record(stream)
+        moe.moe_combine(yb, r["selected"], d["slot"], r["gates_f32"], base_kind="input", base=dv["x"])
+        moe.moe_aux_stats(r["counts"], r["prob_sum"], T, k, True, 0.01)
+
+    sm, im = _time_steps(step_tiny, steps, warmup, flush, stream, inner)
+    f_s = statistics.mean(im) / 1e3
+    flops = 2.0 * T * k * (D * F + F * D)
+    out["tiny_gelu_fp32"] = dict(
+        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+        config=dict(T=T, D=D, E=E, F=F, k=k, capacity=C),
+        roofline=dict(bound="alu", kernel="sgemm_kernel: GELU MLP experts (moe_expert_ffn)",
+                      achieved=flops / f_s / 1e12, peak=FP32_PEAK_TFLOPS, unit="TFLOP/s",
+                      frac=flops / f_s / 1e12 / FP32_PEAK_TFLOPS, traffic=None, avg_launch_ms=1e3 * f_s,
+                      note="launch-latency bound at this size"))
+    del dv
+
+    # forward + backward, fp32, linear experts with residual
+    c = I.fwd_bwd_fp32(seed=0)
+    T, D, E, k = c["T"], c["D"], c["E"], c["k"]
+    C = moe.moe_capacity(T, k, E, c["capacity_factor"])
+    lg, x, w, dy = (c[n].to(dev) for n in ("logits", "x", "w", "dy"))
+    inner = []
+    wsb = torch.empty(B.moe_backward_workspace_size(E, C, D, D), dtype=torch.uint8, device=dev)
+    state = {}
+
+    def step_fb():
+        r = moe.moe_route(lg, k)
+        d = moe.moe_dispatch(r["selected"], E, C, x=x)
+        yb = moe.moe_expert_ffn("linear", d["xbuf"], d["used"], w)
+        moe.moe_combine(yb, r["selected"], d["slot"], r["gates_f32"], base_kind="input", base=x)
+        e0, e1 = events(inner)
+        e0.record(stream)
+        moe.moe_backward(dy, x, lg, r["selected"], r["gates_f32"], d["slot"], d["used"], d["token_of_slot"],
+                         d["xbuf"], yb, w, C, workspace=wsb)
+        e1.record(stream)
+        state["used"] = d["used"]
+
+    sm, im = _time_steps(step_fb, steps, warmup, flush, stream, inner)
+    kept = int(state["used"].sum())
+    b_s = statistics.mean(im) / 1e3
+    flops_b = 2.0 * kept * D * D * 2 + 2.0 * kept * D
+    out["fwd_bwd_fp32"] = dict(
+        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+        config=dict(T=T, D=D, E=E, k=k, capacity=C, kept=kept),
+        roofline=dict(bound="alu", kernel="moe_backward (sgemm_kernel dW + dx, dgate/dlogits, combine)",
+                      achieved=flops_b / b_s / 1e12, peak=FP32_PEAK_TFLOPS, unit="TFLOP/s",
+                      frac=flops_b / b_s / 1e12 / FP32_PEAK_TFLOPS, traffic=None, avg_launch_ms=1e3 * b_s,
+                      peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"))
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -369,6 +545,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=WORKLOAD["T"], help="tokens per rank (smaller for profiling)")
     ap.add_argument("--experts", type=int, default=WORKLOAD["experts"], help="routed experts (smaller for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip timing the router-only, top-1, tiny fp32 and fp32 fwd+bwd workloads")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:

@@ -85,6 +85,10 @@ typedef enum { MOE_FFN_LINEAR = 0, MOE_FFN_GELU_MLP = 1, MOE_FFN_SWIGLU = 2 } mo
 /* Router weight layout: (D, E) as on [P2]; (E, D) as nn.Linear in [P5]. */
 typedef enum { MOE_ROUTER_DE = 0, MOE_ROUTER_ED = 1 } moe_router_layout;
 
+/* Clean router scores ([P3] route_logits): softmax over the experts, or an
+ * independent logistic sigmoid per expert. */
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_scoring;
+
 /* Static string for a moe_status value. */
 MOE_API const char* moe_status_string(int status);
 
@@ -147,6 +151,43 @@ MOE_API int moe_route(const void* x, moe_dtype dtype, int64_t T, int64_t D, int6
               int32_t k, float* logits_out, int64_t* selected, void* gates, float* gates_f32,
               int32_t* counts, float* prob_sum, int32_t* dev_status, void* workspace,
               size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * moe_route_ex -- moe_route with the router variants of [P3] route_logits.
+ *   scoring        MOE_SCORE_SOFTMAX: clean scores p = softmax(s); gates =
+ *                  softmax of the selected logits (moe_route's behaviour).
+ *                  MOE_SCORE_SIGMOID: clean scores sigmoid(s) per expert;
+ *                  gates = the selected sigmoids divided by their sum,
+ *                  computed as a softmax of log-sigmoids so that it stays
+ *                  finite when every sigmoid underflows.
+ *   selection_bias device fp32 (E) or NULL.  When given, the top-k ranks the
+ *                  clean score plus this bias (the bias moves the selection
+ *                  only; gates still come from the clean scores); otherwise the
+ *                  ranking uses the logits themselves.  Ties -> lower index.
+ *                  The ranking is decided in fp32.
+ *   prob_sum[e]    sum over tokens of the clean score of expert e.
+ *   z_loss         device fp32 (1) or NULL: the router z-loss
+ *                  mean_t logsumexp(s_t)^2 ([P3] router_z_loss), fixed-order.
+ * Other arguments as moe_route; the workspace size is the same.
+ */
+MOE_API int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D, int64_t ldx,
+                         const void* w_router, moe_router_layout layout, int32_t E,
+                         const float* logit_bias, int32_t k, moe_scoring scoring,
+                         const float* selection_bias, float* logits_out, int64_t* selected,
+                         void* gates, float* gates_f32, int32_t* counts, float* prob_sum,
+                         float* z_loss, int32_t* dev_status, void* workspace,
+                         size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * moe_renormalize_kept_gates -- [P3] dispatch_with_capacity with
+ * renormalize_kept_gates: out[t,j] = gates[t,j] / sum of token t's kept gates
+ * for kept assignments (slot[t,j] >= 0), 0 for dropped ones, and all zeros for
+ * a token with nothing kept.  gates_f32, out: device fp32 (T, k); slot: device
+ * int64 (T, k) from moe_dispatch.  The default layer keeps the pre-drop gates
+ * ([P1] section 1 item 4); pass this output to moe_combine for the other policy.
+ */
+MOE_API int moe_renormalize_kept_gates(const float* gates_f32, const int64_t* slot, int64_t T,
+                                       int32_t k, float* out, moe_stream_t stream);
 
 /*
  * moe_dispatch -- greedy position-priority slot assignment and the gather

@@ -37,7 +37,9 @@ EXPORTED = [
     "moe_dispatch_workspace_size", "moe_dispatch", "moe_expert_ffn_workspace_size", "moe_expert_ffn",
     "moe_combine", "moe_aux_stats", "moe_backward_workspace_size", "moe_backward", "moe_transpose_weights",
     "moe_clear_status", "moe_read_status", "moe_dispatch_static_max_state_bytes", "moe_dispatch_static",
+    "moe_route_ex", "moe_renormalize_kept_gates",
 ]
+SCORING = {"softmax": 0, "sigmoid": 1}
 
 
 class MoeError(RuntimeError):
@@ -67,6 +69,9 @@ def lib():
         L.moe_route_workspace_size.argtypes = [_i64, _i64, _i32, ctypes.c_int, ctypes.c_int, ctypes.c_int]
         L.moe_route.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, ctypes.c_int, _i32, _vp, _i32, _vp, _vp,
                                 _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_route_ex.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, ctypes.c_int, _i32, _vp, _i32,
+                                   ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_renormalize_kept_gates.argtypes = [_vp, _vp, _i64, _i32, _vp, _vp]
         L.moe_dispatch_workspace_size.restype = _sz
         L.moe_dispatch_workspace_size.argtypes = [_i64, _i32, _i32]
         L.moe_dispatch.argtypes = [_vp, _i64, _i32, _i32, _i64, _vp, ctypes.c_int, _i64, _i64, _vp, _vp, _vp, _vp,
@@ -164,13 +169,16 @@ def moe_route_workspace_size(T, D, E, dtype: int, has_router_weight: bool, layou
 def moe_route(x: torch.Tensor, k: int, w_router: Optional[torch.Tensor] = None, layout: str = "ED",
               E: Optional[int] = None, logit_bias: Optional[torch.Tensor] = None, want_logits: bool = False,
               out: Optional[dict] = None, dev_status: Optional[torch.Tensor] = None,
-              workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
-    """Router scores, softmax, stable top-k, gates, counts and probability sums.
+              workspace: Optional[torch.Tensor] = None, stream=None, scoring: str = "softmax",
+              selection_bias: Optional[torch.Tensor] = None, want_z_loss: bool = False) -> dict:
+    """Router scores, clean scores (softmax or sigmoid), stable top-k, gates, counts, score sums.
 
     ``x`` is (T, D) activations with ``w_router`` given in ``layout`` ("ED" =
     nn.Linear (E, D), "DE" = (D, E)), or (T, E) logits when ``w_router`` is None.
-    Returns a dict of device tensors: selected, gates (x dtype), gates_f32,
-    counts, prob_sum (and logits when requested).
+    ``selection_bias`` (E) moves the selection only.  Calls ``moe_route_ex``
+    (``moe_route`` is its softmax, no-bias case).  Returns a dict of device
+    tensors: selected, gates (x dtype), gates_f32, counts, prob_sum (and logits,
+    z_loss when requested).
     """
     dev = _dev(x)
     dt = _dt(x)
@@ -192,13 +200,27 @@ def moe_route(x: torch.Tensor, k: int, w_router: Optional[torch.Tensor] = None, 
     o.setdefault("prob_sum", torch.empty(E, dtype=torch.float32, device=dev))
     if want_logits:
         o.setdefault("logits", torch.empty(T, E, dtype=torch.float32, device=dev))
+    if want_z_loss:
+        o.setdefault("z_loss", torch.empty(1, dtype=torch.float32, device=dev))
     ws = _workspace(moe_route_workspace_size(T, D, E, dt, w_router is not None, layout), dev, workspace)
     bias = None if logit_bias is None else logit_bias.to(torch.float32).contiguous()
-    rc = lib().moe_route(_p(x), dt, T, D, _rowstride(x), _p(w_router), ROUTER_LAYOUT[layout], E, _p(bias), k,
-                         _p(o.get("logits")), _p(o["selected"]), _p(o["gates"]), _p(o["gates_f32"]),
-                         _p(o["counts"]), _p(o["prob_sum"]), _p(dev_status), _p(ws), ws.numel(), _stream(stream))
-    _check("moe_route", rc)
+    sb = None if selection_bias is None else selection_bias.to(torch.float32).contiguous()
+    rc = lib().moe_route_ex(_p(x), dt, T, D, _rowstride(x), _p(w_router), ROUTER_LAYOUT[layout], E, _p(bias), k,
+                            SCORING[scoring], _p(sb), _p(o.get("logits")), _p(o["selected"]), _p(o["gates"]),
+                            _p(o["gates_f32"]), _p(o["counts"]), _p(o["prob_sum"]), _p(o.get("z_loss")),
+                            _p(dev_status), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_route_ex", rc)
     return o
+
+
+def moe_renormalize_kept_gates(gates_f32: torch.Tensor, slot: torch.Tensor, stream=None) -> torch.Tensor:
+    """Kept gates divided by their per-token sum; dropped assignments and fully dropped tokens get 0."""
+    T, k = gates_f32.shape
+    out = torch.empty_like(gates_f32)
+    rc = lib().moe_renormalize_kept_gates(_p(gates_f32.contiguous()), _p(slot.contiguous()), T, k, _p(out),
+                                          _stream(stream))
+    _check("moe_renormalize_kept_gates", rc)
+    return out
 
 
 def moe_dispatch_workspace_size(T: int, k: int, E: int) -> int:

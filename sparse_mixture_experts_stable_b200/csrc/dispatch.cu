@@ -32,6 +32,19 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
     return v;
 }
 
+constexpr int kBatch = 8;  // chunk keys fetched together per warp
+
+// Expert index of stream element li of this block, or -1 when the element does
+// not exist or (reported to status when given) lies outside [0, E).
+__device__ __forceinline__ int load_key(const int64_t* __restrict__ selected, int64_t base_i, int n_el, int li,
+                                        bool chunk_ok, int E, int32_t* status) {
+    if (!chunk_ok || li >= n_el) return -1;
+    const int64_t e = selected[base_i + li];
+    if (e >= 0 && e < E) return (int)e;
+    if (status) set_status(status, MOE_ERR_BAD_INDEX);
+    return -1;
+}
+
 __global__ void __launch_bounds__(kScanThreads)
     slot_scan_kernel(const int64_t* __restrict__ selected, int64_t T, int k, int E, int64_t C, int nblocks,
                      int64_t* __restrict__ slot, uint8_t* __restrict__ kept, int32_t* __restrict__ used,
@@ -60,17 +73,19 @@ __global__ void __launch_bounds__(kScanThreads)
     const int c_end = (c_begin + cpw) < nchunks ? (c_begin + cpw) : nchunks;
     int* my_off = s_off + warp * E;
 
-    // pass 1: per-warp histogram of the warp's chunks
-    for (int c = c_begin; c < c_end; ++c) {
-        const int li = c * 32 + lane;
-        int key = -1;
-        if (li < n_el) {
-            const int64_t e = selected[base_i + li];
-            if (e >= 0 && e < E) key = (int)e;
-            else set_status(status, MOE_ERR_BAD_INDEX);
+    // pass 1: per-warp histogram of the warp's chunks (keys fetched kBatch chunks at a time)
+    for (int c0 = c_begin; c0 < c_end; c0 += kBatch) {
+        int keys[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) keys[u] = load_key(selected, base_i, n_el, (c0 + u) * 32 + lane, c0 + u < c_end, E,
+                                                          status);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            if (c0 + u >= c_end) break;
+            const int key = keys[u];
+            const uint32_t match = __match_any_sync(0xffffffffu, key);
+            if (key >= 0 && (__ffs(match) - 1) == lane) my_off[key] += __popc(match);
         }
-        const uint32_t match = __match_any_sync(0xffffffffu, key);
-        if (key >= 0 && (__ffs(match) - 1) == lane) my_off[key] += __popc(match);
     }
     __syncthreads();
 
@@ -122,13 +137,17 @@ __global__ void __launch_bounds__(kScanThreads)
     __syncthreads();
 
     // pass 2: ranks -> slots
-    for (int c = c_begin; c < c_end; ++c) {
+    for (int c0 = c_begin; c0 < c_end; c0 += kBatch) {
+      int keys[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+          keys[u] = load_key(selected, base_i, n_el, (c0 + u) * 32 + lane, c0 + u < c_end, E, nullptr);
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int c = c0 + u;
+        if (c >= c_end) break;
         const int li = c * 32 + lane;
-        int key = -1;
-        if (li < n_el) {
-            const int64_t e = selected[base_i + li];
-            if (e >= 0 && e < E) key = (int)e;
-        }
+        const int key = keys[u];
         const uint32_t match = __match_any_sync(0xffffffffu, key);
         int rank = 0;
         if (key >= 0) rank = my_off[key] + __popc(match & lanemask_lt());
@@ -148,6 +167,7 @@ __global__ void __launch_bounds__(kScanThreads)
                 atomicAdd(&s_drop[t - t0], 1);
             }
         }
+      }
     }
     __syncthreads();
     for (int i = threadIdx.x; i < ntok; i += kScanThreads) drops[t0 + i] = s_drop[i];

@@ -4,6 +4,7 @@
 
 #include "common.cuh"
 #include "simt_gemm.cuh"
+#include "tc_expert_gemm.cuh"
 #include "tc_gemm.cuh"
 
 using namespace moe;
@@ -33,46 +34,76 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
     }
 
     if (dtype == MOE_BF16) {
-        // first GEMM: xbuf (E*C, D) x W^T
-        TcGemmProblem p{};
-        p.a = xbuf;
-        p.lda = D;
-        p.a_rows_total = (int64_t)E * C;
-        p.a_rows_per_group = C;
-        p.G = E;
-        p.M = C;
-        p.K = D;
-        p.rows = used;
-        p.out_rows_per_group = C;
-        p.status = dev_status;
-        if (kind == MOE_FFN_LINEAR) {
-            p.b = w1;
-            p.ldb = D;
-            p.b_rows_total = (int64_t)E * Dout;
-            p.b_rows_per_group = Dout;
-            p.N = Dout;
-            p.out = ybuf;
-            p.ldo = Dout;
-            p.epilogue = TC_EPI_BF16;
-            return tc_gemm_run(p, stream);
-        }
-        p.ldb = D;
-        p.b_rows_total = (int64_t)E * F;
-        p.b_rows_per_group = F;
-        p.N = F;
-        p.out = h;
-        p.ldo = F;
-        if (kind == MOE_FFN_SWIGLU) {
-            p.b = w1;   // gate
-            p.b2 = w3;  // up
+        // Kernel choice (measured on B200): the SwiGLU gate/up GEMM over ragged
+        // experts runs with weights on the MMA's M side (tcx_gemm_run: at most
+        // 15 padded token rows per expert); every other bf16 GEMM runs with
+        // token rows on the M side and a single N=256 weight operand
+        // (tc_gemm_run), which reads the fewest shared-memory operand bytes.
+        int rc;
+        if (kind == MOE_FFN_SWIGLU && used != nullptr) {
+            TcxProblem p{};
+            p.w = w1;   // gate
+            p.w2 = w3;  // up
+            p.ldw = D;
+            p.w_rows_total = (int64_t)E * F;
+            p.w_rows_per_group = F;
+            p.x = xbuf;
+            p.ldx = D;
+            p.x_rows_total = (int64_t)E * C;
+            p.x_rows_per_group = C;
+            p.G = E;
+            p.features = F;
+            p.max_tokens = C;
+            p.K = D;
+            p.rows = used;
+            p.out = h;
+            p.ldo = F;
+            p.out_rows_per_group = C;
             p.epilogue = TC_EPI_SWIGLU;
+            p.status = dev_status;
+            rc = tcx_gemm_run(p, stream);
         } else {
-            p.b = w1;
-            p.bias = b1;
-            p.bias_group_stride = F;
-            p.epilogue = TC_EPI_GELU_BIAS;
+            // first GEMM: xbuf (E*C, D) x W^T
+            TcGemmProblem p{};
+            p.a = xbuf;
+            p.lda = D;
+            p.a_rows_total = (int64_t)E * C;
+            p.a_rows_per_group = C;
+            p.G = E;
+            p.M = C;
+            p.K = D;
+            p.rows = used;
+            p.out_rows_per_group = C;
+            p.status = dev_status;
+            if (kind == MOE_FFN_LINEAR) {
+                p.b = w1;
+                p.ldb = D;
+                p.b_rows_total = (int64_t)E * Dout;
+                p.b_rows_per_group = Dout;
+                p.N = Dout;
+                p.out = ybuf;
+                p.ldo = Dout;
+                p.epilogue = TC_EPI_BF16;
+                return tc_gemm_run(p, stream);
+            }
+            p.ldb = D;
+            p.b_rows_total = (int64_t)E * F;
+            p.b_rows_per_group = F;
+            p.N = F;
+            p.out = h;
+            p.ldo = F;
+            if (kind == MOE_FFN_SWIGLU) {
+                p.b = w1;   // gate
+                p.b2 = w3;  // up
+                p.epilogue = TC_EPI_SWIGLU;
+            } else {
+                p.b = w1;
+                p.bias = b1;
+                p.bias_group_stride = F;
+                p.epilogue = TC_EPI_GELU_BIAS;
+            }
+            rc = tc_gemm_run(p, stream);
         }
-        int rc = tc_gemm_run(p, stream);
         if (rc != MOE_OK) return rc;
         // second GEMM: h (E*C, F) x W2^T
         TcGemmProblem q{};

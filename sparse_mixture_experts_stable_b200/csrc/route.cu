@@ -11,7 +11,7 @@
 
 #include "common.cuh"
 #include "simt_gemm.cuh"
-#include "tc_gemm.cuh"
+#include "tc_expert_gemm.cuh"
 #include "util_kernels.cuh"
 
 namespace moe {
@@ -28,37 +28,61 @@ int route_blocks(int64_t T) {
     return (int)(b < kMaxRouteBlocks ? b : kMaxRouteBlocks);
 }
 
-// Is (v, i) ranked ahead of (bv, bi)?  Larger score first, then lower index.
-__device__ __forceinline__ bool ahead(float v, int i, float bv, int bi) {
-    return v > bv || (v == bv && i < bi);
+// Order-preserving map from fp32 to uint32 (larger float -> larger key).  The
+// score is canonicalised first so that -0 and +0 (equal as floats) share a key;
+// NaN never reaches it (non-finite scores are replaced by -inf before).
+__device__ __forceinline__ uint32_t order_key(float v) {
+    if (v == 0.0f) v = 0.0f;
+    const uint32_t b = __float_as_uint(v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 // Each lane holds experts e = m*32 + lane, m < EPL.
+__device__ __forceinline__ float sigmoid_stable_f(float z) {
+    if (z >= 0.f) return 1.f / (1.f + expf(-z));
+    const float ez = expf(z);
+    return ez / (1.f + ez);
+}
+__device__ __forceinline__ float log_sigmoid_f(float z) {
+    return z >= 0.f ? -log1pf(expf(-z)) : z - log1pf(expf(z));
+}
+
+// scoring: 0 softmax, 1 sigmoid.  sel_bias (E) or NULL: added to the clean
+// scores for the selection only.  part_z (gridDim) or NULL: per-block sums of
+// logsumexp(s_t)^2 for the router z-loss.
 template <int EPL, typename InT>
 __global__ void __launch_bounds__(kRouteThreads)
     route_topk_kernel(const InT* __restrict__ logits, int64_t ld, int64_t T, int E, int k,
                       const float* __restrict__ bias, float* __restrict__ logits_out,
                       int64_t* __restrict__ selected, void* __restrict__ gates_out, int gates_bf16,
                       float* __restrict__ gates_f32, int32_t* __restrict__ part_counts,
-                      float* __restrict__ part_psum, int32_t* status) {
+                      float* __restrict__ part_psum, int scoring, const float* __restrict__ sel_bias,
+                      float* __restrict__ part_z, int32_t* status) {
     extern __shared__ float s_dyn[];
     float* s_psum = s_dyn;                                            // [kRouteWarps][E]
     int* s_counts = reinterpret_cast<int*>(s_psum + kRouteWarps * E);  // [E]
     float* s_selv = reinterpret_cast<float*>(s_counts + E);            // [kRouteWarps][k]
+    __shared__ float s_z[kRouteWarps];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_counts[e] = 0;
     __syncthreads();
 
     float bias_r[EPL];
+    float sbias_r[EPL];
     float psum[EPL];
 #pragma unroll
     for (int m = 0; m < EPL; ++m) {
         const int e = m * 32 + lane;
         bias_r[m] = (bias && e < E) ? bias[e] : 0.f;
+        sbias_r[m] = (sel_bias && e < E) ? sel_bias[e] : 0.f;
         psum[m] = 0.f;
     }
     float* selv = s_selv + warp * k;
+    float zacc = 0.f;
 
     const int64_t stride = (int64_t)gridDim.x * kRouteWarps;
     for (int64_t t = (int64_t)blockIdx.x * kRouteWarps + warp; t < T; t += stride) {
@@ -84,57 +108,76 @@ __global__ void __launch_bounds__(kRouteThreads)
         }
         if (!__all_sync(0xffffffffu, finite) && lane == 0) set_status(status, MOE_ERR_NONFINITE);
 
-        // top-k: k rounds of (local best, warp arg-max with index tie-break)
-        float vmax = 0.f;
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
+        // clean scores: softmax over all experts (max-subtracted) or element-wise sigmoid
+        float lmax = v[0];
 #pragma unroll
-            for (int m = 0; m < EPL; ++m) {
-                const int e = m * 32 + lane;
-                if (!((taken >> m) & 1u) && ahead(v[m], e, bv, bi)) {
-                    bv = v[m];
-                    bi = e;
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (ahead(ov, oi, bv, bi)) {
-                    bv = ov;
-                    bi = oi;
-                }
-            }
-            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-            if (j == 0) vmax = bv;
-            if (lane == 0) {
-                selv[j] = bv;
-                selected[t * k + j] = bi;
-                atomicAdd(&s_counts[bi], 1);
-            }
-        }
-        __syncwarp();
-
-        // softmax over all experts (max-subtracted), accumulated per expert
+        for (int m = 1; m < EPL; ++m) lmax = fmaxf(lmax, v[m]);
+        const float smax = warp_max(lmax);
         float part = 0.f;
         float ex[EPL];
 #pragma unroll
         for (int m = 0; m < EPL; ++m) {
             const int e = m * 32 + lane;
-            ex[m] = e < E ? expf(v[m] - vmax) : 0.f;
+            ex[m] = e < E ? expf(v[m] - smax) : 0.f;
             part += ex[m];
         }
-        const float inv = 1.0f / warp_sum(part);
+        const float sum_exp = warp_sum(part);
+        const float inv = 1.0f / sum_exp;
+        float clean[EPL];
 #pragma unroll
-        for (int m = 0; m < EPL; ++m) psum[m] += ex[m] * inv;
+        for (int m = 0; m < EPL; ++m) {
+            const int e = m * 32 + lane;
+            clean[m] = e < E ? (scoring == 0 ? ex[m] * inv : sigmoid_stable_f(v[m])) : 0.f;
+            psum[m] += clean[m];
+        }
+        if (part_z) {
+            const float lse = smax + logf(sum_exp);
+            zacc += lse * lse;
+        }
 
-        // renormalised gates = softmax over the selected scores
+        // top-k: k rounds of (lane-local best key, warp max of keys, lowest
+        // index holding that key).  Keys preserve the float order exactly, so
+        // equal scores tie and the index decides.  The key is the logit, or the
+        // clean score plus the selection bias when one is given.
+        uint32_t key[EPL];
+#pragma unroll
+        for (int m = 0; m < EPL; ++m) {
+            const int e = m * 32 + lane;
+            key[m] = (e < E) ? order_key(sel_bias ? clean[m] + sbias_r[m] : v[m]) : 0u;
+        }
+        for (int j = 0; j < k; ++j) {
+            uint32_t lk = 0;  // below every finite or infinite key
+            uint32_t li = 0xffffffffu;
+            float lv = 0.f;
+#pragma unroll
+            for (int m = 0; m < EPL; ++m) {
+                const bool live = !((taken >> m) & 1u);
+                if (live && key[m] > lk) {  // ascending m: the first of equal keys keeps the lowest index
+                    lk = key[m];
+                    li = (uint32_t)(m * 32 + lane);
+                    lv = v[m];
+                }
+            }
+            const uint32_t gk = __reduce_max_sync(0xffffffffu, lk);
+            const uint32_t bi = __reduce_min_sync(0xffffffffu, lk == gk ? li : 0xffffffffu);
+            if ((int)(bi & 31u) == lane) {
+                taken |= 1u << (bi >> 5);
+                selv[j] = lv;  // the winner's raw logit
+                selected[t * k + j] = (int64_t)bi;
+                atomicAdd(&s_counts[bi], 1);
+            }
+        }
+        __syncwarp();
+
+        // gates: softmax of the selected logits, or of their log-sigmoids
+        float wmax = -INFINITY;
+        for (int j = lane; j < k; j += 32) wmax = fmaxf(wmax, scoring == 0 ? selv[j] : log_sigmoid_f(selv[j]));
+        wmax = warp_max(wmax);
         float gp = 0.f;
-        for (int j = lane; j < k; j += 32) gp += expf(selv[j] - vmax);
+        for (int j = lane; j < k; j += 32) gp += expf((scoring == 0 ? selv[j] : log_sigmoid_f(selv[j])) - wmax);
         const float ginv = 1.0f / warp_sum(gp);
         for (int j = lane; j < k; j += 32) {
-            const float g = expf(selv[j] - vmax) * ginv;
+            const float g = expf((scoring == 0 ? selv[j] : log_sigmoid_f(selv[j])) - wmax) * ginv;
             if (gates_f32) gates_f32[t * k + j] = g;
             if (gates_out) {
                 if (gates_bf16) reinterpret_cast<__nv_bfloat16*>(gates_out)[t * k + j] = __float2bfloat16_rn(g);
@@ -150,7 +193,13 @@ __global__ void __launch_bounds__(kRouteThreads)
         const int e = m * 32 + lane;
         if (e < E) s_psum[warp * E + e] = psum[m];
     }
+    if (lane == 0) s_z[warp] = zacc;
     __syncthreads();
+    if (part_z && threadIdx.x == 0) {
+        float z = 0.f;
+        for (int w = 0; w < kRouteWarps; ++w) z += s_z[w];
+        part_z[blockIdx.x] = z;
+    }
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         float s = 0.f;
         for (int w = 0; w < kRouteWarps; ++w) s += s_psum[w * E + e];
@@ -159,25 +208,56 @@ __global__ void __launch_bounds__(kRouteThreads)
     }
 }
 
-// counts[e] and prob_sum[e] = fixed-order sums of the block partials.
-__global__ void route_reduce_kernel(const int32_t* __restrict__ part_counts, const float* __restrict__ part_psum,
-                                    int nblocks, int E, int32_t* __restrict__ counts, float* __restrict__ prob_sum) {
-    const int e = blockIdx.x * blockDim.x + threadIdx.x;
-    if (e >= E) return;
+// counts[e] and prob_sum[e] = fixed-order sums of the block partials.  A block
+// owns 32 consecutive experts (coalesced loads across experts); its 32 warps
+// each add every 32nd partial row in ascending order, then warp 0 adds the 32
+// warp sums in order.  The order depends only on the partial count, so the
+// result is bitwise reproducible.
+constexpr int kReduceWarps = 32;
+
+__global__ void __launch_bounds__(kReduceWarps * 32)
+    route_reduce_kernel(const int32_t* __restrict__ part_counts, const float* __restrict__ part_psum, int nblocks,
+                        int E, int32_t* __restrict__ counts, float* __restrict__ prob_sum,
+                        const float* __restrict__ part_z, int64_t T, float* __restrict__ z_loss) {
+    __shared__ float s_p[kReduceWarps][32];
+    __shared__ int s_c[kReduceWarps][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 32 + lane;
     int c = 0;
     float s = 0.f;
-    for (int b = 0; b < nblocks; ++b) {
-        c += part_counts[(int64_t)b * E + e];
-        s += part_psum[(int64_t)b * E + e];
+    if (e < E) {
+#pragma unroll 8
+        for (int b = warp; b < nblocks; b += kReduceWarps) {
+            c += part_counts[(int64_t)b * E + e];
+            s += part_psum[(int64_t)b * E + e];
+        }
     }
-    counts[e] = c;
-    prob_sum[e] = s;
+    s_p[warp][lane] = s;
+    s_c[warp][lane] = c;
+    __syncthreads();
+    if (warp == 0 && e < E) {
+        float ts = 0.f;
+        int tc = 0;
+        for (int w = 0; w < kReduceWarps; ++w) {
+            ts += s_p[w][lane];
+            tc += s_c[w][lane];
+        }
+        counts[e] = tc;
+        prob_sum[e] = ts;
+    }
+    // router z-loss: the block partials in ascending order, divided by T
+    if (part_z && blockIdx.x == 0 && threadIdx.x == 0) {
+        float z = 0.f;
+        for (int b = 0; b < nblocks; ++b) z += part_z[b];
+        *z_loss = z / (float)T;
+    }
 }
 
 template <typename InT>
 int launch_topk(int epl, const InT* logits, int64_t ld, int64_t T, int E, int k, const float* bias,
                 float* logits_out, int64_t* selected, void* gates, int gates_bf16, float* gates_f32,
-                int32_t* part_counts, float* part_psum, int32_t* status, cudaStream_t stream) {
+                int32_t* part_counts, float* part_psum, int scoring, const float* sel_bias, float* part_z,
+                int32_t* status, cudaStream_t stream) {
     const int nb = route_blocks(T);
     const size_t smem = sizeof(float) * (size_t)kRouteWarps * E + sizeof(int) * (size_t)E +
                         sizeof(float) * (size_t)kRouteWarps * k;
@@ -187,7 +267,8 @@ int launch_topk(int epl, const InT* logits, int64_t ld, int64_t T, int E, int k,
         if (smem > 48 * 1024)                                                                                 \
             MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); \
         kern<<<nb, kRouteThreads, smem, stream>>>(logits, ld, T, E, k, bias, logits_out, selected, gates,     \
-                                                  gates_bf16, gates_f32, part_counts, part_psum, status);     \
+                                                  gates_bf16, gates_f32, part_counts, part_psum, scoring,     \
+                                                  sel_bias, part_z, status);                                  \
         break;                                                                                                \
     }
     switch (epl) {
@@ -210,7 +291,7 @@ int epl_for(int E) {
 }
 
 struct RouteWs {
-    size_t logits_off, wt_off, pc_off, pp_off, total;
+    size_t logits_off, wt_off, pc_off, pp_off, pz_off, total;
 };
 
 RouteWs route_ws_layout(int64_t T, int64_t D, int32_t E, moe_dtype dtype, int has_w, moe_router_layout layout) {
@@ -225,6 +306,8 @@ RouteWs route_ws_layout(int64_t T, int64_t D, int32_t E, moe_dtype dtype, int ha
     off += align_up((size_t)nb * E * sizeof(int32_t), 256);
     w.pp_off = off;
     off += align_up((size_t)nb * E * sizeof(float), 256);
+    w.pz_off = off;
+    off += align_up((size_t)nb * sizeof(float), 256);
     w.total = off;
     return w;
 }
@@ -240,16 +323,19 @@ extern "C" size_t moe_route_workspace_size(int64_t T, int64_t D, int32_t E, moe_
     return route_ws_layout(T, D, E, dtype, has_router_weight, layout).total;
 }
 
-extern "C" int moe_route(const void* x, moe_dtype dtype, int64_t T, int64_t D, int64_t ldx, const void* w_router,
-                         moe_router_layout layout, int32_t E, const float* logit_bias, int32_t k, float* logits_out,
-                         int64_t* selected, void* gates, float* gates_f32, int32_t* counts, float* prob_sum,
-                         int32_t* dev_status, void* workspace, size_t workspace_bytes, moe_stream_t stream_) {
+extern "C" int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D, int64_t ldx,
+                            const void* w_router, moe_router_layout layout, int32_t E, const float* logit_bias,
+                            int32_t k, moe_scoring scoring, const float* selection_bias, float* logits_out,
+                            int64_t* selected, void* gates, float* gates_f32, int32_t* counts, float* prob_sum,
+                            float* z_loss, int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                            moe_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     MOE_REQUIRE(valid_dtype(dtype), MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(x && selected && counts && prob_sum, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(T >= 1 && E >= 1 && k >= 1 && k <= E, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(E <= kMaxE && k <= kMaxK, MOE_ERR_UNSUPPORTED);
     MOE_REQUIRE(layout == MOE_ROUTER_DE || layout == MOE_ROUTER_ED, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(scoring == MOE_SCORE_SOFTMAX || scoring == MOE_SCORE_SIGMOID, MOE_ERR_INVALID_ARG);
     const int has_w = w_router != nullptr;
     if (has_w) MOE_REQUIRE(D >= 1 && ldx >= D, MOE_ERR_INVALID_ARG);
     else MOE_REQUIRE(ldx >= E, MOE_ERR_INVALID_ARG);
@@ -258,6 +344,8 @@ extern "C" int moe_route(const void* x, moe_dtype dtype, int64_t T, int64_t D, i
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int32_t* part_counts = reinterpret_cast<int32_t*>(ws + wl.pc_off);
     float* part_psum = reinterpret_cast<float*>(ws + wl.pp_off);
+    float* part_z = z_loss ? reinterpret_cast<float*>(ws + wl.pz_off) : nullptr;
+    const int sc = scoring == MOE_SCORE_SIGMOID ? 1 : 0;
     const int epl = epl_for(E);
     const int gates_bf16 = dtype == MOE_BF16;
     int rc = MOE_OK;
@@ -273,29 +361,27 @@ extern "C" int moe_route(const void* x, moe_dtype dtype, int64_t T, int64_t D, i
                 if (rc != MOE_OK) return rc;
                 w_ed = wt;
             }
-            TcGemmProblem p{};
-            p.a = x;
-            p.lda = ldx;
-            p.a_rows_total = T;
-            p.a_rows_per_group = 0;
-            p.b = w_ed;
-            p.b2 = nullptr;
-            p.ldb = D;
-            p.b_rows_total = E;
-            p.b_rows_per_group = 0;
+            TcxProblem p{};
+            p.w = w_ed;  // experts are the output features
+            p.ldw = D;
+            p.w_rows_total = E;
+            p.w_rows_per_group = 0;
+            p.x = x;
+            p.ldx = ldx;
+            p.x_rows_total = T;
+            p.x_rows_per_group = 0;
             p.G = 1;
-            p.M = T;
-            p.N = E;
+            p.features = E;
+            p.max_tokens = T;
             p.K = D;
             p.rows = nullptr;
             p.out = lg;
             p.ldo = E;
             p.out_rows_per_group = 0;
             p.bias = logit_bias;
-            p.bias_group_stride = 0;
             p.epilogue = TC_EPI_F32;
             p.status = dev_status;
-            rc = tc_gemm_run(p, stream);
+            rc = tcx_gemm_run(p, stream);
         } else {
             SimtGemm g{};
             g.A = static_cast<const float*>(x);
@@ -317,18 +403,57 @@ extern "C" int moe_route(const void* x, moe_dtype dtype, int64_t T, int64_t D, i
         }
         if (rc != MOE_OK) return rc;
         rc = launch_topk<float>(epl, lg, E, T, E, k, nullptr, nullptr, selected, gates, gates_bf16, gates_f32,
-                                part_counts, part_psum, dev_status, stream);
+                                part_counts, part_psum, sc, selection_bias, part_z, dev_status, stream);
     } else if (dtype == MOE_BF16) {
         rc = launch_topk<__nv_bfloat16>(epl, static_cast<const __nv_bfloat16*>(x), ldx, T, E, k, logit_bias,
                                         logits_out, selected, gates, gates_bf16, gates_f32, part_counts, part_psum,
-                                        dev_status, stream);
+                                        sc, selection_bias, part_z, dev_status, stream);
     } else {
         rc = launch_topk<float>(epl, static_cast<const float*>(x), ldx, T, E, k, logit_bias, logits_out, selected,
-                                gates, gates_bf16, gates_f32, part_counts, part_psum, dev_status, stream);
+                                gates, gates_bf16, gates_f32, part_counts, part_psum, sc, selection_bias, part_z,
+                                dev_status, stream);
     }
     if (rc != MOE_OK) return rc;
     const int nb = route_blocks(T);
-    route_reduce_kernel<<<(E + 255) / 256, 256, 0, stream>>>(part_counts, part_psum, nb, E, counts, prob_sum);
+    route_reduce_kernel<<<(E + 31) / 32, kReduceWarps * 32, 0, stream>>>(part_counts, part_psum, nb, E, counts,
+                                                                         prob_sum, part_z, T, z_loss);
+    return launch_status();
+}
+
+extern "C" int moe_route(const void* x, moe_dtype dtype, int64_t T, int64_t D, int64_t ldx, const void* w_router,
+                         moe_router_layout layout, int32_t E, const float* logit_bias, int32_t k, float* logits_out,
+                         int64_t* selected, void* gates, float* gates_f32, int32_t* counts, float* prob_sum,
+                         int32_t* dev_status, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+    return moe_route_ex(x, dtype, T, D, ldx, w_router, layout, E, logit_bias, k, MOE_SCORE_SOFTMAX, nullptr,
+                        logits_out, selected, gates, gates_f32, counts, prob_sum, nullptr, dev_status, workspace,
+                        workspace_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// moe_renormalize_kept_gates
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+__global__ void renormalize_kernel(const float* __restrict__ gates, const int64_t* __restrict__ slot, int64_t T,
+                                   int k, float* __restrict__ out) {
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    float mass = 0.f;
+    for (int j = 0; j < k; ++j)
+        if (slot[t * k + j] >= 0) mass += gates[t * k + j];
+    const float inv = mass > 0.f ? 1.0f / mass : 0.f;
+    for (int j = 0; j < k; ++j) out[t * k + j] = slot[t * k + j] >= 0 ? gates[t * k + j] * inv : 0.f;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_renormalize_kept_gates(const float* gates_f32, const int64_t* slot, int64_t T, int32_t k,
+                                          float* out, moe_stream_t stream) {
+    MOE_REQUIRE(gates_f32 && slot && out && T >= 1 && k >= 1, MOE_ERR_INVALID_ARG);
+    renormalize_kernel<<<(unsigned)((T + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        gates_f32, slot, T, k, out);
     return launch_status();
 }
 

@@ -1,0 +1,39 @@
+// Grouped bf16 tensor-core GEMM with weights on the M side (see tc_expert_gemm.cu).
+#pragma once
+
+#include <stdint.h>
+
+#include "common.cuh"
+#include "tc_gemm.cuh"
+
+namespace moe {
+
+struct TcxProblem {
+    const void* w;             // bf16 weights (w_rows_total, K), row stride ldw: row g*w_rows_per_group + f
+    const void* w2;            // second weight matrix for TC_EPI_SWIGLU (the up projection), else NULL
+    int64_t ldw;
+    int64_t w_rows_total;
+    int64_t w_rows_per_group;
+    const void* x;             // bf16 tokens (x_rows_total, K), row stride ldx: row g*x_rows_per_group + n
+    int64_t ldx;
+    int64_t x_rows_total;
+    int64_t x_rows_per_group;
+    int G;                     // groups (experts)
+    int64_t features;          // output features per group
+    int64_t max_tokens;        // token rows per group (C)
+    int64_t K;
+    const int32_t* rows;       // device (G) valid token rows per group, or NULL (= max_tokens)
+    void* out;                 // (G*out_rows_per_group, ldo): fp32 for TC_EPI_F32, else bf16
+    int64_t ldo;
+    int64_t out_rows_per_group;
+    const void* bias;          // per feature: fp32 (TC_EPI_F32, shared by groups) or bf16 (+ g*bias_group_stride)
+    int64_t bias_group_stride;
+    int epilogue;              // TcEpilogue
+    int32_t* status;
+};
+
+// Single-CTA kernel: 256 weight rows x up to 128 tokens per tile.
+int tcx_gemm_run(const TcxProblem& p, cudaStream_t stream);
+
+
+}  // namespace moe

@@ -50,4 +50,8 @@ struct TcGemmProblem {
 // Validates alignment, encodes the tensor maps and launches.  Returns a moe_status.
 int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream);
 
+// 2-D bf16 TMA map over a (rows, inner) row-major matrix with row stride
+// ld_elems: box = box_rows x 64 elements, 128-byte swizzle, zero fill outside.
+bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld_elems, int box_rows);
+
 }  // namespace moe
