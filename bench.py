@@ -248,7 +248,17 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     ffn_ev = []
 
+    side = torch.cuda.Stream(device=dev)
+    ev_x, ev_shared = torch.cuda.Event(), torch.cuda.Event()
+
     def step(x):
+        # shared expert on a second stream, overlapping the routing chain (as SwiGLUMoE.forward does)
+        ev_x.record(stream)
+        side.wait_event(ev_x)
+        moe.moe_expert_ffn("swiglu", x.view(1, T, H), None, dv["s_gate"], w2=dv["s_down"], w3=dv["s_up"],
+                           ybuf=layer.shared.view(1, T, H), dev_status=layer.status, workspace=layer.ws_shared,
+                           stream=side)
+        ev_shared.record(side)
         r = moe.moe_route(x, k, w_router=dv["w_router"], layout="ED", logit_bias=dv["router_bias"],
                           out=layer.route_out, dev_status=layer.status, workspace=layer.ws_route)
         d = moe.moe_dispatch(r["selected"], E, layer.C, x=x, out=layer.disp_out, dev_status=layer.status,
@@ -259,8 +269,7 @@ def run_ours(args, world, rank, local):
                            ybuf=layer.ybuf, dev_status=layer.status, workspace=layer.ws_ffn)
         e1.record(stream)
         ffn_ev.append((e0, e1))
-        moe.moe_expert_ffn("swiglu", x.view(1, T, H), None, dv["s_gate"], w2=dv["s_down"], w3=dv["s_up"],
-                           ybuf=layer.shared.view(1, T, H), dev_status=layer.status, workspace=layer.ws_shared)
+        stream.wait_event(ev_shared)
         y = moe.moe_combine(layer.ybuf, r["selected"], d["slot"], r["gates_f32"], base_kind="tensor",
                             base=layer.shared, y=layer.y, dev_status=layer.status)
         f, P, aux = moe.moe_aux_stats(r["counts"], r["prob_sum"], T, k, True, cfg["aux_coef"],

@@ -50,16 +50,16 @@ __device__ __forceinline__ float log_sigmoid_f(float z) {
     return z >= 0.f ? -log1pf(expf(-z)) : z - log1pf(expf(z));
 }
 
-// scoring: 0 softmax, 1 sigmoid.  sel_bias (E) or NULL: added to the clean
-// scores for the selection only.  part_z (gridDim) or NULL: per-block sums of
-// logsumexp(s_t)^2 for the router z-loss.
-template <int EPL, typename InT>
+// SC: 0 softmax, 1 sigmoid clean scores.  SB: a selection bias is given
+// (sel_bias (E), added to the clean scores for the selection only).  part_z
+// (gridDim) or NULL: per-block sums of logsumexp(s_t)^2 for the router z-loss.
+template <int EPL, typename InT, int SC, bool SB>
 __global__ void __launch_bounds__(kRouteThreads)
     route_topk_kernel(const InT* __restrict__ logits, int64_t ld, int64_t T, int E, int k,
                       const float* __restrict__ bias, float* __restrict__ logits_out,
                       int64_t* __restrict__ selected, void* __restrict__ gates_out, int gates_bf16,
                       float* __restrict__ gates_f32, int32_t* __restrict__ part_counts,
-                      float* __restrict__ part_psum, int scoring, const float* __restrict__ sel_bias,
+                      float* __restrict__ part_psum, const float* __restrict__ sel_bias,
                       float* __restrict__ part_z, int32_t* status) {
     extern __shared__ float s_dyn[];
     float* s_psum = s_dyn;                                            // [kRouteWarps][E]
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kRouteThreads)
     for (int m = 0; m < EPL; ++m) {
         const int e = m * 32 + lane;
         bias_r[m] = (bias && e < E) ? bias[e] : 0.f;
-        sbias_r[m] = (sel_bias && e < E) ? sel_bias[e] : 0.f;
+        sbias_r[m] = (SB && e < E) ? sel_bias[e] : 0.f;
         psum[m] = 0.f;
     }
     float* selv = s_selv + warp * k;
@@ -127,7 +127,8 @@ __global__ void __launch_bounds__(kRouteThreads)
 #pragma unroll
         for (int m = 0; m < EPL; ++m) {
             const int e = m * 32 + lane;
-            clean[m] = e < E ? (scoring == 0 ? ex[m] * inv : sigmoid_stable_f(v[m])) : 0.f;
+            if (SC == 0) clean[m] = e < E ? ex[m] * inv : 0.f;
+            else clean[m] = e < E ? sigmoid_stable_f(v[m]) : 0.f;
             psum[m] += clean[m];
         }
         if (part_z) {
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(kRouteThreads)
 #pragma unroll
         for (int m = 0; m < EPL; ++m) {
             const int e = m * 32 + lane;
-            key[m] = (e < E) ? order_key(sel_bias ? clean[m] + sbias_r[m] : v[m]) : 0u;
+            key[m] = (e < E) ? order_key(SB ? clean[m] + sbias_r[m] : v[m]) : 0u;
         }
         for (int j = 0; j < k; ++j) {
             uint32_t lk = 0;  // below every finite or infinite key
@@ -169,15 +170,17 @@ __global__ void __launch_bounds__(kRouteThreads)
         }
         __syncwarp();
 
-        // gates: softmax of the selected logits, or of their log-sigmoids
-        float wmax = -INFINITY;
-        for (int j = lane; j < k; j += 32) wmax = fmaxf(wmax, scoring == 0 ? selv[j] : log_sigmoid_f(selv[j]));
-        wmax = warp_max(wmax);
-        float gp = 0.f;
-        for (int j = lane; j < k; j += 32) gp += expf((scoring == 0 ? selv[j] : log_sigmoid_f(selv[j])) - wmax);
-        const float ginv = 1.0f / warp_sum(gp);
+        // gates: softmax of the selected logits, or of their log-sigmoids (k <= 64:
+        // each lane owns j = lane and j = lane + 32)
+        float w0 = -INFINITY, w1 = -INFINITY;
+        if (lane < k) w0 = SC == 0 ? selv[lane] : log_sigmoid_f(selv[lane]);
+        if (lane + 32 < k) w1 = SC == 0 ? selv[lane + 32] : log_sigmoid_f(selv[lane + 32]);
+        const float wmax = warp_max(fmaxf(w0, w1));
+        const float e0 = lane < k ? expf(w0 - wmax) : 0.f;
+        const float e1 = lane + 32 < k ? expf(w1 - wmax) : 0.f;
+        const float ginv = 1.0f / warp_sum(e0 + e1);
         for (int j = lane; j < k; j += 32) {
-            const float g = expf((scoring == 0 ? selv[j] : log_sigmoid_f(selv[j])) - wmax) * ginv;
+            const float g = (j == lane ? e0 : e1) * ginv;
             if (gates_f32) gates_f32[t * k + j] = g;
             if (gates_out) {
                 if (gates_bf16) reinterpret_cast<__nv_bfloat16*>(gates_out)[t * k + j] = __float2bfloat16_rn(g);
@@ -263,12 +266,13 @@ int launch_topk(int epl, const InT* logits, int64_t ld, int64_t T, int E, int k,
                         sizeof(float) * (size_t)kRouteWarps * k;
 #define MOE_TOPK_CASE(N)                                                                                      \
     case N: {                                                                                                 \
-        auto kern = route_topk_kernel<N, InT>;                                                                \
+        auto kern = scoring == 0 ? (sel_bias ? route_topk_kernel<N, InT, 0, true> : route_topk_kernel<N, InT, 0, false>) \
+                                 : (sel_bias ? route_topk_kernel<N, InT, 1, true> : route_topk_kernel<N, InT, 1, false>); \
         if (smem > 48 * 1024)                                                                                 \
             MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)); \
         kern<<<nb, kRouteThreads, smem, stream>>>(logits, ld, T, E, k, bias, logits_out, selected, gates,     \
-                                                  gates_bf16, gates_f32, part_counts, part_psum, scoring,     \
-                                                  sel_bias, part_z, status);                                  \
+                                                  gates_bf16, gates_f32, part_counts, part_psum, sel_bias,    \
+                                                  part_z, status);                                            \
         break;                                                                                                \
     }
     switch (epl) {

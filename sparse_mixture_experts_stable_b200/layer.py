@@ -52,21 +52,36 @@ class SwiGLUMoE:
                                   dtype=torch.uint8, device=dev)
         self.ws_shared = (torch.empty(max(B.moe_expert_ffn_workspace_size("swiglu", dt, 1, T, F_shared), 256),
                                       dtype=torch.uint8, device=dev) if F_shared else None)
+        self.side = None  # stream for the shared expert, created on first use
 
     def forward(self, x, w_router, router_bias, w_gate, w_up, w_down, s_gate=None, s_up=None, s_down=None):
-        """x (T,H); w_router (E,H); w_gate/w_up (E,F,H); w_down (E,H,F); shared (1,F_s,H)/(1,H,F_s)."""
+        """x (T,H); w_router (E,H); w_gate/w_up (E,F,H); w_down (E,H,F); shared (1,F_s,H)/(1,H,F_s).
+
+        The shared expert only needs x, so it runs on a second stream while the
+        router, the slot scan and the gather (short, latency- and memory-bound
+        kernels) run on the current one; the combine waits for both.
+        """
+        main = torch.cuda.current_stream(x.device)
+        base_kind, base = "zero", None
+        if self.F_shared:
+            if self.side is None:
+                self.side = torch.cuda.Stream(device=x.device)
+                self.ev_x, self.ev_shared = torch.cuda.Event(), torch.cuda.Event()
+            self.ev_x.record(main)
+            self.side.wait_event(self.ev_x)
+            B.moe_expert_ffn("swiglu", x.view(1, self.T, self.H), None, s_gate, w2=s_down, w3=s_up,
+                             ybuf=self.shared.view(1, self.T, self.H), dev_status=self.status,
+                             workspace=self.ws_shared, stream=self.side)
+            self.ev_shared.record(self.side)
+            base_kind, base = "tensor", self.shared
         r = B.moe_route(x, self.k, w_router=w_router, layout="ED", logit_bias=router_bias, out=self.route_out,
                         dev_status=self.status, workspace=self.ws_route)
         d = B.moe_dispatch(r["selected"], self.E, self.C, x=x, out=self.disp_out, dev_status=self.status,
                            workspace=self.ws_disp)
         B.moe_expert_ffn("swiglu", d["xbuf"], d["used"], w_gate, w2=w_down, w3=w_up, ybuf=self.ybuf,
                          dev_status=self.status, workspace=self.ws_ffn)
-        base_kind, base = "zero", None
         if self.F_shared:
-            B.moe_expert_ffn("swiglu", x.view(1, self.T, self.H), None, s_gate, w2=s_down, w3=s_up,
-                             ybuf=self.shared.view(1, self.T, self.H), dev_status=self.status,
-                             workspace=self.ws_shared)
-            base_kind, base = "tensor", self.shared
+            main.wait_event(self.ev_shared)
         B.moe_combine(self.ybuf, r["selected"], d["slot"], r["gates_f32"], base_kind=base_kind, base=base, y=self.y,
                       dev_status=self.status)
         f, P, aux = B.moe_aux_stats(r["counts"], r["prob_sum"], self.T, self.k, True, self.aux_coef,
