@@ -38,6 +38,13 @@ UNIT = "tokens/s"
 WORKLOAD = dict(workload="full_layer_bf16", T=16384, hidden=2048, experts=256, top_k=8, expert_intermediate=512,
                 shared_experts=1, shared_intermediate=512, capacity_factor=1.25, capacity=640, aux_coef=0.001)
 KERNELS_PER_STEP = 11  # router GEMM, top-k, reduce, scan, gather, 2 routed GEMMs, 2 shared GEMMs, combine, aux
+# DRAM bytes (read + write) per algorithmic byte of the two routed expert-FFN
+# launches, from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum
+# on the same kernels at T = 4096, E = 64 (profiles/expert_gemm_dram_traffic_T4096_E64.md).
+# Both operands and outputs scale with E and the kept rows, so the full-size
+# traffic is these ratios times the full-size algorithmic bytes.
+TRAFFIC_PER_ALG_BYTE = {"gate_up": 1.017, "down": 0.857}
+TRAFFIC_SOURCE = "ncu DRAM bytes at T=4096, E=64, scaled by algorithmic bytes"
 
 
 def measured_peaks():
@@ -313,8 +320,12 @@ def run_ours(args, world, rank, local):
     ffn_avg_s = statistics.mean(ffn_ms) / 1e3
     pk = measured_peaks()
     achieved = flops / ffn_avg_s / 1e12
-    roof = dict(bound="tensor", kernel="tcx_kernel: routed SwiGLU gate/up + down launches", achieved=achieved,
-                peak=pk["bf16_sustained"], unit="TFLOP/s", frac=achieved / pk["bf16_sustained"], traffic=None,
+    alg_gate_up = E * 2 * F * H * 2 + kept * H * 2 + kept * F * 2
+    alg_down = E * H * F * 2 + kept * F * 2 + kept * H * 2
+    traffic = (TRAFFIC_PER_ALG_BYTE["gate_up"] * alg_gate_up + TRAFFIC_PER_ALG_BYTE["down"] * alg_down)
+    roof = dict(bound="tensor", kernel="routed expert FFN: tcx_kernel<SWIGLU> gate/up + tc_gemm_kernel<BF16> down",
+                achieved=achieved, peak=pk["bf16_sustained"], unit="TFLOP/s", frac=achieved / pk["bf16_sustained"],
+                traffic=traffic, traffic_source=TRAFFIC_SOURCE, bytes_alg=alg_gate_up + alg_down,
                 peak_source=f"{pk['source']} bf16 sustained", frac_of_burst=achieved / pk["bf16"],
                 flops_per_launch=flops, kept_rows=kept, avg_launch_ms=1e3 * ffn_avg_s)
 
