@@ -10,6 +10,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "route_scores.cuh"
 #include "simt_gemm.cuh"
 #include "tc_expert_gemm.cuh"
 #include "util_kernels.cuh"
@@ -26,28 +27,6 @@ constexpr int kMaxE = 1024;
 int route_blocks(int64_t T) {
     int64_t b = (T + kRouteWarps - 1) / kRouteWarps;
     return (int)(b < kMaxRouteBlocks ? b : kMaxRouteBlocks);
-}
-
-// Order-preserving map from fp32 to uint32 (larger float -> larger key).  The
-// score is canonicalised first so that -0 and +0 (equal as floats) share a key;
-// NaN never reaches it (non-finite scores are replaced by -inf before).
-__device__ __forceinline__ uint32_t order_key(float v) {
-    if (v == 0.0f) v = 0.0f;
-    const uint32_t b = __float_as_uint(v);
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-__device__ __forceinline__ float key_value(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-// Each lane holds experts e = m*32 + lane, m < EPL.
-__device__ __forceinline__ float sigmoid_stable_f(float z) {
-    if (z >= 0.f) return 1.f / (1.f + expf(-z));
-    const float ez = expf(z);
-    return ez / (1.f + ez);
-}
-__device__ __forceinline__ float log_sigmoid_f(float z) {
-    return z >= 0.f ? -log1pf(expf(-z)) : z - log1pf(expf(z));
 }
 
 // SC: 0 softmax, 1 sigmoid clean scores.  SB: a selection bias is given

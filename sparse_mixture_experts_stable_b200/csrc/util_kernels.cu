@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 // in shared memory first, so the row loops below contain no warp shuffles and
 // may diverge freely over ragged row lengths.
 constexpr int kMaxKCombine = 64;
+constexpr int kCombineBatch = 8;  // row loads issued before the first add
 
 template <typename T, typename G, bool VEC>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
@@ -121,25 +122,36 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
     if (t >= Ttok) return;
-    // compact the kept, in-range assignments in ascending j (lane 0 keeps the order)
-    if (lane == 0) {
-        int n = 0;
-        bool bad = false;
-        for (int j = 0; j < k; ++j) {
+    // compact the kept, in-range assignments in ascending j: lanes read 32
+    // assignments at a time and a ballot gives each kept one its position
+    int nk = 0;
+    for (int j0 = 0; j0 < k; j0 += 32) {
+        const int j = j0 + lane;
+        bool keep = false;
+        int64_t row = 0;
+        float g = 1.f;
+        if (j < k) {
             const int64_t s = slot[t * k + j];
-            if (s < 0) continue;
-            const int64_t e = selected[t * k + j];
-            if (e < 0 || e >= E || s >= C) {
-                bad = true;
-                continue;
+            if (s >= 0) {
+                const int64_t e = selected[t * k + j];
+                if (e < 0 || e >= E || s >= C) {
+                    set_status(status, MOE_ERR_BAD_INDEX);
+                } else {
+                    keep = true;
+                    row = (e * C + s) * N;
+                    if (gates) g = to_f32(gates[t * k + j]);
+                }
             }
-            s_row[warp][n] = (e * C + s) * N;
-            s_gate[warp][n] = gates ? to_f32(gates[t * k + j]) : 1.f;
-            ++n;
         }
-        s_n[warp] = n;
-        if (bad) set_status(status, MOE_ERR_BAD_INDEX);
+        const uint32_t m = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+            const int pos = nk + __popc(m & lanemask_lt());
+            s_row[warp][pos] = row;
+            s_gate[warp][pos] = g;
+        }
+        nk += __popc(m);
     }
+    if (lane == 0) s_n[warp] = nk;
     __syncwarp();
     const int n_terms = s_n[warp];
     const int64_t* rows = s_row[warp];
@@ -160,12 +172,21 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 #pragma unroll
                 for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
             }
-            for (int j = 0; j < n_terms; ++j) {
-                const float g = gs[j];
-                const uint4 r = reinterpret_cast<const uint4*>(ybuf + rows[j])[v];
-                const T* rv = reinterpret_cast<const T*>(&r);
+            // up to kCombineBatch rows in flight per lane, added in ascending j
+            for (int j0 = 0; j0 < n_terms; j0 += kCombineBatch) {
+                uint4 r[kCombineBatch];
 #pragma unroll
-                for (int i = 0; i < EPV; ++i) acc[i] = fmaf(g, to_f32(rv[i]), acc[i]);
+                for (int u = 0; u < kCombineBatch; ++u)
+                    if (j0 + u < n_terms) r[u] = reinterpret_cast<const uint4*>(ybuf + rows[j0 + u])[v];
+#pragma unroll
+                for (int u = 0; u < kCombineBatch; ++u) {
+                    if (j0 + u < n_terms) {
+                        const float g = gs[j0 + u];
+                        const T* rv = reinterpret_cast<const T*>(&r[u]);
+#pragma unroll
+                        for (int i = 0; i < EPV; ++i) acc[i] = fmaf(g, to_f32(rv[i]), acc[i]);
+                    }
+                }
             }
             uint4 o;
             T* ov = reinterpret_cast<T*>(&o);

@@ -146,6 +146,19 @@ def full_layer_bf16(seed: int = 0, T: int = 16384, H: int = 2048, E: int = 256, 
                 s_gate=_bf16(s_gate[None]), s_up=_bf16(s_up[None]), s_down=_bf16(s_down[None]))
 
 
+def router_spread_bf16(seed: int = 0, T: int = 1500, D: int = 512, E: int = 64) -> dict:
+    """Router inputs with the full layer's score spread (std about 0.5 at D = 512).
+
+    Same recipe as the router part of full_layer_bf16: x = a/8, router weight
+    b * 2^-7 with a, b uniform in the integers [-8, 8], so every score is a
+    multiple of 2^-10 below 2^6 in magnitude for D <= 512 and exact in fp32.
+    """
+    rng = np.random.default_rng(seed)
+    x = rng.integers(-8, 9, size=(T, D)).astype(np.float32) / 8.0
+    w_router = rng.integers(-8, 9, size=(E, D)).astype(np.float32) / 128.0
+    return dict(name="router_spread_bf16", T=T, D=D, E=E, x=_bf16(x), w_router=_bf16(w_router))
+
+
 def fwd_bwd_fp32(seed: int = 0, T: int = 8192, D: int = 1024, E: int = 64, k: int = 2,
                  capacity_factor: float = 1.0) -> dict:
     """Forward + backward of a top-2 linear-expert layer with residual, fp32.
