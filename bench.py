@@ -320,9 +320,10 @@ def run_ours(args, world, rank, local):
     ffn_avg_s = statistics.mean(ffn_ms) / 1e3
     pk = measured_peaks()
     achieved = flops / ffn_avg_s / 1e12
-    alg_gate_up = E * 2 * F * H * 2 + kept * H * 2 + kept * F * 2
+    alg_gate_up = E * 2 * F * H * 2 + kept * H * 2 + kept * F * 2  # weights, gathered rows, h written
     alg_down = E * H * F * 2 + kept * F * 2 + kept * H * 2
-    traffic = (TRAFFIC_PER_ALG_BYTE["gate_up"] * alg_gate_up + TRAFFIC_PER_ALG_BYTE["down"] * alg_down)
+    traffic = (None if TRAFFIC_PER_ALG_BYTE is None else
+               TRAFFIC_PER_ALG_BYTE["gate_up"] * alg_gate_up + TRAFFIC_PER_ALG_BYTE["down"] * alg_down)
     roof = dict(bound="tensor", kernel="routed expert FFN: tcx_kernel<SWIGLU> gate/up + tc_gemm_kernel<BF16> down",
                 achieved=achieved, peak=pk["bf16_sustained"], unit="TFLOP/s", frac=achieved / pk["bf16_sustained"],
                 traffic=traffic, traffic_source=TRAFFIC_SOURCE, bytes_alg=alg_gate_up + alg_down,

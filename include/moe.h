@@ -297,6 +297,33 @@ MOE_API int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf,
                    moe_stream_t stream);
 
 /*
+ * moe_expert_ffn_gathered -- moe_expert_ffn (SwiGLU, bf16) reading each
+ * expert's rows straight from the token matrix through the dispatch's
+ * inverse map, without the expert-major copy:
+ *   ybuf[e,c,:] = Expert_e(x[token_of_slot[e,c], :])   for c < used[e]
+ * which equals moe_dispatch's gather into xbuf followed by moe_expert_ffn
+ * ([P4] steps 5 and 6 fused; [P3] swiglu_expert).  The gate/up kernel copies
+ * the token rows into the tensor-core tiles itself, so the (E, C, D) buffer
+ * is neither written nor read.
+ *
+ * Arguments:
+ *   kind, dtype   MOE_FFN_SWIGLU and MOE_BF16 only (else MOE_ERR_UNSUPPORTED).
+ *   x             device bf16 (T, D), row stride ldx (multiple of 8, 16-byte
+ *                 aligned base); D a multiple of 8.
+ *   token_of_slot device int32 (E, C) from moe_dispatch; an entry outside
+ *                 [0, T) for c < used[e] sets MOE_ERR_BAD_INDEX and reads a zero row.
+ *   used          device int32 (E) from moe_dispatch (required).
+ *   w1 = gate (E, F, D), w3 = up (E, F, D), w2 = down (E, Dout, F), bf16.
+ *   ybuf          device bf16 (E, C, Dout); rows c >= used[e] are not written.
+ *   workspace     device, >= moe_expert_ffn_workspace_size(MOE_FFN_SWIGLU, MOE_BF16, E, C, F).
+ */
+MOE_API int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const void* x, int64_t T, int64_t ldx,
+                                    const int32_t* token_of_slot, const int32_t* used, int32_t E, int64_t C,
+                                    int64_t D, int64_t F, int64_t Dout, const void* w1, const void* w2,
+                                    const void* w3, void* ybuf, int32_t* dev_status, void* workspace,
+                                    size_t workspace_bytes, moe_stream_t stream);
+
+/*
  * moe_combine -- gate-weighted combine back to token order.
  *   y[t,:] = base[t,:] + sum_{j : slot[t,j] >= 0} gate[t,j] * ybuf[e_{t,j}, slot[t,j], :]
  * ([P1] section 1 item 4: y = x + sum over kept; [P2] y = shared + sum;

@@ -37,7 +37,7 @@ EXPORTED = [
     "moe_dispatch_workspace_size", "moe_dispatch", "moe_expert_ffn_workspace_size", "moe_expert_ffn",
     "moe_combine", "moe_aux_stats", "moe_backward_workspace_size", "moe_backward", "moe_transpose_weights",
     "moe_clear_status", "moe_read_status", "moe_dispatch_static_max_state_bytes", "moe_dispatch_static",
-    "moe_route_ex", "moe_renormalize_kept_gates",
+    "moe_route_ex", "moe_renormalize_kept_gates", "moe_expert_ffn_gathered",
 ]
 SCORING = {"softmax": 0, "sigmoid": 1}
 
@@ -84,6 +84,8 @@ def lib():
         L.moe_expert_ffn_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, _i32, _i64, _i64]
         L.moe_expert_ffn.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _vp,
                                      _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_expert_ffn_gathered.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _i64, _i64, _vp, _vp, _i32, _i64,
+                                              _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
         L.moe_combine.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, _i64, _i32, _i32, _i64, _i64, ctypes.c_int,
                                   _vp, _i64, _vp, _i64, ctypes.c_int, _vp, _vp]
         L.moe_aux_stats.argtypes = [_vp, _vp, _i64, _i32, _i32, ctypes.c_int, _f32, _vp, _vp, ctypes.c_int, _vp,
@@ -313,6 +315,35 @@ def moe_expert_ffn(kind: str, xbuf: torch.Tensor, used: Optional[torch.Tensor], 
     rc = lib().moe_expert_ffn(FFN[kind], dt, _p(xbuf), _p(used), E, C, D, F, Dout, _p(w1), _p(b1), _p(w2), _p(b2),
                               _p(w3), _p(ybuf), _p(dev_status), _p(ws), ws.numel(), _stream(stream))
     _check("moe_expert_ffn", rc)
+    return ybuf
+
+
+def moe_expert_ffn_gathered(x: torch.Tensor, token_of_slot: torch.Tensor, used: torch.Tensor, w_gate: torch.Tensor,
+                            w_down: torch.Tensor, w_up: torch.Tensor, ybuf: Optional[torch.Tensor] = None,
+                            dev_status: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                            stream=None) -> torch.Tensor:
+    """SwiGLU experts on the rows token_of_slot picks from x (no expert-major copy of x), bf16.
+
+    x (T, D); token_of_slot (E, C) int32 and used (E) int32 from moe_dispatch;
+    w_gate/w_up (E, F, D), w_down (E, Dout, F).  Returns ybuf (E, C, Dout).
+    """
+    dev = _dev(x)
+    dt = _dt(x)
+    T, D = x.shape
+    E, C = token_of_slot.shape
+    F, Dout = w_gate.shape[1], w_down.shape[1]
+    for w in (w_gate, w_up, w_down):
+        if w.dtype != x.dtype or not w.is_contiguous():
+            raise TypeError("weights must be contiguous and share x's dtype")
+    if token_of_slot.dtype != torch.int32 or used.dtype != torch.int32:
+        raise TypeError("token_of_slot and used must be int32")
+    if ybuf is None:
+        ybuf = torch.empty(E, C, Dout, dtype=x.dtype, device=dev)
+    ws = _workspace(moe_expert_ffn_workspace_size("swiglu", dt, E, C, F), dev, workspace)
+    rc = lib().moe_expert_ffn_gathered(FFN["swiglu"], dt, _p(x), T, _rowstride(x), _p(token_of_slot.contiguous()),
+                                       _p(used), E, C, D, F, Dout, _p(w_gate), _p(w_down), _p(w_up), _p(ybuf),
+                                       _p(dev_status), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_expert_ffn_gathered", rc)
     return ybuf
 
 

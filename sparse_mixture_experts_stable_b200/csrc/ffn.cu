@@ -15,6 +15,42 @@ extern "C" size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dty
     return align_up((size_t)E * C * F * dtype_size(dtype), 1024);
 }
 
+namespace {
+
+// Second GEMM of the bf16 MLP experts: ybuf = h (E*C, F) x W2^T (+ b2).
+int down_projection(moe_ffn_kind kind, const void* h, const int32_t* used, int32_t E, int64_t C, int64_t F,
+                    int64_t Dout, const void* w2, const void* b2, void* ybuf, int32_t* dev_status,
+                    cudaStream_t stream) {
+    TcGemmProblem q{};
+    q.a = h;
+    q.lda = F;
+    q.a_rows_total = (int64_t)E * C;
+    q.a_rows_per_group = C;
+    q.b = w2;
+    q.ldb = F;
+    q.b_rows_total = (int64_t)E * Dout;
+    q.b_rows_per_group = Dout;
+    q.G = E;
+    q.M = C;
+    q.N = Dout;
+    q.K = F;
+    q.rows = used;
+    q.out = ybuf;
+    q.ldo = Dout;
+    q.out_rows_per_group = C;
+    q.status = dev_status;
+    if (kind == MOE_FFN_GELU_MLP) {
+        q.bias = b2;
+        q.bias_group_stride = Dout;
+        q.epilogue = TC_EPI_BF16_BIAS;
+    } else {
+        q.epilogue = TC_EPI_BF16;
+    }
+    return tc_gemm_run(q, stream);
+}
+
+}  // namespace
+
 extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32_t* used, int32_t E,
                               int64_t C, int64_t D, int64_t F, int64_t Dout, const void* w1, const void* b1,
                               const void* w2, const void* b2, const void* w3, void* ybuf, int32_t* dev_status,
@@ -105,33 +141,7 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
             rc = tc_gemm_run(p, stream);
         }
         if (rc != MOE_OK) return rc;
-        // second GEMM: h (E*C, F) x W2^T
-        TcGemmProblem q{};
-        q.a = h;
-        q.lda = F;
-        q.a_rows_total = (int64_t)E * C;
-        q.a_rows_per_group = C;
-        q.b = w2;
-        q.ldb = F;
-        q.b_rows_total = (int64_t)E * Dout;
-        q.b_rows_per_group = Dout;
-        q.G = E;
-        q.M = C;
-        q.N = Dout;
-        q.K = F;
-        q.rows = used;
-        q.out = ybuf;
-        q.ldo = Dout;
-        q.out_rows_per_group = C;
-        q.status = dev_status;
-        if (kind == MOE_FFN_GELU_MLP) {
-            q.bias = b2;
-            q.bias_group_stride = Dout;
-            q.epilogue = TC_EPI_BF16_BIAS;
-        } else {
-            q.epilogue = TC_EPI_BF16;
-        }
-        return tc_gemm_run(q, stream);
+        return down_projection(kind, h, used, E, C, F, Dout, w2, b2, ybuf, dev_status, stream);
     }
 
     // fp32: FFMA GEMMs, B = weights in (out, in) layout -> transposed operand
@@ -201,4 +211,44 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
         d.epilogue = SIMT_EPI_BIAS;
     }
     return simt_gemm_run(d, stream);
+}
+
+extern "C" int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const void* x, int64_t T, int64_t ldx,
+                                       const int32_t* token_of_slot, const int32_t* used, int32_t E, int64_t C,
+                                       int64_t D, int64_t F, int64_t Dout, const void* w1, const void* w2,
+                                       const void* w3, void* ybuf, int32_t* dev_status, void* workspace,
+                                       size_t workspace_bytes, moe_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    MOE_REQUIRE(kind == MOE_FFN_SWIGLU && dtype == MOE_BF16, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(x && token_of_slot && used && ybuf && w1 && w2 && w3, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(T >= 1 && ldx >= D && E >= 1 && C >= 0 && D >= 1 && F >= 1 && Dout >= 1, MOE_ERR_INVALID_ARG);
+    if (C == 0) return MOE_OK;
+    MOE_REQUIRE(workspace && workspace_bytes >= moe_expert_ffn_workspace_size(kind, dtype, E, C, F),
+                MOE_ERR_WORKSPACE);
+    void* h = workspace;
+    // gate/up with the token rows read from x through token_of_slot
+    TcxProblem p{};
+    p.w = w1;   // gate
+    p.w2 = w3;  // up
+    p.ldw = D;
+    p.w_rows_total = (int64_t)E * F;
+    p.w_rows_per_group = F;
+    p.x = x;
+    p.ldx = ldx;
+    p.x_rows_total = T;
+    p.x_rows_per_group = 0;
+    p.G = E;
+    p.features = F;
+    p.max_tokens = C;
+    p.K = D;
+    p.rows = used;
+    p.gather_index = token_of_slot;
+    p.out = h;
+    p.ldo = F;
+    p.out_rows_per_group = C;
+    p.epilogue = TC_EPI_SWIGLU;
+    p.status = dev_status;
+    const int rc = tcx_gemm_run(p, stream);
+    if (rc != MOE_OK) return rc;
+    return down_projection(kind, h, used, E, C, F, Dout, w2, nullptr, ybuf, dev_status, stream);
 }

@@ -37,6 +37,8 @@ constexpr int kM = 128;       // features per tile (UMMA M)
 constexpr int kBK = 64;       // K per stage (one 128-byte swizzle row of bf16)
 constexpr int kStages = 4;
 constexpr int kThreads = 192;
+constexpr int kGatherThreads = 128;  // gathered token rows: four more warps fill the token tile
+constexpr int kGatherLag = 2;       // stages a gather thread keeps in flight before signalling
 constexpr int kMaxGroups = 1024;
 constexpr int kStageBytes = 48 * 1024;  // two weight tiles (2 x 16 KB) + 128 token rows (16 KB)
 constexpr int kNT = 128;                // token rows per tile (TMA box height)
@@ -62,6 +64,11 @@ struct XParams {
     int64_t bias_group_stride;
     int vec_ok;
     int32_t* status;
+    const __nv_bfloat16* xg;  // gathered mode: token source rows (row stride ldxg)
+    int64_t ldxg;
+    int64_t kdim;             // K (gathered mode: chunks past K are zero-filled)
+    int64_t xrows;            // gathered mode: rows of the source matrix
+    const int32_t* gidx;      // gathered mode: (G, max_tokens) source row per token slot
 };
 
 __device__ __forceinline__ int64_t group_rows(const XParams& p, int g) {
@@ -84,8 +91,8 @@ __device__ __forceinline__ void decode(int tile, const int* prefix, int G, int f
     ft = local - tt * f_tiles;
 }
 
-template <int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int EPI, bool GATHER>
+__global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads, 1)
     tcx_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmW2,
                const __grid_constant__ CUtensorMap tmX, const XParams p) {
     constexpr bool kDual = EPI == TC_EPI_SWIGLU;
@@ -108,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], GATHER ? 1 + kGatherThreads : 1);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -160,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(st, &tmW, kb * kBK, w_y, &full[stage]);
                     if (kDual) tma_load_2d(st + 16 * 1024, &tmW2, kb * kBK, w_y, &full[stage]);
                     else tma_load_2d(st + 16 * 1024, &tmW, kb * kBK, w_y + kM, &full[stage]);
-                    tma_load_2d(st + x_off, &tmX, kb * kBK, x_y, &full[stage]);
+                    if (!GATHER) tma_load_2d(st + x_off, &tmX, kb * kBK, x_y, &full[stage]);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -216,6 +223,82 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_commit(&tfull[acc]);
             }
+        }
+        __syncwarp();
+    } else if (GATHER && warp >= kThreads / 32) {
+        // ------------------------- gathered token rows -------------------------
+        // kGatherThreads threads fill the 128 x 64 token tile of each stage with
+        // 16-byte cp.async copies from the source rows, in the 128-byte swizzled
+        // layout the TMA would produce (chunk j of row r at chunk j ^ (r & 7)).
+        // Thread gt copies chunk j = gt & 7 of rows kRowStep*i + (gt >> 3), so
+        // eight consecutive threads read one contiguous 128-byte row segment.  A
+        // stage is signalled once its copies have landed (kGatherLag stages
+        // later), after a proxy fence that makes them visible to the tensor core.
+        constexpr int kRowStep = kGatherThreads / 8;
+        constexpr int kPasses = kNT / kRowStep;
+        const int gt = threadIdx.x - kThreads;
+        const int j = gt & 7;
+        const int rsub = gt >> 3;
+        // row kRowStep*i + rsub has (row & 7) == (rsub & 7) for every i
+        const uint32_t dst_off = (uint32_t)(rsub * 128 + ((j ^ (rsub & 7)) << 4));
+        int stage = 0;
+        uint32_t phase = 0;
+        int pending = 0;    // stages issued and not yet signalled
+        int sig_stage = 0;  // oldest of them
+        bool abort = false;
+        for (int tile = blockIdx.x; tile < total && !abort; tile += gridDim.x) {
+            int g, ft, tt;
+            decode(tile, s_prefix, p.G, p.f_tiles, g, ft, tt);
+            const int64_t n0 = (int64_t)tt * p.nt;
+            const int64_t rows_g = group_rows(p, g);
+            const int32_t* gi = p.gidx + (int64_t)g * p.max_tokens;
+            const __nv_bfloat16* src[kPasses];
+            uint32_t srcb[kPasses];
+#pragma unroll
+            for (int i = 0; i < kPasses; ++i) {
+                const int64_t n = n0 + kRowStep * i + rsub;
+                int32_t t = n < rows_g ? gi[n] : -1;
+                if (t >= p.xrows) {  // outside the source matrix: report, read zeros
+                    set_status(p.status, MOE_ERR_BAD_INDEX);
+                    t = -1;
+                }
+                src[i] = p.xg + (t >= 0 ? (int64_t)t * p.ldxg : 0) + 8 * j;
+                srcb[i] = t >= 0 ? 16u : 0u;
+            }
+            for (int kb = 0; kb < p.k_blocks; ++kb) {
+                int ok = 1;
+                if ((threadIdx.x & 31) == 0) ok = mbar_wait(&empty[stage], phase ^ 1u, p.status) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok || s_abort) {
+                    s_abort = 1;
+                    abort = true;
+                    break;
+                }
+                const uint32_t dst = smem_u32(stages + stage * kStageBytes + x_off) + dst_off;
+                const bool in_k = (int64_t)kb * kBK + 8 * j < p.kdim;
+#pragma unroll
+                for (int i = 0; i < kPasses; ++i)  // a zero-byte copy reads nothing; give it the base address anyway
+                    cp_async_16(dst + i * kRowStep * 128, in_k ? src[i] + kb * kBK : p.xg, in_k ? srcb[i] : 0u);
+                cp_async_commit();
+                ++pending;
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (pending > kGatherLag) {
+                    cp_async_wait_group<kGatherLag>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full[sig_stage]);
+                    sig_stage = sig_stage + 1 == kStages ? 0 : sig_stage + 1;
+                    --pending;
+                }
+            }
+        }
+        cp_async_wait_group<0>();
+        fence_proxy_async_smem();
+        for (; pending > 0; --pending) {
+            mbar_arrive(&full[sig_stage]);
+            sig_stage = sig_stage + 1 == kStages ? 0 : sig_stage + 1;
         }
         __syncwarp();
     } else {
@@ -304,18 +387,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int EPI>
+template <int EPI, bool GATHER = false>
 int launch(const CUtensorMap& w, const CUtensorMap& w2, const CUtensorMap& x, const XParams& kp, int grid,
            cudaStream_t stream) {
     static bool attr_set[64] = {false};
     int dev = 0;
     MOE_CUDA_TRY(cudaGetDevice(&dev));
-    if (dev < 64 && !attr_set[dev]) {
-        MOE_CUDA_TRY(
-            cudaFuncSetAttribute(tcx_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes));
-        attr_set[dev] = true;
+    if (dev >= 64 || !attr_set[dev]) {
+        MOE_CUDA_TRY(cudaFuncSetAttribute(tcx_kernel<EPI, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)kSmemBytes));
+        if (dev < 64) attr_set[dev] = true;
     }
-    tcx_kernel<EPI><<<grid, kThreads, kSmemBytes, stream>>>(w, w2, x, kp);
+    tcx_kernel<EPI, GATHER><<<grid, GATHER ? kThreads + kGatherThreads : kThreads, kSmemBytes, stream>>>(w, w2, x,
+                                                                                                         kp);
     return launch_status();
 }
 
@@ -331,6 +415,8 @@ int tcx_gemm_run(const TcxProblem& p, cudaStream_t stream) {
                 MOE_ERR_UNSUPPORTED);
     MOE_REQUIRE(p.ldw >= p.K && p.ldx >= p.K, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(p.w_rows_total < (int64_t(1) << 31) && p.x_rows_total < (int64_t(1) << 31), MOE_ERR_UNSUPPORTED);
+    const bool gather = p.gather_index != nullptr;
+    if (gather) MOE_REQUIRE(dual && p.K % 8 == 0, MOE_ERR_UNSUPPORTED);
     if (p.max_tokens == 0) return MOE_OK;
 
     XParams kp{};
@@ -343,7 +429,7 @@ int tcx_gemm_run(const TcxProblem& p, cudaStream_t stream) {
     kp.f_tiles = (int)((p.features + kp.feat_per_tile - 1) / kp.feat_per_tile);
     kp.nt = kNT;
     kp.k_blocks = (int)((p.K + kBK - 1) / kBK);
-    kp.tx_bytes = (uint32_t)(2 * kM * kBK * 2 + kp.nt * kBK * 2);
+    kp.tx_bytes = (uint32_t)(2 * kM * kBK * 2 + (gather ? 0 : kp.nt * kBK * 2));
     kp.rows = p.rows;
     kp.out = p.out;
     kp.ldo = p.ldo;
@@ -353,12 +439,18 @@ int tcx_gemm_run(const TcxProblem& p, cudaStream_t stream) {
     const size_t esz = p.epilogue == TC_EPI_F32 ? 4 : 2;
     kp.vec_ok = aligned16(p.out) && (p.ldo * (int64_t)esz) % 16 == 0;
     kp.status = p.status;
+    kp.xg = static_cast<const __nv_bfloat16*>(p.x);
+    kp.ldxg = p.ldx;
+    kp.kdim = p.K;
+    kp.gidx = p.gather_index;
+    kp.xrows = p.x_rows_total;
 
     CUtensorMap mw, mw2, mx;
     MOE_REQUIRE(make_map(&mw, p.w, p.K, p.w_rows_total, p.ldw, kM), MOE_ERR_CUDA);
     if (dual) MOE_REQUIRE(make_map(&mw2, p.w2, p.K, p.w_rows_total, p.ldw, kM), MOE_ERR_CUDA);
     else mw2 = mw;
-    MOE_REQUIRE(make_map(&mx, p.x, p.K, p.x_rows_total, p.ldx, kp.nt), MOE_ERR_CUDA);
+    if (gather) mx = mw;  // token rows are copied by the kernel's gather warps
+    else MOE_REQUIRE(make_map(&mx, p.x, p.K, p.x_rows_total, p.ldx, kp.nt), MOE_ERR_CUDA);
 
     const int64_t max_tiles = (int64_t)p.G * kp.f_tiles * ((p.max_tokens + kp.nt - 1) / kp.nt);
     MOE_REQUIRE(max_tiles < (int64_t(1) << 30), MOE_ERR_UNSUPPORTED);
@@ -371,7 +463,9 @@ int tcx_gemm_run(const TcxProblem& p, cudaStream_t stream) {
         case TC_EPI_BF16: return launch<TC_EPI_BF16>(mw, mw2, mx, kp, grid, stream);
         case TC_EPI_BF16_BIAS: return launch<TC_EPI_BF16_BIAS>(mw, mw2, mx, kp, grid, stream);
         case TC_EPI_GELU_BIAS: return launch<TC_EPI_GELU_BIAS>(mw, mw2, mx, kp, grid, stream);
-        case TC_EPI_SWIGLU: return launch<TC_EPI_SWIGLU>(mw, mw2, mx, kp, grid, stream);
+        case TC_EPI_SWIGLU:
+            return gather ? launch<TC_EPI_SWIGLU, true>(mw, mw2, mx, kp, grid, stream)
+                          : launch<TC_EPI_SWIGLU>(mw, mw2, mx, kp, grid, stream);
         default: return MOE_ERR_INVALID_ARG;
     }
 }

@@ -23,6 +23,11 @@ struct TcxProblem {
     int64_t max_tokens;        // token rows per group (C)
     int64_t K;
     const int32_t* rows;       // device (G) valid token rows per group, or NULL (= max_tokens)
+    // Gathered token rows (TC_EPI_SWIGLU only): when non-NULL, token row n of group g
+    // is row gather_index[g*max_tokens + n] of x (x_rows_total rows), read directly by
+    // the kernel instead of from an expert-major copy; a negative index or n >= rows[g]
+    // reads zeros.  x_rows_per_group is then unused.
+    const int32_t* gather_index;
     void* out;                 // (G*out_rows_per_group, ldo): fp32 for TC_EPI_F32, else bf16
     int64_t ldo;
     int64_t out_rows_per_group;

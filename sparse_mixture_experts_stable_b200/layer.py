@@ -18,7 +18,7 @@ class SwiGLUMoE:
     """
 
     def __init__(self, T: int, H: int, E: int, F: int, k: int, capacity_factor: float, F_shared: int = 0,
-                 aux_coef: float = 0.0, dtype=torch.bfloat16, device="cuda"):
+                 aux_coef: float = 0.0, dtype=torch.bfloat16, device="cuda", gathered: bool = False):
         self.T, self.H, self.E, self.F, self.k = T, H, E, F, k
         self.F_shared, self.aux_coef, self.dtype = F_shared, aux_coef, dtype
         self.C = B.moe_capacity(T, k, E, capacity_factor)
@@ -39,8 +39,13 @@ class SwiGLUMoE:
             overflow=torch.empty(E, dtype=torch.int32, device=dev),
             drops=torch.empty(T, dtype=torch.int32, device=dev),
             token_of_slot=torch.empty(E, C, dtype=torch.int32, device=dev),
-            xbuf=torch.empty(E, C, H, dtype=dtype, device=dev),
         )
+        # gathered=True (bf16 only) skips the (E, C, H) copy of the token rows: the
+        # expert kernel reads them from x, which saves that memory at about the
+        # same step time; otherwise the dispatch gathers them into xbuf.
+        self.gathered = gathered and dtype == torch.bfloat16
+        if not self.gathered:
+            self.disp_out["xbuf"] = torch.empty(E, C, H, dtype=dtype, device=dev)
         self.ybuf = torch.empty(E, C, H, dtype=dtype, device=dev)
         self.y = torch.empty(T, H, dtype=dtype, device=dev)
         self.shared = torch.empty(T, H, dtype=dtype, device=dev) if F_shared else None
@@ -76,10 +81,16 @@ class SwiGLUMoE:
             base_kind, base = "tensor", self.shared
         r = B.moe_route(x, self.k, w_router=w_router, layout="ED", logit_bias=router_bias, out=self.route_out,
                         dev_status=self.status, workspace=self.ws_route)
-        d = B.moe_dispatch(r["selected"], self.E, self.C, x=x, out=self.disp_out, dev_status=self.status,
-                           workspace=self.ws_disp)
-        B.moe_expert_ffn("swiglu", d["xbuf"], d["used"], w_gate, w2=w_down, w3=w_up, ybuf=self.ybuf,
-                         dev_status=self.status, workspace=self.ws_ffn)
+        if self.gathered:  # slots only: the expert kernel reads its rows from x through token_of_slot
+            d = B.moe_dispatch(r["selected"], self.E, self.C, out=self.disp_out, dev_status=self.status,
+                               workspace=self.ws_disp)
+            B.moe_expert_ffn_gathered(x, d["token_of_slot"], d["used"], w_gate, w_down, w_up, ybuf=self.ybuf,
+                                      dev_status=self.status, workspace=self.ws_ffn)
+        else:
+            d = B.moe_dispatch(r["selected"], self.E, self.C, x=x, out=self.disp_out, dev_status=self.status,
+                               workspace=self.ws_disp)
+            B.moe_expert_ffn("swiglu", d["xbuf"], d["used"], w_gate, w2=w_down, w3=w_up, ybuf=self.ybuf,
+                             dev_status=self.status, workspace=self.ws_ffn)
         if self.F_shared:
             main.wait_event(self.ev_shared)
         B.moe_combine(self.ybuf, r["selected"], d["slot"], r["gates_f32"], base_kind=base_kind, base=base, y=self.y,

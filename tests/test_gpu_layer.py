@@ -97,14 +97,15 @@ def _swiglu_oracle_rows(cfg, o, tokens, shared_rows):
     return np.stack(ys)
 
 
-@pytest.mark.parametrize("full_size", [False, True])
-def test_full_swiglu_layer_bf16(full_size):
+@pytest.mark.parametrize("full_size,gathered", [(False, False), (False, True), (True, False), (True, True)])
+def test_full_swiglu_layer_bf16(full_size, gathered):
     if full_size:
         cfg = I.full_layer_bf16(seed=0)
     else:
         cfg = I.full_layer_bf16(seed=7, T=2048, H=512, E=32, F=256, k=8, F_shared=256)
     T, H, E, F, k = cfg["T"], cfg["H"], cfg["E"], cfg["F"], cfg["k"]
-    layer = SwiGLUMoE(T, H, E, F, k, cfg["capacity_factor"], F_shared=cfg["F_shared"], aux_coef=cfg["aux_coef"])
+    layer = SwiGLUMoE(T, H, E, F, k, cfg["capacity_factor"], F_shared=cfg["F_shared"], aux_coef=cfg["aux_coef"],
+                      gathered=gathered)
     C = layer.C
     dv = {n: cfg[n].to(DEV) for n in ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down", "s_gate", "s_up",
                                        "s_down")}
