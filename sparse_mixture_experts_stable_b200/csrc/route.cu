@@ -20,13 +20,21 @@ namespace {
 
 constexpr int kRouteWarps = 8;
 constexpr int kRouteThreads = kRouteWarps * 32;
-constexpr int kMaxRouteBlocks = 1024;
+constexpr int kMaxRouteBlocks = 1024;  // bound on the per-block partials (workspace sizing)
+constexpr int kRouteBlocksPerSm = 4;    // blocks launched per SM; each warp then walks several tokens
 constexpr int kMaxK = 64;
 constexpr int kMaxE = 1024;
 
 int route_blocks(int64_t T) {
     int64_t b = (T + kRouteWarps - 1) / kRouteWarps;
     return (int)(b < kMaxRouteBlocks ? b : kMaxRouteBlocks);
+}
+
+// Blocks the top-k kernel launches (<= route_blocks(T), the partials' capacity).
+int topk_grid(int64_t T) {
+    const int cap = kRouteBlocksPerSm * device_sm_count();
+    const int b = route_blocks(T);
+    return b < cap ? b : cap;
 }
 
 // SC: 0 softmax, 1 sigmoid clean scores.  SB: a selection bias is given
@@ -43,7 +51,6 @@ __global__ void __launch_bounds__(kRouteThreads)
     extern __shared__ float s_dyn[];
     float* s_psum = s_dyn;                                            // [kRouteWarps][E]
     int* s_counts = reinterpret_cast<int*>(s_psum + kRouteWarps * E);  // [E]
-    float* s_selv = reinterpret_cast<float*>(s_counts + E);            // [kRouteWarps][k]
     __shared__ float s_z[kRouteWarps];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -60,12 +67,25 @@ __global__ void __launch_bounds__(kRouteThreads)
         sbias_r[m] = (SB && e < E) ? sel_bias[e] : 0.f;
         psum[m] = 0.f;
     }
-    float* selv = s_selv + warp * k;
     float zacc = 0.f;
 
     const int64_t stride = (int64_t)gridDim.x * kRouteWarps;
-    for (int64_t t = (int64_t)blockIdx.x * kRouteWarps + warp; t < T; t += stride) {
-        const InT* row = logits + t * ld;
+    // the next token's scores are loaded while the current token is processed
+    InT nxt[EPL];
+    int64_t t = (int64_t)blockIdx.x * kRouteWarps + warp;
+    if (t < T) {
+#pragma unroll
+        for (int m = 0; m < EPL; ++m) nxt[m] = (m * 32 + lane < E) ? logits[t * ld + m * 32 + lane] : InT(0.f);
+    }
+    for (; t < T; t += stride) {
+        InT cur[EPL];
+#pragma unroll
+        for (int m = 0; m < EPL; ++m) cur[m] = nxt[m];
+        if (t + stride < T) {
+            const InT* nrow = logits + (t + stride) * ld;
+#pragma unroll
+            for (int m = 0; m < EPL; ++m) nxt[m] = (m * 32 + lane < E) ? nrow[m * 32 + lane] : InT(0.f);
+        }
         float v[EPL];
         uint32_t taken = 0;
         bool finite = true;
@@ -73,7 +93,7 @@ __global__ void __launch_bounds__(kRouteThreads)
         for (int m = 0; m < EPL; ++m) {
             const int e = m * 32 + lane;
             if (e < E) {
-                float x = to_f32(row[e]) + bias_r[m];
+                float x = to_f32(cur[m]) + bias_r[m];
                 if (!isfinite(x)) {
                     finite = false;
                     x = -INFINITY;
@@ -125,6 +145,10 @@ __global__ void __launch_bounds__(kRouteThreads)
             const int e = m * 32 + lane;
             key[m] = (e < E) ? order_key(SB ? clean[m] + sbias_r[m] : v[m]) : 0u;
         }
+        // Winner j is kept by lane j (j < 32) or lane j - 32 in registers; the
+        // rounds contain no divergent branch and no memory access.
+        uint32_t sel0 = 0, sel1 = 0;
+        float val0 = 0.f, val1 = 0.f;
         for (int j = 0; j < k; ++j) {
             uint32_t lk = 0;  // below every finite or infinite key
             uint32_t li = 0xffffffffu;
@@ -140,20 +164,32 @@ __global__ void __launch_bounds__(kRouteThreads)
             }
             const uint32_t gk = __reduce_max_sync(0xffffffffu, lk);
             const uint32_t bi = __reduce_min_sync(0xffffffffu, lk == gk ? li : 0xffffffffu);
-            if ((int)(bi & 31u) == lane) {
-                taken |= 1u << (bi >> 5);
-                selv[j] = lv;  // the winner's raw logit
-                selected[t * k + j] = (int64_t)bi;
-                atomicAdd(&s_counts[bi], 1);
+            const int wl = (int)(bi & 31u);
+            // the winner's raw logit: its key when ranking by logit, else from the winning lane
+            const float wv = SB ? __shfl_sync(0xffffffffu, lv, wl) : key_to_float(gk);
+            taken |= wl == lane ? 1u << (bi >> 5) : 0u;
+            if (j < 32) {
+                sel0 = lane == j ? bi : sel0;
+                val0 = lane == j ? wv : val0;
+            } else {
+                sel1 = lane == j - 32 ? bi : sel1;
+                val1 = lane == j - 32 ? wv : val1;
             }
         }
-        __syncwarp();
+        if (lane < k) {
+            selected[t * k + lane] = (int64_t)sel0;
+            atomicAdd(&s_counts[sel0], 1);
+        }
+        if (lane + 32 < k) {
+            selected[t * k + lane + 32] = (int64_t)sel1;
+            atomicAdd(&s_counts[sel1], 1);
+        }
 
         // gates: softmax of the selected logits, or of their log-sigmoids (k <= 64:
         // each lane owns j = lane and j = lane + 32)
         float w0 = -INFINITY, w1 = -INFINITY;
-        if (lane < k) w0 = SC == 0 ? selv[lane] : log_sigmoid_f(selv[lane]);
-        if (lane + 32 < k) w1 = SC == 0 ? selv[lane + 32] : log_sigmoid_f(selv[lane + 32]);
+        if (lane < k) w0 = SC == 0 ? val0 : log_sigmoid_f(val0);
+        if (lane + 32 < k) w1 = SC == 0 ? val1 : log_sigmoid_f(val1);
         const float wmax = warp_max(fmaxf(w0, w1));
         const float e0 = lane < k ? expf(w0 - wmax) : 0.f;
         const float e1 = lane + 32 < k ? expf(w1 - wmax) : 0.f;
@@ -240,9 +276,8 @@ int launch_topk(int epl, const InT* logits, int64_t ld, int64_t T, int E, int k,
                 float* logits_out, int64_t* selected, void* gates, int gates_bf16, float* gates_f32,
                 int32_t* part_counts, float* part_psum, int scoring, const float* sel_bias, float* part_z,
                 int32_t* status, cudaStream_t stream) {
-    const int nb = route_blocks(T);
-    const size_t smem = sizeof(float) * (size_t)kRouteWarps * E + sizeof(int) * (size_t)E +
-                        sizeof(float) * (size_t)kRouteWarps * k;
+    const int nb = topk_grid(T);
+    const size_t smem = sizeof(float) * (size_t)kRouteWarps * E + sizeof(int) * (size_t)E;
 #define MOE_TOPK_CASE(N)                                                                                      \
     case N: {                                                                                                 \
         auto kern = scoring == 0 ? (sel_bias ? route_topk_kernel<N, InT, 0, true> : route_topk_kernel<N, InT, 0, false>) \
@@ -397,7 +432,7 @@ extern "C" int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D
                                 dev_status, stream);
     }
     if (rc != MOE_OK) return rc;
-    const int nb = route_blocks(T);
+    const int nb = topk_grid(T);
     route_reduce_kernel<<<(E + 31) / 32, kReduceWarps * 32, 0, stream>>>(part_counts, part_psum, nb, E, counts,
                                                                          prob_sum, part_z, T, z_loss);
     return launch_status();

@@ -18,6 +18,11 @@ __device__ __forceinline__ uint32_t order_key(float v) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// Inverse of order_key (-0 comes back as +0).
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 __device__ __forceinline__ float sigmoid_stable_f(float z) {
     if (z >= 0.f) return 1.f / (1.f + expf(-z));
     const float ez = expf(z);
