@@ -130,7 +130,8 @@ MOE_API int moe_capacity(int64_t T, int32_t k, int32_t E, double capacity_factor
  *              (row stride ldx, dtype `dtype`) and D is ignored.
  *   w_router   device or NULL; router weight in `layout`, dtype `dtype`.
  *              bf16 scores are computed on the tensor cores (fp32
- *              accumulate); fp32 scores with fp32 FFMA.
+ *              accumulate); fp32 scores on the tensor cores as split-tf32
+ *              products (fp32 accuracy).
  *   logit_bias device fp32 (E) or NULL.
  *   k          1 <= k <= E; this build requires k <= 64 and E <= 1024.
  *   logits_out device fp32 (T, E) or NULL; receives s.
@@ -275,7 +276,10 @@ MOE_API int moe_dispatch_static(const int64_t* selected, int64_t T, int32_t k, i
  *   SWIGLU   : (silu(x W1_e^T) * (x W3_e^T)) W2_e^T                 [P3]
  *              W1 = gate (E, F, D), W3 = up (E, F, D), W2 = down (E, Dout, F)
  * bf16: tcgen05 tensor cores, fp32 accumulation, the intermediate
- * activation rounded to bf16, outputs bf16.  fp32: fp32 FFMA throughout.
+ * activation rounded to bf16, outputs bf16.  fp32: tcgen05 tensor cores on
+ * split-tf32 operands (x = hi + lo, three tf32 products per term, fp32
+ * accumulation), which keeps fp32 accuracy; the split operands live in the
+ * workspace.
  * Rows c >= rows(e) of ybuf are not written.  An always-on shared expert
  * ([P3] EducationalMoE) is this call with E = 1, C = T, used = NULL and the
  * token matrix as xbuf.
@@ -286,10 +290,11 @@ MOE_API int moe_dispatch_static(const int64_t* selected, int64_t T, int32_t k, i
  *   w1,b1,w2,b2,w3 device, layouts above, dtype `dtype` (biases too);
  *             unused ones may be NULL.
  *   ybuf      device (E, C, Dout) contiguous, dtype `dtype`.
- *   workspace device, >= moe_expert_ffn_workspace_size(...) bytes.
+ *   workspace device, >= moe_expert_ffn_workspace_size(kind, dtype, E, C, D, F, Dout)
+ *             bytes (0 for bf16 LINEAR; fp32 needs room for the split operands).
  */
 MOE_API size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dtype, int32_t E, int64_t C,
-                                     int64_t F);
+                                             int64_t D, int64_t F, int64_t Dout);
 MOE_API int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32_t* used,
                    int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout, const void* w1,
                    const void* b1, const void* w2, const void* b2, const void* w3, void* ybuf,
@@ -315,7 +320,7 @@ MOE_API int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf,
  *   used          device int32 (E) from moe_dispatch (required).
  *   w1 = gate (E, F, D), w3 = up (E, F, D), w2 = down (E, Dout, F), bf16.
  *   ybuf          device bf16 (E, C, Dout); rows c >= used[e] are not written.
- *   workspace     device, >= moe_expert_ffn_workspace_size(MOE_FFN_SWIGLU, MOE_BF16, E, C, F).
+ *   workspace     device, >= moe_expert_ffn_workspace_size(MOE_FFN_SWIGLU, MOE_BF16, E, C, D, F, Dout).
  */
 MOE_API int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const void* x, int64_t T, int64_t ldx,
                                     const int32_t* token_of_slot, const int32_t* used, int32_t E, int64_t C,

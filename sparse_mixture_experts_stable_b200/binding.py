@@ -81,7 +81,7 @@ def lib():
         L.moe_dispatch_static.argtypes = [_vp, _i64, _i32, _i32, _i64, _vp, ctypes.c_int, _i64, _i64, _vp, _vp, _vp,
                                           _vp, _vp, _vp, _vp, _vp, _vp]
         L.moe_expert_ffn_workspace_size.restype = _sz
-        L.moe_expert_ffn_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, _i32, _i64, _i64]
+        L.moe_expert_ffn_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, _i32, _i64, _i64, _i64, _i64]
         L.moe_expert_ffn.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _vp,
                                      _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
         L.moe_expert_ffn_gathered.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _i64, _i64, _vp, _vp, _i32, _i64,
@@ -287,8 +287,8 @@ def moe_dispatch_static(selected: torch.Tensor, E: int, C: int, x: Optional[torc
     return o
 
 
-def moe_expert_ffn_workspace_size(kind: str, dtype: int, E: int, C: int, F: int) -> int:
-    return int(lib().moe_expert_ffn_workspace_size(FFN[kind], dtype, E, C, F))
+def moe_expert_ffn_workspace_size(kind: str, dtype: int, E: int, C: int, D: int, F: int, Dout: int) -> int:
+    return int(lib().moe_expert_ffn_workspace_size(FFN[kind], dtype, E, C, D, F, Dout))
 
 
 def moe_expert_ffn(kind: str, xbuf: torch.Tensor, used: Optional[torch.Tensor], w1: torch.Tensor,
@@ -311,7 +311,7 @@ def moe_expert_ffn(kind: str, xbuf: torch.Tensor, used: Optional[torch.Tensor], 
         raise ValueError("xbuf must be contiguous")
     if ybuf is None:
         ybuf = torch.empty(E, C, Dout, dtype=xbuf.dtype, device=dev)
-    ws = _workspace(moe_expert_ffn_workspace_size(kind, dt, E, C, max(F, 1)), dev, workspace)
+    ws = _workspace(moe_expert_ffn_workspace_size(kind, dt, E, C, D, max(F, 1), Dout), dev, workspace)
     rc = lib().moe_expert_ffn(FFN[kind], dt, _p(xbuf), _p(used), E, C, D, F, Dout, _p(w1), _p(b1), _p(w2), _p(b2),
                               _p(w3), _p(ybuf), _p(dev_status), _p(ws), ws.numel(), _stream(stream))
     _check("moe_expert_ffn", rc)
@@ -339,7 +339,7 @@ def moe_expert_ffn_gathered(x: torch.Tensor, token_of_slot: torch.Tensor, used: 
         raise TypeError("token_of_slot and used must be int32")
     if ybuf is None:
         ybuf = torch.empty(E, C, Dout, dtype=x.dtype, device=dev)
-    ws = _workspace(moe_expert_ffn_workspace_size("swiglu", dt, E, C, F), dev, workspace)
+    ws = _workspace(moe_expert_ffn_workspace_size("swiglu", dt, E, C, D, F, Dout), dev, workspace)
     rc = lib().moe_expert_ffn_gathered(FFN["swiglu"], dt, _p(x), T, _rowstride(x), _p(token_of_slot.contiguous()),
                                        _p(used), E, C, D, F, Dout, _p(w_gate), _p(w_down), _p(w_up), _p(ybuf),
                                        _p(dev_status), _p(ws), ws.numel(), _stream(stream))

@@ -1,14 +1,15 @@
 // moe_backward: backward of the linear-expert layer with the kept mask fixed.
 //   1. dgate / dlogits       one warp per token (row dots, quotient rule, aux term)
 //   2. dybuf[e,c] = gate * dy[token]     token-major gather with scale
-//   3. dW[e]   = dybuf_e^T xbuf_e        FFMA GEMM, K = used[e] rows
-//   4. dxbuf_e = dybuf_e W_e             FFMA GEMM, M = used[e] rows
+//   3. dW[e]   = dybuf_e^T xbuf_e        split-tf32 tensor-core GEMM, K = used[e] rows
+//   4. dxbuf_e = dybuf_e W_e             split-tf32 tensor-core GEMM, M = used[e] rows
 //   5. dx[t]   = [dy[t]] + sum_kept dxbuf[e, slot]   deterministic combine
 #include <cuda_runtime.h>
 #include <math.h>
 
 #include "common.cuh"
-#include "simt_gemm.cuh"
+#include "f32_gemm.cuh"
+#include "tc_tf32.cuh"
 #include "util_kernels.cuh"
 
 namespace moe {
@@ -92,9 +93,32 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 using namespace moe;
 
+namespace moe {
+namespace {
+
+// The two GEMMs' shapes (for the split-operand workspace).
+size_t backward_split_bytes(int32_t E, int64_t C, int64_t D, int64_t Dout) {
+    F32Gemm w{};  // dW: (Dout x D), K = C
+    w.M = Dout;
+    w.N = D;
+    w.K = C;
+    w.groups = E;
+    F32Gemm x{};  // dxbuf: (C x D), K = Dout
+    x.M = C;
+    x.N = D;
+    x.K = Dout;
+    x.groups = E;
+    const size_t a = tf32x3_workspace_size(w), b = tf32x3_workspace_size(x);
+    return a > b ? a : b;
+}
+
+}  // namespace
+}  // namespace moe
+
 extern "C" size_t moe_backward_workspace_size(int32_t E, int64_t C, int64_t D, int64_t Dout) {
     if (E < 1 || C < 1) return 256;
-    return align_up((size_t)E * C * Dout * 4, 256) + align_up((size_t)E * C * D * 4, 256);
+    return align_up((size_t)E * C * Dout * 4, 256) + align_up((size_t)E * C * D * 4, 256) +
+           backward_split_bytes(E, C, D, Dout);
 }
 
 extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, const void* x, const float* logits,
@@ -118,7 +142,10 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
     MOE_REQUIRE(workspace && workspace_bytes >= moe_backward_workspace_size(E, C, D, Dout), MOE_ERR_WORKSPACE);
     const int64_t Cw = C > 0 ? C : 1;
     float* dybuf = static_cast<float*>(workspace);
-    float* dxbuf = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align_up((size_t)E * Cw * Dout * 4, 256));
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* dxbuf = reinterpret_cast<float*>(ws + align_up((size_t)E * Cw * Dout * 4, 256));
+    uint8_t* split = ws + align_up((size_t)E * Cw * Dout * 4, 256) + align_up((size_t)E * Cw * D * 4, 256);
+    const size_t split_bytes = workspace_bytes - (size_t)(split - ws);
 
     const unsigned grid = (unsigned)((T + kWarps - 1) / kWarps);
     dgate_dlogits_kernel<<<grid, kWarps * 32, 0, stream>>>(
@@ -141,7 +168,7 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
     if (rc != MOE_OK) return rc;
 
     // dW[e] (Dout x D) = sum_c dybuf[e,c,:]^T xbuf[e,c,:]
-    SimtGemm w{};
+    F32Gemm w{};
     w.A = dybuf;
     w.lda = Dout;
     w.a_trans = true;
@@ -159,11 +186,11 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
     w.groups = E;
     w.rows = used;
     w.rows_mode = 2;
-    rc = simt_gemm_run(w, stream);
+    rc = tf32x3_gemm_run(w, split, split_bytes, dev_status, stream);
     if (rc != MOE_OK) return rc;
 
     // dxbuf[e] (rows x D) = dybuf[e] (rows x Dout) * W[e] (Dout x D)
-    SimtGemm g{};
+    F32Gemm g{};
     g.A = dybuf;
     g.lda = Dout;
     g.a_group_stride = C * Dout;
@@ -180,7 +207,7 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
     g.groups = E;
     g.rows = used;
     g.rows_mode = 1;
-    rc = simt_gemm_run(g, stream);
+    rc = tf32x3_gemm_run(g, split, split_bytes, dev_status, stream);
     if (rc != MOE_OK) return rc;
 
     return combine_rows(dxbuf, selected, slot, nullptr, MOE_F32, T, k, E, C, D, use_residual ? dy : nullptr, D, dx, D,

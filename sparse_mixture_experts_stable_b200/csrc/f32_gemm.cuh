@@ -1,4 +1,5 @@
-// fp32 grouped GEMM on the CUDA cores (FFMA), for the fp32 paths.
+// Problem form of the fp32 grouped GEMMs (run on the tensor cores as
+// split-tf32 products by tf32x3_gemm_run, tc_tf32.cuh).
 //
 // C[g](m, n) = epilogue( sum_k A[g](m, k) * B[g](k, n) )
 //   A(m, k) = a_trans ? A[k * lda + m] : A[m * lda + k]
@@ -13,14 +14,14 @@
 
 namespace moe {
 
-enum SimtEpilogue : int {
-    SIMT_EPI_NONE = 0,
-    SIMT_EPI_BIAS = 1,       // + bias[n]
-    SIMT_EPI_BIAS_GELU = 2,  // gelu(acc + bias[n])
-    SIMT_EPI_SILU_MUL = 3    // silu(acc) * C_old  (read-modify-write of C)
+enum F32Epilogue : int {
+    F32_EPI_NONE = 0,
+    F32_EPI_BIAS = 1,       // + bias[n]
+    F32_EPI_BIAS_GELU = 2,  // gelu(acc + bias[n])
+    F32_EPI_SILU_MUL = 3    // silu(acc) * C_old  (read-modify-write of C)
 };
 
-struct SimtGemm {
+struct F32Gemm {
     const float* A = nullptr;
     int64_t lda = 0;
     bool a_trans = false;
@@ -38,9 +39,7 @@ struct SimtGemm {
     int rows_mode = 0;
     const float* bias = nullptr;
     int64_t bias_group_stride = 0;
-    int epilogue = SIMT_EPI_NONE;
+    int epilogue = F32_EPI_NONE;
 };
-
-int simt_gemm_run(const SimtGemm& g, cudaStream_t stream);
 
 }  // namespace moe

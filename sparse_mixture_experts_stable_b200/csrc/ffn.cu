@@ -1,18 +1,55 @@
 // moe_expert_ffn: the expert FFNs as grouped GEMMs over variable-occupancy
-// experts.  bf16 runs on the tcgen05 tensor cores (tc_gemm), fp32 on FFMA.
+// experts, on the tcgen05 tensor cores: bf16 operands directly (tc_gemm,
+// tcx), fp32 operands as split-tf32 products (tc_tf32).
 #include <cuda_runtime.h>
 
 #include "common.cuh"
-#include "simt_gemm.cuh"
+#include "f32_gemm.cuh"
 #include "tc_expert_gemm.cuh"
 #include "tc_gemm.cuh"
+#include "tc_tf32.cuh"
 
 using namespace moe;
 
-extern "C" size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dtype, int32_t E, int64_t C,
-                                                int64_t F) {
-    if (kind == MOE_FFN_LINEAR || E < 1 || C < 1 || F < 1) return 0;
-    return align_up((size_t)E * C * F * dtype_size(dtype), 1024);
+namespace {
+
+// The fp32 GEMMs of one moe_expert_ffn call in F32Gemm form (operand
+// pointers left empty): [0] the first projection (LINEAR: the only one),
+// [1] the second projection of the MLP experts.
+void fp32_shapes(moe_ffn_kind kind, int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout, F32Gemm (&s)[2]) {
+    s[0] = F32Gemm{};
+    s[0].M = C;
+    s[0].K = D;
+    s[0].N = kind == MOE_FFN_LINEAR ? Dout : F;
+    s[0].groups = E;
+    s[1] = F32Gemm{};
+    s[1].M = C;
+    s[1].K = F;
+    s[1].N = Dout;
+    s[1].groups = E;
+}
+
+size_t fp32_split_bytes(moe_ffn_kind kind, int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout) {
+    F32Gemm s[2];
+    fp32_shapes(kind, E, C, D, F, Dout, s);
+    size_t b = tf32x3_workspace_size(s[0]);
+    if (kind != MOE_FFN_LINEAR) {
+        const size_t b2 = tf32x3_workspace_size(s[1]);
+        b = b2 > b ? b2 : b;
+    }
+    return b;
+}
+
+}  // namespace
+
+extern "C" size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dtype, int32_t E, int64_t C, int64_t D,
+                                                int64_t F, int64_t Dout) {
+    if (E < 1 || C < 1) return 0;
+    size_t h = 0;
+    if (kind != MOE_FFN_LINEAR && F >= 1) h = align_up((size_t)E * C * F * dtype_size(dtype), 1024);
+    if (dtype == MOE_F32 && D >= 1 && Dout >= 1 && (kind == MOE_FFN_LINEAR || F >= 1))
+        return h + fp32_split_bytes(kind, E, C, D, F, Dout);
+    return h;
 }
 
 namespace {
@@ -63,10 +100,12 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
     if (kind == MOE_FFN_GELU_MLP) MOE_REQUIRE(b1 && w2 && b2 && F >= 1, MOE_ERR_INVALID_ARG);
     if (kind == MOE_FFN_SWIGLU) MOE_REQUIRE(w2 && w3 && F >= 1, MOE_ERR_INVALID_ARG);
     void* h = nullptr;
+    const size_t need = moe_expert_ffn_workspace_size(kind, dtype, E, C, D, F, Dout);
+    MOE_REQUIRE(need == 0 || (workspace && workspace_bytes >= need), MOE_ERR_WORKSPACE);
+    size_t h_bytes = 0;
     if (kind != MOE_FFN_LINEAR) {
-        MOE_REQUIRE(workspace && workspace_bytes >= moe_expert_ffn_workspace_size(kind, dtype, E, C, F),
-                    MOE_ERR_WORKSPACE);
         h = workspace;
+        h_bytes = align_up((size_t)E * C * F * dtype_size(dtype), 1024);
     }
 
     if (dtype == MOE_BF16) {
@@ -144,8 +183,11 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
         return down_projection(kind, h, used, E, C, F, Dout, w2, b2, ybuf, dev_status, stream);
     }
 
-    // fp32: FFMA GEMMs, B = weights in (out, in) layout -> transposed operand
-    SimtGemm g{};
+    // fp32: split-tf32 tensor-core GEMMs, B = weights in (out, in) layout -> transposed operand
+    void* split = static_cast<uint8_t*>(workspace) + h_bytes;
+    const size_t split_bytes = workspace_bytes - h_bytes;
+    auto run = [&](const F32Gemm& q) { return tf32x3_gemm_run(q, split, split_bytes, dev_status, stream); };
+    F32Gemm g{};
     g.A = static_cast<const float*>(xbuf);
     g.lda = D;
     g.a_group_stride = C * D;
@@ -163,7 +205,7 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
         g.ldc = Dout;
         g.c_group_stride = C * Dout;
         g.N = Dout;
-        return simt_gemm_run(g, stream);
+        return run(g);
     }
     float* hf = static_cast<float*>(h);
     g.ldb = D;
@@ -177,18 +219,18 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
         g.B = static_cast<const float*>(w1);
         g.bias = static_cast<const float*>(b1);
         g.bias_group_stride = F;
-        g.epilogue = SIMT_EPI_BIAS_GELU;
-        rc = simt_gemm_run(g, stream);
+        g.epilogue = F32_EPI_BIAS_GELU;
+        rc = run(g);
     } else {
         g.B = static_cast<const float*>(w3);  // up -> h
-        rc = simt_gemm_run(g, stream);
+        rc = run(g);
         if (rc != MOE_OK) return rc;
         g.B = static_cast<const float*>(w1);  // gate: h = silu(gate) * up
-        g.epilogue = SIMT_EPI_SILU_MUL;
-        rc = simt_gemm_run(g, stream);
+        g.epilogue = F32_EPI_SILU_MUL;
+        rc = run(g);
     }
     if (rc != MOE_OK) return rc;
-    SimtGemm d{};
+    F32Gemm d{};
     d.A = hf;
     d.lda = F;
     d.a_group_stride = C * F;
@@ -208,9 +250,9 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
     if (kind == MOE_FFN_GELU_MLP) {
         d.bias = static_cast<const float*>(b2);
         d.bias_group_stride = Dout;
-        d.epilogue = SIMT_EPI_BIAS;
+        d.epilogue = F32_EPI_BIAS;
     }
-    return simt_gemm_run(d, stream);
+    return run(d);
 }
 
 extern "C" int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const void* x, int64_t T, int64_t ldx,
@@ -223,7 +265,7 @@ extern "C" int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const
     MOE_REQUIRE(x && token_of_slot && used && ybuf && w1 && w2 && w3, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(T >= 1 && ldx >= D && E >= 1 && C >= 0 && D >= 1 && F >= 1 && Dout >= 1, MOE_ERR_INVALID_ARG);
     if (C == 0) return MOE_OK;
-    MOE_REQUIRE(workspace && workspace_bytes >= moe_expert_ffn_workspace_size(kind, dtype, E, C, F),
+    MOE_REQUIRE(workspace && workspace_bytes >= moe_expert_ffn_workspace_size(kind, dtype, E, C, D, F, Dout),
                 MOE_ERR_WORKSPACE);
     void* h = workspace;
     // gate/up with the token rows read from x through token_of_slot

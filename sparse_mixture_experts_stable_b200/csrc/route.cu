@@ -1,6 +1,6 @@
 // moe_route and moe_aux_stats.
 //
-// Router scores come from the tensor-core GEMM (bf16) or the FFMA GEMM (fp32),
+// Router scores come from the tensor-core GEMM (bf16, or split-tf32 for fp32),
 // written as fp32 logits; then one warp per token does softmax, top-k and the
 // renormalised gates entirely in registers, and each block leaves per-expert
 // partial counts and probability sums that a second kernel adds up in a fixed
@@ -11,8 +11,9 @@
 
 #include "common.cuh"
 #include "route_scores.cuh"
-#include "simt_gemm.cuh"
+#include "f32_gemm.cuh"
 #include "tc_expert_gemm.cuh"
+#include "tc_tf32.cuh"
 #include "util_kernels.cuh"
 
 namespace moe {
@@ -309,8 +310,18 @@ int epl_for(int E) {
 }
 
 struct RouteWs {
-    size_t logits_off, wt_off, pc_off, pp_off, pz_off, total;
+    size_t logits_off, wt_off, pc_off, pp_off, pz_off, split_off, total;
 };
+
+// The fp32 router GEMM in F32Gemm form (operands filled in by the caller).
+F32Gemm router_f32_shape(int64_t T, int64_t D, int32_t E) {
+    F32Gemm g{};
+    g.M = T;
+    g.N = E;
+    g.K = D;
+    g.groups = 1;
+    return g;
+}
 
 RouteWs route_ws_layout(int64_t T, int64_t D, int32_t E, moe_dtype dtype, int has_w, moe_router_layout layout) {
     RouteWs w{};
@@ -326,6 +337,8 @@ RouteWs route_ws_layout(int64_t T, int64_t D, int32_t E, moe_dtype dtype, int ha
     off += align_up((size_t)nb * E * sizeof(float), 256);
     w.pz_off = off;
     off += align_up((size_t)nb * sizeof(float), 256);
+    w.split_off = off;
+    if (has_w && dtype == MOE_F32) off += align_up(tf32x3_workspace_size(router_f32_shape(T, D, E)), 256);
     w.total = off;
     return w;
 }
@@ -401,7 +414,7 @@ extern "C" int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D
             p.status = dev_status;
             rc = tcx_gemm_run(p, stream);
         } else {
-            SimtGemm g{};
+            F32Gemm g{};
             g.A = static_cast<const float*>(x);
             g.lda = ldx;
             g.a_trans = false;
@@ -416,8 +429,8 @@ extern "C" int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D
             g.K = D;
             g.groups = 1;
             g.bias = logit_bias;
-            g.epilogue = SIMT_EPI_BIAS;
-            rc = simt_gemm_run(g, stream);
+            g.epilogue = F32_EPI_BIAS;
+            rc = tf32x3_gemm_run(g, ws + wl.split_off, wl.total - wl.split_off, dev_status, stream);
         }
         if (rc != MOE_OK) return rc;
         rc = launch_topk<float>(epl, lg, E, T, E, k, nullptr, nullptr, selected, gates, gates_bf16, gates_f32,

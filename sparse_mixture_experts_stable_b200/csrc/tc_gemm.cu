@@ -370,6 +370,21 @@ bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int
     return r == CUDA_SUCCESS;
 }
 
+// 2-D fp32 map over a (rows, inner) row-major matrix: box = box_rows x 32
+// elements (128 bytes), 128-byte swizzle, zero fill outside the matrix.
+bool make_map_f32(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld_elems, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld_elems * 4};
+    cuuint32_t box[2] = {32u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 template <int EPI>

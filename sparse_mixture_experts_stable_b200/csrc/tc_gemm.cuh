@@ -54,4 +54,7 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream);
 // ld_elems: box = box_rows x 64 elements, 128-byte swizzle, zero fill outside.
 bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld_elems, int box_rows);
 
+// The same for fp32 elements: box = box_rows x 32 elements (128 bytes).
+bool make_map_f32(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld_elems, int box_rows);
+
 }  // namespace moe

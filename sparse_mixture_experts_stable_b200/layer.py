@@ -53,9 +53,9 @@ class SwiGLUMoE:
         self.ws_route = torch.empty(max(B.moe_route_workspace_size(T, H, E, dt, True, "ED"), 256),
                                     dtype=torch.uint8, device=dev)
         self.ws_disp = torch.empty(max(B.moe_dispatch_workspace_size(T, k, E), 256), dtype=torch.uint8, device=dev)
-        self.ws_ffn = torch.empty(max(B.moe_expert_ffn_workspace_size("swiglu", dt, E, C, F), 256),
+        self.ws_ffn = torch.empty(max(B.moe_expert_ffn_workspace_size("swiglu", dt, E, C, H, F, H), 256),
                                   dtype=torch.uint8, device=dev)
-        self.ws_shared = (torch.empty(max(B.moe_expert_ffn_workspace_size("swiglu", dt, 1, T, F_shared), 256),
+        self.ws_shared = (torch.empty(max(B.moe_expert_ffn_workspace_size("swiglu", dt, 1, T, H, F_shared, H), 256),
                                       dtype=torch.uint8, device=dev) if F_shared else None)
         self.side = None  # stream for the shared expert, created on first use
 

@@ -92,6 +92,8 @@ def test_host_validation_before_any_launch():
 def test_workspace_sizes():
     assert moe.binding.moe_dispatch_workspace_size(16384, 8, 256) >= 32 * 256 * 4
     assert moe.binding.moe_route_workspace_size(65536, 2048, 256, B.MOE_BF16, True, "DE") > 65536 * 256 * 4
-    assert moe.binding.moe_expert_ffn_workspace_size("linear", B.MOE_BF16, 8, 16, 32) == 0
-    assert moe.binding.moe_expert_ffn_workspace_size("swiglu", B.MOE_BF16, 256, 640, 512) >= 256 * 640 * 512 * 2
+    assert moe.binding.moe_expert_ffn_workspace_size("linear", B.MOE_BF16, 8, 16, 64, 32, 64) == 0
+    assert moe.binding.moe_expert_ffn_workspace_size("swiglu", B.MOE_BF16, 256, 640, 2048, 512, 2048) >= 256 * 640 * 512 * 2
+    # fp32 adds the split-tf32 operands: hi and lo of rows and weights, K rounded up to 32
+    assert moe.binding.moe_expert_ffn_workspace_size("linear", B.MOE_F32, 8, 16, 64, 0, 48) >= 2 * 4 * (8 * 16 * 64 + 8 * 48 * 64)
     assert moe.binding.moe_backward_workspace_size(64, 256, 1024, 1024) >= 2 * 64 * 256 * 1024 * 4
