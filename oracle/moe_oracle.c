@@ -421,6 +421,127 @@ void oracle_backward_linear(const double* dy, const double* x, const double* s,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Backward of the SwiGLU-expert layer with the kept mask constant (the        */
+/* [P1] section 1 item 7 backward carried over to [P3] swiglu_expert).  For a   */
+/* kept assignment of token t to expert e with gate g:                          */
+/*   a = x Wg_e, b = x Wu_e, h = silu(a) * b, o = h Wd_e,  y_t += g o           */
+/* and for the upstream gradient dy_t:                                          */
+/*   dgate = dy_t . o,  do = g dy_t,  dh = do Wd_e^T,                           */
+/*   da = dh * b * silu'(a),  db = dh * silu(a),  silu'(a) = s (1 + a (1 - s)), */
+/*   s = sigmoid(a);  dWd_e += h^T do,  dWg_e += x^T da,  dWu_e += x^T db,      */
+/*   dx_t += da Wg_e^T + db Wu_e^T  (+ dy_t with the residual base).           */
+/* dlogits follows from dgate exactly as in the linear case.  Weights in the    */
+/* x@W layout: Wg, Wu (E, D, F); Wd (E, F, N).                                  */
+/* ------------------------------------------------------------------------ */
+
+/* One kept assignment: recompute the forward quantities and the gradients of
+ * the expert's hidden layer.  a, b, h, da, db: (F); o: (N). */
+static void swiglu_assignment(const double* xrow, const double* dyrow, double g, const double* Wge,
+                              const double* Wue, const double* Wde, int64_t D, int64_t F, int64_t N,
+                              double* a, double* b, double* h, double* o, double* da, double* db,
+                              double* dgate_out) {
+    for (int64_t f = 0; f < F; ++f) { a[f] = 0.0; b[f] = 0.0; }
+    for (int64_t d = 0; d < D; ++d)
+        for (int64_t f = 0; f < F; ++f) {
+            a[f] += xrow[d] * Wge[d * F + f];
+            b[f] += xrow[d] * Wue[d * F + f];
+        }
+    for (int64_t f = 0; f < F; ++f) h[f] = a[f] * sigmoid_stable(a[f]) * b[f];
+    for (int64_t n = 0; n < N; ++n) o[n] = 0.0;
+    for (int64_t f = 0; f < F; ++f)
+        for (int64_t n = 0; n < N; ++n) o[n] += h[f] * Wde[f * N + n];
+    double dg = 0.0;
+    for (int64_t n = 0; n < N; ++n) dg += dyrow[n] * o[n];
+    *dgate_out = dg;
+    for (int64_t f = 0; f < F; ++f) {
+        double dh = 0.0;
+        for (int64_t n = 0; n < N; ++n) dh += g * dyrow[n] * Wde[f * N + n];
+        const double sg = sigmoid_stable(a[f]);
+        da[f] = dh * b[f] * sg * (1.0 + a[f] * (1.0 - sg));
+        db[f] = dh * a[f] * sg;
+    }
+}
+
+void oracle_backward_swiglu(const double* dy, const double* x, const double* s,
+                            const int64_t* selected, const uint8_t* kept, const double* gates,
+                            const double* Wg, const double* Wu, const double* Wd, int64_t T,
+                            int32_t k, int32_t E, int64_t D, int64_t F, int64_t N,
+                            int use_residual, double aux_coef, int normalize_by_k,
+                            const int64_t* counts, double* dx, double* dWg, double* dWu,
+                            double* dWd, double* dlogits, double* dgate) {
+    /* per token: dgate, dlogits, dx */
+    OMP_FOR
+    for (int64_t t = 0; t < T; ++t) {
+        double* a = (double*)malloc((size_t)(5 * F + N) * sizeof(double));
+        double *b = a + F, *h = b + F, *da = h + F, *db = da + F, *o = db + F;
+        for (int64_t d = 0; d < D; ++d) dx[t * D + d] = use_residual ? dy[t * N + d] : 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            dgate[t * k + j] = 0.0;
+            if (!kept[t * k + j]) continue;
+            const int64_t e = selected[t * k + j];
+            const double* Wge = Wg + e * D * F;
+            const double* Wue = Wu + e * D * F;
+            swiglu_assignment(x + t * D, dy + t * N, gates[t * k + j], Wge, Wue, Wd + e * F * N, D, F, N,
+                              a, b, h, o, da, db, &dgate[t * k + j]);
+            for (int64_t d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int64_t f = 0; f < F; ++f) acc += da[f] * Wge[d * F + f] + db[f] * Wue[d * F + f];
+                dx[t * D + d] += acc;
+            }
+        }
+        free(a);
+        for (int32_t e = 0; e < E; ++e) dlogits[t * E + e] = 0.0;
+        double gdot = 0.0;
+        for (int32_t j = 0; j < k; ++j) gdot += gates[t * k + j] * dgate[t * k + j];
+        for (int32_t i = 0; i < k; ++i)
+            dlogits[t * E + selected[t * k + i]] += gates[t * k + i] * (dgate[t * k + i] - gdot);
+        if (aux_coef != 0.0) {
+            double kn = normalize_by_k ? (double)k : 1.0;
+            const double* st = s + t * E;
+            double mx = st[0];
+            for (int32_t e = 1; e < E; ++e) if (st[e] > mx) mx = st[e];
+            double den = 0.0;
+            for (int32_t e = 0; e < E; ++e) den += exp(st[e] - mx);
+            double cp = 0.0;
+            for (int32_t e = 0; e < E; ++e) cp += (double)counts[e] * (exp(st[e] - mx) / den);
+            double scale = aux_coef * (double)E / ((double)T * (double)T * kn);
+            for (int32_t e = 0; e < E; ++e) {
+                double p = exp(st[e] - mx) / den;
+                dlogits[t * E + e] += scale * p * ((double)counts[e] - cp);
+            }
+        }
+    }
+    /* weight gradients, one expert per iteration */
+    OMP_FOR
+    for (int32_t e = 0; e < E; ++e) {
+        double* a = (double*)malloc((size_t)(5 * F + N) * sizeof(double));
+        double *b = a + F, *h = b + F, *da = h + F, *db = da + F, *o = db + F;
+        double* dWge = dWg + (int64_t)e * D * F;
+        double* dWue = dWu + (int64_t)e * D * F;
+        double* dWde = dWd + (int64_t)e * F * N;
+        for (int64_t i = 0; i < D * F; ++i) { dWge[i] = 0.0; dWue[i] = 0.0; }
+        for (int64_t i = 0; i < F * N; ++i) dWde[i] = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            for (int32_t j = 0; j < k; ++j) {
+                if (!kept[t * k + j] || selected[t * k + j] != e) continue;
+                const double g = gates[t * k + j];
+                double unused;
+                swiglu_assignment(x + t * D, dy + t * N, g, Wg + (int64_t)e * D * F, Wu + (int64_t)e * D * F,
+                                  Wd + (int64_t)e * F * N, D, F, N, a, b, h, o, da, db, &unused);
+                for (int64_t f = 0; f < F; ++f)
+                    for (int64_t n = 0; n < N; ++n) dWde[f * N + n] += h[f] * g * dy[t * N + n];
+                for (int64_t d = 0; d < D; ++d)
+                    for (int64_t f = 0; f < F; ++f) {
+                        dWge[d * F + f] += x[t * D + d] * da[f];
+                        dWue[d * F + f] += x[t * D + d] * db[f];
+                    }
+            }
+        }
+        free(a);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Dense reference with the explicit (T,E,C) tensors ([P1] section 1 item 5:   */
 /* dispatch_mask (T,E,C) bool and combine_weights (T,E,C), zero on dropped     */
 /* slots; section 2: M = combine.sum(axis=2), xe = x @ W for every (t,e),      */

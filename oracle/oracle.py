@@ -63,6 +63,8 @@ def _load():
         lib.oracle_z_loss.argtypes = [_D, i64, i32]
         lib.oracle_backward_linear.argtypes = [_D, _D, _D, _I64, _U8, _D, _D, i64, i32, i32, i64, i64,
                                                ctypes.c_int, dbl, ctypes.c_int, _I64, _D, _D, _D, _D]
+        lib.oracle_backward_swiglu.argtypes = [_D, _D, _D, _I64, _U8, _D, _D, _D, _D, i64, i32, i32, i64, i64,
+                                               i64, ctypes.c_int, dbl, ctypes.c_int, _I64, _D, _D, _D, _D, _D, _D]
         lib.oracle_combine_precomputed.argtypes = [_D, i64, i32, i64, _I64, _U8, _D, i32, ctypes.c_int,
                                                    _D, _D]
         lib.oracle_combine_slots.argtypes = [_D, i64, i32, i64, i64, _I64, _I64, _U8, _D, i32,
@@ -293,6 +295,37 @@ def backward_linear(dy, x, s, selected, kept, gates, W, use_residual: bool = Tru
                                    float(aux_coef), int(bool(normalize_by_k)), _p(cnt, _I64),
                                    _p(dx, _D), _p(dW, _D), _p(dl, _D), _p(dg, _D))
     return dx, dW, dl, dg
+
+
+def backward_swiglu(dy, x, s, selected, kept, gates, Wg, Wu, Wd, use_residual: bool = False,
+                    aux_coef: float = 0.0, normalize_by_k: bool = True, counts=None):
+    """Backward of the SwiGLU-expert layer with the kept mask constant.
+
+    ``Wg, Wu`` are ``(E, D, F)``, ``Wd`` is ``(E, F, N)`` (pages' x@W layout).
+    Returns ``(dx, dWg, dWu, dWd, dlogits, dgate)``.
+    """
+    dy, x, s = _f64(dy), _f64(x), _f64(s)
+    Wg, Wu, Wd = _f64(Wg), _f64(Wu), _f64(Wd)
+    T, D = x.shape
+    E = s.shape[1]
+    F, N = Wg.shape[2], Wd.shape[2]
+    sel = _i64(selected).reshape(T, -1)
+    k = sel.shape[1]
+    kp = _u8(kept).reshape(T, k)
+    g = _f64(gates).reshape(T, k)
+    cnt = _i64(counts if counts is not None else np.bincount(sel.ravel(), minlength=E))
+    dx = np.empty((T, D), np.float64)
+    dWg = np.empty((E, D, F), np.float64)
+    dWu = np.empty((E, D, F), np.float64)
+    dWd = np.empty((E, F, N), np.float64)
+    dl = np.empty((T, E), np.float64)
+    dg = np.empty((T, k), np.float64)
+    _load().oracle_backward_swiglu(_p(dy, _D), _p(x, _D), _p(s, _D), _p(sel, _I64), _p(kp, _U8), _p(g, _D),
+                                   _p(Wg, _D), _p(Wu, _D), _p(Wd, _D), T, k, E, D, F, N,
+                                   int(bool(use_residual)), float(aux_coef), int(bool(normalize_by_k)),
+                                   _p(cnt, _I64), _p(dx, _D), _p(dWg, _D), _p(dWu, _D), _p(dWd, _D),
+                                   _p(dl, _D), _p(dg, _D))
+    return dx, dWg, dWu, dWd, dl, dg
 
 
 def combine_precomputed(u, selected, kept, gates, base=None) -> np.ndarray:

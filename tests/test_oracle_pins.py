@@ -422,6 +422,87 @@ def test_backward_top1_logit_gradient_is_zero():
     assert np.abs(dl).max() < 1e-12
 
 
+def _loss_swiglu(x, s, w, dy, sel0, kept, k, aux_coef, counts0, residual):
+    probs, sel, gates, _, psum = O.route(s, k)
+    assert (sel == sel0).all(), "perturbation changed the top-k decision"
+    y = O.layer_rows("swiglu", x, sel, kept, gates, w, base_kind="input" if residual else "zero")
+    _, _, aux = O.aux(counts0, psum, x.shape[0], k, normalize_by_k=True)
+    return float((dy * y).sum() + aux_coef * aux)
+
+
+@pytest.mark.parametrize("aux_coef,residual", [(0.0, False), (0.29, True)])
+def test_backward_swiglu_finite_differences(aux_coef, residual):
+    # The module-7 SwiGLU expert under the numpy-layer page's backward rules:
+    # every analytic gradient against central differences of y . dy (+ aux).
+    ver = _golden("numpy_layer_verification.json")
+    rng = np.random.default_rng(21)
+    T, D, F, E, k = 7, 4, 3, 4, 2
+    x = rng.standard_normal((T, D))
+    s = rng.standard_normal((T, E))
+    w = {"w1": rng.standard_normal((E, D, F)) * 0.7, "w3": rng.standard_normal((E, D, F)) * 0.7,
+         "w2": rng.standard_normal((E, F, D)) * 0.7}
+    dy = rng.standard_normal((T, D))
+    C = 3  # forces drops
+    out = O.forward("swiglu", x, s, k, C, w, base_kind="input" if residual else "zero")
+    sel, kept, counts = out["selected"], out["kept"], out["counts"]
+    assert (~kept).any()
+    dx, dWg, dWu, dWd, dl, dg = O.backward_swiglu(dy, x, s, sel, kept, out["gates"], w["w1"], w["w3"], w["w2"],
+                                                  use_residual=residual, aux_coef=aux_coef, counts=counts)
+    h = 1e-6
+
+    def fd(arr):
+        g = np.zeros_like(arr)
+        it = np.nditer(arr, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            a0 = arr[i]
+            arr[i] = a0 + h
+            lp = _loss_swiglu(x, s, w, dy, sel, kept, k, aux_coef, counts, residual)
+            arr[i] = a0 - h
+            lm = _loss_swiglu(x, s, w, dy, sel, kept, k, aux_coef, counts, residual)
+            arr[i] = a0
+            g[i] = (lp - lm) / (2 * h)
+        return g
+
+    bound = 10 * max(ver["backward_vs_finite_difference_max_err"].values())
+    assert np.abs(fd(x) - dx).max() < bound
+    assert np.abs(fd(s) - dl).max() < bound
+    assert np.abs(fd(w["w1"]) - dWg).max() < bound
+    assert np.abs(fd(w["w3"]) - dWu).max() < bound
+    assert np.abs(fd(w["w2"]) - dWd).max() < bound
+    assert (dg[~kept] == 0).all()
+    # dgate is dy . (ungated expert output) on kept assignments
+    t, j = np.argwhere(kept)[0]
+    o = O.expert_rows("swiglu", x, [t], [sel[t, j]], w)[0]
+    assert math.isclose(dg[t, j], float(dy[t] @ o), rel_tol=1e-12)
+
+
+def test_backward_swiglu_down_gradient_closed_form_and_top1():
+    # With one hidden unit (F = 1) the down-projection gradient has a closed
+    # form: dWd_e = sum over kept tokens of e of g * silu(a) * b * dy, with
+    # a = x . wg_e and b = x . wu_e, written out here by hand.
+    rng = np.random.default_rng(22)
+    T, D, E, k = 5, 3, 2, 1
+    x = rng.standard_normal((T, D))
+    s = rng.standard_normal((T, E))
+    w = {"w1": rng.standard_normal((E, D, 1)), "w3": rng.standard_normal((E, D, 1)),
+         "w2": rng.standard_normal((E, 1, D))}
+    dy = rng.standard_normal((T, D))
+    out = O.forward("swiglu", x, s, k, T, w)
+    sel, kept, gates = out["selected"], out["kept"], out["gates"]
+    _, _, _, dWd, dl, _ = O.backward_swiglu(dy, x, s, sel, kept, gates, w["w1"], w["w3"], w["w2"])
+    want = np.zeros((E, 1, D))
+    for t in range(T):
+        e = sel[t, 0]
+        a = x[t] @ w["w1"][e][:, 0]
+        b = x[t] @ w["w3"][e][:, 0]
+        hval = a / (1 + math.exp(-a)) * b
+        want[e, 0] += gates[t, 0] * hval * dy[t]
+    np.testing.assert_allclose(dWd, want, rtol=1e-12, atol=1e-14)
+    # k = 1: the renormalised gate is identically 1, so the logits get no gradient
+    assert np.abs(dl).max() < 1e-12
+
+
 # --------------------------------------------------------------------------
 # negative cases (module-7 negative tests)
 # --------------------------------------------------------------------------
