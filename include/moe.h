@@ -370,7 +370,8 @@ MOE_API int moe_aux_stats(const int32_t* counts, const float* prob_sum, int64_t 
 /*
  * moe_backward -- backward of the linear-expert layer, the kept mask and the
  * drops held constant ([P1] section 1 item 7 and section 2 moe_backward).
- * fp32 only in this build (kind must be MOE_FFN_LINEAR, dtype MOE_F32).
+ * fp32 linear experts (kind MOE_FFN_LINEAR, dtype MOE_F32); the bf16 SwiGLU
+ * experts have moe_backward_swiglu.
  *
  * With out_{t,j} = x_t W_e^T (e = selected[t,j], kept) and the loss
  * L = sum_t dy_t . y_t + aux_coef * aux:
@@ -401,6 +402,43 @@ MOE_API int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, con
                  int normalize_by_k, const int32_t* counts, void* dx, void* dW, float* dlogits,
                  float* dgate, int32_t* dev_status, void* workspace, size_t workspace_bytes,
                  moe_stream_t stream);
+
+/*
+ * moe_backward_swiglu -- backward of the SwiGLU-expert layer ([P3]
+ * swiglu_expert, [P3] EducationalMoE routed experts) under the same rules as
+ * moe_backward: kept mask and drops constant, gates = softmax of the selected
+ * logits.  bf16 activations and weights, fp32 accumulation; weight gradients
+ * in fp32.  For a kept (t,j) -> e with a = x_t Wg_e^T, b = x_t Wu_e^T,
+ * h = silu(a) * b, o = h Wd_e^T:
+ *   dgate[t,j] = dy_t . o        (o read from the forward's ybuf)
+ *   dlogits    as in moe_backward
+ *   do = gate dy_t,  dh = do Wd_e,  s = sigmoid(a),
+ *   da = dh * b * s * (1 + a (1 - s)),  db = dh * a * s
+ *   dw_down[e] += do^T h         (E, H, F)
+ *   dw_gate[e] += da^T x_t       (E, F, H)
+ *   dw_up[e]   += db^T x_t       (E, F, H)
+ *   dx[t]      = [dy_t] + sum_kept (da Wg_e + db Wu_e)     (T, H), bf16
+ * a and b are recomputed from xbuf; h, da, db are rounded to bf16 before the
+ * weight-gradient and dx products.
+ *
+ * Arguments (device): dy bf16 (T, H); logits fp32 (T, E); selected int64,
+ *   gates fp32, slot int64 (T, k); used int32 (E); xbuf bf16 (E, C, H) and
+ *   ybuf bf16 (E, C, H) from the forward; w_gate, w_up bf16 (E, F, H);
+ *   w_down bf16 (E, H, F); counts int32 (E) when aux_coef != 0.
+ *   H and F multiples of 8, k <= 64, dtype MOE_BF16 (else MOE_ERR_UNSUPPORTED).
+ *   Outputs: dx bf16 (T, H); dw_gate, dw_up fp32 (E, F, H); dw_down fp32
+ *   (E, H, F); dlogits fp32 (T, E); dgate fp32 (T, k).
+ *   workspace >= moe_backward_swiglu_workspace_size(E, C, H, F) bytes.
+ */
+MOE_API size_t moe_backward_swiglu_workspace_size(int32_t E, int64_t C, int64_t H, int64_t F);
+MOE_API int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float* logits, const int64_t* selected,
+                                const float* gates, const int64_t* slot, const int32_t* used, const void* xbuf,
+                                const void* ybuf, const void* w_gate, const void* w_up, const void* w_down,
+                                int64_t T, int32_t k, int32_t E, int64_t C, int64_t H, int64_t F, int use_residual,
+                                float aux_coef, int normalize_by_k, const int32_t* counts, void* dx,
+                                float* dw_gate, float* dw_up, float* dw_down, float* dlogits, float* dgate,
+                                int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                                moe_stream_t stream);
 
 /*
  * moe_transpose_weights -- convert expert matrices from the pages' x @ W

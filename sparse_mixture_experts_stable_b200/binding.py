@@ -37,7 +37,8 @@ EXPORTED = [
     "moe_dispatch_workspace_size", "moe_dispatch", "moe_expert_ffn_workspace_size", "moe_expert_ffn",
     "moe_combine", "moe_aux_stats", "moe_backward_workspace_size", "moe_backward", "moe_transpose_weights",
     "moe_clear_status", "moe_read_status", "moe_dispatch_static_max_state_bytes", "moe_dispatch_static",
-    "moe_route_ex", "moe_renormalize_kept_gates", "moe_expert_ffn_gathered",
+    "moe_route_ex", "moe_renormalize_kept_gates", "moe_expert_ffn_gathered", "moe_backward_swiglu_workspace_size",
+    "moe_backward_swiglu",
 ]
 SCORING = {"softmax": 0, "sigmoid": 1}
 
@@ -90,6 +91,11 @@ def lib():
                                   _vp, _i64, _vp, _i64, ctypes.c_int, _vp, _vp]
         L.moe_aux_stats.argtypes = [_vp, _vp, _i64, _i32, _i32, ctypes.c_int, _f32, _vp, _vp, ctypes.c_int, _vp,
                                     _vp]
+        L.moe_backward_swiglu_workspace_size.restype = _sz
+        L.moe_backward_swiglu_workspace_size.argtypes = [_i32, _i64, _i64, _i64]
+        L.moe_backward_swiglu.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+                                          _i32, _i32, _i64, _i64, _i64, ctypes.c_int, _f32, ctypes.c_int, _vp, _vp,
+                                          _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
         L.moe_backward_workspace_size.restype = _sz
         L.moe_backward_workspace_size.argtypes = [_i32, _i64, _i64, _i64]
         L.moe_backward.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -405,6 +411,38 @@ def moe_backward(dy, x, logits, selected, gates_f32, slot, used, token_of_slot, 
                             _p(dW), _p(dl), _p(dg), _p(dev_status), _p(ws), ws.numel(), _stream(stream))
     _check("moe_backward", rc)
     return dx, dW, dl, dg
+
+
+def moe_backward_swiglu_workspace_size(E: int, C: int, H: int, F: int) -> int:
+    return int(lib().moe_backward_swiglu_workspace_size(E, C, H, F))
+
+
+def moe_backward_swiglu(dy, logits, selected, gates_f32, slot, used, xbuf, ybuf, w_gate, w_up, w_down, C: int,
+                        use_residual: bool = False, aux_coef: float = 0.0, normalize_by_k: bool = True, counts=None,
+                        dev_status=None, workspace=None, stream=None):
+    """Backward of the bf16 SwiGLU-expert layer.
+
+    Returns (dx bf16 (T,H), dw_gate fp32 (E,F,H), dw_up fp32 (E,F,H), dw_down fp32 (E,H,F),
+    dlogits fp32 (T,E), dgate fp32 (T,k)).
+    """
+    dev = _dev(dy)
+    T, H = dy.shape
+    E, F = w_gate.shape[0], w_gate.shape[1]
+    k = selected.shape[1]
+    dx = torch.empty(T, H, dtype=dy.dtype, device=dev)
+    dwg = torch.empty(E, F, H, dtype=torch.float32, device=dev)
+    dwu = torch.empty(E, F, H, dtype=torch.float32, device=dev)
+    dwd = torch.empty(E, H, F, dtype=torch.float32, device=dev)
+    dl = torch.empty(T, E, dtype=torch.float32, device=dev)
+    dg = torch.empty(T, k, dtype=torch.float32, device=dev)
+    ws = _workspace(moe_backward_swiglu_workspace_size(E, C, H, F), dev, workspace)
+    rc = lib().moe_backward_swiglu(_dt(dy), _p(dy), _p(logits), _p(selected), _p(gates_f32), _p(slot), _p(used),
+                                   _p(xbuf), _p(ybuf), _p(w_gate), _p(w_up), _p(w_down), T, k, E, C, H, F,
+                                   int(bool(use_residual)), float(aux_coef), int(bool(normalize_by_k)), _p(counts),
+                                   _p(dx), _p(dwg), _p(dwu), _p(dwd), _p(dl), _p(dg), _p(dev_status), _p(ws),
+                                   ws.numel(), _stream(stream))
+    _check("moe_backward_swiglu", rc)
+    return dx, dwg, dwu, dwd, dl, dg
 
 
 def moe_transpose_weights(src: torch.Tensor, stream=None) -> torch.Tensor:

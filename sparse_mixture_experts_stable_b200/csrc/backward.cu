@@ -4,10 +4,12 @@
 //   3. dW[e]   = dybuf_e^T xbuf_e        split-tf32 tensor-core GEMM, K = used[e] rows
 //   4. dxbuf_e = dybuf_e W_e             split-tf32 tensor-core GEMM, M = used[e] rows
 //   5. dx[t]   = [dy[t]] + sum_kept dxbuf[e, slot]   deterministic combine
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
 #include "common.cuh"
+#include "tc_gemm.cuh"
 #include "f32_gemm.cuh"
 #include "tc_tf32.cuh"
 #include "util_kernels.cuh"
@@ -17,8 +19,9 @@ namespace {
 
 constexpr int kWarps = 8;
 
+template <typename In>
 __global__ void __launch_bounds__(kWarps * 32)
-    dgate_dlogits_kernel(const float* __restrict__ dy, int64_t Dout, const float* __restrict__ ybuf,
+    dgate_dlogits_kernel(const In* __restrict__ dy, int64_t Dout, const In* __restrict__ ybuf,
                          const float* __restrict__ logits, const int64_t* __restrict__ selected,
                          const float* __restrict__ gates, const int64_t* __restrict__ slot, int64_t T, int k, int E,
                          int64_t C, float aux_coef, float kn, const int32_t* __restrict__ counts,
@@ -26,7 +29,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * kWarps + warp;
     if (t >= T) return;
-    const float* dyr = dy + t * Dout;
+    const In* dyr = dy + t * Dout;
     // dgate_j (all lanes end up with every dgate_j through the warp sums)
     float gdot = 0.f;
     float my_dg0 = 0.f, my_dg1 = 0.f;  // dgate for j = lane, lane + 32
@@ -38,9 +41,9 @@ __global__ void __launch_bounds__(kWarps * 32)
             if (e < 0 || e >= E || s >= C) {
                 if (lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
             } else {
-                const float* yr = ybuf + (e * C + s) * Dout;
+                const In* yr = ybuf + (e * C + s) * Dout;
                 float part = 0.f;
-                for (int64_t n = lane; n < Dout; n += 32) part = fmaf(dyr[n], yr[n], part);
+                for (int64_t n = lane; n < Dout; n += 32) part = fmaf(to_f32(dyr[n]), to_f32(yr[n]), part);
                 dg = warp_sum(part);
             }
         }
@@ -148,7 +151,7 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
     const size_t split_bytes = workspace_bytes - (size_t)(split - ws);
 
     const unsigned grid = (unsigned)((T + kWarps - 1) / kWarps);
-    dgate_dlogits_kernel<<<grid, kWarps * 32, 0, stream>>>(
+    dgate_dlogits_kernel<float><<<grid, kWarps * 32, 0, stream>>>(
         static_cast<const float*>(dy), Dout, static_cast<const float*>(ybuf), logits, selected, gates, slot, T, k, E,
         C, aux_coef, normalize_by_k ? (float)k : 1.0f, counts, dlogits, dgate, dev_status);
     int rc = launch_status();
@@ -212,4 +215,253 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
 
     return combine_rows(dxbuf, selected, slot, nullptr, MOE_F32, T, k, E, C, D, use_residual ? dy : nullptr, D, dx, D,
                         MOE_F32, dev_status, stream);
+}
+
+// ---------------------------------------------------------------------------
+// moe_backward_swiglu: bf16 SwiGLU experts, the kept mask held constant.
+//   1. dgate / dlogits                       as above, on bf16 rows
+//   2. dybuf[e,c] = gate * dy[token]         scaled gather (bf16)
+//   3. [a | b] = xbuf [Wg; Wu]^T             two tensor-core GEMMs, fp32 out
+//   4. dh = dybuf Wd                         tensor-core GEMM on Wd^T, fp32 out
+//   5. h, da, db from (a, b, dh)             elementwise (silu and its derivative)
+//   6. dWd = dybuf^T h, dWg = da^T xbuf, dWu = db^T xbuf
+//                                            tensor-core GEMMs on zero-padded,
+//                                            token-transposed operands, fp32 out
+//   7. dxbuf = [da | db] [Wg; Wu]            tensor-core GEMM on the transposed
+//                                            stacked weights, bf16 out
+//   8. dx[t] = [dy[t]] + sum_kept dxbuf[e, slot]
+// All GEMMs are the K-major tcgen05 kernel; operands that the products need
+// with the token index as K are transposed (with zeros past used[e]) first.
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+// dst[g][c][r] = r < valid[g] ? src[g][r][c] : 0   for r < Rp, c < Cc
+// (valid = NULL: every r < R is valid).  bf16; 32 x 32 tiles through shared memory.
+__global__ void __launch_bounds__(256)
+    transpose_valid_kernel(const __nv_bfloat16* __restrict__ src, int64_t lds, int64_t sgs, int64_t R, int64_t Cc,
+                           const int32_t* __restrict__ valid, int64_t Rp, __nv_bfloat16* __restrict__ dst,
+                           int64_t ldd, int64_t dgs) {
+    __shared__ __nv_bfloat16 tile[32][34];
+    const int g = blockIdx.z;
+    int64_t Rv = R;
+    if (valid) {
+        const int64_t v = valid[g];
+        Rv = v < 0 ? 0 : (v < R ? v : R);
+    }
+    const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+    const __nv_bfloat16* s = src + g * sgs;
+    __nv_bfloat16* d = dst + g * dgs;
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int64_t r = r0 + i, c = c0 + threadIdx.x;
+        tile[i][threadIdx.x] = (r < Rv && c < Cc) ? s[r * lds + c] : __float2bfloat16_rn(0.f);
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int64_t c = c0 + i, r = r0 + threadIdx.x;
+        if (c < Cc && r < Rp) d[c * ldd + r] = tile[threadIdx.x][i];
+    }
+}
+
+int transpose_valid(const __nv_bfloat16* src, int64_t lds, int64_t sgs, int G, int64_t R, int64_t Cc,
+                    const int32_t* valid, int64_t Rp, __nv_bfloat16* dst, int64_t ldd, int64_t dgs,
+                    cudaStream_t stream) {
+    MOE_REQUIRE(G <= 65535 && (Rp + 31) / 32 <= 65535, MOE_ERR_UNSUPPORTED);
+    const dim3 grid((unsigned)((Cc + 31) / 32), (unsigned)((Rp + 31) / 32), (unsigned)G), block(32, 8);
+    transpose_valid_kernel<<<grid, block, 0, stream>>>(src, lds, sgs, R, Cc, valid, Rp, dst, ldd, dgs);
+    return launch_status();
+}
+
+// h, da, db from a, b (ab rows: [a | b], fp32) and dh (fp32), for c < used[e]:
+//   s = sigmoid(a), h = a s b, da = dh b s (1 + a (1 - s)), db = dh a s.
+__global__ void swiglu_bwd_elem_kernel(const float* __restrict__ ab, const float* __restrict__ dh,
+                                       const int32_t* __restrict__ used, int64_t C, int64_t F,
+                                       __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ dab) {
+    const int e = blockIdx.y;
+    const int64_t u = used[e] < 0 ? 0 : (used[e] < C ? used[e] : C);
+    const int64_t n = u * F;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t c = i / F, f = i - c * F;
+        const int64_t row = (int64_t)e * C + c;
+        const float a = ab[row * 2 * F + f], b = ab[row * 2 * F + F + f];
+        const float g = dh[row * F + f];
+        const float s = 1.0f / (1.0f + expf(-a));
+        h[row * F + f] = __float2bfloat16_rn(a * s * b);
+        dab[row * 2 * F + f] = __float2bfloat16_rn(g * b * s * (1.0f + a * (1.0f - s)));
+        dab[row * 2 * F + F + f] = __float2bfloat16_rn(g * a * s);
+    }
+}
+
+// Grouped bf16 GEMM out[g] (M x N, fp32 or bf16) = A[g] (M x K) B[g]^T, K-major operands.
+int gemm(const void* a, int64_t lda, int64_t a_rows_total, int64_t a_rows_per_group, const void* b, int64_t ldb,
+         int64_t b_rows_total, int64_t b_rows_per_group, int G, int64_t M, int64_t N, int64_t K, const int32_t* rows,
+         void* out, int64_t ldo, int64_t out_rows_per_group, int epilogue, int32_t* status, cudaStream_t stream) {
+    TcGemmProblem p{};
+    p.a = a;
+    p.lda = lda;
+    p.a_rows_total = a_rows_total;
+    p.a_rows_per_group = a_rows_per_group;
+    p.b = b;
+    p.ldb = ldb;
+    p.b_rows_total = b_rows_total;
+    p.b_rows_per_group = b_rows_per_group;
+    p.G = G;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.rows = rows;
+    p.out = out;
+    p.ldo = ldo;
+    p.out_rows_per_group = out_rows_per_group;
+    p.epilogue = epilogue;
+    p.status = status;
+    return tc_gemm_run(p, stream);
+}
+
+struct SwigluBwdWs {
+    size_t dybuf, ab, dh, h, dab, wdT, wguT, dybufT, hT, dabT, xbufT, dxbuf, total;
+    int64_t Cp;
+};
+
+SwigluBwdWs swiglu_bwd_layout(int32_t E, int64_t C, int64_t H, int64_t F) {
+    SwigluBwdWs w{};
+    w.Cp = (C + 7) / 8 * 8;  // token count padded for 16-byte TMA rows
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += align_up(bytes, 1024);
+        return o;
+    };
+    w.dybuf = take((size_t)E * C * H * 2);
+    w.ab = take((size_t)E * C * 2 * F * 4);
+    w.dh = take((size_t)E * C * F * 4);
+    w.h = take((size_t)E * C * F * 2);
+    w.dab = take((size_t)E * C * 2 * F * 2);
+    w.wdT = take((size_t)E * F * H * 2);
+    w.wguT = take((size_t)E * H * 2 * F * 2);
+    w.dybufT = take((size_t)E * H * w.Cp * 2);
+    w.hT = take((size_t)E * F * w.Cp * 2);
+    w.dabT = take((size_t)E * 2 * F * w.Cp * 2);
+    w.xbufT = take((size_t)E * H * w.Cp * 2);
+    w.dxbuf = take((size_t)E * C * H * 2);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" size_t moe_backward_swiglu_workspace_size(int32_t E, int64_t C, int64_t H, int64_t F) {
+    if (E < 1 || C < 1 || H < 1 || F < 1) return 256;
+    return swiglu_bwd_layout(E, C, H, F).total;
+}
+
+extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float* logits, const int64_t* selected,
+                                   const float* gates, const int64_t* slot, const int32_t* used, const void* xbuf,
+                                   const void* ybuf, const void* w_gate, const void* w_up, const void* w_down,
+                                   int64_t T, int32_t k, int32_t E, int64_t C, int64_t H, int64_t F, int use_residual,
+                                   float aux_coef, int normalize_by_k, const int32_t* counts, void* dx,
+                                   float* dw_gate, float* dw_up, float* dw_down, float* dlogits, float* dgate,
+                                   int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                                   moe_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    using bf16 = __nv_bfloat16;
+    MOE_REQUIRE(dtype == MOE_BF16, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(dy && logits && selected && gates && slot && used && dx && dw_gate && dw_up && dw_down && dlogits &&
+                    dgate,
+                MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(C == 0 || (xbuf && ybuf && w_gate && w_up && w_down), MOE_ERR_INVALID_ARG);  // unread when C == 0
+    MOE_REQUIRE(T >= 1 && k >= 1 && k <= E && E >= 1 && C >= 0 && H >= 1 && F >= 1, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(k <= 64 && H % 8 == 0 && F % 8 == 0, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(aux_coef == 0.f || counts != nullptr, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(workspace && workspace_bytes >= moe_backward_swiglu_workspace_size(E, C, H, F), MOE_ERR_WORKSPACE);
+
+    const unsigned grid = (unsigned)((T + kWarps - 1) / kWarps);
+    dgate_dlogits_kernel<bf16><<<grid, kWarps * 32, 0, stream>>>(
+        static_cast<const bf16*>(dy), H, static_cast<const bf16*>(ybuf), logits, selected, gates, slot, T, k, E, C,
+        aux_coef, normalize_by_k ? (float)k : 1.0f, counts, dlogits, dgate, dev_status);
+    int rc = launch_status();
+    if (rc != MOE_OK) return rc;
+
+    if (C == 0) {  // nothing kept: no expert gradient
+        MOE_CUDA_TRY(cudaMemsetAsync(dw_gate, 0, (size_t)E * F * H * 4, stream));
+        MOE_CUDA_TRY(cudaMemsetAsync(dw_up, 0, (size_t)E * F * H * 4, stream));
+        MOE_CUDA_TRY(cudaMemsetAsync(dw_down, 0, (size_t)E * H * F * 4, stream));
+        if (use_residual)
+            MOE_CUDA_TRY(cudaMemcpyAsync(dx, dy, (size_t)T * H * 2, cudaMemcpyDeviceToDevice, stream));
+        else
+            MOE_CUDA_TRY(cudaMemsetAsync(dx, 0, (size_t)T * H * 2, stream));
+        return MOE_OK;
+    }
+
+    const SwigluBwdWs l = swiglu_bwd_layout(E, C, H, F);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    bf16* dybuf = reinterpret_cast<bf16*>(ws + l.dybuf);
+    float* ab = reinterpret_cast<float*>(ws + l.ab);
+    float* dh = reinterpret_cast<float*>(ws + l.dh);
+    bf16* h = reinterpret_cast<bf16*>(ws + l.h);
+    bf16* dab = reinterpret_cast<bf16*>(ws + l.dab);
+    bf16* wdT = reinterpret_cast<bf16*>(ws + l.wdT);
+    bf16* wguT = reinterpret_cast<bf16*>(ws + l.wguT);
+    bf16* dybufT = reinterpret_cast<bf16*>(ws + l.dybufT);
+    bf16* hT = reinterpret_cast<bf16*>(ws + l.hT);
+    bf16* dabT = reinterpret_cast<bf16*>(ws + l.dabT);
+    bf16* xbufT = reinterpret_cast<bf16*>(ws + l.xbufT);
+    bf16* dxbuf = reinterpret_cast<bf16*>(ws + l.dxbuf);
+    const int64_t Cp = l.Cp, F2 = 2 * F;
+    const bf16* xb = static_cast<const bf16*>(xbuf);
+
+    // 2. dybuf[e,c] = gate * dy[token]
+    rc = gather_rows(dy, H, T, k, selected, slot, E, C, gates, dybuf, H, MOE_BF16, dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    // 3. [a | b] = xbuf [Wg; Wu]^T  (fp32)
+    rc = gemm(xbuf, H, (int64_t)E * C, C, w_gate, H, (int64_t)E * F, F, E, C, F, H, used, ab, F2, C, TC_EPI_F32,
+              dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    rc = gemm(xbuf, H, (int64_t)E * C, C, w_up, H, (int64_t)E * F, F, E, C, F, H, used, ab + F, F2, C, TC_EPI_F32,
+              dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    // 4. dh = dybuf Wd, with Wd (E, H, F) transposed to (E, F, H)
+    rc = transpose_valid(static_cast<const bf16*>(w_down), F, H * F, E, H, F, nullptr, H, wdT, H, F * H, stream);
+    if (rc != MOE_OK) return rc;
+    rc = gemm(dybuf, H, (int64_t)E * C, C, wdT, H, (int64_t)E * F, F, E, C, F, H, used, dh, F, C, TC_EPI_F32,
+              dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    // 5. h, da, db
+    {
+        const dim3 g2((unsigned)((C * F + 255) / 256 < 1024 ? (C * F + 255) / 256 : 1024), (unsigned)E);
+        MOE_REQUIRE(E <= 65535, MOE_ERR_UNSUPPORTED);
+        swiglu_bwd_elem_kernel<<<g2, 256, 0, stream>>>(ab, dh, used, C, F, h, dab);
+        rc = launch_status();
+        if (rc != MOE_OK) return rc;
+    }
+    // 6. weight gradients over the token index: transposed operands, zeros past used[e]
+    rc = transpose_valid(dybuf, H, C * H, E, C, H, used, Cp, dybufT, Cp, H * Cp, stream);
+    if (rc != MOE_OK) return rc;
+    rc = transpose_valid(h, F, C * F, E, C, F, used, Cp, hT, Cp, F * Cp, stream);
+    if (rc != MOE_OK) return rc;
+    rc = transpose_valid(dab, F2, C * F2, E, C, F2, used, Cp, dabT, Cp, F2 * Cp, stream);
+    if (rc != MOE_OK) return rc;
+    rc = transpose_valid(xb, H, C * H, E, C, H, used, Cp, xbufT, Cp, H * Cp, stream);
+    if (rc != MOE_OK) return rc;
+    rc = gemm(dybufT, Cp, (int64_t)E * H, H, hT, Cp, (int64_t)E * F, F, E, H, F, Cp, nullptr, dw_down, F, H,
+              TC_EPI_F32, dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    rc = gemm(dabT, Cp, (int64_t)E * F2, F2, xbufT, Cp, (int64_t)E * H, H, E, F, H, Cp, nullptr, dw_gate, H, F,
+              TC_EPI_F32, dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    rc = gemm(dabT + F * Cp, Cp, (int64_t)E * F2 - F, F2, xbufT, Cp, (int64_t)E * H, H, E, F, H, Cp, nullptr, dw_up,
+              H, F, TC_EPI_F32, dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    // 7. dxbuf = [da | db] [Wg; Wu], with the stacked weights transposed to (E, H, 2F)
+    rc = transpose_valid(static_cast<const bf16*>(w_gate), H, F * H, E, F, H, nullptr, F, wguT, F2, H * F2, stream);
+    if (rc != MOE_OK) return rc;
+    rc = transpose_valid(static_cast<const bf16*>(w_up), H, F * H, E, F, H, nullptr, F, wguT + F, F2, H * F2, stream);
+    if (rc != MOE_OK) return rc;
+    rc = gemm(dab, F2, (int64_t)E * C, C, wguT, F2, (int64_t)E * H, H, E, C, H, F2, used, dxbuf, H, C, TC_EPI_BF16,
+              dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    // 8. dx
+    return combine_rows(dxbuf, selected, slot, nullptr, MOE_F32, T, k, E, C, H, use_residual ? dy : nullptr, H, dx,
+                        H, MOE_BF16, dev_status, stream);
 }

@@ -89,9 +89,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             for (int64_t v = lane; v < nv; v += 32) {
                 uint4 x = reinterpret_cast<const uint4*>(srow)[v];
                 if (scale) {
-                    float4 f = *reinterpret_cast<float4*>(&x);
-                    f.x *= g; f.y *= g; f.z *= g; f.w *= g;
-                    x = *reinterpret_cast<uint4*>(&f);
+                    T* xv = reinterpret_cast<T*>(&x);
+#pragma unroll
+                    for (int i = 0; i < EPV; ++i) xv[i] = from_f32<T>(to_f32(xv[i]) * g);
                 }
                 reinterpret_cast<uint4*>(drow)[v] = x;
             }
@@ -224,7 +224,6 @@ int gather_rows(const void* src, int64_t lds, int64_t T, int32_t k, const int64_
                 int32_t E, int64_t C, const float* scale, void* dst, int64_t D, moe_dtype dtype, int32_t* status,
                 cudaStream_t stream) {
     MOE_REQUIRE(k >= 1 && k <= 64, MOE_ERR_UNSUPPORTED);
-    MOE_REQUIRE(!(scale && dtype != MOE_F32), MOE_ERR_UNSUPPORTED);
     if (T == 0 || C == 0 || D == 0) return MOE_OK;
     const size_t es = dtype_size(dtype);
     const bool vec = aligned16(src) && aligned16(dst) && ((size_t)lds * es) % 16 == 0 && ((size_t)D * es) % 16 == 0;

@@ -12,7 +12,7 @@ int transpose_matrices(const void* src, void* dst, int64_t batches, int64_t rows
                        cudaStream_t stream);
 
 // Token-major scatter into an expert-major buffer: for every kept assignment
-// (slot[t,j] >= 0) copy src row t (times scale[t,j] if scale != NULL, fp32 only)
+// (slot[t,j] >= 0) copy src row t (times scale[t,j] if scale != NULL, in fp32)
 // into dst[(selected[t,j] * C + slot[t,j]) * D ...].  Each src row is read once.
 int gather_rows(const void* src, int64_t lds, int64_t T, int32_t k, const int64_t* selected, const int64_t* slot,
                 int32_t E, int64_t C, const float* scale, void* dst, int64_t D, moe_dtype dtype,

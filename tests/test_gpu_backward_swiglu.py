@@ -1,0 +1,92 @@
+"""moe_backward_swiglu (bf16 SwiGLU experts) against the fp64 oracle backward.
+
+The forward runs on the GPU (route on given logits, dispatch, SwiGLU experts);
+the oracle recomputes everything in fp64 from the same bf16 inputs.  Integer
+routing is exact; the gradients carry bf16 roundings of the forward output, of
+the scaled upstream rows and of h, da, db, so they are held to the bf16
+tolerance, scaled by the largest magnitude of each gradient tensor.
+"""
+import numpy as np
+import pytest
+import torch
+
+import sparse_mixture_experts_stable_b200 as moe
+from oracle import oracle as O
+from sparse_mixture_experts_stable_b200.inputs import pages_layout
+from tests.gpu_util import BF16_RTOL, DEV, assert_close, cpu, cpu64
+
+pytestmark = pytest.mark.gpu
+
+
+def _close(got, want, what):
+    scale = float(np.abs(want).max()) if want.size else 1.0
+    assert_close(got, want, BF16_RTOL, BF16_RTOL * scale, what)
+
+
+@pytest.mark.parametrize("T,H,F,E,k,cf,residual,aux", [
+    (300, 128, 96, 6, 2, 0.8, False, 0.0),   # capacity binds: drops
+    (517, 64, 48, 4, 3, 1.5, True, 0.1),     # ragged token count, residual, aux term
+    (64, 72, 40, 3, 1, 2.0, False, 0.0),     # top-1; H, F not multiples of 64
+])
+def test_backward_swiglu_matches_oracle(T, H, F, E, k, cf, residual, aux):
+    g = torch.Generator().manual_seed(T + H)
+
+    def rnd(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=g) * scale).to(torch.bfloat16)
+
+    x = rnd(T, H)
+    lg = torch.randn(T, E, generator=g)
+    wg, wu, wd = rnd(E, F, H, scale=H ** -0.5), rnd(E, F, H, scale=H ** -0.5), rnd(E, H, F, scale=F ** -0.5)
+    dy = rnd(T, H)
+    C = moe.moe_capacity(T, k, E, cf)
+
+    xd, lgd, dyd = x.to(DEV), lg.to(DEV), dy.to(DEV)
+    wgd, wud, wdd = wg.to(DEV), wu.to(DEV), wd.to(DEV)
+    r = moe.moe_route(lgd, k)
+    d = moe.moe_dispatch(r["selected"], E, C, x=xd)
+    st = moe.new_status()
+    ybuf = moe.moe_expert_ffn("swiglu", d["xbuf"], d["used"], wgd, w2=wdd, w3=wud, dev_status=st)
+    dx, dwg, dwu, dwd, dl, dg = moe.moe_backward_swiglu(
+        dyd, lgd, r["selected"], r["gates_f32"], d["slot"], d["used"], d["xbuf"], ybuf, wgd, wud, wdd, C,
+        use_residual=residual, aux_coef=aux, counts=r["counts"], dev_status=st)
+    assert moe.moe_read_status(st) == 0
+
+    s64 = cpu64(lg)
+    probs, sel, gates, counts, _ = O.route(s64, k)
+    np.testing.assert_array_equal(cpu(r["selected"]), sel)
+    disp = O.dispatch(sel, E, C)
+    kept = disp["kept"]
+    if cf < 1.0:
+        assert (~kept).any()
+    want = O.backward_swiglu(cpu64(dy), cpu64(x), s64, sel, kept, gates, pages_layout(wg), pages_layout(wu),
+                             pages_layout(wd), use_residual=residual, aux_coef=aux, counts=counts)
+    wdx, wdWg, wdWu, wdWd, wdl, wdg = want
+    _close(cpu64(dg), wdg, "dgate")
+    assert (cpu64(dg)[~kept] == 0).all()
+    _close(cpu64(dl), wdl, "dlogits")
+    _close(cpu64(dx), wdx, "dx")
+    # the oracle's weight gradients are in the x@W layout: (E, D, F) and (E, F, N)
+    _close(cpu64(dwg), wdWg.transpose(0, 2, 1), "dw_gate")
+    _close(cpu64(dwu), wdWu.transpose(0, 2, 1), "dw_up")
+    _close(cpu64(dwd), wdWd.transpose(0, 2, 1), "dw_down")
+    # an expert that received no token has an exactly zero gradient
+    for e in np.flatnonzero(disp["used"] == 0):
+        assert (cpu64(dwg)[e] == 0).all() and (cpu64(dwd)[e] == 0).all()
+
+
+def test_backward_swiglu_with_nothing_kept():
+    T, H, F, E, k = 50, 64, 32, 2, 1
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16).to(DEV)
+    lg = torch.randn(T, E, generator=g).to(DEV)
+    dy = torch.randn(T, H, generator=g).to(torch.bfloat16).to(DEV)
+    w = [torch.randn(*s, generator=g).to(torch.bfloat16).to(DEV) for s in ((E, F, H), (E, F, H), (E, H, F))]
+    r = moe.moe_route(lg, k)
+    d = moe.moe_dispatch(r["selected"], E, 0)
+    ybuf = torch.empty(E, 0, H, dtype=torch.bfloat16, device=DEV)
+    xbuf = torch.empty(E, 0, H, dtype=torch.bfloat16, device=DEV)
+    dx, dwg, dwu, dwd, dl, dg = moe.moe_backward_swiglu(dy, lg, r["selected"], r["gates_f32"], d["slot"], d["used"],
+                                                        xbuf, ybuf, *w, 0, use_residual=True)
+    assert torch.equal(dx, dy)
+    assert (dwg == 0).all() and (dwu == 0).all() and (dwd == 0).all()
+    assert (dl == 0).all() and (dg == 0).all()
