@@ -180,6 +180,28 @@ MOE_API int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D, i
                          size_t workspace_bytes, moe_stream_t stream);
 
 /*
+ * moe_router_backward -- gradients of the router scores s = x W (+ b) for a
+ * given dL/ds (dlogits, e.g. from moe_backward or moe_backward_swiglu):
+ *   dx_router[t,d] = sum_e dlogits[t,e] W(e,d)           fp32 (T, D)
+ *   dw_router      = x^T dlogits in w_router's layout     fp32 ((E,D) or (D,E))
+ *   db_router[e]   = sum_t dlogits[t,e]                   fp32 (E), fixed order
+ * ([P2] s = x . w_e is linear in x, w and b.)  The layer's full input
+ * gradient is the expert backward's dx plus dx_router.  Both products run on
+ * the tensor cores as split-tf32 (fp32 accuracy; bf16 x and w are read as
+ * they are).  Any of the three outputs may be NULL to skip it.
+ *   x          device (T, D), row stride ldx, dtype `dtype`.
+ *   w_router   device, layout `layout`, dtype `dtype`.
+ *   dlogits    device fp32 (T, E).
+ *   workspace  device, >= moe_router_backward_workspace_size(T, D, E, dtype, layout).
+ */
+MOE_API size_t moe_router_backward_workspace_size(int64_t T, int64_t D, int32_t E, moe_dtype dtype,
+                                                  moe_router_layout layout);
+MOE_API int moe_router_backward(moe_dtype dtype, const void* x, int64_t T, int64_t D, int64_t ldx,
+                                const void* w_router, moe_router_layout layout, int32_t E, const float* dlogits,
+                                float* dx_router, float* dw_router, float* db_router, int32_t* dev_status,
+                                void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/*
  * moe_renormalize_kept_gates -- [P3] dispatch_with_capacity with
  * renormalize_kept_gates: out[t,j] = gates[t,j] / sum of token t's kept gates
  * for kept assignments (slot[t,j] >= 0), 0 for dropped ones, and all zeros for

@@ -75,6 +75,33 @@ void oracle_router_logits(const double* x, const double* w_router, const double*
     }
 }
 
+/* Router backward: s = x w_router + b is linear in x, w_router and b, so for
+ * the gradient g = dL/ds (T, E):
+ *   dx[t,d] = sum_e g[t,e] w_router[d,e],  dw[d,e] = sum_t x[t,d] g[t,e],
+ *   db[e] = sum_t g[t,e].                                                     */
+void oracle_router_backward(const double* x, const double* w_router, const double* g, int64_t T,
+                            int64_t D, int32_t E, double* dx, double* dw, double* db) {
+    OMP_FOR
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (int32_t e = 0; e < E; ++e) acc += g[t * E + e] * w_router[d * E + e];
+            dx[t * D + d] = acc;
+        }
+    OMP_FOR
+    for (int64_t d = 0; d < D; ++d)
+        for (int32_t e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int64_t t = 0; t < T; ++t) acc += x[t * D + d] * g[t * E + e];
+            dw[d * E + e] = acc;
+        }
+    for (int32_t e = 0; e < E; ++e) {
+        double acc = 0.0;
+        for (int64_t t = 0; t < T; ++t) acc += g[t * E + e];
+        db[e] = acc;
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Routing.  For each token:                                                  */
 /*  - softmax over all E experts with the maximum subtracted first           */

@@ -65,6 +65,7 @@ def _load():
                                                ctypes.c_int, dbl, ctypes.c_int, _I64, _D, _D, _D, _D]
         lib.oracle_backward_swiglu.argtypes = [_D, _D, _D, _I64, _U8, _D, _D, _D, _D, i64, i32, i32, i64, i64,
                                                i64, ctypes.c_int, dbl, ctypes.c_int, _I64, _D, _D, _D, _D, _D, _D]
+        lib.oracle_router_backward.argtypes = [_D, _D, _D, i64, i64, i32, _D, _D, _D]
         lib.oracle_combine_precomputed.argtypes = [_D, i64, i32, i64, _I64, _U8, _D, i32, ctypes.c_int,
                                                    _D, _D]
         lib.oracle_combine_slots.argtypes = [_D, i64, i32, i64, i64, _I64, _I64, _U8, _D, i32,
@@ -117,6 +118,18 @@ def router_logits(x, w_router, bias=None) -> np.ndarray:
     s = np.empty((T, E), np.float64)
     _load().oracle_router_logits(_p(x, _D), _p(w, _D), _p(b, _D), T, D, E, _p(s, _D))
     return s
+
+
+def router_backward(x, w_router, dlogits):
+    """``(dx, dw_router, db)`` of ``s = x @ w_router + b`` for the gradient ``dlogits`` (w_router is (D, E))."""
+    x, w, g = _f64(x), _f64(w_router), _f64(dlogits)
+    T, D = x.shape
+    E = w.shape[1]
+    dx = np.empty((T, D), np.float64)
+    dw = np.empty((D, E), np.float64)
+    db = np.empty(E, np.float64)
+    _load().oracle_router_backward(_p(x, _D), _p(w, _D), _p(g, _D), T, D, E, _p(dx, _D), _p(dw, _D), _p(db, _D))
+    return dx, dw, db
 
 
 def route(s, k: int):

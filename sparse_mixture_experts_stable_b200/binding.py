@@ -38,7 +38,7 @@ EXPORTED = [
     "moe_combine", "moe_aux_stats", "moe_backward_workspace_size", "moe_backward", "moe_transpose_weights",
     "moe_clear_status", "moe_read_status", "moe_dispatch_static_max_state_bytes", "moe_dispatch_static",
     "moe_route_ex", "moe_renormalize_kept_gates", "moe_expert_ffn_gathered", "moe_backward_swiglu_workspace_size",
-    "moe_backward_swiglu",
+    "moe_backward_swiglu", "moe_router_backward_workspace_size", "moe_router_backward",
 ]
 SCORING = {"softmax": 0, "sigmoid": 1}
 
@@ -91,6 +91,10 @@ def lib():
                                   _vp, _i64, _vp, _i64, ctypes.c_int, _vp, _vp]
         L.moe_aux_stats.argtypes = [_vp, _vp, _i64, _i32, _i32, ctypes.c_int, _f32, _vp, _vp, ctypes.c_int, _vp,
                                     _vp]
+        L.moe_router_backward_workspace_size.restype = _sz
+        L.moe_router_backward_workspace_size.argtypes = [_i64, _i64, _i32, ctypes.c_int, ctypes.c_int]
+        L.moe_router_backward.argtypes = [ctypes.c_int, _vp, _i64, _i64, _i64, _vp, ctypes.c_int, _i32, _vp, _vp,
+                                          _vp, _vp, _vp, _vp, _sz, _vp]
         L.moe_backward_swiglu_workspace_size.restype = _sz
         L.moe_backward_swiglu_workspace_size.argtypes = [_i32, _i64, _i64, _i64]
         L.moe_backward_swiglu.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
@@ -411,6 +415,26 @@ def moe_backward(dy, x, logits, selected, gates_f32, slot, used, token_of_slot, 
                             _p(dW), _p(dl), _p(dg), _p(dev_status), _p(ws), ws.numel(), _stream(stream))
     _check("moe_backward", rc)
     return dx, dW, dl, dg
+
+
+def moe_router_backward(x: torch.Tensor, w_router: torch.Tensor, dlogits: torch.Tensor, layout: str = "ED",
+                        dev_status=None, workspace=None, stream=None):
+    """Gradients of s = x W (+ b) for dL/ds: returns (dx_router fp32 (T,D), dw_router fp32 in W's layout, db fp32 (E))."""
+    dev = _dev(x)
+    T, D = x.shape
+    E = dlogits.shape[1]
+    if w_router.dtype != x.dtype:
+        raise TypeError("w_router must have x's dtype")
+    dx = torch.empty(T, D, dtype=torch.float32, device=dev)
+    dw = torch.empty(tuple(w_router.shape), dtype=torch.float32, device=dev)
+    db = torch.empty(E, dtype=torch.float32, device=dev)
+    dt = _dt(x)
+    ws = _workspace(int(lib().moe_router_backward_workspace_size(T, D, E, dt, ROUTER_LAYOUT[layout])), dev, workspace)
+    rc = lib().moe_router_backward(dt, _p(x), T, D, _rowstride(x), _p(w_router.contiguous()), ROUTER_LAYOUT[layout], E,
+                                   _p(dlogits.to(torch.float32).contiguous()), _p(dx), _p(dw), _p(db),
+                                   _p(dev_status), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_router_backward", rc)
+    return dx, dw, db
 
 
 def moe_backward_swiglu_workspace_size(E: int, C: int, H: int, F: int) -> int:

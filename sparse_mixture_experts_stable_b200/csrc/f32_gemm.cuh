@@ -22,6 +22,8 @@ enum F32Epilogue : int {
 };
 
 struct F32Gemm {
+    // A and B are fp32, or bf16 when a_bf16 / b_bf16 is set (read through the
+    // same pointers; products still in fp32 accuracy).
     const float* A = nullptr;
     int64_t lda = 0;
     bool a_trans = false;
@@ -40,6 +42,8 @@ struct F32Gemm {
     const float* bias = nullptr;
     int64_t bias_group_stride = 0;
     int epilogue = F32_EPI_NONE;
+    bool a_bf16 = false;
+    bool b_bf16 = false;
 };
 
 }  // namespace moe

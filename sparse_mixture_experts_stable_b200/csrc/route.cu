@@ -539,3 +539,118 @@ extern "C" int moe_aux_stats(const int32_t* counts, const float* prob_sum, int64
                                              out_dtype == MOE_BF16, aux);
     return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// moe_router_backward
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+// db[e] = sum_t g[t,e] in a fixed order: warp w of block b adds rows t = w,
+// w + 32, ... for experts 32b + lane, then warp 0 adds the 32 warp sums.
+__global__ void __launch_bounds__(1024)
+    column_sum_kernel(const float* __restrict__ g, int64_t T, int E, float* __restrict__ out) {
+    __shared__ float s[32][33];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 32 + lane;
+    float acc = 0.f;
+    if (e < E)
+        for (int64_t t = warp; t < T; t += 32) acc += g[t * E + e];
+    s[warp][lane] = acc;
+    __syncthreads();
+    if (warp == 0 && e < E) {
+        float tot = 0.f;
+        for (int w = 0; w < 32; ++w) tot += s[w][lane];
+        out[e] = tot;
+    }
+}
+
+// The two GEMMs of the router backward in F32Gemm form.
+void router_bwd_gemms(moe_dtype dtype, const void* x, int64_t T, int64_t D, int64_t ldx, const void* w,
+                      moe_router_layout layout, int32_t E, const float* g, float* dx, float* dw, F32Gemm& gx,
+                      F32Gemm& gw) {
+    const bool bf16 = dtype == MOE_BF16;
+    // dx[t,d] = sum_e g[t,e] W(e,d)
+    gx = F32Gemm{};
+    gx.A = g;
+    gx.lda = E;
+    gx.B = static_cast<const float*>(w);
+    gx.b_bf16 = bf16;
+    if (layout == MOE_ROUTER_ED) {  // W(e,d) = w[e*D + d]: B(k=e, n=d) not transposed
+        gx.ldb = D;
+        gx.b_trans = false;
+    } else {  // W(e,d) = w[d*E + e]: B(k=e, n=d) = w[n*E + k]
+        gx.ldb = E;
+        gx.b_trans = true;
+    }
+    gx.C = dx;
+    gx.ldc = D;
+    gx.M = T;
+    gx.N = D;
+    gx.K = E;
+    // dw in the weight's layout; reduction over t
+    gw = F32Gemm{};
+    if (layout == MOE_ROUTER_ED) {  // dw[e,d] = sum_t g[t,e] x[t,d]
+        gw.A = g;
+        gw.lda = E;
+        gw.a_trans = true;
+        gw.B = static_cast<const float*>(x);
+        gw.b_bf16 = bf16;
+        gw.ldb = ldx;
+        gw.M = E;
+        gw.N = D;
+        gw.ldc = D;
+    } else {  // dw[d,e] = sum_t x[t,d] g[t,e]
+        gw.A = static_cast<const float*>(x);
+        gw.a_bf16 = bf16;
+        gw.lda = ldx;
+        gw.a_trans = true;
+        gw.B = g;
+        gw.ldb = E;
+        gw.M = D;
+        gw.N = E;
+        gw.ldc = E;
+    }
+    gw.C = dw;
+    gw.K = T;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" size_t moe_router_backward_workspace_size(int64_t T, int64_t D, int32_t E, moe_dtype dtype,
+                                                     moe_router_layout layout) {
+    if (T < 1 || D < 1 || E < 1) return 0;
+    F32Gemm gx, gw;
+    router_bwd_gemms(dtype, nullptr, T, D, D, nullptr, layout, E, nullptr, nullptr, nullptr, gx, gw);
+    const size_t a = tf32x3_workspace_size(gx), b = tf32x3_workspace_size(gw);
+    return a > b ? a : b;
+}
+
+extern "C" int moe_router_backward(moe_dtype dtype, const void* x, int64_t T, int64_t D, int64_t ldx,
+                                   const void* w_router, moe_router_layout layout, int32_t E, const float* dlogits,
+                                   float* dx_router, float* dw_router, float* db_router, int32_t* dev_status,
+                                   void* workspace, size_t workspace_bytes, moe_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    MOE_REQUIRE(valid_dtype(dtype), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(layout == MOE_ROUTER_DE || layout == MOE_ROUTER_ED, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(x && w_router && dlogits && T >= 1 && D >= 1 && E >= 1 && ldx >= D, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(workspace_bytes >= moe_router_backward_workspace_size(T, D, E, dtype, layout) && workspace,
+                MOE_ERR_WORKSPACE);
+    F32Gemm gx, gw;
+    router_bwd_gemms(dtype, x, T, D, ldx, w_router, layout, E, dlogits, dx_router, dw_router, gx, gw);
+    int rc;
+    if (dx_router) {
+        rc = tf32x3_gemm_run(gx, workspace, workspace_bytes, dev_status, stream);
+        if (rc != MOE_OK) return rc;
+    }
+    if (dw_router) {
+        rc = tf32x3_gemm_run(gw, workspace, workspace_bytes, dev_status, stream);
+        if (rc != MOE_OK) return rc;
+    }
+    if (db_router) {
+        column_sum_kernel<<<(E + 31) / 32, 1024, 0, stream>>>(dlogits, T, E, db_router);
+        return launch_status();
+    }
+    return MOE_OK;
+}

@@ -11,6 +11,7 @@
 //    tcgen05.mma.kind::tf32 into one accumulator; warps 2..5 read TMEM and apply
 //    the epilogue.  Every mbarrier wait is bounded.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -45,9 +46,9 @@ __device__ __forceinline__ float tf32_round(float x) {
 //   TRANS: src(g, r, k) = src[g*gs + k*ld + r]   (r contiguous in memory)
 //   else : src(g, r, k) = src[g*gs + r*ld + k]   (k contiguous)
 // Block 32 x 8 threads covers 32 rows x 32 k; grid (Kp/32, ceil(R/32), G).
-template <bool TRANS>
+template <bool TRANS, typename In>
 __global__ void __launch_bounds__(256)
-    split_kernel(const float* __restrict__ src, int64_t ld, int64_t gs, int64_t R, int64_t K, int64_t Kp,
+    split_kernel(const In* __restrict__ src, int64_t ld, int64_t gs, int64_t R, int64_t K, int64_t Kp,
                  const int32_t* __restrict__ krows, float* __restrict__ hi, float* __restrict__ lo) {
     __shared__ float tile[32][33];
     const int g = blockIdx.z;
@@ -57,13 +58,13 @@ __global__ void __launch_bounds__(256)
         Kg = r < 0 ? 0 : (r < K ? r : K);
     }
     const int64_t r0 = (int64_t)blockIdx.y * 32, k0 = (int64_t)blockIdx.x * 32;
-    const float* s = src + g * gs;
+    const In* s = src + g * gs;
     const int tx = threadIdx.x, ty = threadIdx.y;
     if (TRANS) {
         // read 32 k-rows of 32 consecutive r, write transposed
         for (int i = ty; i < 32; i += 8) {
             const int64_t k = k0 + i, r = r0 + tx;
-            tile[i][tx] = (k < Kg && r < R) ? s[k * ld + r] : 0.f;
+            tile[i][tx] = (k < Kg && r < R) ? to_f32(s[k * ld + r]) : 0.f;
         }
         __syncthreads();
         for (int i = ty; i < 32; i += 8) {
@@ -80,7 +81,7 @@ __global__ void __launch_bounds__(256)
         for (int i = ty; i < 32; i += 8) {
             const int64_t r = r0 + i, k = k0 + tx;
             if (r < R) {
-                const float x = k < Kg ? s[r * ld + k] : 0.f;
+                const float x = k < Kg ? to_f32(s[r * ld + k]) : 0.f;
                 const float h = tf32_round(x);
                 const size_t o = ((size_t)g * R + r) * Kp + k;
                 hi[o] = h;
@@ -367,12 +368,19 @@ SplitLayout split_layout(const F32Gemm& g) {
     return l;
 }
 
-int launch_split(bool trans, const float* src, int64_t ld, int64_t gs, int groups, int64_t R, int64_t K, int64_t Kp,
-                 const int32_t* krows, float* hi, float* lo, cudaStream_t stream) {
+int launch_split(bool trans, bool bf16, const void* src, int64_t ld, int64_t gs, int groups, int64_t R, int64_t K,
+                 int64_t Kp, const int32_t* krows, float* hi, float* lo, cudaStream_t stream) {
     MOE_REQUIRE(groups <= 65535 && (R + 31) / 32 <= 65535, MOE_ERR_UNSUPPORTED);
     const dim3 grid((unsigned)(Kp / 32), (unsigned)((R + 31) / 32), (unsigned)groups), block(32, 8);
-    if (trans) split_kernel<true><<<grid, block, 0, stream>>>(src, ld, gs, R, K, Kp, krows, hi, lo);
-    else split_kernel<false><<<grid, block, 0, stream>>>(src, ld, gs, R, K, Kp, krows, hi, lo);
+    if (bf16) {
+        const __nv_bfloat16* s = static_cast<const __nv_bfloat16*>(src);
+        if (trans) split_kernel<true><<<grid, block, 0, stream>>>(s, ld, gs, R, K, Kp, krows, hi, lo);
+        else split_kernel<false><<<grid, block, 0, stream>>>(s, ld, gs, R, K, Kp, krows, hi, lo);
+    } else {
+        const float* s = static_cast<const float*>(src);
+        if (trans) split_kernel<true><<<grid, block, 0, stream>>>(s, ld, gs, R, K, Kp, krows, hi, lo);
+        else split_kernel<false><<<grid, block, 0, stream>>>(s, ld, gs, R, K, Kp, krows, hi, lo);
+    }
     return launch_status();
 }
 
@@ -400,11 +408,11 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
     const int32_t* krows = g.rows_mode == 2 ? g.rows : nullptr;
 
     // K-major split operands: A as (groups, M, Kp), B^T as (groups, N, Kp)
-    int rc = launch_split(g.a_trans, g.A, g.lda, g.a_group_stride, g.groups, g.M, g.K, l.Kp, krows, a_hi, a_lo,
-                          stream);
+    int rc = launch_split(g.a_trans, g.a_bf16, g.A, g.lda, g.a_group_stride, g.groups, g.M, g.K, l.Kp, krows, a_hi,
+                          a_lo, stream);
     if (rc != MOE_OK) return rc;
-    rc = launch_split(!g.b_trans, g.B, g.ldb, g.b_group_stride, g.groups, g.N, g.K, l.Kp, krows, b_hi, b_lo,
-                      stream);
+    rc = launch_split(!g.b_trans, g.b_bf16, g.B, g.ldb, g.b_group_stride, g.groups, g.N, g.K, l.Kp, krows, b_hi,
+                      b_lo, stream);
     if (rc != MOE_OK) return rc;
 
     T3Params kp{};

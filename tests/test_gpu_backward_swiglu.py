@@ -1,4 +1,5 @@
-"""moe_backward_swiglu (bf16 SwiGLU experts) against the fp64 oracle backward.
+"""moe_backward_swiglu (bf16 SwiGLU experts) and moe_router_backward against the
+fp64 oracle backward.
 
 The forward runs on the GPU (route on given logits, dispatch, SwiGLU experts);
 the oracle recomputes everything in fp64 from the same bf16 inputs.  Integer
@@ -13,7 +14,7 @@ import torch
 import sparse_mixture_experts_stable_b200 as moe
 from oracle import oracle as O
 from sparse_mixture_experts_stable_b200.inputs import pages_layout
-from tests.gpu_util import BF16_RTOL, DEV, assert_close, cpu, cpu64
+from tests.gpu_util import BF16_RTOL, DEV, F32_ATOL, F32_RTOL, assert_close, assert_close_mag, cpu, cpu64
 
 pytestmark = pytest.mark.gpu
 
@@ -90,3 +91,21 @@ def test_backward_swiglu_with_nothing_kept():
     assert torch.equal(dx, dy)
     assert (dwg == 0).all() and (dwu == 0).all() and (dwd == 0).all()
     assert (dl == 0).all() and (dg == 0).all()
+
+
+@pytest.mark.parametrize("dtype,layout", [(torch.bfloat16, "ED"), (torch.bfloat16, "DE"), (torch.float32, "ED")])
+def test_router_backward_matches_oracle(dtype, layout):
+    # s = x W (+ b): dx = dlogits W^T, dW = x^T dlogits, db = column sums (fp32 accuracy)
+    T, D, E = 700, 192, 40
+    g = torch.Generator().manual_seed(5 + (layout == "DE"))
+    x = torch.randn(T, D, generator=g).to(dtype)
+    w_ed = (torch.randn(E, D, generator=g) * 0.1).to(dtype)
+    dl = torch.randn(T, E, generator=g)
+    w = w_ed if layout == "ED" else w_ed.t().contiguous()
+    dx, dw, db = moe.moe_router_backward(x.to(DEV), w.to(DEV), dl.to(DEV), layout=layout)
+    wdx, wdw, wdb = O.router_backward(cpu64(x), cpu64(w_ed).T, cpu64(dl))  # oracle weight is (D, E)
+    mdx, mdw, mdb = O.router_backward(np.abs(cpu64(x)), np.abs(cpu64(w_ed)).T, np.abs(cpu64(dl)))
+    assert_close_mag(cpu64(dx), wdx, mdx, F32_RTOL, F32_ATOL, "dx_router")
+    got_dw = cpu64(dw) if layout == "DE" else cpu64(dw).T
+    assert_close_mag(got_dw, wdw, mdw, F32_RTOL, F32_ATOL, "dw_router")
+    assert_close_mag(cpu64(db), wdb, mdb, F32_RTOL, F32_ATOL, "db_router")

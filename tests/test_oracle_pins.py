@@ -503,6 +503,56 @@ def test_backward_swiglu_down_gradient_closed_form_and_top1():
     assert np.abs(dl).max() < 1e-12
 
 
+def test_router_and_expert_backward_compose_to_the_full_gradient():
+    # Module 7's layer end to end: s = x W_r + b, SwiGLU experts, y = x + sum gate * out.
+    # With the routing decisions fixed, dL/dx = expert path + residual + dlogits W_r^T,
+    # dL/dW_r = x^T dlogits, dL/db = sum_t dlogits; checked by central differences.
+    ver = _golden("numpy_layer_verification.json")
+    rng = np.random.default_rng(23)
+    T, D, F, E, k = 6, 4, 3, 4, 2
+    x = rng.standard_normal((T, D))
+    wr = rng.standard_normal((D, E))
+    b = rng.standard_normal(E) * 0.3
+    w = {"w1": rng.standard_normal((E, D, F)) * 0.7, "w3": rng.standard_normal((E, D, F)) * 0.7,
+         "w2": rng.standard_normal((E, F, D)) * 0.7}
+    dy = rng.standard_normal((T, D))
+    C = 3
+    s0 = O.router_logits(x, wr, b)
+    out = O.forward("swiglu", x, s0, k, C, w, base_kind="input")
+    sel0, kept = out["selected"], out["kept"]
+
+    def loss():
+        s = O.router_logits(x, wr, b)
+        _, sel, gates, _, _ = O.route(s, k)
+        assert (sel == sel0).all()
+        y = O.layer_rows("swiglu", x, sel, kept, gates, w, base_kind="input")
+        return float((dy * y).sum())
+
+    dxe, _, _, _, dl, _ = O.backward_swiglu(dy, x, s0, sel0, kept, out["gates"], w["w1"], w["w3"], w["w2"],
+                                            use_residual=True)
+    dxr, dwr, dbr = O.router_backward(x, wr, dl)
+    h = 1e-6
+
+    def fd(arr):
+        g = np.zeros_like(arr)
+        it = np.nditer(arr, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            a0 = arr[i]
+            arr[i] = a0 + h
+            lp = loss()
+            arr[i] = a0 - h
+            lm = loss()
+            arr[i] = a0
+            g[i] = (lp - lm) / (2 * h)
+        return g
+
+    bound = 10 * max(ver["backward_vs_finite_difference_max_err"].values())
+    assert np.abs(fd(x) - (dxe + dxr)).max() < bound
+    assert np.abs(fd(wr) - dwr).max() < bound
+    assert np.abs(fd(b) - dbr).max() < bound
+
+
 # --------------------------------------------------------------------------
 # negative cases (module-7 negative tests)
 # --------------------------------------------------------------------------
