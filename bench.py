@@ -38,13 +38,12 @@ UNIT = "tokens/s"
 WORKLOAD = dict(workload="full_layer_bf16", T=16384, hidden=2048, experts=256, top_k=8, expert_intermediate=512,
                 shared_experts=1, shared_intermediate=512, capacity_factor=1.25, capacity=640, aux_coef=0.001)
 KERNELS_PER_STEP = 11  # router GEMM, top-k, reduce, scan, gather, 2 routed GEMMs, 2 shared GEMMs, combine, aux
-# DRAM bytes (read + write) per algorithmic byte of the two routed expert-FFN
-# launches, from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum
-# on the same kernels at T = 4096, E = 64 (profiles/expert_gemm_dram_traffic_T4096_E64.md).
-# Both operands and outputs scale with E and the kept rows, so the full-size
-# traffic is these ratios times the full-size algorithmic bytes.
-TRAFFIC_PER_ALG_BYTE = {"gate_up": 1.017, "down": 0.857}
-TRAFFIC_SOURCE = "ncu DRAM bytes at T=4096, E=64, scaled by algorithmic bytes"
+# DRAM bytes (read + write) per launch of the two routed expert-FFN kernels,
+# from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum on this
+# workload (profiles/expert_gemm_dram_traffic.md; a one-pass metric set).  For
+# other sizes the same capture's ratio to the algorithmic bytes is applied.
+TRAFFIC_MEASURED = {"gate_up": 1618.1e6, "down": 982.9e6}
+TRAFFIC_PER_ALG_BYTE = {"gate_up": 1.047, "down": 0.975}
 
 
 def measured_peaks():
@@ -330,11 +329,15 @@ def run_ours(args, world, rank, local):
     achieved = flops / ffn_avg_s / 1e12
     alg_gate_up = E * 2 * F * H * 2 + kept * H * 2 + kept * F * 2  # weights, gathered rows, h written
     alg_down = E * H * F * 2 + kept * F * 2 + kept * H * 2
-    traffic = (None if TRAFFIC_PER_ALG_BYTE is None else
-               TRAFFIC_PER_ALG_BYTE["gate_up"] * alg_gate_up + TRAFFIC_PER_ALG_BYTE["down"] * alg_down)
+    if T == WORKLOAD["T"] and E == WORKLOAD["experts"]:
+        traffic = TRAFFIC_MEASURED["gate_up"] + TRAFFIC_MEASURED["down"]
+        traffic_source = "ncu dram__bytes_read.sum + dram__bytes_write.sum of both launches, this workload"
+    else:
+        traffic = TRAFFIC_PER_ALG_BYTE["gate_up"] * alg_gate_up + TRAFFIC_PER_ALG_BYTE["down"] * alg_down
+        traffic_source = "full-workload ncu DRAM bytes per algorithmic byte, times this size's algorithmic bytes"
     roof = dict(bound="tensor", kernel="routed expert FFN: tcx_kernel<SWIGLU> gate/up + tc_gemm_kernel<BF16> down",
                 achieved=achieved, peak=pk["bf16_sustained"], unit="TFLOP/s", frac=achieved / pk["bf16_sustained"],
-                traffic=traffic, traffic_source=TRAFFIC_SOURCE, bytes_alg=alg_gate_up + alg_down,
+                traffic=traffic, traffic_source=traffic_source, bytes_alg=alg_gate_up + alg_down,
                 peak_source=f"{pk['source']} bf16 sustained", frac_of_burst=achieved / pk["bf16"],
                 flops_per_launch=flops, kept_rows=kept, avg_launch_ms=1e3 * ffn_avg_s)
 
@@ -566,6 +569,43 @@ def run_other_workloads(steps, warmup, flush, stream, dev):
                       achieved=3 * flops_b / b_s / 1e12, peak=tf32_peak(pk), unit="TFLOP/s",
                       frac=3 * flops_b / b_s / 1e12 / tf32_peak(pk), traffic=None, avg_launch_ms=1e3 * b_s,
                       fp32_tflops=flops_b / b_s / 1e12, peak_source=TF32_PEAK_SOURCE))
+    del lg, x, w, dy, wsb, state
+
+    # training step of the full layer: forward, SwiGLU-expert backward and router backward (bf16)
+    from sparse_mixture_experts_stable_b200.layer import SwiGLUMoE
+    c = I.full_layer_bf16(seed=0)
+    T, H, E, F, k = c["T"], c["H"], c["E"], c["F"], c["k"]
+    dv = {n: c[n].to(dev) for n in ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down")}
+    dyt = (torch.randn(T, H, generator=torch.Generator().manual_seed(1)) * 0.1).to(torch.bfloat16).to(dev)
+    layer = SwiGLUMoE(T, H, E, F, k, c["capacity_factor"], F_shared=0, aux_coef=c["aux_coef"], device=dev)
+    wsbs = torch.empty(B.moe_backward_swiglu_workspace_size(E, layer.C, H, F), dtype=torch.uint8, device=dev)
+    kept_box = {}
+    inner = []
+
+    def step_train():
+        o = layer.forward(dv["x"], dv["w_router"], dv["router_bias"], dv["w_gate"], dv["w_up"], dv["w_down"])
+        lg_t = layer.route_out.get("logits")
+        e0, e1 = events(inner)
+        e0.record(stream)
+        dxe, dwg, dwu, dwd, dl, dg = moe.moe_backward_swiglu(
+            dyt, lg_t, o["selected"], o["gates_f32"], o["slot"], o["used"], o["xbuf"], layer.ybuf, dv["w_gate"],
+            dv["w_up"], dv["w_down"], layer.C, aux_coef=c["aux_coef"], counts=o["counts"], workspace=wsbs)
+        e1.record(stream)
+        moe.moe_router_backward(dv["x"], dv["w_router"], dl)
+        kept_box["used"] = o["used"]
+
+    layer.route_out["logits"] = torch.empty(T, E, dtype=torch.float32, device=dev)
+    sm, im = _time_steps(step_train, max(steps // 5, 3), warmup, flush, stream, inner)
+    kept = int(kept_box["used"].sum())
+    bw_s = statistics.mean(im) / 1e3
+    flops_bw = 16.0 * kept * H * F  # recomputed gate/up (4), dh (2), three weight gradients (6), dx (4): x kept*H*F
+    out["full_layer_bf16_train"] = dict(
+        value=T * len(sm) / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / len(sm), steps=len(sm),
+        config=dict(T=T, H=H, E=E, F=F, k=k, capacity=layer.C, kept=kept, shared_experts=0,
+                    step="forward + moe_backward_swiglu + moe_router_backward"),
+        roofline=dict(bound="tensor", kernel="moe_backward_swiglu (tcgen05 GEMMs + transposes)",
+                      achieved=flops_bw / bw_s / 1e12, peak=pk["bf16_sustained"], unit="TFLOP/s",
+                      frac=flops_bw / bw_s / 1e12 / pk["bf16_sustained"], traffic=None, avg_launch_ms=1e3 * bw_s))
     return out
 
 
