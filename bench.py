@@ -486,7 +486,7 @@ def run_other_workloads(steps, warmup, flush, stream, dev):
     out["router_bf16"] = dict(
         value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
         config=dict(T=T, D=D, E=E, k=k),
-        roofline=dict(bound="hbm/tensor ridge", kernel="moe_route: tcx_kernel<F32> scores + route_topk_kernel + route_reduce_kernel",
+        roofline=dict(bound="hbm/tensor ridge", kernel="moe_route: tc_gemm_kernel<F32> scores + route_topk_kernel + route_reduce_kernel",
                       achieved=bytes_alg / r_s / 1e9, peak=pk["hbm"], unit="GB/s", frac=bytes_alg / r_s / 1e9 / pk["hbm"],
                       tflops=flops / r_s / 1e12, frac_tensor=flops / r_s / 1e12 / pk["bf16"], traffic=None,
                       bytes_per_launch=bytes_alg, flops_per_launch=flops, avg_launch_ms=1e3 * r_s))

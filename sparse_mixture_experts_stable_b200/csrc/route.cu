@@ -12,7 +12,7 @@
 #include "common.cuh"
 #include "route_scores.cuh"
 #include "f32_gemm.cuh"
-#include "tc_expert_gemm.cuh"
+#include "tc_gemm.cuh"
 #include "tc_tf32.cuh"
 #include "util_kernels.cuh"
 
@@ -392,27 +392,28 @@ extern "C" int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D
                 if (rc != MOE_OK) return rc;
                 w_ed = wt;
             }
-            TcxProblem p{};
-            p.w = w_ed;  // experts are the output features
-            p.ldw = D;
-            p.w_rows_total = E;
-            p.w_rows_per_group = 0;
-            p.x = x;
-            p.ldx = ldx;
-            p.x_rows_total = T;
-            p.x_rows_per_group = 0;
-            p.G = 1;
-            p.features = E;
-            p.max_tokens = T;
-            p.K = D;
-            p.rows = nullptr;
-            p.out = lg;
-            p.ldo = E;
-            p.out_rows_per_group = 0;
-            p.bias = logit_bias;
-            p.epilogue = TC_EPI_F32;
-            p.status = dev_status;
-            rc = tcx_gemm_run(p, stream);
+            // tokens on the MMA's M side, all E experts in one N tile
+            TcGemmProblem q{};
+            q.a = x;
+            q.lda = ldx;
+            q.a_rows_total = T;
+            q.a_rows_per_group = 0;
+            q.b = w_ed;
+            q.ldb = D;
+            q.b_rows_total = E;
+            q.b_rows_per_group = 0;
+            q.G = 1;
+            q.M = T;
+            q.N = E;
+            q.K = D;
+            q.rows = nullptr;
+            q.out = lg;
+            q.ldo = E;
+            q.out_rows_per_group = 0;
+            q.bias = logit_bias;
+            q.epilogue = TC_EPI_F32;
+            q.status = dev_status;
+            rc = tc_gemm_run(q, stream);
         } else {
             F32Gemm g{};
             g.A = static_cast<const float*>(x);

@@ -458,16 +458,10 @@ int tcx_gemm_run(const TcxProblem& p, cudaStream_t stream) {
     if (max_tiles < grid) grid = (int)max_tiles;
     if (grid < 1) grid = 1;
 
-    switch (p.epilogue) {
-        case TC_EPI_F32: return launch<TC_EPI_F32>(mw, mw2, mx, kp, grid, stream);
-        case TC_EPI_BF16: return launch<TC_EPI_BF16>(mw, mw2, mx, kp, grid, stream);
-        case TC_EPI_BF16_BIAS: return launch<TC_EPI_BF16_BIAS>(mw, mw2, mx, kp, grid, stream);
-        case TC_EPI_GELU_BIAS: return launch<TC_EPI_GELU_BIAS>(mw, mw2, mx, kp, grid, stream);
-        case TC_EPI_SWIGLU:
-            return gather ? launch<TC_EPI_SWIGLU, true>(mw, mw2, mx, kp, grid, stream)
-                          : launch<TC_EPI_SWIGLU>(mw, mw2, mx, kp, grid, stream);
-        default: return MOE_ERR_INVALID_ARG;
-    }
+    // The library uses this kernel for the SwiGLU gate/up projection only.
+    if (p.epilogue != TC_EPI_SWIGLU) return MOE_ERR_UNSUPPORTED;
+    return gather ? launch<TC_EPI_SWIGLU, true>(mw, mw2, mx, kp, grid, stream)
+                  : launch<TC_EPI_SWIGLU>(mw, mw2, mx, kp, grid, stream);
 }
 
 }  // namespace moe
