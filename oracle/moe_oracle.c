@@ -569,6 +569,130 @@ void oracle_backward_swiglu(const double* dy, const double* x, const double* s,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Backward of the GELU-MLP-expert layer ([P5] Expert, fc2(gelu(fc1(x)))),     */
+/* the kept mask constant as in [P1] section 1 item 7.  For a kept assignment   */
+/* of token t to expert e with gate g:                                          */
+/*   z = x W1_e + b1_e,  h = gelu(z),  o = h W2_e + b2_e,  y_t += g o           */
+/* and for the upstream gradient dy_t:                                          */
+/*   dgate = dy_t . o,  do = g dy_t,  dh = do W2_e^T,                           */
+/*   dz = dh * gelu'(z),  gelu'(z) = Phi(z) + z phi(z)  (the derivative of     */
+/*   z Phi(z), Phi the standard normal CDF, phi its density),                   */
+/*   dW2_e += h^T do,  db2_e += do,  dW1_e += x^T dz,  db1_e += dz,             */
+/*   dx_t += dz W1_e^T  (+ dy_t with the residual base).                        */
+/* dlogits follows from dgate as in the linear case.  Weights in the x@W        */
+/* layout: W1 (E, D, F), b1 (E, F), W2 (E, F, N), b2 (E, N).                    */
+/* ------------------------------------------------------------------------ */
+
+static double gelu_erf_grad(double z) {
+    const double cdf = 0.5 * (1.0 + erf(z / sqrt(2.0)));
+    const double pdf = exp(-0.5 * z * z) / sqrt(2.0 * acos(-1.0));
+    return cdf + z * pdf;
+}
+
+/* One kept assignment: z, h (F), o (N), dz (F) and dgate. */
+static void gelu_assignment(const double* xrow, const double* dyrow, double g, const double* W1e,
+                            const double* b1e, const double* W2e, const double* b2e, int64_t D, int64_t F,
+                            int64_t N, double* z, double* h, double* o, double* dz, double* dgate_out) {
+    for (int64_t f = 0; f < F; ++f) z[f] = 0.0;
+    for (int64_t d = 0; d < D; ++d)
+        for (int64_t f = 0; f < F; ++f) z[f] += xrow[d] * W1e[d * F + f];
+    for (int64_t f = 0; f < F; ++f) {
+        z[f] += b1e[f];
+        h[f] = gelu_erf(z[f]);
+    }
+    for (int64_t n = 0; n < N; ++n) o[n] = b2e[n];
+    for (int64_t f = 0; f < F; ++f)
+        for (int64_t n = 0; n < N; ++n) o[n] += h[f] * W2e[f * N + n];
+    double dg = 0.0;
+    for (int64_t n = 0; n < N; ++n) dg += dyrow[n] * o[n];
+    *dgate_out = dg;
+    for (int64_t f = 0; f < F; ++f) {
+        double dh = 0.0;
+        for (int64_t n = 0; n < N; ++n) dh += g * dyrow[n] * W2e[f * N + n];
+        dz[f] = dh * gelu_erf_grad(z[f]);
+    }
+}
+
+void oracle_backward_gelu(const double* dy, const double* x, const double* s, const int64_t* selected,
+                          const uint8_t* kept, const double* gates, const double* W1, const double* b1,
+                          const double* W2, const double* b2, int64_t T, int32_t k, int32_t E, int64_t D,
+                          int64_t F, int64_t N, int use_residual, double aux_coef, int normalize_by_k,
+                          const int64_t* counts, double* dx, double* dW1, double* db1, double* dW2, double* db2,
+                          double* dlogits, double* dgate) {
+    /* per token: dgate, dlogits, dx */
+    OMP_FOR
+    for (int64_t t = 0; t < T; ++t) {
+        double* z = (double*)malloc((size_t)(3 * F + N) * sizeof(double));
+        double *h = z + F, *dz = h + F, *o = dz + F;
+        for (int64_t d = 0; d < D; ++d) dx[t * D + d] = use_residual ? dy[t * N + d] : 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            dgate[t * k + j] = 0.0;
+            if (!kept[t * k + j]) continue;
+            const int64_t e = selected[t * k + j];
+            const double* W1e = W1 + e * D * F;
+            gelu_assignment(x + t * D, dy + t * N, gates[t * k + j], W1e, b1 + e * F, W2 + e * F * N, b2 + e * N,
+                            D, F, N, z, h, o, dz, &dgate[t * k + j]);
+            for (int64_t d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int64_t f = 0; f < F; ++f) acc += dz[f] * W1e[d * F + f];
+                dx[t * D + d] += acc;
+            }
+        }
+        free(z);
+        for (int32_t e = 0; e < E; ++e) dlogits[t * E + e] = 0.0;
+        double gdot = 0.0;
+        for (int32_t j = 0; j < k; ++j) gdot += gates[t * k + j] * dgate[t * k + j];
+        for (int32_t i = 0; i < k; ++i)
+            dlogits[t * E + selected[t * k + i]] += gates[t * k + i] * (dgate[t * k + i] - gdot);
+        if (aux_coef != 0.0) {
+            double kn = normalize_by_k ? (double)k : 1.0;
+            const double* st = s + t * E;
+            double mx = st[0];
+            for (int32_t e = 1; e < E; ++e) if (st[e] > mx) mx = st[e];
+            double den = 0.0;
+            for (int32_t e = 0; e < E; ++e) den += exp(st[e] - mx);
+            double cp = 0.0;
+            for (int32_t e = 0; e < E; ++e) cp += (double)counts[e] * (exp(st[e] - mx) / den);
+            double scale = aux_coef * (double)E / ((double)T * (double)T * kn);
+            for (int32_t e = 0; e < E; ++e) {
+                double p = exp(st[e] - mx) / den;
+                dlogits[t * E + e] += scale * p * ((double)counts[e] - cp);
+            }
+        }
+    }
+    /* weight and bias gradients, one expert per iteration */
+    OMP_FOR
+    for (int32_t e = 0; e < E; ++e) {
+        double* z = (double*)malloc((size_t)(3 * F + N) * sizeof(double));
+        double *h = z + F, *dz = h + F, *o = dz + F;
+        double* dW1e = dW1 + (int64_t)e * D * F;
+        double* dW2e = dW2 + (int64_t)e * F * N;
+        double* db1e = db1 + (int64_t)e * F;
+        double* db2e = db2 + (int64_t)e * N;
+        for (int64_t i = 0; i < D * F; ++i) dW1e[i] = 0.0;
+        for (int64_t i = 0; i < F * N; ++i) dW2e[i] = 0.0;
+        for (int64_t f = 0; f < F; ++f) db1e[f] = 0.0;
+        for (int64_t n = 0; n < N; ++n) db2e[n] = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            for (int32_t j = 0; j < k; ++j) {
+                if (!kept[t * k + j] || selected[t * k + j] != e) continue;
+                const double g = gates[t * k + j];
+                double unused;
+                gelu_assignment(x + t * D, dy + t * N, g, W1 + (int64_t)e * D * F, b1 + (int64_t)e * F,
+                                W2 + (int64_t)e * F * N, b2 + (int64_t)e * N, D, F, N, z, h, o, dz, &unused);
+                for (int64_t f = 0; f < F; ++f)
+                    for (int64_t n = 0; n < N; ++n) dW2e[f * N + n] += h[f] * g * dy[t * N + n];
+                for (int64_t n = 0; n < N; ++n) db2e[n] += g * dy[t * N + n];
+                for (int64_t d = 0; d < D; ++d)
+                    for (int64_t f = 0; f < F; ++f) dW1e[d * F + f] += x[t * D + d] * dz[f];
+                for (int64_t f = 0; f < F; ++f) db1e[f] += dz[f];
+            }
+        }
+        free(z);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Dense reference with the explicit (T,E,C) tensors ([P1] section 1 item 5:   */
 /* dispatch_mask (T,E,C) bool and combine_weights (T,E,C), zero on dropped     */
 /* slots; section 2: M = combine.sum(axis=2), xe = x @ W for every (t,e),      */

@@ -65,6 +65,9 @@ def _load():
                                                ctypes.c_int, dbl, ctypes.c_int, _I64, _D, _D, _D, _D]
         lib.oracle_backward_swiglu.argtypes = [_D, _D, _D, _I64, _U8, _D, _D, _D, _D, i64, i32, i32, i64, i64,
                                                i64, ctypes.c_int, dbl, ctypes.c_int, _I64, _D, _D, _D, _D, _D, _D]
+        lib.oracle_backward_gelu.argtypes = [_D, _D, _D, _I64, _U8, _D, _D, _D, _D, _D, i64, i32, i32, i64, i64,
+                                             i64, ctypes.c_int, dbl, ctypes.c_int, _I64, _D, _D, _D, _D, _D, _D,
+                                             _D]
         lib.oracle_router_backward.argtypes = [_D, _D, _D, i64, i64, i32, _D, _D, _D]
         lib.oracle_combine_precomputed.argtypes = [_D, i64, i32, i64, _I64, _U8, _D, i32, ctypes.c_int,
                                                    _D, _D]
@@ -339,6 +342,38 @@ def backward_swiglu(dy, x, s, selected, kept, gates, Wg, Wu, Wd, use_residual: b
                                    _p(cnt, _I64), _p(dx, _D), _p(dWg, _D), _p(dWu, _D), _p(dWd, _D),
                                    _p(dl, _D), _p(dg, _D))
     return dx, dWg, dWu, dWd, dl, dg
+
+
+def backward_gelu(dy, x, s, selected, kept, gates, W1, b1, W2, b2, use_residual: bool = False,
+                  aux_coef: float = 0.0, normalize_by_k: bool = True, counts=None):
+    """Backward of the GELU-MLP-expert layer with the kept mask constant.
+
+    ``W1`` is ``(E, D, F)``, ``b1`` ``(E, F)``, ``W2`` ``(E, F, N)``, ``b2`` ``(E, N)``
+    (pages' x@W layout).  Returns ``(dx, dW1, db1, dW2, db2, dlogits, dgate)``.
+    """
+    dy, x, s = _f64(dy), _f64(x), _f64(s)
+    W1, b1, W2, b2 = _f64(W1), _f64(b1), _f64(W2), _f64(b2)
+    T, D = x.shape
+    E = s.shape[1]
+    F, N = W1.shape[2], W2.shape[2]
+    sel = _i64(selected).reshape(T, -1)
+    k = sel.shape[1]
+    kp = _u8(kept).reshape(T, k)
+    g = _f64(gates).reshape(T, k)
+    cnt = _i64(counts if counts is not None else np.bincount(sel.ravel(), minlength=E))
+    dx = np.empty((T, D), np.float64)
+    dW1 = np.empty((E, D, F), np.float64)
+    db1 = np.empty((E, F), np.float64)
+    dW2 = np.empty((E, F, N), np.float64)
+    db2 = np.empty((E, N), np.float64)
+    dl = np.empty((T, E), np.float64)
+    dg = np.empty((T, k), np.float64)
+    _load().oracle_backward_gelu(_p(dy, _D), _p(x, _D), _p(s, _D), _p(sel, _I64), _p(kp, _U8), _p(g, _D),
+                                 _p(W1, _D), _p(b1, _D), _p(W2, _D), _p(b2, _D), T, k, E, D, F, N,
+                                 int(bool(use_residual)), float(aux_coef), int(bool(normalize_by_k)),
+                                 _p(cnt, _I64), _p(dx, _D), _p(dW1, _D), _p(db1, _D), _p(dW2, _D), _p(db2, _D),
+                                 _p(dl, _D), _p(dg, _D))
+    return dx, dW1, db1, dW2, db2, dl, dg
 
 
 def combine_precomputed(u, selected, kept, gates, base=None) -> np.ndarray:

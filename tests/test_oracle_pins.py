@@ -477,6 +477,89 @@ def test_backward_swiglu_finite_differences(aux_coef, residual):
     assert math.isclose(dg[t, j], float(dy[t] @ o), rel_tol=1e-12)
 
 
+def _loss_gelu(x, s, w, dy, sel0, kept, k, aux_coef, counts0, residual):
+    probs, sel, gates, _, psum = O.route(s, k)
+    assert (sel == sel0).all(), "perturbation changed the top-k decision"
+    y = O.layer_rows("gelu_mlp", x, sel, kept, gates, w, base_kind="input" if residual else "zero")
+    _, _, aux = O.aux(counts0, psum, x.shape[0], k, normalize_by_k=True)
+    return float((dy * y).sum() + aux_coef * aux)
+
+
+@pytest.mark.parametrize("aux_coef,residual", [(0.0, True), (0.41, False)])
+def test_backward_gelu_finite_differences(aux_coef, residual):
+    # The GELU-MLP expert (fc2(gelu(fc1 x)), biases on both layers) under the
+    # numpy-layer page's backward rules, against central differences of y . dy (+ aux).
+    ver = _golden("numpy_layer_verification.json")
+    rng = np.random.default_rng(31)
+    T, D, F, E, k = 7, 4, 5, 4, 2
+    x = rng.standard_normal((T, D))
+    s = rng.standard_normal((T, E))
+    w = {"w1": rng.standard_normal((E, D, F)) * 0.8, "b1": rng.standard_normal((E, F)) * 0.5,
+         "w2": rng.standard_normal((E, F, D)) * 0.8, "b2": rng.standard_normal((E, D)) * 0.5}
+    dy = rng.standard_normal((T, D))
+    C = 3  # forces drops
+    out = O.forward("gelu_mlp", x, s, k, C, w, base_kind="input" if residual else "zero")
+    sel, kept, counts = out["selected"], out["kept"], out["counts"]
+    assert (~kept).any()
+    dx, dW1, db1, dW2, db2, dl, dg = O.backward_gelu(dy, x, s, sel, kept, out["gates"], w["w1"], w["b1"],
+                                                     w["w2"], w["b2"], use_residual=residual,
+                                                     aux_coef=aux_coef, counts=counts)
+    h = 1e-6
+
+    def fd(arr):
+        g = np.zeros_like(arr)
+        it = np.nditer(arr, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            a0 = arr[i]
+            arr[i] = a0 + h
+            lp = _loss_gelu(x, s, w, dy, sel, kept, k, aux_coef, counts, residual)
+            arr[i] = a0 - h
+            lm = _loss_gelu(x, s, w, dy, sel, kept, k, aux_coef, counts, residual)
+            arr[i] = a0
+            g[i] = (lp - lm) / (2 * h)
+        return g
+
+    bound = 10 * max(ver["backward_vs_finite_difference_max_err"].values())
+    assert np.abs(fd(x) - dx).max() < bound
+    assert np.abs(fd(s) - dl).max() < bound
+    assert np.abs(fd(w["w1"]) - dW1).max() < bound
+    assert np.abs(fd(w["b1"]) - db1).max() < bound
+    assert np.abs(fd(w["w2"]) - dW2).max() < bound
+    assert np.abs(fd(w["b2"]) - db2).max() < bound
+    assert (dg[~kept] == 0).all()
+    t, j = np.argwhere(kept)[0]
+    o = O.expert_rows("gelu_mlp", x, [t], [sel[t, j]], w)[0]
+    assert math.isclose(dg[t, j], float(dy[t] @ o), rel_tol=1e-12)
+
+
+def test_backward_gelu_bias_gradients_closed_form():
+    # One expert, top-1, D = F = N = 1, x = 0: z = b1, so
+    #   db2 = sum_t dy_t,  db1 = W2 * gelu'(b1) * sum_t dy_t,  dW1 = 0,
+    # with gelu'(z) = Phi(z) + z phi(z) from scipy's normal distribution.
+    from scipy.stats import norm
+    T = 5
+    x = np.zeros((T, 1))
+    s = np.zeros((T, 1))
+    dy = np.arange(1.0, T + 1.0).reshape(T, 1)
+    b1v, w2v = 0.7, -1.3
+    w = {"w1": np.full((1, 1, 1), 2.0), "b1": np.full((1, 1), b1v), "w2": np.full((1, 1, 1), w2v),
+         "b2": np.full((1, 1), 0.25)}
+    out = O.forward("gelu_mlp", x, s, 1, T, w)
+    dx, dW1, db1, dW2, db2, dl, dg = O.backward_gelu(dy, x, s, out["selected"], out["kept"], out["gates"],
+                                                     w["w1"], w["b1"], w["w2"], w["b2"])
+    S = float(dy.sum())
+    gprime = norm.cdf(b1v) + b1v * norm.pdf(b1v)
+    assert math.isclose(float(db2[0, 0]), S, rel_tol=1e-14)
+    assert math.isclose(float(db1[0, 0]), w2v * gprime * S, rel_tol=1e-13)
+    assert float(dW1[0, 0, 0]) == 0.0
+    # dW2 = gelu(b1) * sum dy with gelu(z) = z Phi(z)
+    assert math.isclose(float(dW2[0, 0, 0]), b1v * norm.cdf(b1v) * S, rel_tol=1e-13)
+    # dx_t = dy_t * W2 * gelu'(b1) * W1
+    np.testing.assert_allclose(dx[:, 0], dy[:, 0] * w2v * gprime * 2.0, rtol=1e-13)
+    assert np.abs(dl).max() == 0.0
+
+
 def test_backward_swiglu_down_gradient_closed_form_and_top1():
     # With one hidden unit (F = 1) the down-projection gradient has a closed
     # form: dWd_e = sum over kept tokens of e of g * silu(a) * b * dy, with
