@@ -558,7 +558,40 @@ def run_other_workloads(steps, warmup, flush, stream, dev):
                       frac=3 * flops / f_s / 1e12 / tf32_peak(pk), traffic=None, avg_launch_ms=1e3 * f_s,
                       fp32_tflops=flops / f_s / 1e12, peak_source=TF32_PEAK_SOURCE,
                       note="three tf32 MMAs per fp32 product; launch-latency bound at this size"))
-    del dv
+
+    # the same layer's training step: forward, GELU-expert backward, router backward (fp32)
+    dyg = torch.randn(T, D, generator=torch.Generator().manual_seed(2)).to(dev)
+    wsg = torch.empty(B.moe_backward_gelu_workspace_size(E, C, D, F, D), dtype=torch.uint8, device=dev)
+    inner = []
+    kept_box = {}
+
+    def step_tiny_train():
+        r = moe.moe_route(dv["x"], k, w_router=dv["w_router"], want_logits=True)
+        d = moe.moe_dispatch(r["selected"], E, C, x=dv["x"])
+        yb = moe.moe_expert_ffn("gelu_mlp", d["xbuf"], d["used"], dv["w1"], b1=dv["b1"], w2=dv["w2"], b2=dv["b2"])
+        moe.moe_combine(yb, r["selected"], d["slot"], r["gates_f32"], base_kind="input", base=dv["x"])
+        e0, e1 = events(inner)
+        e0.record(stream)
+        g = moe.moe_backward_gelu(dyg, r["logits"], r["selected"], r["gates_f32"], d["slot"], d["used"], d["xbuf"],
+                                  yb, dv["w1"], dv["b1"], dv["w2"], C, use_residual=True, workspace=wsg)
+        e1.record(stream)
+        moe.moe_router_backward(dv["x"], dv["w_router"], g[5])
+        kept_box["used"] = d["used"]
+
+    sm, im = _time_steps(step_tiny_train, steps, warmup, flush, stream, inner)
+    kept = int(kept_box["used"].sum())
+    b_s = statistics.mean(im) / 1e3
+    flops_b = 2.0 * kept * D * F * 5  # recomputed z, dh, dW2, dW1, dx: 2*kept*D*F each
+    out["tiny_gelu_fp32_train"] = dict(
+        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+        config=dict(T=T, D=D, E=E, F=F, k=k, capacity=C, kept=kept,
+                    step="forward + moe_backward_gelu + moe_router_backward"),
+        roofline=dict(bound="tensor", kernel="moe_backward_gelu (tf32x3_kernel x5, elementwise, sums, combine)",
+                      achieved=3 * flops_b / b_s / 1e12, peak=tf32_peak(pk), unit="TFLOP/s",
+                      frac=3 * flops_b / b_s / 1e12 / tf32_peak(pk), traffic=None, avg_launch_ms=1e3 * b_s,
+                      fp32_tflops=flops_b / b_s / 1e12, peak_source=TF32_PEAK_SOURCE,
+                      note="launch-latency bound at this size"))
+    del dv, dyg, wsg
 
     # forward + backward, fp32, linear experts with residual
     c = I.fwd_bwd_fp32(seed=0)

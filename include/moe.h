@@ -263,13 +263,13 @@ MOE_API int moe_dispatch(const int64_t* selected, int64_t T, int32_t k, int32_t 
  *
  * This entry point takes no workspace.  The slot scan's look-back state lives
  * in one fixed file-scope device array of moe_dispatch_static_max_state_bytes()
- * bytes (1 MiB) that every GPU which loads the library holds until the process
+ * bytes (4 MiB) that every GPU which loads the library holds until the process
  * exits.  The call allocates nothing: no cudaMalloc, cudaFree or allocating
  * library routine.
  *
  * Arguments and outputs: as moe_dispatch, without workspace/workspace_bytes.
- * Limit: ceil(T/512) * E * 4 + 4 bytes of state, rounded up to 256, must fit in
- * the array (E = 256 allows T <= 523776); a larger problem returns
+ * Limit: ceil(T/128) * E * 4 + 4 bytes of state, rounded up to 256, must fit in
+ * the array (E = 256 allows T <= 524160); a larger problem returns
  * MOE_ERR_UNSUPPORTED and enqueues nothing.
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
@@ -461,6 +461,43 @@ MOE_API int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float* lo
                                 float* dw_gate, float* dw_up, float* dw_down, float* dlogits, float* dgate,
                                 int32_t* dev_status, void* workspace, size_t workspace_bytes,
                                 moe_stream_t stream);
+
+/*
+ * moe_backward_gelu -- backward of the GELU-MLP-expert layer ([P5] Expert:
+ * fc2(gelu(fc1(x))) with biases, exact erf GELU) under the same rules as
+ * moe_backward: kept mask and drops constant, gates = softmax of the
+ * selected logits.  fp32 throughout; the products run on the tensor cores as
+ * split-tf32 (fp32 accuracy).  For a kept (t,j) -> e with
+ * z = x_t W1_e^T + b1_e, h = gelu(z), o = h W2_e^T + b2_e:
+ *   dgate[t,j] = dy_t . o        (o read from the forward's ybuf)
+ *   dlogits    as in moe_backward
+ *   do = gate dy_t,  dh = do W2_e,  dz = dh * gelu'(z),
+ *   gelu'(z) = Phi(z) + z phi(z)  (standard normal CDF and density)
+ *   dw2[e] += do^T h   (E, Dout, F)     db2[e] += do   (E, Dout)
+ *   dw1[e] += dz^T x_t (E, F, D)        db1[e] += dz   (E, F)
+ *   dx[t]   = [dy_t] + sum_kept dz W1_e                 (T, D)
+ * z is recomputed from xbuf.  Bias gradients are summed over the kept rows
+ * of each expert in slot order.
+ *
+ * Arguments (device): dy (T, Dout); logits fp32 (T, E); selected int64,
+ *   gates fp32, slot int64 (T, k); used int32 (E); xbuf (E, C, D) and ybuf
+ *   (E, C, Dout) from the forward; w1 (E, F, D), b1 (E, F), w2 (E, Dout, F)
+ *   as for moe_expert_ffn (b2 does not enter the gradients); counts int32
+ *   (E) when aux_coef != 0.  dtype MOE_F32 (else MOE_ERR_UNSUPPORTED), k <= 64.
+ *   The residual term [dy_t] needs Dout == D.
+ *   Outputs: dx (T, D); dw1 (E, F, D); db1 (E, F); dw2 (E, Dout, F);
+ *   db2 (E, Dout); dlogits fp32 (T, E); dgate fp32 (T, k).
+ *   workspace >= moe_backward_gelu_workspace_size(E, C, D, F, Dout) bytes.
+ */
+MOE_API size_t moe_backward_gelu_workspace_size(int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout);
+MOE_API int moe_backward_gelu(moe_dtype dtype, const void* dy, const float* logits, const int64_t* selected,
+                              const float* gates, const int64_t* slot, const int32_t* used, const void* xbuf,
+                              const void* ybuf, const void* w1, const void* b1, const void* w2, int64_t T,
+                              int32_t k, int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout,
+                              int use_residual, float aux_coef, int normalize_by_k, const int32_t* counts,
+                              void* dx, float* dw1, float* db1, float* dw2, float* db2, float* dlogits,
+                              float* dgate, int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                              moe_stream_t stream);
 
 /*
  * moe_transpose_weights -- convert expert matrices from the pages' x @ W

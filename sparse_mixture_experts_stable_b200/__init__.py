@@ -7,8 +7,8 @@ preallocated buffers (``layer.py``) and the seeded synthetic workloads
 (``inputs.py``).
 """
 from .binding import (  # noqa: F401
-    EXPORTED, LIB_PATH, MoeError, lib, moe_aux_stats, moe_backward, moe_backward_swiglu, moe_capacity,
-    moe_clear_status, moe_combine, moe_dispatch, moe_dispatch_static, moe_expert_ffn, moe_expert_ffn_gathered,
-    moe_read_status, moe_renormalize_kept_gates, moe_route, moe_router_backward, moe_transpose_weights, new_status,
+    EXPORTED, LIB_PATH, MoeError, lib, moe_aux_stats, moe_backward, moe_backward_gelu, moe_backward_swiglu,
+    moe_capacity, moe_clear_status, moe_combine, moe_dispatch, moe_dispatch_static, moe_expert_ffn,
+    moe_expert_ffn_gathered, moe_read_status, moe_renormalize_kept_gates, moe_route, moe_router_backward, moe_transpose_weights, new_status,
     status_string,
 )

@@ -39,6 +39,7 @@ EXPORTED = [
     "moe_clear_status", "moe_read_status", "moe_dispatch_static_max_state_bytes", "moe_dispatch_static",
     "moe_route_ex", "moe_renormalize_kept_gates", "moe_expert_ffn_gathered", "moe_backward_swiglu_workspace_size",
     "moe_backward_swiglu", "moe_router_backward_workspace_size", "moe_router_backward",
+    "moe_backward_gelu_workspace_size", "moe_backward_gelu",
 ]
 SCORING = {"softmax": 0, "sigmoid": 1}
 
@@ -100,6 +101,11 @@ def lib():
         L.moe_backward_swiglu.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                           _i32, _i32, _i64, _i64, _i64, ctypes.c_int, _f32, ctypes.c_int, _vp, _vp,
                                           _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_backward_gelu_workspace_size.restype = _sz
+        L.moe_backward_gelu_workspace_size.argtypes = [_i32, _i64, _i64, _i64, _i64]
+        L.moe_backward_gelu.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+                                        _i32, _i32, _i64, _i64, _i64, _i64, ctypes.c_int, _f32, ctypes.c_int, _vp,
+                                        _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
         L.moe_backward_workspace_size.restype = _sz
         L.moe_backward_workspace_size.argtypes = [_i32, _i64, _i64, _i64]
         L.moe_backward.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -467,6 +473,40 @@ def moe_backward_swiglu(dy, logits, selected, gates_f32, slot, used, xbuf, ybuf,
                                    ws.numel(), _stream(stream))
     _check("moe_backward_swiglu", rc)
     return dx, dwg, dwu, dwd, dl, dg
+
+
+def moe_backward_gelu_workspace_size(E: int, C: int, D: int, F: int, Dout: int) -> int:
+    return int(lib().moe_backward_gelu_workspace_size(E, C, D, F, Dout))
+
+
+def moe_backward_gelu(dy, logits, selected, gates_f32, slot, used, xbuf, ybuf, w1, b1, w2, C: int,
+                      use_residual: bool = False, aux_coef: float = 0.0, normalize_by_k: bool = True, counts=None,
+                      dev_status=None, workspace=None, stream=None):
+    """Backward of the fp32 GELU-MLP-expert layer (weights in the (out, in) layout:
+    w1 (E,F,D), b1 (E,F), w2 (E,Dout,F)).
+
+    Returns (dx (T,D), dw1 (E,F,D), db1 (E,F), dw2 (E,Dout,F), db2 (E,Dout),
+    dlogits (T,E), dgate (T,k)), all fp32.
+    """
+    dev = _dev(dy)
+    T, Dout = dy.shape
+    E, F, D = w1.shape
+    k = selected.shape[1]
+    dx = torch.empty(T, D, dtype=torch.float32, device=dev)
+    dw1 = torch.empty(E, F, D, dtype=torch.float32, device=dev)
+    db1 = torch.empty(E, F, dtype=torch.float32, device=dev)
+    dw2 = torch.empty(E, Dout, F, dtype=torch.float32, device=dev)
+    db2 = torch.empty(E, Dout, dtype=torch.float32, device=dev)
+    dl = torch.empty(T, E, dtype=torch.float32, device=dev)
+    dg = torch.empty(T, k, dtype=torch.float32, device=dev)
+    ws = _workspace(moe_backward_gelu_workspace_size(E, C, D, F, Dout), dev, workspace)
+    rc = lib().moe_backward_gelu(_dt(dy), _p(dy), _p(logits), _p(selected), _p(gates_f32), _p(slot), _p(used),
+                                 _p(xbuf), _p(ybuf), _p(w1), _p(b1), _p(w2), T, k, E, C, D, F, Dout,
+                                 int(bool(use_residual)), float(aux_coef), int(bool(normalize_by_k)), _p(counts),
+                                 _p(dx), _p(dw1), _p(db1), _p(dw2), _p(db2), _p(dl), _p(dg), _p(dev_status),
+                                 _p(ws), ws.numel(), _stream(stream))
+    _check("moe_backward_gelu", rc)
+    return dx, dw1, db1, dw2, db2, dl, dg
 
 
 def moe_transpose_weights(src: torch.Tensor, stream=None) -> torch.Tensor:

@@ -465,3 +465,223 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     return combine_rows(dxbuf, selected, slot, nullptr, MOE_F32, T, k, E, C, H, use_residual ? dy : nullptr, H, dx,
                         H, MOE_BF16, dev_status, stream);
 }
+
+// ---------------------------------------------------------------------------
+// moe_backward_gelu: fp32 GELU-MLP experts (fc2(gelu(fc1 x)), both layers with
+// bias), the kept mask held constant.
+//   1. dgate / dlogits                       as above
+//   2. dybuf[e,c] = gate * dy[token]         scaled gather
+//   3. z  = xbuf W1^T + b1                   split-tf32 GEMM, bias epilogue
+//   4. dh = dybuf W2                         split-tf32 GEMM
+//   5. h = gelu(z), dz = dh * gelu'(z)       elementwise, in place over z and dh
+//   6. dW2 = dybuf^T h,  dW1 = dz^T xbuf     split-tf32 GEMMs, K = used[e] tokens
+//   7. db2 = column sums of dybuf, db1 = column sums of dz (c < used[e], fixed order)
+//   8. dxbuf = dz W1                         split-tf32 GEMM
+//   9. dx[t] = [dy[t]] + sum_kept dxbuf[e, slot]
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+// In place over the first used[e] rows of expert e:
+//   z  <- gelu(z)                       = z Phi(z)
+//   dh <- dh * gelu'(z),  gelu'(z)      = Phi(z) + z phi(z)
+// with Phi the standard normal CDF (through erff) and phi its density.
+__global__ void gelu_bwd_elem_kernel(float* __restrict__ z, float* __restrict__ dh, const int32_t* __restrict__ used,
+                                     int64_t C, int64_t F) {
+    const int e = blockIdx.y;
+    const int64_t u = used[e] < 0 ? 0 : (used[e] < C ? used[e] : C);
+    const int64_t n = u * F;
+    float* ze = z + (int64_t)e * C * F;
+    float* de = dh + (int64_t)e * C * F;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = ze[i];
+        const float cdf = 0.5f * (1.0f + erff(v * 0.70710678118654752f));
+        const float pdf = 0.39894228040143268f * expf(-0.5f * v * v);
+        ze[i] = v * cdf;
+        de[i] *= cdf + v * pdf;
+    }
+}
+
+// out[g][n] = sum_{r < valid[g]} src[g][r][n], r ascending (one thread per column).
+__global__ void group_column_sum_kernel(const float* __restrict__ src, int64_t R, int64_t N,
+                                        const int32_t* __restrict__ valid, float* __restrict__ out) {
+    const int g = blockIdx.y;
+    const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= N) return;
+    const int64_t u = valid[g] < 0 ? 0 : (valid[g] < R ? valid[g] : R);
+    const float* s = src + (int64_t)g * R * N + n;
+    float acc = 0.f;
+    for (int64_t r = 0; r < u; ++r) acc += s[r * N];
+    out[(int64_t)g * N + n] = acc;
+}
+
+struct GeluBwdWs {
+    size_t dybuf, z, dh, dxbuf, split, total;
+};
+
+// The five split-tf32 GEMMs (operand pointers filled in by the caller).
+void gelu_bwd_shapes(int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout, F32Gemm (&s)[5]) {
+    for (auto& q : s) {
+        q = F32Gemm{};
+        q.groups = E;
+    }
+    // 0: z (C x F) = xbuf (C x D) . W1^T, W1 (F, D)
+    s[0].lda = D; s[0].a_group_stride = C * D;
+    s[0].ldb = D; s[0].b_trans = true; s[0].b_group_stride = F * D;
+    s[0].ldc = F; s[0].c_group_stride = C * F;
+    s[0].M = C; s[0].N = F; s[0].K = D; s[0].rows_mode = 1;
+    s[0].bias_group_stride = F; s[0].epilogue = F32_EPI_BIAS;
+    // 1: dh (C x F) = dybuf (C x Dout) . W2, W2 (Dout, F)
+    s[1].lda = Dout; s[1].a_group_stride = C * Dout;
+    s[1].ldb = F; s[1].b_group_stride = Dout * F;
+    s[1].ldc = F; s[1].c_group_stride = C * F;
+    s[1].M = C; s[1].N = F; s[1].K = Dout; s[1].rows_mode = 1;
+    // 2: dW2 (Dout x F) = dybuf^T (Dout x C) . h (C x F)
+    s[2].lda = Dout; s[2].a_trans = true; s[2].a_group_stride = C * Dout;
+    s[2].ldb = F; s[2].b_group_stride = C * F;
+    s[2].ldc = F; s[2].c_group_stride = Dout * F;
+    s[2].M = Dout; s[2].N = F; s[2].K = C; s[2].rows_mode = 2;
+    // 3: dW1 (F x D) = dz^T (F x C) . xbuf (C x D)
+    s[3].lda = F; s[3].a_trans = true; s[3].a_group_stride = C * F;
+    s[3].ldb = D; s[3].b_group_stride = C * D;
+    s[3].ldc = D; s[3].c_group_stride = F * D;
+    s[3].M = F; s[3].N = D; s[3].K = C; s[3].rows_mode = 2;
+    // 4: dxbuf (C x D) = dz (C x F) . W1 (F x D)
+    s[4].lda = F; s[4].a_group_stride = C * F;
+    s[4].ldb = D; s[4].b_group_stride = F * D;
+    s[4].ldc = D; s[4].c_group_stride = C * D;
+    s[4].M = C; s[4].N = D; s[4].K = F; s[4].rows_mode = 1;
+}
+
+GeluBwdWs gelu_bwd_layout(int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout) {
+    GeluBwdWs w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += align_up(bytes, 1024);
+        return o;
+    };
+    w.dybuf = take((size_t)E * C * Dout * 4);
+    w.z = take((size_t)E * C * F * 4);
+    w.dh = take((size_t)E * C * F * 4);
+    w.dxbuf = take((size_t)E * C * D * 4);
+    F32Gemm s[5];
+    gelu_bwd_shapes(E, C, D, F, Dout, s);
+    size_t split = 0;
+    for (const auto& q : s) {
+        const size_t b = tf32x3_workspace_size(q);
+        split = b > split ? b : split;
+    }
+    w.split = take(split);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" size_t moe_backward_gelu_workspace_size(int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout) {
+    if (E < 1 || C < 1 || D < 1 || F < 1 || Dout < 1) return 256;
+    return gelu_bwd_layout(E, C, D, F, Dout).total;
+}
+
+extern "C" int moe_backward_gelu(moe_dtype dtype, const void* dy, const float* logits, const int64_t* selected,
+                                 const float* gates, const int64_t* slot, const int32_t* used, const void* xbuf,
+                                 const void* ybuf, const void* w1, const void* b1, const void* w2, int64_t T,
+                                 int32_t k, int32_t E, int64_t C, int64_t D, int64_t F, int64_t Dout,
+                                 int use_residual, float aux_coef, int normalize_by_k, const int32_t* counts,
+                                 void* dx, float* dw1, float* db1, float* dw2, float* db2, float* dlogits,
+                                 float* dgate, int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                                 moe_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    MOE_REQUIRE(dtype == MOE_F32, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(dy && logits && selected && gates && slot && used && dx && dw1 && db1 && dw2 && db2 && dlogits &&
+                    dgate,
+                MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(C == 0 || (xbuf && ybuf && w1 && b1 && w2), MOE_ERR_INVALID_ARG);  // unread when C == 0
+    MOE_REQUIRE(T >= 1 && k >= 1 && k <= E && E >= 1 && C >= 0 && D >= 1 && F >= 1 && Dout >= 1,
+                MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(k <= 64 && E <= 65535, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(!use_residual || Dout == D, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aux_coef == 0.f || counts != nullptr, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(workspace && workspace_bytes >= moe_backward_gelu_workspace_size(E, C, D, F, Dout),
+                MOE_ERR_WORKSPACE);
+
+    const unsigned grid = (unsigned)((T + kWarps - 1) / kWarps);
+    dgate_dlogits_kernel<float><<<grid, kWarps * 32, 0, stream>>>(
+        static_cast<const float*>(dy), Dout, static_cast<const float*>(ybuf), logits, selected, gates, slot, T, k, E,
+        C, aux_coef, normalize_by_k ? (float)k : 1.0f, counts, dlogits, dgate, dev_status);
+    int rc = launch_status();
+    if (rc != MOE_OK) return rc;
+
+    if (C == 0) {  // nothing kept: no expert gradient
+        MOE_CUDA_TRY(cudaMemsetAsync(dw1, 0, (size_t)E * F * D * 4, stream));
+        MOE_CUDA_TRY(cudaMemsetAsync(db1, 0, (size_t)E * F * 4, stream));
+        MOE_CUDA_TRY(cudaMemsetAsync(dw2, 0, (size_t)E * Dout * F * 4, stream));
+        MOE_CUDA_TRY(cudaMemsetAsync(db2, 0, (size_t)E * Dout * 4, stream));
+        if (use_residual)
+            MOE_CUDA_TRY(cudaMemcpyAsync(dx, dy, (size_t)T * D * 4, cudaMemcpyDeviceToDevice, stream));
+        else
+            MOE_CUDA_TRY(cudaMemsetAsync(dx, 0, (size_t)T * D * 4, stream));
+        return MOE_OK;
+    }
+
+    const GeluBwdWs l = gelu_bwd_layout(E, C, D, F, Dout);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* dybuf = reinterpret_cast<float*>(ws + l.dybuf);
+    float* z = reinterpret_cast<float*>(ws + l.z);
+    float* dh = reinterpret_cast<float*>(ws + l.dh);
+    float* dxbuf = reinterpret_cast<float*>(ws + l.dxbuf);
+    void* split = ws + l.split;
+    const size_t split_bytes = workspace_bytes - l.split;
+    const float* xb = static_cast<const float*>(xbuf);
+    F32Gemm s[5];
+    gelu_bwd_shapes(E, C, D, F, Dout, s);
+    for (auto& q : s) q.rows = used;
+    auto run = [&](const F32Gemm& q) { return tf32x3_gemm_run(q, split, split_bytes, dev_status, stream); };
+
+    // 2. dybuf[e,c] = gate * dy[token]
+    rc = gather_rows(dy, Dout, T, k, selected, slot, E, C, gates, dybuf, Dout, MOE_F32, dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    // 3. z = xbuf W1^T + b1
+    s[0].A = xb;
+    s[0].B = static_cast<const float*>(w1);
+    s[0].bias = static_cast<const float*>(b1);
+    s[0].C = z;
+    if ((rc = run(s[0])) != MOE_OK) return rc;
+    // 4. dh = dybuf W2
+    s[1].A = dybuf;
+    s[1].B = static_cast<const float*>(w2);
+    s[1].C = dh;
+    if ((rc = run(s[1])) != MOE_OK) return rc;
+    // 5. h = gelu(z) (into z), dz = dh * gelu'(z) (into dh)
+    {
+        const int64_t blocks = (C * F + 255) / 256;
+        const dim3 g2((unsigned)(blocks < 1024 ? blocks : 1024), (unsigned)E);
+        gelu_bwd_elem_kernel<<<g2, 256, 0, stream>>>(z, dh, used, C, F);
+        if ((rc = launch_status()) != MOE_OK) return rc;
+    }
+    // 6. dW2 = dybuf^T h,  dW1 = dz^T xbuf
+    s[2].A = dybuf;
+    s[2].B = z;
+    s[2].C = dw2;
+    if ((rc = run(s[2])) != MOE_OK) return rc;
+    s[3].A = dh;
+    s[3].B = xb;
+    s[3].C = dw1;
+    if ((rc = run(s[3])) != MOE_OK) return rc;
+    // 7. bias gradients
+    group_column_sum_kernel<<<dim3((unsigned)((Dout + 255) / 256), (unsigned)E), 256, 0, stream>>>(dybuf, C, Dout,
+                                                                                                   used, db2);
+    if ((rc = launch_status()) != MOE_OK) return rc;
+    group_column_sum_kernel<<<dim3((unsigned)((F + 255) / 256), (unsigned)E), 256, 0, stream>>>(dh, C, F, used, db1);
+    if ((rc = launch_status()) != MOE_OK) return rc;
+    // 8. dxbuf = dz W1
+    s[4].A = dh;
+    s[4].B = static_cast<const float*>(w1);
+    s[4].C = dxbuf;
+    if ((rc = run(s[4])) != MOE_OK) return rc;
+    // 9. dx
+    return combine_rows(dxbuf, selected, slot, nullptr, MOE_F32, T, k, E, C, D, use_residual ? dy : nullptr, D, dx, D,
+                        MOE_F32, dev_status, stream);
+}

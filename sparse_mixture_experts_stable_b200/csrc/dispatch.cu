@@ -18,7 +18,7 @@ namespace {
 
 constexpr int kScanThreads = 512;
 constexpr int kScanWarps = kScanThreads / 32;
-constexpr int kScanTokens = 512;
+constexpr int kScanTokens = 128;  // 128 blocks at T = 16384: most SMs take part
 constexpr uint32_t kFlagAgg = 1u << 30;   // block aggregate published
 constexpr uint32_t kFlagPre = 2u << 30;   // inclusive prefix published
 constexpr uint32_t kValMask = (1u << 30) - 1;
@@ -205,7 +205,7 @@ int dispatch_check_args(const int64_t* selected, int64_t T, int32_t k, int32_t E
     MOE_REQUIRE(C == 0 || token_of_slot != nullptr, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(T >= 1 && k >= 1 && E >= 1 && C >= 0, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(T * (int64_t)k < (int64_t(1) << 30) && C < (int64_t(1) << 30), MOE_ERR_UNSUPPORTED);
-    MOE_REQUIRE(E <= 2048 && k <= 64, MOE_ERR_UNSUPPORTED);  // scan smem: (16 E + 512) * 4 bytes
+    MOE_REQUIRE(E <= 2048 && k <= 64, MOE_ERR_UNSUPPORTED);  // scan smem: (16 E + 128) * 4 bytes
     if (x) {
         MOE_REQUIRE(valid_dtype(dtype) && (xbuf || C == 0) && D >= 1 && ldx >= D, MOE_ERR_INVALID_ARG);
     }

@@ -18,8 +18,8 @@
 namespace moe {
 namespace {
 
-// 1 MiB of look-back state: ceil(T / 512) * E + 1 words must fit.
-constexpr size_t kStaticScanWords = size_t(1) << 18;
+// 4 MiB of look-back state: ceil(T / 128) * E + 1 words must fit.
+constexpr size_t kStaticScanWords = size_t(1) << 20;
 static __device__ __align__(256) uint32_t g_scan_scratch[kStaticScanWords];
 
 constexpr int kMaxDevices = 64;

@@ -97,3 +97,21 @@ def test_workspace_sizes():
     # fp32 adds the split-tf32 operands: hi and lo of rows and weights, K rounded up to 32
     assert moe.binding.moe_expert_ffn_workspace_size("linear", B.MOE_F32, 8, 16, 64, 0, 48) >= 2 * 4 * (8 * 16 * 64 + 8 * 48 * 64)
     assert moe.binding.moe_backward_workspace_size(64, 256, 1024, 1024) >= 2 * 64 * 256 * 1024 * 4
+    # GELU backward: dybuf, z, dh, dxbuf (fp32) plus the split operands
+    E, C, D, F = 8, 160, 64, 256
+    assert moe.binding.moe_backward_gelu_workspace_size(E, C, D, F, D) >= 4 * E * C * (D + 2 * F + D)
+    assert moe.binding.moe_backward_gelu_workspace_size(E, 0, D, F, D) > 0
+
+
+def test_backward_gelu_host_checks():
+    L = moe.lib()
+    p, nul = ctypes.c_void_p(16), None
+
+    def call(dtype, T=8, k=2, E=4, C=4, D=16, F=16, Dout=16, residual=0, ws_bytes=1 << 30):
+        return L.moe_backward_gelu(dtype, p, p, p, p, p, p, p, p, p, p, p, T, k, E, C, D, F, Dout, residual, 0.0, 1,
+                                   nul, p, p, p, p, p, p, p, nul, p, ws_bytes, nul)
+
+    assert call(B.MOE_BF16) == B.MOE_ERR_UNSUPPORTED        # fp32 only
+    assert call(B.MOE_F32, k=5) == B.MOE_ERR_INVALID_ARG     # k > E
+    assert call(B.MOE_F32, residual=1, Dout=8) == B.MOE_ERR_INVALID_ARG  # residual needs Dout == D
+    assert call(B.MOE_F32, ws_bytes=64) == B.MOE_ERR_WORKSPACE

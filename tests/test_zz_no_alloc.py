@@ -49,7 +49,7 @@ def test_static_dispatch_matches_workspace_dispatch_twice():
 def test_static_dispatch_rejects_problems_beyond_its_array():
     L = B.lib()
     limit = L.moe_dispatch_static_max_state_bytes()
-    assert limit == 1 << 20
+    assert limit == 4 << 20
     p = ctypes.c_void_p(16)
     # E = 256 and T = 600000 need more look-back state than the array holds
     rc = L.moe_dispatch_static(p, 600000, 1, 256, 10, None, 0, 0, 0, p, p, p, p, p, p, None, None, None)
