@@ -500,6 +500,102 @@ MOE_API int moe_backward_gelu(moe_dtype dtype, const void* dy, const float* logi
                               moe_stream_t stream);
 
 /*
+ * Expert parallelism over R ranks (one process per GPU).  Rank r holds T_r
+ * tokens and experts [r E/R, (r+1) E/R) with their weights.  The layer over
+ * the R ranks equals the layer over the whole batch with the tokens in rank
+ * order: expert e keeps at most C assignments, C = ceil(cf * T * k / E) for
+ * the global T, which is also ceil(cf * T_r * k / (E/R)) when every rank has
+ * T_r = T / R tokens ([P1] section 1 item 2: the capacity does not change
+ * with the expert-parallel world size).  Greedy position priority across
+ * ranks: rank r's assignments to expert e take the slots after those of
+ * ranks 0..r-1.  [P3]'s expert-parallel payload (T k D values each way) is
+ * moved by moe_ep_dispatch and moe_ep_combine themselves, reading and
+ * writing the other ranks' buffers through peer memory.
+ *
+ * One step on rank r:
+ *   1. moe_route on the local tokens -> selected, gates, counts (E).
+ *   2. gather every rank's counts into counts_all (R, E) (caller: e.g. an
+ *      NCCL all-gather), then moe_ep_plan.
+ *   3. moe_ep_dispatch: slots and rows into the owner ranks' xbuf.
+ *   4. barrier (every rank's rows have landed).
+ *   5. moe_expert_ffn on the local (E/R, C, D) xbuf with used + r E/R.
+ *   6. barrier (every expert output is written).
+ *   7. moe_ep_combine from the owner ranks' ybuf.
+ * Barrier 4 of the next step also orders this step's combine reads before
+ * the next expert FFN overwrites ybuf.  The buffers of the other ranks are
+ * mapped once with moe_ipc_export / moe_ipc_import.
+ */
+
+/*
+ * moe_ep_plan -- from every rank's pre-drop counts, this rank's slot base per
+ * expert and the global per-expert statistics.
+ *   counts_all   device int32 (R, E): row q = rank q's counts from moe_route.
+ *   rank_base    device int32 (E): sum_{q < rank} counts_all[q][e].
+ *   used         device int32 (E) or NULL: min(sum_q counts_all[q][e], C).
+ *   overflow     device int32 (E) or NULL: sum - used.
+ *   counts_total device int32 (E) or NULL: sum_q counts_all[q][e] (the global
+ *                counts for moe_aux_stats).
+ * Sums saturate at 2^31 - 1.
+ */
+MOE_API int moe_ep_plan(const int32_t* counts_all, int32_t R, int32_t rank, int32_t E, int64_t C,
+                        int32_t* rank_base, int32_t* used, int32_t* overflow, int32_t* counts_total,
+                        moe_stream_t stream);
+
+/*
+ * moe_ep_dispatch -- moe_dispatch for rank `rank` of an expert-parallel group:
+ * slot[t,j] = rank_base[e] + #{earlier local assignments to e}, kept iff
+ * slot < C; each kept row x[t] is written to row (e mod E/R) * C + slot of
+ * the expert-major buffer of rank e / (E/R).
+ *   selected     device int64 (T, k) local assignments; rank_base from
+ *                moe_ep_plan; token_base = global index of local token 0
+ *                (recorded in token_of_slot).
+ *   x            device (T, D), row stride ldx, dtype `dtype`; NULL skips the
+ *                row movement.
+ *   xbuf_ranks   HOST array of R device pointers: rank q's (E/R, C, D) buffer,
+ *                as mapped into this process (this rank's own buffer at q =
+ *                rank).  Rows are written with 16-byte vectors when every
+ *                pointer and the row pitch allow it.
+ *   slot (T, k) int64, kept (T, k) uint8, drops_per_token (T) int32: as
+ *                moe_dispatch, with global slots.
+ *   token_of_slot device int32 (E, C) or NULL: filled with -1, then
+ *                token_base + t at the slots this rank's tokens hold.
+ *   workspace    >= moe_dispatch_workspace_size(T, k, E) bytes.
+ * E must be a multiple of R; R <= 64; E <= 2048, k <= 64.
+ */
+MOE_API int moe_ep_dispatch(const int64_t* selected, int64_t T, int32_t k, int32_t E, int64_t C,
+                            const int32_t* rank_base, int64_t token_base, const void* x, moe_dtype dtype,
+                            int64_t D, int64_t ldx, void* const* xbuf_ranks, int32_t R, int64_t* slot,
+                            uint8_t* kept, int32_t* drops_per_token, int32_t* token_of_slot, int32_t* dev_status,
+                            void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * moe_ep_combine -- moe_combine reading each kept row from the owner rank:
+ *   y[t] = base[t] + sum_{j kept, ascending} gate[t,j] * ybuf_{e / (E/R)}[e mod E/R, slot[t,j]]
+ *   ybuf_ranks   HOST array of R device pointers to every rank's (E/R, C, N)
+ *                expert output buffer, as mapped into this process.
+ * Other arguments and the status word as moe_combine (E is the global
+ * expert count, a multiple of R).
+ */
+MOE_API int moe_ep_combine(const void* const* ybuf_ranks, int32_t R, const int64_t* selected, const int64_t* slot,
+                           const void* gates, moe_dtype gate_dtype, int64_t T, int32_t k, int32_t E, int64_t C,
+                           int64_t N, moe_base base_kind, const void* base, int64_t ldbase, void* y, int64_t ldy,
+                           moe_dtype dtype, int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * Peer mapping of device buffers between processes (CUDA IPC).
+ * moe_ipc_export: handle (host, MOE_IPC_HANDLE_BYTES) of the device
+ *   allocation holding dev_ptr, and the byte offset of dev_ptr in it.  The
+ *   memory must come from cudaMalloc (PyTorch's default allocator).
+ * moe_ipc_import: maps another process's allocation into this one; the
+ *   buffer is at *mapping + offset.  Release with moe_ipc_close(*mapping).
+ * Errors are returned as MOE_ERR_CUDA (nothing is left pending).
+ */
+#define MOE_IPC_HANDLE_BYTES 64
+MOE_API int moe_ipc_export(const void* dev_ptr, void* handle, int64_t* offset);
+MOE_API int moe_ipc_import(const void* handle, void** mapping);
+MOE_API int moe_ipc_close(void* mapping);
+
+/*
  * moe_transpose_weights -- convert expert matrices from the pages' x @ W
  * layout (E, K_in, N_out) to this library's (E, N_out, K_in), on device.
  * src and dst must not overlap.  dtype f32 or bf16.

@@ -39,8 +39,10 @@ EXPORTED = [
     "moe_clear_status", "moe_read_status", "moe_dispatch_static_max_state_bytes", "moe_dispatch_static",
     "moe_route_ex", "moe_renormalize_kept_gates", "moe_expert_ffn_gathered", "moe_backward_swiglu_workspace_size",
     "moe_backward_swiglu", "moe_router_backward_workspace_size", "moe_router_backward",
-    "moe_backward_gelu_workspace_size", "moe_backward_gelu",
+    "moe_backward_gelu_workspace_size", "moe_backward_gelu", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine",
+    "moe_ipc_export", "moe_ipc_import", "moe_ipc_close",
 ]
+IPC_HANDLE_BYTES = 64
 SCORING = {"softmax": 0, "sigmoid": 1}
 
 
@@ -111,6 +113,14 @@ def lib():
         L.moe_backward.argtypes = [ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, _i64, _i32, _i32, _i64, _i64, _i64, ctypes.c_int, _f32, ctypes.c_int, _vp,
                                    _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_ep_plan.argtypes = [_vp, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp]
+        L.moe_ep_dispatch.argtypes = [_vp, _i64, _i32, _i32, _i64, _vp, _i64, _vp, ctypes.c_int, _i64, _i64, _vp,
+                                      _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.moe_ep_combine.argtypes = [_vp, _i32, _vp, _vp, _vp, ctypes.c_int, _i64, _i32, _i32, _i64, _i64,
+                                     ctypes.c_int, _vp, _i64, _vp, _i64, ctypes.c_int, _vp, _vp]
+        L.moe_ipc_export.argtypes = [_vp, _vp, ctypes.POINTER(_i64)]
+        L.moe_ipc_import.argtypes = [_vp, ctypes.POINTER(_vp)]
+        L.moe_ipc_close.argtypes = [_vp]
         L.moe_transpose_weights.argtypes = [_vp, _vp, _i32, _i64, _i64, ctypes.c_int, _vp]
         L.moe_clear_status.argtypes = [_vp, _vp]
         L.moe_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_i32)]
@@ -507,6 +517,96 @@ def moe_backward_gelu(dy, logits, selected, gates_f32, slot, used, xbuf, ybuf, w
                                  _p(ws), ws.numel(), _stream(stream))
     _check("moe_backward_gelu", rc)
     return dx, dw1, db1, dw2, db2, dl, dg
+
+
+def _ptr_table(bufs):
+    """Host array of device pointers from tensors or integer addresses."""
+    addrs = [b.data_ptr() if isinstance(b, torch.Tensor) else int(b) for b in bufs]
+    return (ctypes.c_void_p * len(addrs))(*addrs), len(addrs)
+
+
+def moe_ep_plan(counts_all: torch.Tensor, rank: int, C: int, out: Optional[dict] = None, stream=None) -> dict:
+    """This rank's per-expert slot base and the global used/overflow/counts from every rank's counts (R, E)."""
+    dev = _dev(counts_all)
+    R, E = counts_all.shape
+    ca = counts_all.to(torch.int32).contiguous()
+    o = dict(out or {})
+    for key in ("rank_base", "used", "overflow", "counts_total"):
+        o.setdefault(key, torch.empty(E, dtype=torch.int32, device=dev))
+    rc = lib().moe_ep_plan(_p(ca), R, rank, E, C, _p(o["rank_base"]), _p(o["used"]), _p(o["overflow"]),
+                           _p(o["counts_total"]), _stream(stream))
+    _check("moe_ep_plan", rc)
+    return o
+
+
+def moe_ep_dispatch(selected: torch.Tensor, E: int, C: int, rank_base: torch.Tensor, token_base: int,
+                    x: Optional[torch.Tensor], xbuf_ranks, out: Optional[dict] = None,
+                    dev_status: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream=None) -> dict:
+    """Slots from this rank's base and the rows written into the owner ranks' buffers (list, one per rank)."""
+    dev = _dev(selected)
+    if selected.dtype != torch.int64:
+        raise TypeError("selected must be int64")
+    sel = selected.reshape(selected.shape[0], -1).contiguous()
+    T, k = sel.shape
+    o = dict(out or {})
+    o.setdefault("slot", torch.empty(T, k, dtype=torch.int64, device=dev))
+    o.setdefault("kept", torch.empty(T, k, dtype=torch.uint8, device=dev))
+    o.setdefault("drops", torch.empty(T, dtype=torch.int32, device=dev))
+    o.setdefault("token_of_slot", torch.empty(E, max(C, 0), dtype=torch.int32, device=dev))
+    dt, D, ldx = MOE_F32, 0, 0
+    if x is not None:
+        dt, D, ldx = _dt(x), x.shape[1], _rowstride(x)
+    tab, R = _ptr_table(xbuf_ranks)
+    ws = _workspace(moe_dispatch_workspace_size(T, k, E), dev, workspace)
+    rc = lib().moe_ep_dispatch(_p(sel), T, k, E, C, _p(rank_base), int(token_base), _p(x), dt, D, ldx, tab, R,
+                               _p(o["slot"]), _p(o["kept"]), _p(o["drops"]), _p(o["token_of_slot"]),
+                               _p(dev_status), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_ep_dispatch", rc)
+    return o
+
+
+def moe_ep_combine(ybuf_ranks, selected: torch.Tensor, slot: torch.Tensor, gates: Optional[torch.Tensor], E: int,
+                   C: int, N: int, dtype: torch.dtype, base_kind: str = "zero", base: Optional[torch.Tensor] = None,
+                   y: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """moe_combine reading every kept row from its owner rank's output buffer (list, one per rank)."""
+    dev = _dev(selected)
+    sel = selected.reshape(selected.shape[0], -1).contiguous()
+    T, k = sel.shape
+    sl = slot.reshape(T, k).contiguous()
+    g = None if gates is None else gates.reshape(T, k).contiguous()
+    gdt = MOE_F32 if g is None else _dt(g)
+    if y is None:
+        y = torch.empty(T, N, dtype=dtype, device=dev)
+    tab, R = _ptr_table(ybuf_ranks)
+    ldb = _rowstride(base) if base is not None else 0
+    rc = lib().moe_ep_combine(tab, R, _p(sel), _p(sl), _p(g), gdt, T, k, E, C, N, BASE[base_kind], _p(base), ldb,
+                              _p(y), _rowstride(y), _dt(y), _p(dev_status), _stream(stream))
+    _check("moe_ep_combine", rc)
+    return y
+
+
+def moe_ipc_export(t: torch.Tensor):
+    """(handle bytes, byte offset) of the device allocation holding ``t``."""
+    h = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = _i64(0)
+    _check("moe_ipc_export", lib().moe_ipc_export(_p(t), h, ctypes.byref(off)))
+    return h.raw, int(off.value)
+
+
+def moe_ipc_import(handle: bytes) -> int:
+    """Maps another process's allocation; returns the mapping's device address."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("IPC handle must be %d bytes" % IPC_HANDLE_BYTES)
+    m = _vp(0)
+    _check("moe_ipc_import", lib().moe_ipc_import(ctypes.create_string_buffer(handle, IPC_HANDLE_BYTES),
+                                                  ctypes.byref(m)))
+    return int(m.value)
+
+
+def moe_ipc_close(mapping: int):
+    _check("moe_ipc_close", lib().moe_ipc_close(_vp(mapping)))
 
 
 def moe_transpose_weights(src: torch.Tensor, stream=None) -> torch.Tensor:

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kScanThreads)
                      int64_t* __restrict__ slot, uint8_t* __restrict__ kept, int32_t* __restrict__ used,
                      int32_t* __restrict__ overflow, int32_t* __restrict__ drops,
                      int32_t* __restrict__ token_of_slot, uint32_t* __restrict__ state, uint32_t* ticket,
-                     int32_t* status) {
+                     int32_t* status, const int32_t* __restrict__ rank_base, int64_t token_base) {
     extern __shared__ int s_dyn[];
     int* s_off = s_dyn;                          // [kScanWarps][E]: per-warp running rank
     int* s_drop = s_off + kScanWarps * E;        // [kScanTokens]
@@ -126,8 +126,10 @@ __global__ void __launch_bounds__(kScanThreads)
             if (timed_out) set_status(status, MOE_ERR_TIMEOUT);
             st_release(mine, kFlagPre | ((excl + agg) & kValMask));
         }
-        for (int w = 0; w < kScanWarps; ++w) s_off[w * E + e] += (int)excl;
-        if (bid == nblocks - 1) {
+        // expert parallelism: the assignments of lower ranks come first
+        const int rb = rank_base ? rank_base[e] : 0;
+        for (int w = 0; w < kScanWarps; ++w) s_off[w * E + e] += (int)excl + rb;
+        if (bid == nblocks - 1 && rank_base == nullptr) {
             const int64_t total = (int64_t)excl + agg;
             const int64_t u = total < C ? total : C;
             used[e] = (int32_t)u;
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(kScanThreads)
             if (key >= 0 && rank < C) {
                 slot[i] = rank;
                 kept[i] = 1;
-                token_of_slot[(int64_t)key * C + rank] = (int32_t)t;
+                if (token_of_slot) token_of_slot[(int64_t)key * C + rank] = (int32_t)(token_base + t);
             } else {
                 slot[i] = -1;
                 kept[i] = 0;
@@ -182,18 +184,20 @@ size_t dispatch_scan_state_bytes(int64_t T, int32_t E) {
 
 int dispatch_scan_launch(const int64_t* selected, int64_t T, int32_t k, int32_t E, int64_t C, int64_t* slot,
                          uint8_t* kept, int32_t* used, int32_t* overflow, int32_t* drops, int32_t* token_of_slot,
-                         void* state_mem, int32_t* status, cudaStream_t stream) {
+                         void* state_mem, int32_t* status, cudaStream_t stream, const int32_t* rank_base,
+                         int64_t token_base) {
     const int64_t nb = (T + kScanTokens - 1) / kScanTokens;
     uint32_t* state = static_cast<uint32_t*>(state_mem);
     uint32_t* ticket = state + nb * E;
     MOE_CUDA_TRY(cudaMemsetAsync(state, 0, (size_t)nb * E * sizeof(uint32_t) + sizeof(uint32_t), stream));
-    if (C > 0) MOE_CUDA_TRY(cudaMemsetAsync(token_of_slot, 0xFF, (size_t)E * C * sizeof(int32_t), stream));
+    if (C > 0 && token_of_slot)
+        MOE_CUDA_TRY(cudaMemsetAsync(token_of_slot, 0xFF, (size_t)E * C * sizeof(int32_t), stream));
     const size_t smem = sizeof(int) * ((size_t)kScanWarps * E + kScanTokens);
     if (smem > 48 * 1024)
         MOE_CUDA_TRY(cudaFuncSetAttribute(slot_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     slot_scan_kernel<<<(unsigned)nb, kScanThreads, smem, stream>>>(selected, T, k, E, C, (int)nb, slot, kept, used,
                                                                    overflow, drops, token_of_slot, state, ticket,
-                                                                   status);
+                                                                   status, rank_base, token_base);
     return launch_status();
 }
 

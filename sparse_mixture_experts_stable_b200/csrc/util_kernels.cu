@@ -58,13 +58,31 @@ __device__ __forceinline__ float get_gate(const Assign& a, int j) {
     return j < 32 ? g0 : g1;
 }
 
+// x <- x * g elementwise for the 16 bytes of x (rounded back to T).
+template <typename T>
+__device__ __forceinline__ void scale_vec(uint4& x, float g) {
+    T* xv = reinterpret_cast<T*>(&x);
+#pragma unroll
+    for (int i = 0; i < 16 / (int)sizeof(T); ++i) xv[i] = from_f32<T>(to_f32(xv[i]) * g);
+}
+
+template <>
+__device__ __forceinline__ void scale_vec<float>(uint4& x, float g) {
+    x.x = __float_as_uint(__uint_as_float(x.x) * g);
+    x.y = __float_as_uint(__uint_as_float(x.y) * g);
+    x.z = __float_as_uint(__uint_as_float(x.z) * g);
+    x.w = __float_as_uint(__uint_as_float(x.w) * g);
+}
+
 // ------------------------------- gather -------------------------------------
 // One warp per token; 16-byte vectors when every row start is 16-byte aligned.
-template <typename T, bool VEC>
+// EP: the destination of expert e is rank e / epr's buffer (tab), row
+// (e % epr) * C + slot; otherwise dst row e * C + slot.
+template <typename T, bool VEC, bool EP>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     gather_kernel(const T* __restrict__ src, int64_t lds, int64_t Ttok, int k, const int64_t* __restrict__ selected,
                   const int64_t* __restrict__ slot, int E, int64_t C, const float* __restrict__ scale,
-                  T* __restrict__ dst, int64_t D, int32_t* status) {
+                  T* __restrict__ dst, int64_t D, int32_t* status, const RankTable tab) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
     if (t >= Ttok) return;
@@ -83,16 +101,12 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             continue;
         }
         const float g = get_gate(a, j);
-        T* drow = dst + (e * C + s) * D;
+        T* drow = EP ? static_cast<T*>(tab.base[e / tab.epr]) + ((e % tab.epr) * C + s) * D : dst + (e * C + s) * D;
         if (VEC) {
             const int64_t nv = D / EPV;
             for (int64_t v = lane; v < nv; v += 32) {
                 uint4 x = reinterpret_cast<const uint4*>(srow)[v];
-                if (scale) {
-                    T* xv = reinterpret_cast<T*>(&x);
-#pragma unroll
-                    for (int i = 0; i < EPV; ++i) xv[i] = from_f32<T>(to_f32(xv[i]) * g);
-                }
+                if (scale) scale_vec<T>(x, g);
                 reinterpret_cast<uint4*>(drow)[v] = x;
             }
         } else {
@@ -102,6 +116,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             }
         }
     }
+    if (EP) __threadfence_system();  // rows written to peer memory are visible before the kernel ends
 }
 
 // ------------------------------- combine ------------------------------------
@@ -111,11 +126,14 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 constexpr int kMaxKCombine = 64;
 constexpr int kCombineBatch = 4;  // row loads issued before the first add (4 measured faster than 8)
 
-template <typename T, typename G, bool VEC>
+// EP: the row of expert e is read from rank e / epr's buffer (tab), and the
+// staged table holds its address instead of an offset into ybuf.
+template <typename T, typename G, bool VEC, bool EP>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     combine_kernel(const T* __restrict__ ybuf, const int64_t* __restrict__ selected, const int64_t* __restrict__ slot,
                    const G* __restrict__ gates, int64_t Ttok, int k, int E, int64_t C, int64_t N,
-                   const T* __restrict__ base, int64_t ldbase, T* __restrict__ y, int64_t ldy, int32_t* status) {
+                   const T* __restrict__ base, int64_t ldbase, T* __restrict__ y, int64_t ldy, int32_t* status,
+                   const RankTable tab) {
     __shared__ int64_t s_row[kWarpsPerBlock][kMaxKCombine];
     __shared__ float s_gate[kWarpsPerBlock][kMaxKCombine];
     __shared__ int s_n[kWarpsPerBlock];
@@ -138,7 +156,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                     set_status(status, MOE_ERR_BAD_INDEX);
                 } else {
                     keep = true;
-                    row = (e * C + s) * N;
+                    if (EP)
+                        row = reinterpret_cast<int64_t>(static_cast<const T*>(tab.base[e / tab.epr]) +
+                                                        ((e % tab.epr) * C + s) * N);
+                    else
+                        row = (e * C + s) * N;
                     if (gates) g = to_f32(gates[t * k + j]);
                 }
             }
@@ -177,7 +199,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                 uint4 r[kCombineBatch];
 #pragma unroll
                 for (int u = 0; u < kCombineBatch; ++u)
-                    if (j0 + u < n_terms) r[u] = reinterpret_cast<const uint4*>(ybuf + rows[j0 + u])[v];
+                    if (j0 + u < n_terms) {
+                        const T* rp = EP ? reinterpret_cast<const T*>(rows[j0 + u]) : ybuf + rows[j0 + u];
+                        r[u] = reinterpret_cast<const uint4*>(rp)[v];
+                    }
 #pragma unroll
                 for (int u = 0; u < kCombineBatch; ++u) {
                     if (j0 + u < n_terms) {
@@ -197,7 +222,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     } else {
         for (int64_t n = lane; n < N; n += 32) {
             float acc = brow ? to_f32(brow[n]) : 0.f;
-            for (int j = 0; j < n_terms; ++j) acc = fmaf(gs[j], to_f32(ybuf[rows[j] + n]), acc);
+            for (int j = 0; j < n_terms; ++j) {
+                const T* rp = EP ? reinterpret_cast<const T*>(rows[j]) : ybuf + rows[j];
+                acc = fmaf(gs[j], to_f32(rp[n]), acc);
+            }
             yrow[n] = from_f32<T>(acc);
         }
     }
@@ -220,67 +248,100 @@ int transpose_matrices(const void* src, void* dst, int64_t batches, int64_t rows
     return launch_status();
 }
 
+bool RankTable::aligned16_all() const {
+    for (int r = 0; r < ranks; ++r)
+        if (!aligned16(base[r])) return false;
+    return true;
+}
+
+template <typename T>
+static void launch_gather(bool vec, const RankTable* tab, unsigned grid, const void* src, int64_t lds, int64_t T_,
+                          int k, const int64_t* selected, const int64_t* slot, int E, int64_t C, const float* scale,
+                          void* dst, int64_t D, int32_t* status, cudaStream_t stream) {
+    const int threads = kWarpsPerBlock * 32;
+    auto s = static_cast<const T*>(src);
+    auto d = static_cast<T*>(dst);
+    const RankTable t = tab ? *tab : RankTable{};
+    if (tab) {
+        if (vec) gather_kernel<T, true, true><<<grid, threads, 0, stream>>>(s, lds, T_, k, selected, slot, E, C, scale, d, D, status, t);
+        else gather_kernel<T, false, true><<<grid, threads, 0, stream>>>(s, lds, T_, k, selected, slot, E, C, scale, d, D, status, t);
+    } else {
+        if (vec) gather_kernel<T, true, false><<<grid, threads, 0, stream>>>(s, lds, T_, k, selected, slot, E, C, scale, d, D, status, t);
+        else gather_kernel<T, false, false><<<grid, threads, 0, stream>>>(s, lds, T_, k, selected, slot, E, C, scale, d, D, status, t);
+    }
+}
+
 int gather_rows(const void* src, int64_t lds, int64_t T, int32_t k, const int64_t* selected, const int64_t* slot,
                 int32_t E, int64_t C, const float* scale, void* dst, int64_t D, moe_dtype dtype, int32_t* status,
-                cudaStream_t stream) {
+                cudaStream_t stream, const RankTable* tab) {
     MOE_REQUIRE(k >= 1 && k <= 64, MOE_ERR_UNSUPPORTED);
     if (T == 0 || C == 0 || D == 0) return MOE_OK;
     const size_t es = dtype_size(dtype);
-    const bool vec = aligned16(src) && aligned16(dst) && ((size_t)lds * es) % 16 == 0 && ((size_t)D * es) % 16 == 0;
+    const bool dst_ok = tab ? tab->aligned16_all() : aligned16(dst);
+    const bool vec = aligned16(src) && dst_ok && ((size_t)lds * es) % 16 == 0 && ((size_t)D * es) % 16 == 0;
     const unsigned grid = (unsigned)((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
-    const int threads = kWarpsPerBlock * 32;
-    if (dtype == MOE_BF16) {
-        auto s = static_cast<const __nv_bfloat16*>(src);
-        auto d = static_cast<__nv_bfloat16*>(dst);
-        if (vec) gather_kernel<__nv_bfloat16, true><<<grid, threads, 0, stream>>>(s, lds, T, k, selected, slot, E, C, scale, d, D, status);
-        else gather_kernel<__nv_bfloat16, false><<<grid, threads, 0, stream>>>(s, lds, T, k, selected, slot, E, C, scale, d, D, status);
-    } else {
-        auto s = static_cast<const float*>(src);
-        auto d = static_cast<float*>(dst);
-        if (vec) gather_kernel<float, true><<<grid, threads, 0, stream>>>(s, lds, T, k, selected, slot, E, C, scale, d, D, status);
-        else gather_kernel<float, false><<<grid, threads, 0, stream>>>(s, lds, T, k, selected, slot, E, C, scale, d, D, status);
-    }
+    if (dtype == MOE_BF16)
+        launch_gather<__nv_bfloat16>(vec, tab, grid, src, lds, T, k, selected, slot, E, C, scale, dst, D, status,
+                                     stream);
+    else
+        launch_gather<float>(vec, tab, grid, src, lds, T, k, selected, slot, E, C, scale, dst, D, status, stream);
     return launch_status();
+}
+
+template <typename T, typename G, bool EP>
+static void launch_combine_ep(bool vec, unsigned grid, const void* ybuf, const int64_t* selected, const int64_t* slot,
+                              const void* gates, int64_t T_, int k, int E, int64_t C, int64_t N, const void* base,
+                              int64_t ldbase, void* y, int64_t ldy, int32_t* status, const RankTable& tab,
+                              cudaStream_t stream) {
+    const int threads = kWarpsPerBlock * 32;
+    if (vec)
+        combine_kernel<T, G, true, EP><<<grid, threads, 0, stream>>>(
+            static_cast<const T*>(ybuf), selected, slot, static_cast<const G*>(gates), T_, k, E, C, N,
+            static_cast<const T*>(base), ldbase, static_cast<T*>(y), ldy, status, tab);
+    else
+        combine_kernel<T, G, false, EP><<<grid, threads, 0, stream>>>(
+            static_cast<const T*>(ybuf), selected, slot, static_cast<const G*>(gates), T_, k, E, C, N,
+            static_cast<const T*>(base), ldbase, static_cast<T*>(y), ldy, status, tab);
 }
 
 template <typename T, typename G>
 static void launch_combine(bool vec, unsigned grid, const void* ybuf, const int64_t* selected, const int64_t* slot,
                            const void* gates, int64_t T_, int k, int E, int64_t C, int64_t N, const void* base,
-                           int64_t ldbase, void* y, int64_t ldy, int32_t* status, cudaStream_t stream) {
-    const int threads = kWarpsPerBlock * 32;
-    if (vec)
-        combine_kernel<T, G, true><<<grid, threads, 0, stream>>>(
-            static_cast<const T*>(ybuf), selected, slot, static_cast<const G*>(gates), T_, k, E, C, N,
-            static_cast<const T*>(base), ldbase, static_cast<T*>(y), ldy, status);
+                           int64_t ldbase, void* y, int64_t ldy, int32_t* status, const RankTable* tab,
+                           cudaStream_t stream) {
+    if (tab)
+        launch_combine_ep<T, G, true>(vec, grid, ybuf, selected, slot, gates, T_, k, E, C, N, base, ldbase, y, ldy,
+                                      status, *tab, stream);
     else
-        combine_kernel<T, G, false><<<grid, threads, 0, stream>>>(
-            static_cast<const T*>(ybuf), selected, slot, static_cast<const G*>(gates), T_, k, E, C, N,
-            static_cast<const T*>(base), ldbase, static_cast<T*>(y), ldy, status);
+        launch_combine_ep<T, G, false>(vec, grid, ybuf, selected, slot, gates, T_, k, E, C, N, base, ldbase, y, ldy,
+                                       status, RankTable{}, stream);
 }
 
 int combine_rows(const void* ybuf, const int64_t* selected, const int64_t* slot, const void* gates,
                  moe_dtype gate_dtype, int64_t T, int32_t k, int32_t E, int64_t C, int64_t N, const void* base,
-                 int64_t ldbase, void* y, int64_t ldy, moe_dtype dtype, int32_t* status, cudaStream_t stream) {
+                 int64_t ldbase, void* y, int64_t ldy, moe_dtype dtype, int32_t* status, cudaStream_t stream,
+                 const RankTable* tab) {
     MOE_REQUIRE(k >= 1 && k <= kMaxKCombine, MOE_ERR_UNSUPPORTED);
     if (T == 0 || N == 0) return MOE_OK;
     const size_t es = dtype_size(dtype);
-    const bool vec = aligned16(ybuf) && aligned16(y) && (!base || aligned16(base)) && ((size_t)N * es) % 16 == 0 &&
+    const bool src_ok = tab ? tab->aligned16_all() : aligned16(ybuf);
+    const bool vec = src_ok && aligned16(y) && (!base || aligned16(base)) && ((size_t)N * es) % 16 == 0 &&
                      ((size_t)ldy * es) % 16 == 0 && (!base || ((size_t)ldbase * es) % 16 == 0);
     const unsigned grid = (unsigned)((T + kWarpsPerBlock - 1) / kWarpsPerBlock);
     if (dtype == MOE_BF16) {
         if (gate_dtype == MOE_BF16)
             launch_combine<__nv_bfloat16, __nv_bfloat16>(vec, grid, ybuf, selected, slot, gates, T, k, E, C, N, base,
-                                                         ldbase, y, ldy, status, stream);
+                                                         ldbase, y, ldy, status, tab, stream);
         else
             launch_combine<__nv_bfloat16, float>(vec, grid, ybuf, selected, slot, gates, T, k, E, C, N, base, ldbase,
-                                                 y, ldy, status, stream);
+                                                 y, ldy, status, tab, stream);
     } else {
         if (gate_dtype == MOE_BF16)
             launch_combine<float, __nv_bfloat16>(vec, grid, ybuf, selected, slot, gates, T, k, E, C, N, base, ldbase,
-                                                 y, ldy, status, stream);
+                                                 y, ldy, status, tab, stream);
         else
             launch_combine<float, float>(vec, grid, ybuf, selected, slot, gates, T, k, E, C, N, base, ldbase, y, ldy,
-                                         status, stream);
+                                         status, tab, stream);
     }
     return launch_status();
 }
