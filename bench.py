@@ -627,6 +627,64 @@ def run_other_workloads(steps, warmup, flush, stream, dev):
                       fp32_tflops=flops_b / b_s / 1e12, peak_source=TF32_PEAK_SOURCE))
     del lg, x, w, dy, wsb, state
 
+    # expert parallelism, 4 ranks emulated on this GPU: the full-layer batch split over the ranks, every rank's
+    # rows written into and read from the other ranks' buffers through the peer-pointer tables
+    from sparse_mixture_experts_stable_b200 import ep
+    c = I.full_layer_bf16(seed=0)
+    T, H, E, F, k = c["T"], c["H"], c["E"], c["F"], c["k"]
+    R, epr = 4, c["E"] // 4
+    C = moe.moe_capacity(T, k, E, c["capacity_factor"])
+    dv = {n: c[n].to(dev) for n in ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down")}
+    xs = [t.contiguous() for t in torch.chunk(dv["x"], R)]
+    wr = [{"w1": dv["w_gate"][q * epr:(q + 1) * epr], "w3": dv["w_up"][q * epr:(q + 1) * epr],
+           "w2": dv["w_down"][q * epr:(q + 1) * epr]} for q in range(R)]
+    xbufs = [torch.empty(epr, C, H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    ybufs = [torch.empty(epr, C, H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    ys = [torch.empty_like(t) for t in xs]
+    tb = ep.token_bases([t.shape[0] for t in xs])
+    wsd = torch.empty(B.moe_dispatch_workspace_size(T // R, k, E), dtype=torch.uint8, device=dev)
+    inner_d, inner_c = [], []
+    kept_box = {}
+
+    def step_ep():
+        routes = [moe.moe_route(xs[q], k, w_router=dv["w_router"], logit_bias=dv["router_bias"]) for q in range(R)]
+        counts_all = torch.stack([r["counts"] for r in routes])
+        plans = [moe.moe_ep_plan(counts_all, q, C) for q in range(R)]
+        e0, e1 = events(inner_d)
+        e0.record(stream)
+        disp = [moe.moe_ep_dispatch(routes[q]["selected"], E, C, plans[q]["rank_base"], tb[q], xs[q], xbufs,
+                                    workspace=wsd) for q in range(R)]
+        e1.record(stream)
+        for q in range(R):
+            moe.moe_expert_ffn("swiglu", xbufs[q], plans[q]["used"][q * epr:(q + 1) * epr], wr[q]["w1"],
+                               w2=wr[q]["w2"], w3=wr[q]["w3"], ybuf=ybufs[q])
+        e0, e1 = events(inner_c)
+        e0.record(stream)
+        for q in range(R):
+            moe.moe_ep_combine(ybufs, routes[q]["selected"], disp[q]["slot"], routes[q]["gates_f32"], E, C, H,
+                               torch.bfloat16, base_kind="input", base=xs[q], y=ys[q])
+        e1.record(stream)
+        kept_box["used"] = plans[0]["used"]
+
+    sm, _ = _time_steps(step_ep, steps, warmup, flush, stream)
+    kept = int(kept_box["used"].sum())
+    d_s = statistics.mean(a.elapsed_time(b) for a, b in inner_d[-steps:]) / 1e3
+    c_s = statistics.mean(a.elapsed_time(b) for a, b in inner_c[-steps:]) / 1e3
+    moved = 2 * kept * H * 2  # kept rows out to their owner ranks and back (bf16)
+    bytes_alg = (T * H * 2 + kept * H * 2) + (kept * H * 2 + 2 * T * H * 2)  # dispatch + combine (x and y base/out)
+    out["full_layer_bf16_ep4_one_device"] = dict(
+        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+        config=dict(T=T, H=H, E=E, F=F, k=k, capacity=C, kept=kept, ranks=R, experts_per_rank=epr,
+                    step="4 ranks on one GPU: route, counts, moe_ep_plan, moe_ep_dispatch, experts, moe_ep_combine",
+                    shared_experts=0),
+        roofline=dict(bound="hbm", kernel="moe_ep_dispatch gather + moe_ep_combine (peer-pointer row exchange)",
+                      achieved=bytes_alg / (d_s + c_s) / 1e9, peak=pk["hbm"], unit="GB/s",
+                      frac=bytes_alg / (d_s + c_s) / 1e9 / pk["hbm"], traffic=None,
+                      dispatch_ms=1e3 * d_s, combine_ms=1e3 * c_s, bytes_per_step=bytes_alg,
+                      exchanged_bytes=moved, payload_bytes_no_drops=ep.payload_bytes(T, H, k, 2),
+                      note="on one GPU the peer buffers are local HBM; across GPUs the exchanged bytes cross NVLink"))
+    del dv, xs, wr, xbufs, ybufs, ys, wsd
+
     # training step of the full layer: forward, SwiGLU-expert backward and router backward (bf16)
     from sparse_mixture_experts_stable_b200.layer import SwiGLUMoE
     c = I.full_layer_bf16(seed=0)

@@ -48,6 +48,16 @@ def partition(E: int, R: int) -> int:
     return E // R
 
 
+def payload_bytes(tokens: int, hidden: int, k: int, bytes_per_value: int, include_return: bool = True) -> int:
+    """Activation bytes an expert-parallel step moves with no drops (Module 7 page,
+    expert-parallel payload): T*k rows of ``hidden`` values out, and as many back."""
+    for v in (tokens, hidden, k, bytes_per_value):
+        if int(v) < 1:
+            raise ValueError("sizes must be positive")
+    one_way = int(tokens) * int(hidden) * int(k) * int(bytes_per_value)
+    return one_way * (2 if include_return else 1)
+
+
 def token_bases(tokens_per_rank: Sequence[int]) -> List[int]:
     """Global index of every rank's first token (tokens in rank order)."""
     out, acc = [], 0

@@ -125,6 +125,9 @@ def test_two_rank_expert_parallel_host_logic():
 
 def test_expert_parallel_partition_rules():
     from sparse_mixture_experts_stable_b200 import ep
+    # Module 7 page, expert-parallel payload: 2048 tokens, hidden 7168, top-8, bf16 -> 448 MiB round trip
+    assert ep.payload_bytes(2048, 7168, 8, 2) == 448 * 2 ** 20
+    assert ep.payload_bytes(2048, 7168, 8, 2, include_return=False) == 224 * 2 ** 20
     assert ep.partition(256, 8) == 32
     assert ep.token_bases([5, 0, 7]) == [0, 5, 5]
     for E, R in [(10, 4), (8, 0), (128, 128)]:
