@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "tc_gemm.cuh"
 #include "f32_gemm.cuh"
+#include "tc_ptx.cuh"
 #include "tc_tf32.cuh"
 #include "util_kernels.cuh"
 
@@ -19,7 +20,43 @@ namespace {
 
 constexpr int kWarps = 8;
 
-template <typename In>
+// This lane's part of the dot product of two rows of n elements: 16-byte
+// vectors when VEC (n a multiple of the vector width, rows 16-byte aligned).
+__device__ __forceinline__ float dot16(const uint4& a, const uint4& b, float acc, const float*) {
+    acc = fmaf(__uint_as_float(a.x), __uint_as_float(b.x), acc);
+    acc = fmaf(__uint_as_float(a.y), __uint_as_float(b.y), acc);
+    acc = fmaf(__uint_as_float(a.z), __uint_as_float(b.z), acc);
+    return fmaf(__uint_as_float(a.w), __uint_as_float(b.w), acc);
+}
+__device__ __forceinline__ float dot16(const uint4& a, const uint4& b, float acc, const __nv_bfloat16*) {
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[i]));
+        const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb[i]));
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+    }
+    return acc;
+}
+
+template <typename In, bool VEC>
+__device__ __forceinline__ float row_dot_part(const In* __restrict__ a, const In* __restrict__ b, int64_t n,
+                                              int lane) {
+    float part = 0.f;
+    if (VEC) {
+        constexpr int EPV = 16 / sizeof(In);
+        const int64_t nv = n / EPV;
+        const uint4* va = reinterpret_cast<const uint4*>(a);
+        const uint4* vb = reinterpret_cast<const uint4*>(b);
+        for (int64_t v = lane; v < nv; v += 32) part = dot16(va[v], vb[v], part, a);
+    } else {
+        for (int64_t i = lane; i < n; i += 32) part = fmaf(to_f32(a[i]), to_f32(b[i]), part);
+    }
+    return part;
+}
+
+template <typename In, bool VEC>
 __global__ void __launch_bounds__(kWarps * 32)
     dgate_dlogits_kernel(const In* __restrict__ dy, int64_t Dout, const In* __restrict__ ybuf,
                          const float* __restrict__ logits, const int64_t* __restrict__ selected,
@@ -42,9 +79,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                 if (lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
             } else {
                 const In* yr = ybuf + (e * C + s) * Dout;
-                float part = 0.f;
-                for (int64_t n = lane; n < Dout; n += 32) part = fmaf(to_f32(dyr[n]), to_f32(yr[n]), part);
-                dg = warp_sum(part);
+                dg = warp_sum(row_dot_part<In, VEC>(dyr, yr, Dout, lane));
             }
         }
         gdot = fmaf(gates[t * k + j], dg, gdot);
@@ -89,6 +124,23 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
         __syncwarp();
     }
+}
+
+template <typename In>
+void launch_dgate(unsigned grid, cudaStream_t stream, const In* dy, int64_t Dout, const In* ybuf,
+                  const float* logits, const int64_t* selected, const float* gates, const int64_t* slot, int64_t T,
+                  int k, int E, int64_t C, float aux_coef, float kn, const int32_t* counts, float* dlogits,
+                  float* dgate, int32_t* status) {
+    constexpr int EPV = 16 / sizeof(In);
+    const bool vec = Dout % EPV == 0 && aligned16(dy) && (ybuf == nullptr || aligned16(ybuf));
+    if (vec)
+        dgate_dlogits_kernel<In, true><<<grid, kWarps * 32, 0, stream>>>(dy, Dout, ybuf, logits, selected, gates, slot,
+                                                                        T, k, E, C, aux_coef, kn, counts, dlogits,
+                                                                        dgate, status);
+    else
+        dgate_dlogits_kernel<In, false><<<grid, kWarps * 32, 0, stream>>>(dy, Dout, ybuf, logits, selected, gates,
+                                                                         slot, T, k, E, C, aux_coef, kn, counts,
+                                                                         dlogits, dgate, status);
 }
 
 }  // namespace
@@ -151,9 +203,9 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
     const size_t split_bytes = workspace_bytes - (size_t)(split - ws);
 
     const unsigned grid = (unsigned)((T + kWarps - 1) / kWarps);
-    dgate_dlogits_kernel<float><<<grid, kWarps * 32, 0, stream>>>(
-        static_cast<const float*>(dy), Dout, static_cast<const float*>(ybuf), logits, selected, gates, slot, T, k, E,
-        C, aux_coef, normalize_by_k ? (float)k : 1.0f, counts, dlogits, dgate, dev_status);
+    launch_dgate<float>(grid, stream, static_cast<const float*>(dy), Dout, static_cast<const float*>(ybuf), logits,
+                        selected, gates, slot, T, k, E, C, aux_coef, normalize_by_k ? (float)k : 1.0f, counts, dlogits,
+                        dgate, dev_status);
     int rc = launch_status();
     if (rc != MOE_OK) return rc;
 
@@ -263,32 +315,108 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// The same transpose on 64 x 64 tiles moving 16-byte vectors on both sides
+// (needs 16-byte aligned bases, strides that are multiples of 8 elements,
+// Cc and Rp multiples of 8).  Tile rows are 66 elements wide (33 words), so
+// the column reads of the second phase hit at most two lanes per bank.
+constexpr int kTT = 64;
+__global__ void __launch_bounds__(256)
+    transpose_valid_v8_kernel(const __nv_bfloat16* __restrict__ src, int64_t lds, int64_t sgs, int64_t R, int64_t Cc,
+                              const int32_t* __restrict__ valid, int64_t Rp, __nv_bfloat16* __restrict__ dst,
+                              int64_t ldd, int64_t dgs) {
+    __shared__ uint16_t tile[kTT][kTT + 2];
+    const int g = blockIdx.z;
+    int64_t Rv = R;
+    if (valid) {
+        const int64_t v = valid[g];
+        Rv = v < 0 ? 0 : (v < R ? v : R);
+    }
+    const int64_t r0 = (int64_t)blockIdx.y * kTT, c0 = (int64_t)blockIdx.x * kTT;
+    const __nv_bfloat16* s = src + g * sgs;
+    __nv_bfloat16* d = dst + g * dgs;
+    const int q = threadIdx.x & 7, rr = threadIdx.x >> 3;  // 8-element chunk, row within a 32-row half
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int64_t r = r0 + rr + 32 * i, c = c0 + 8 * q;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < Rv && c < Cc) v = *reinterpret_cast<const uint4*>(s + r * lds + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            tile[rr + 32 * i][8 * q + 2 * j] = (uint16_t)(w[j] & 0xFFFFu);
+            tile[rr + 32 * i][8 * q + 2 * j + 1] = (uint16_t)(w[j] >> 16);
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int64_t c = c0 + rr + 32 * i, r = r0 + 8 * q;
+        if (c < Cc && r < Rp) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                w[j] = (uint32_t)tile[8 * q + 2 * j][rr + 32 * i] | ((uint32_t)tile[8 * q + 2 * j + 1][rr + 32 * i] << 16);
+            *reinterpret_cast<uint4*>(d + c * ldd + r) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
 int transpose_valid(const __nv_bfloat16* src, int64_t lds, int64_t sgs, int G, int64_t R, int64_t Cc,
                     const int32_t* valid, int64_t Rp, __nv_bfloat16* dst, int64_t ldd, int64_t dgs,
                     cudaStream_t stream) {
     MOE_REQUIRE(G <= 65535 && (Rp + 31) / 32 <= 65535, MOE_ERR_UNSUPPORTED);
-    const dim3 grid((unsigned)((Cc + 31) / 32), (unsigned)((Rp + 31) / 32), (unsigned)G), block(32, 8);
-    transpose_valid_kernel<<<grid, block, 0, stream>>>(src, lds, sgs, R, Cc, valid, Rp, dst, ldd, dgs);
+    const bool v8 = aligned16(src) && aligned16(dst) && lds % 8 == 0 && sgs % 8 == 0 && ldd % 8 == 0 &&
+                    dgs % 8 == 0 && Cc % 8 == 0 && Rp % 8 == 0;
+    if (v8) {
+        const dim3 grid((unsigned)((Cc + kTT - 1) / kTT), (unsigned)((Rp + kTT - 1) / kTT), (unsigned)G);
+        transpose_valid_v8_kernel<<<grid, 256, 0, stream>>>(src, lds, sgs, R, Cc, valid, Rp, dst, ldd, dgs);
+    } else {
+        const dim3 grid((unsigned)((Cc + 31) / 32), (unsigned)((Rp + 31) / 32), (unsigned)G), block(32, 8);
+        transpose_valid_kernel<<<grid, block, 0, stream>>>(src, lds, sgs, R, Cc, valid, Rp, dst, ldd, dgs);
+    }
     return launch_status();
 }
 
 // h, da, db from a, b (ab rows: [a | b], fp32) and dh (fp32), for c < used[e]:
 //   s = sigmoid(a), h = a s b, da = dh b s (1 + a (1 - s)), db = dh a s.
+// Eight consecutive f per thread (F a multiple of 8): 32-byte fp32 loads,
+// 16-byte bf16 stores.
 __global__ void swiglu_bwd_elem_kernel(const float* __restrict__ ab, const float* __restrict__ dh,
                                        const int32_t* __restrict__ used, int64_t C, int64_t F,
                                        __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ dab) {
     const int e = blockIdx.y;
     const int64_t u = used[e] < 0 ? 0 : (used[e] < C ? used[e] : C);
-    const int64_t n = u * F;
+    const int64_t F8 = F / 8;
+    const int64_t n = u * F8;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t c = i / F, f = i - c * F;
+        const int64_t c = i / F8, f = (i - c * F8) * 8;
         const int64_t row = (int64_t)e * C + c;
-        const float a = ab[row * 2 * F + f], b = ab[row * 2 * F + F + f];
-        const float g = dh[row * F + f];
-        const float s = 1.0f / (1.0f + expf(-a));
-        h[row * F + f] = __float2bfloat16_rn(a * s * b);
-        dab[row * 2 * F + f] = __float2bfloat16_rn(g * b * s * (1.0f + a * (1.0f - s)));
-        dab[row * 2 * F + F + f] = __float2bfloat16_rn(g * a * s);
+        const float4* pa = reinterpret_cast<const float4*>(ab + row * 2 * F + f);
+        const float4* pb = reinterpret_cast<const float4*>(ab + row * 2 * F + F + f);
+        const float4* pg = reinterpret_cast<const float4*>(dh + row * F + f);
+        const float4 a0 = pa[0], a1 = pa[1], b0 = pb[0], b1 = pb[1], g0 = pg[0], g1 = pg[1];
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        uint32_t ph[4], pda[4], pdb[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float hv[2], dav[2], dbv[2];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const float a = av[2 * j + m], b = bv[2 * j + m], g = gv[2 * j + m];
+                const float s = 1.0f / (1.0f + expf(-a));
+                hv[m] = a * s * b;
+                dav[m] = g * b * s * (1.0f + a * (1.0f - s));
+                dbv[m] = g * a * s;
+            }
+            ph[j] = tc::pack_bf16x2(hv[0], hv[1]);
+            pda[j] = tc::pack_bf16x2(dav[0], dav[1]);
+            pdb[j] = tc::pack_bf16x2(dbv[0], dbv[1]);
+        }
+        *reinterpret_cast<uint4*>(h + row * F + f) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(dab + row * 2 * F + f) = make_uint4(pda[0], pda[1], pda[2], pda[3]);
+        *reinterpret_cast<uint4*>(dab + row * 2 * F + F + f) = make_uint4(pdb[0], pdb[1], pdb[2], pdb[3]);
     }
 }
 
@@ -377,9 +505,9 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     MOE_REQUIRE(workspace && workspace_bytes >= moe_backward_swiglu_workspace_size(E, C, H, F), MOE_ERR_WORKSPACE);
 
     const unsigned grid = (unsigned)((T + kWarps - 1) / kWarps);
-    dgate_dlogits_kernel<bf16><<<grid, kWarps * 32, 0, stream>>>(
-        static_cast<const bf16*>(dy), H, static_cast<const bf16*>(ybuf), logits, selected, gates, slot, T, k, E, C,
-        aux_coef, normalize_by_k ? (float)k : 1.0f, counts, dlogits, dgate, dev_status);
+    launch_dgate<bf16>(grid, stream, static_cast<const bf16*>(dy), H, static_cast<const bf16*>(ybuf), logits, selected,
+                       gates, slot, T, k, E, C, aux_coef, normalize_by_k ? (float)k : 1.0f, counts, dlogits, dgate,
+                       dev_status);
     int rc = launch_status();
     if (rc != MOE_OK) return rc;
 
@@ -429,7 +557,8 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     if (rc != MOE_OK) return rc;
     // 5. h, da, db
     {
-        const dim3 g2((unsigned)((C * F + 255) / 256 < 1024 ? (C * F + 255) / 256 : 1024), (unsigned)E);
+        const int64_t nb = (C * (F / 8) + 255) / 256;
+        const dim3 g2((unsigned)(nb < 1024 ? nb : 1024), (unsigned)E);
         MOE_REQUIRE(E <= 65535, MOE_ERR_UNSUPPORTED);
         swiglu_bwd_elem_kernel<<<g2, 256, 0, stream>>>(ab, dh, used, C, F, h, dab);
         rc = launch_status();
@@ -608,9 +737,9 @@ extern "C" int moe_backward_gelu(moe_dtype dtype, const void* dy, const float* l
                 MOE_ERR_WORKSPACE);
 
     const unsigned grid = (unsigned)((T + kWarps - 1) / kWarps);
-    dgate_dlogits_kernel<float><<<grid, kWarps * 32, 0, stream>>>(
-        static_cast<const float*>(dy), Dout, static_cast<const float*>(ybuf), logits, selected, gates, slot, T, k, E,
-        C, aux_coef, normalize_by_k ? (float)k : 1.0f, counts, dlogits, dgate, dev_status);
+    launch_dgate<float>(grid, stream, static_cast<const float*>(dy), Dout, static_cast<const float*>(ybuf), logits,
+                        selected, gates, slot, T, k, E, C, aux_coef, normalize_by_k ? (float)k : 1.0f, counts, dlogits,
+                        dgate, dev_status);
     int rc = launch_status();
     if (rc != MOE_OK) return rc;
 

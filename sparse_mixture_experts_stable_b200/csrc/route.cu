@@ -547,23 +547,47 @@ extern "C" int moe_aux_stats(const int32_t* counts, const float* prob_sum, int64
 namespace moe {
 namespace {
 
-// db[e] = sum_t g[t,e] in a fixed order: warp w of block b adds rows t = w,
-// w + 32, ... for experts 32b + lane, then warp 0 adds the 32 warp sums.
+// Column sums of g (T, E) in a fixed order, in two passes.  Pass 1: block
+// (b, c) covers experts 32b + lane over the rows of chunk c; warp w adds rows
+// t = chunk start + w, + 32, ..., warp 0 adds the 32 warp sums into part[c][e].
+// Pass 2: out[e] = sum over the chunks in ascending order (plus add[s][e] of
+// `nadd` further partial rows when given).
+constexpr int kColChunks = 64;
 __global__ void __launch_bounds__(1024)
-    column_sum_kernel(const float* __restrict__ g, int64_t T, int E, float* __restrict__ out) {
+    column_sum_part_kernel(const float* __restrict__ g, int64_t T, int E, int64_t chunk, float* __restrict__ part) {
     __shared__ float s[32][33];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 32 + lane;
+    const int64_t t0 = (int64_t)blockIdx.y * chunk;
+    const int64_t t1 = t0 + chunk < T ? t0 + chunk : T;
     float acc = 0.f;
     if (e < E)
-        for (int64_t t = warp; t < T; t += 32) acc += g[t * E + e];
+        for (int64_t t = t0 + warp; t < t1; t += 32) acc += g[t * E + e];
     s[warp][lane] = acc;
     __syncthreads();
     if (warp == 0 && e < E) {
         float tot = 0.f;
         for (int w = 0; w < 32; ++w) tot += s[w][lane];
-        out[e] = tot;
+        part[(int64_t)blockIdx.y * E + e] = tot;
     }
+}
+
+// out[i] = sum_{s < n} part[s][i], s ascending (i < len).
+__global__ void sum_rows_kernel(const float* __restrict__ part, int n, int64_t len, float* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < len; i += (int64_t)gridDim.x * blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < n; ++s) acc += part[(int64_t)s * len + i];
+        out[i] = acc;
+    }
+}
+
+// K splits of the weight-gradient product (reduction over the T tokens): enough
+// tiles for the SMs while T splits evenly.
+int wgrad_splits(int64_t T, int64_t M, int64_t N) {
+    const int64_t tiles = ((M + 127) / 128) * ((N + 127) / 128);
+    int s = 1;
+    while (s < 8 && tiles * s * 2 <= 160 && T % (2 * s) == 0 && T / (2 * s) >= 512) s *= 2;
+    return s;
 }
 
 // The two GEMMs of the router backward in F32Gemm form.
@@ -614,6 +638,36 @@ void router_bwd_gemms(moe_dtype dtype, const void* x, int64_t T, int64_t D, int6
     }
     gw.C = dw;
     gw.K = T;
+    // split the reduction over t into S groups of T/S rows, partial products summed afterwards
+    const int S = wgrad_splits(T, gw.M, gw.N);
+    if (S > 1) {
+        gw.groups = S;
+        gw.K = T / S;
+        if (layout == MOE_ROUTER_ED) {
+            gw.a_group_stride = gw.K * E;
+            gw.b_group_stride = gw.K * ldx;
+        } else {
+            gw.a_group_stride = gw.K * ldx;
+            gw.b_group_stride = gw.K * E;
+        }
+        gw.c_group_stride = gw.M * gw.N;
+    }
+}
+
+// Workspace of the router backward: the split operands, then (when the
+// weight gradient is split) the partial products, then the column-sum partials.
+struct RouterBwdWs {
+    size_t split, partials, colsum, total;
+};
+
+RouterBwdWs router_bwd_layout(const F32Gemm& gx, const F32Gemm& gw, int32_t E) {
+    RouterBwdWs l{};
+    const size_t a = tf32x3_workspace_size(gx), b = tf32x3_workspace_size(gw);
+    l.split = align_up(a > b ? a : b, 256);
+    l.partials = gw.groups > 1 ? align_up((size_t)gw.groups * gw.M * gw.N * 4, 256) : 0;
+    l.colsum = align_up((size_t)kColChunks * E * 4, 256);
+    l.total = l.split + l.partials + l.colsum;
+    return l;
 }
 
 }  // namespace
@@ -624,8 +678,7 @@ extern "C" size_t moe_router_backward_workspace_size(int64_t T, int64_t D, int32
     if (T < 1 || D < 1 || E < 1) return 0;
     F32Gemm gx, gw;
     router_bwd_gemms(dtype, nullptr, T, D, D, nullptr, layout, E, nullptr, nullptr, nullptr, gx, gw);
-    const size_t a = tf32x3_workspace_size(gx), b = tf32x3_workspace_size(gw);
-    return a > b ? a : b;
+    return router_bwd_layout(gx, gw, E).total;
 }
 
 extern "C" int moe_router_backward(moe_dtype dtype, const void* x, int64_t T, int64_t D, int64_t ldx,
@@ -640,17 +693,35 @@ extern "C" int moe_router_backward(moe_dtype dtype, const void* x, int64_t T, in
                 MOE_ERR_WORKSPACE);
     F32Gemm gx, gw;
     router_bwd_gemms(dtype, x, T, D, ldx, w_router, layout, E, dlogits, dx_router, dw_router, gx, gw);
+    const RouterBwdWs l = router_bwd_layout(gx, gw, E);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
     int rc;
     if (dx_router) {
-        rc = tf32x3_gemm_run(gx, workspace, workspace_bytes, dev_status, stream);
+        rc = tf32x3_gemm_run(gx, ws, l.split, dev_status, stream);
         if (rc != MOE_OK) return rc;
     }
     if (dw_router) {
-        rc = tf32x3_gemm_run(gw, workspace, workspace_bytes, dev_status, stream);
+        float* part = reinterpret_cast<float*>(ws + l.split);
+        if (gw.groups > 1) gw.C = part;
+        rc = tf32x3_gemm_run(gw, ws, l.split, dev_status, stream);
         if (rc != MOE_OK) return rc;
+        if (gw.groups > 1) {
+            const int64_t len = gw.M * gw.N;
+            const int64_t nb = (len + 255) / 256;
+            sum_rows_kernel<<<(unsigned)(nb < 4096 ? nb : 4096), 256, 0, stream>>>(part, gw.groups, len, dw_router);
+            rc = launch_status();
+            if (rc != MOE_OK) return rc;
+        }
     }
     if (db_router) {
-        column_sum_kernel<<<(E + 31) / 32, 1024, 0, stream>>>(dlogits, T, E, db_router);
+        float* part = reinterpret_cast<float*>(ws + l.split + l.partials);
+        const int64_t chunk = (T + kColChunks - 1) / kColChunks;
+        const int chunks = (int)((T + chunk - 1) / chunk);
+        column_sum_part_kernel<<<dim3((unsigned)((E + 31) / 32), (unsigned)chunks), 1024, 0, stream>>>(dlogits, T, E,
+                                                                                                      chunk, part);
+        rc = launch_status();
+        if (rc != MOE_OK) return rc;
+        sum_rows_kernel<<<(unsigned)((E + 255) / 256), 256, 0, stream>>>(part, chunks, E, db_router);
         return launch_status();
     }
     return MOE_OK;
