@@ -273,9 +273,10 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
 // moe_backward_swiglu: bf16 SwiGLU experts, the kept mask held constant.
 //   1. dgate / dlogits                       as above, on bf16 rows
 //   2. dybuf[e,c] = gate * dy[token]         scaled gather (bf16)
-//   3. [a | b] = xbuf [Wg; Wu]^T             two tensor-core GEMMs, fp32 out
-//   4. dh = dybuf Wd                         tensor-core GEMM on Wd^T, fp32 out
-//   5. h, da, db from (a, b, dh)             elementwise (silu and its derivative)
+//   3. [a | b] = xbuf [Wg; Wu]^T             one tensor-core GEMM (both weights), fp32 out
+//   4. dh = dybuf Wd -> h, da, db            tensor-core GEMM on Wd^T whose epilogue takes
+//                                            a, b and forms h = silu(a) b and the
+//                                            derivatives (dh never leaves the SM)
 //   6. dWd = dybuf^T h, dWg = da^T xbuf, dWu = db^T xbuf
 //                                            tensor-core GEMMs on zero-padded,
 //                                            token-transposed operands, fp32 out
@@ -316,6 +317,8 @@ __global__ void __launch_bounds__(256)
 }
 
 // The same transpose on 64 x 64 tiles moving 16-byte vectors on both sides
+// (with `valid`, 64-wide row blocks wholly past the valid rows, other than the
+// first, are left unwritten: the GEMMs that read them stop at the valid count)
 // (needs 16-byte aligned bases, strides that are multiples of 8 elements,
 // Cc and Rp multiples of 8).  Tile rows are 66 elements wide (33 words), so
 // the column reads of the second phase hit at most two lanes per bank.
@@ -332,6 +335,9 @@ __global__ void __launch_bounds__(256)
         Rv = v < 0 ? 0 : (v < R ? v : R);
     }
     const int64_t r0 = (int64_t)blockIdx.y * kTT, c0 = (int64_t)blockIdx.x * kTT;
+    // with a valid count, only the 64-wide blocks a K-limited product reads are
+    // needed: those up to the one holding row Rv - 1 (at least the first)
+    if (valid && r0 >= kTT && r0 >= Rv) return;
     const __nv_bfloat16* s = src + g * sgs;
     __nv_bfloat16* d = dst + g * dgs;
     const int q = threadIdx.x & 7, rr = threadIdx.x >> 3;  // 8-element chunk, row within a 32-row half
@@ -377,53 +383,11 @@ int transpose_valid(const __nv_bfloat16* src, int64_t lds, int64_t sgs, int G, i
     return launch_status();
 }
 
-// h, da, db from a, b (ab rows: [a | b], fp32) and dh (fp32), for c < used[e]:
-//   s = sigmoid(a), h = a s b, da = dh b s (1 + a (1 - s)), db = dh a s.
-// Eight consecutive f per thread (F a multiple of 8): 32-byte fp32 loads,
-// 16-byte bf16 stores.
-__global__ void swiglu_bwd_elem_kernel(const float* __restrict__ ab, const float* __restrict__ dh,
-                                       const int32_t* __restrict__ used, int64_t C, int64_t F,
-                                       __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ dab) {
-    const int e = blockIdx.y;
-    const int64_t u = used[e] < 0 ? 0 : (used[e] < C ? used[e] : C);
-    const int64_t F8 = F / 8;
-    const int64_t n = u * F8;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t c = i / F8, f = (i - c * F8) * 8;
-        const int64_t row = (int64_t)e * C + c;
-        const float4* pa = reinterpret_cast<const float4*>(ab + row * 2 * F + f);
-        const float4* pb = reinterpret_cast<const float4*>(ab + row * 2 * F + F + f);
-        const float4* pg = reinterpret_cast<const float4*>(dh + row * F + f);
-        const float4 a0 = pa[0], a1 = pa[1], b0 = pb[0], b1 = pb[1], g0 = pg[0], g1 = pg[1];
-        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-        uint32_t ph[4], pda[4], pdb[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float hv[2], dav[2], dbv[2];
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const float a = av[2 * j + m], b = bv[2 * j + m], g = gv[2 * j + m];
-                const float s = 1.0f / (1.0f + expf(-a));
-                hv[m] = a * s * b;
-                dav[m] = g * b * s * (1.0f + a * (1.0f - s));
-                dbv[m] = g * a * s;
-            }
-            ph[j] = tc::pack_bf16x2(hv[0], hv[1]);
-            pda[j] = tc::pack_bf16x2(dav[0], dav[1]);
-            pdb[j] = tc::pack_bf16x2(dbv[0], dbv[1]);
-        }
-        *reinterpret_cast<uint4*>(h + row * F + f) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-        *reinterpret_cast<uint4*>(dab + row * 2 * F + f) = make_uint4(pda[0], pda[1], pda[2], pda[3]);
-        *reinterpret_cast<uint4*>(dab + row * 2 * F + F + f) = make_uint4(pdb[0], pdb[1], pdb[2], pdb[3]);
-    }
-}
-
 // Grouped bf16 GEMM out[g] (M x N, fp32 or bf16) = A[g] (M x K) B[g]^T, K-major operands.
 int gemm(const void* a, int64_t lda, int64_t a_rows_total, int64_t a_rows_per_group, const void* b, int64_t ldb,
          int64_t b_rows_total, int64_t b_rows_per_group, int G, int64_t M, int64_t N, int64_t K, const int32_t* rows,
-         void* out, int64_t ldo, int64_t out_rows_per_group, int epilogue, int32_t* status, cudaStream_t stream) {
+         void* out, int64_t ldo, int64_t out_rows_per_group, int epilogue, int32_t* status, cudaStream_t stream,
+         const int32_t* k_rows = nullptr) {
     TcGemmProblem p{};
     p.a = a;
     p.lda = lda;
@@ -438,6 +402,7 @@ int gemm(const void* a, int64_t lda, int64_t a_rows_total, int64_t a_rows_per_gr
     p.N = N;
     p.K = K;
     p.rows = rows;
+    p.k_rows = k_rows;
     p.out = out;
     p.ldo = ldo;
     p.out_rows_per_group = out_rows_per_group;
@@ -447,7 +412,7 @@ int gemm(const void* a, int64_t lda, int64_t a_rows_total, int64_t a_rows_per_gr
 }
 
 struct SwigluBwdWs {
-    size_t dybuf, ab, dh, h, dab, wdT, wguT, dybufT, hT, dabT, xbufT, dxbuf, total;
+    size_t dybuf, ab, h, dab, wdT, wguT, dybufT, hT, dabT, xbufT, dxbuf, total;
     int64_t Cp;
 };
 
@@ -462,7 +427,6 @@ SwigluBwdWs swiglu_bwd_layout(int32_t E, int64_t C, int64_t H, int64_t F) {
     };
     w.dybuf = take((size_t)E * C * H * 2);
     w.ab = take((size_t)E * C * 2 * F * 4);
-    w.dh = take((size_t)E * C * F * 4);
     w.h = take((size_t)E * C * F * 2);
     w.dab = take((size_t)E * C * 2 * F * 2);
     w.wdT = take((size_t)E * F * H * 2);
@@ -526,7 +490,6 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     bf16* dybuf = reinterpret_cast<bf16*>(ws + l.dybuf);
     float* ab = reinterpret_cast<float*>(ws + l.ab);
-    float* dh = reinterpret_cast<float*>(ws + l.dh);
     bf16* h = reinterpret_cast<bf16*>(ws + l.h);
     bf16* dab = reinterpret_cast<bf16*>(ws + l.dab);
     bf16* wdT = reinterpret_cast<bf16*>(ws + l.wdT);
@@ -542,26 +505,59 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     // 2. dybuf[e,c] = gate * dy[token]
     rc = gather_rows(dy, H, T, k, selected, slot, E, C, gates, dybuf, H, MOE_BF16, dev_status, stream);
     if (rc != MOE_OK) return rc;
-    // 3. [a | b] = xbuf [Wg; Wu]^T  (fp32)
-    rc = gemm(xbuf, H, (int64_t)E * C, C, w_gate, H, (int64_t)E * F, F, E, C, F, H, used, ab, F2, C, TC_EPI_F32,
-              dev_status, stream);
-    if (rc != MOE_OK) return rc;
-    rc = gemm(xbuf, H, (int64_t)E * C, C, w_up, H, (int64_t)E * F, F, E, C, F, H, used, ab + F, F2, C, TC_EPI_F32,
-              dev_status, stream);
-    if (rc != MOE_OK) return rc;
-    // 4. dh = dybuf Wd, with Wd (E, H, F) transposed to (E, F, H)
+    // 3. [a | b] = xbuf [Wg; Wu]^T  (fp32), both weights in one pass over xbuf
+    {
+        TcGemmProblem p{};
+        p.a = xbuf;
+        p.lda = H;
+        p.a_rows_total = (int64_t)E * C;
+        p.a_rows_per_group = C;
+        p.b = w_gate;
+        p.b2 = w_up;
+        p.ldb = H;
+        p.b_rows_total = (int64_t)E * F;
+        p.b_rows_per_group = F;
+        p.G = E;
+        p.M = C;
+        p.N = F;
+        p.K = H;
+        p.rows = used;
+        p.out = ab;
+        p.ldo = F2;
+        p.out_rows_per_group = C;
+        p.epilogue = TC_EPI_F32_DUAL;
+        p.status = dev_status;
+        rc = tc_gemm_run(p, stream);
+        if (rc != MOE_OK) return rc;
+    }
+    // 4. dh = dybuf Wd (Wd (E, H, F) transposed to (E, F, H)); the epilogue turns dh and [a | b] into h, [da | db]
     rc = transpose_valid(static_cast<const bf16*>(w_down), F, H * F, E, H, F, nullptr, H, wdT, H, F * H, stream);
     if (rc != MOE_OK) return rc;
-    rc = gemm(dybuf, H, (int64_t)E * C, C, wdT, H, (int64_t)E * F, F, E, C, F, H, used, dh, F, C, TC_EPI_F32,
-              dev_status, stream);
-    if (rc != MOE_OK) return rc;
-    // 5. h, da, db
     {
-        const int64_t nb = (C * (F / 8) + 255) / 256;
-        const dim3 g2((unsigned)(nb < 1024 ? nb : 1024), (unsigned)E);
-        MOE_REQUIRE(E <= 65535, MOE_ERR_UNSUPPORTED);
-        swiglu_bwd_elem_kernel<<<g2, 256, 0, stream>>>(ab, dh, used, C, F, h, dab);
-        rc = launch_status();
+        TcGemmProblem p{};
+        p.a = dybuf;
+        p.lda = H;
+        p.a_rows_total = (int64_t)E * C;
+        p.a_rows_per_group = C;
+        p.b = wdT;
+        p.ldb = H;
+        p.b_rows_total = (int64_t)E * F;
+        p.b_rows_per_group = F;
+        p.G = E;
+        p.M = C;
+        p.N = F;
+        p.K = H;
+        p.rows = used;
+        p.out = h;
+        p.ldo = F;
+        p.out_rows_per_group = C;
+        p.aux = ab;
+        p.aux_ld = F2;
+        p.out2 = dab;
+        p.ldo2 = F2;
+        p.epilogue = TC_EPI_SWIGLU_BWD;
+        p.status = dev_status;
+        rc = tc_gemm_run(p, stream);
         if (rc != MOE_OK) return rc;
     }
     // 6. weight gradients over the token index: transposed operands, zeros past used[e]
@@ -573,14 +569,15 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     if (rc != MOE_OK) return rc;
     rc = transpose_valid(xb, H, C * H, E, C, H, used, Cp, xbufT, Cp, H * Cp, stream);
     if (rc != MOE_OK) return rc;
+    // K = the expert's kept tokens only (the transposed operands are zero past used[e])
     rc = gemm(dybufT, Cp, (int64_t)E * H, H, hT, Cp, (int64_t)E * F, F, E, H, F, Cp, nullptr, dw_down, F, H,
-              TC_EPI_F32, dev_status, stream);
+              TC_EPI_F32, dev_status, stream, used);
     if (rc != MOE_OK) return rc;
     rc = gemm(dabT, Cp, (int64_t)E * F2, F2, xbufT, Cp, (int64_t)E * H, H, E, F, H, Cp, nullptr, dw_gate, H, F,
-              TC_EPI_F32, dev_status, stream);
+              TC_EPI_F32, dev_status, stream, used);
     if (rc != MOE_OK) return rc;
     rc = gemm(dabT + F * Cp, Cp, (int64_t)E * F2 - F, F2, xbufT, Cp, (int64_t)E * H, H, E, F, H, Cp, nullptr, dw_up,
-              H, F, TC_EPI_F32, dev_status, stream);
+              H, F, TC_EPI_F32, dev_status, stream, used);
     if (rc != MOE_OK) return rc;
     // 7. dxbuf = [da | db] [Wg; Wu], with the stacked weights transposed to (E, H, 2F)
     rc = transpose_valid(static_cast<const bf16*>(w_gate), H, F * H, E, F, H, nullptr, F, wguT, F2, H * F2, stream);

@@ -46,14 +46,21 @@ struct KParams {
     int k_blocks;
     uint32_t tx_bytes;
     const int32_t* rows;
+    const int32_t* k_rows;
     void* out;
     int64_t ldo;
     int64_t out_rows_per_group;
     const void* bias;
     int64_t bias_group_stride;
+    const float* aux;
+    int64_t aux_ld;
+    void* out2;
+    int64_t ldo2;
     int vec_ok;
     int32_t* status;
 };
+
+constexpr bool is_dual(int epi) { return epi == TC_EPI_SWIGLU || epi == TC_EPI_F32_DUAL; }
 
 using namespace tc;
 
@@ -73,6 +80,16 @@ __device__ __forceinline__ void decode_tile(int tile, const int* prefix, int G, 
     const int mtiles = (prefix[g + 1] - prefix[g]) / n_tiles;
     nt = local / mtiles;
     mt = local - nt * mtiles;
+}
+
+// K blocks of group g: all of them, or (k_rows given) those holding its first
+// k_rows[g] K positions, at least one (the operands are zero past k_rows[g], so
+// a group with none still produces its zero tile).
+__device__ __forceinline__ int group_k_blocks(const KParams& p, int g) {
+    if (p.k_rows == nullptr) return p.k_blocks;
+    const int v = p.k_rows[g];
+    const int kb = v <= 0 ? 1 : (v + kBK - 1) / kBK;
+    return kb < p.k_blocks ? kb : p.k_blocks;
 }
 
 // Store 32 bf16 values (already packed in pairs) for columns n0..n0+31 of one row.
@@ -162,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_tile(tile, s_prefix, p.G, p.n_tiles, g, mt, nt);
                 const int32_t a_y = (int32_t)(g * p.a_rows_per_group + (int64_t)mt * kBM);
                 const int32_t b_y = (int32_t)(g * p.b_rows_per_group + (int64_t)nt * p.b_box_rows);
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                const int kbg = group_k_blocks(p, g);
+                for (int kb = 0; kb < kbg; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) {
                         s_abort = 1;
                         break;
@@ -172,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* b_dst = smB + stage * kBBytes;
                     tma_load_2d(a_dst, &tmA, kb * kBK, a_y, &full[stage]);
                     tma_load_2d(b_dst, &tmB, kb * kBK, b_y, &full[stage]);
-                    if (EPI == TC_EPI_SWIGLU)
+                    if (is_dual(EPI))
                         tma_load_2d(b_dst + p.b_box_rows * (kBK * 2), &tmB2, kb * kBK, b_y, &full[stage]);
                     if (++stage == kStages) {
                         stage = 0;
@@ -199,7 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * kBN;
                 bool ok = true;
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                int g_, mt_, nt_;
+                decode_tile(tile, s_prefix, p.G, p.n_tiles, g_, mt_, nt_);
+                const int kbg = group_k_blocks(p, g_);
+                for (int kb = 0; kb < kbg; ++kb) {
                     if (!mbar_wait(&full[stage], phase, p.status)) {
                         s_abort = 1;
                         ok = false;
@@ -265,6 +286,82 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
                     if (row_ok) store_bf16_32(orow, n0, p.N, pk, p.vec_ok);
+                }
+            } else if (EPI == TC_EPI_F32_DUAL) {
+                // gate half of the accumulator -> columns [0, N), up half -> [N, 2N)
+                float* orow = reinterpret_cast<float*>(p.out) + out_row * p.ldo;
+                const int half = p.n_mma / 2;
+                for (int c = 0; c < p.n_mma / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(t_row + c * 32, r);
+                    tmem_ld_wait(r);
+                    const bool up = c * 32 >= half;
+                    const int64_t n0 = (int64_t)nt * p.tile_n_out + (up ? c * 32 - half : c * 32);
+                    float* dst = orow + (up ? p.N : 0);
+                    if (row_ok) {
+                        if (p.vec_ok && n0 + 32 <= p.N) {
+                            float4* d4 = reinterpret_cast<float4*>(dst + n0);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                    __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (n0 + i < p.N) dst[n0 + i] = __uint_as_float(r[i]);
+                        }
+                    }
+                }
+            } else if (EPI == TC_EPI_SWIGLU_BWD) {
+                // dh in the accumulator; a, b from aux:
+                //   h = silu(a) b, da = dh b s (1 + a (1 - s)), db = dh a s,  s = sigmoid(a)
+                __nv_bfloat16* hrow = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * p.ldo;
+                __nv_bfloat16* drow = reinterpret_cast<__nv_bfloat16*>(p.out2) + out_row * p.ldo2;
+                const float* arow = p.aux + out_row * p.aux_ld;
+                for (int c = 0; c < p.n_mma / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(t_row + c * 32, r);
+                    tmem_ld_wait(r);
+                    const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
+                    if (!row_ok || n0 >= p.N) continue;
+                    float av[32], bv[32];
+                    if (p.vec_ok && n0 + 32 <= p.N) {
+                        const float4* a4 = reinterpret_cast<const float4*>(arow + n0);
+                        const float4* b4 = reinterpret_cast<const float4*>(arow + p.N + n0);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 x = a4[i], y = b4[i];
+                            av[4 * i] = x.x; av[4 * i + 1] = x.y; av[4 * i + 2] = x.z; av[4 * i + 3] = x.w;
+                            bv[4 * i] = y.x; bv[4 * i + 1] = y.y; bv[4 * i + 2] = y.z; bv[4 * i + 3] = y.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const bool in = n0 + i < p.N;
+                            av[i] = in ? arow[n0 + i] : 0.f;
+                            bv[i] = in ? arow[p.N + n0 + i] : 0.f;
+                        }
+                    }
+                    uint32_t ph[16], pa[16], pb[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float hv[2], dav[2], dbv[2];
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            const float a = av[2 * i + m], b = bv[2 * i + m];
+                            const float g = __uint_as_float(r[2 * i + m]);
+                            const float s = 1.0f / (1.0f + expf(-a));
+                            hv[m] = a * s * b;
+                            dav[m] = g * b * s * (1.0f + a * (1.0f - s));
+                            dbv[m] = g * a * s;
+                        }
+                        ph[i] = pack_bf16x2(hv[0], hv[1]);
+                        pa[i] = pack_bf16x2(dav[0], dav[1]);
+                        pb[i] = pack_bf16x2(dbv[0], dbv[1]);
+                    }
+                    store_bf16_32(hrow, n0, p.N, ph, p.vec_ok);
+                    store_bf16_32(drow, n0, p.N, pa, p.vec_ok);
+                    store_bf16_32(drow + p.N, n0, p.N, pb, p.vec_ok);
                 }
             } else if (EPI == TC_EPI_F32) {
                 float* orow = reinterpret_cast<float*>(p.out) + out_row * p.ldo;
@@ -412,7 +509,9 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     MOE_REQUIRE(aligned16(p.a) && aligned16(p.b) && (p.lda * 2) % 16 == 0 && (p.ldb * 2) % 16 == 0,
                 MOE_ERR_UNSUPPORTED);
     MOE_REQUIRE(p.lda >= p.K && p.ldb >= p.K, MOE_ERR_INVALID_ARG);
-    const bool dual = p.epilogue == TC_EPI_SWIGLU;
+    const bool dual = p.epilogue == TC_EPI_SWIGLU || p.epilogue == TC_EPI_F32_DUAL;
+    if (p.epilogue == TC_EPI_SWIGLU_BWD)
+        MOE_REQUIRE(p.aux && p.out2 && p.aux_ld >= 2 * p.N && p.ldo2 >= 2 * p.N, MOE_ERR_INVALID_ARG);
     if (dual) MOE_REQUIRE(p.b2 && aligned16(p.b2), MOE_ERR_INVALID_ARG);
     // TMA coordinates are 32-bit.
     MOE_REQUIRE(p.a_rows_total < (int64_t(1) << 31) && p.b_rows_total < (int64_t(1) << 31), MOE_ERR_UNSUPPORTED);
@@ -437,13 +536,23 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     kp.k_blocks = (int)((p.K + kBK - 1) / kBK);
     kp.tx_bytes = (uint32_t)(kABytes + kp.n_mma * kBK * 2);
     kp.rows = p.rows;
+    kp.k_rows = p.k_rows;
     kp.out = p.out;
     kp.ldo = p.ldo;
     kp.out_rows_per_group = p.out_rows_per_group;
     kp.bias = p.bias;
     kp.bias_group_stride = p.bias_group_stride;
-    const size_t esz = p.epilogue == TC_EPI_F32 ? 4 : 2;
+    kp.aux = p.aux;
+    kp.aux_ld = p.aux_ld;
+    kp.out2 = p.out2;
+    kp.ldo2 = p.ldo2;
+    const bool f32_out = p.epilogue == TC_EPI_F32 || p.epilogue == TC_EPI_F32_DUAL;
+    const size_t esz = f32_out ? 4 : 2;
     kp.vec_ok = aligned16(p.out) && (p.ldo * (int64_t)esz) % 16 == 0;
+    if (p.epilogue == TC_EPI_F32_DUAL) kp.vec_ok = kp.vec_ok && (p.N * 4) % 16 == 0;
+    if (p.epilogue == TC_EPI_SWIGLU_BWD)
+        kp.vec_ok = kp.vec_ok && aligned16(p.out2) && (p.ldo2 * 2) % 16 == 0 && (p.N * 2) % 16 == 0 &&
+                    aligned16(p.aux) && (p.aux_ld * 4) % 16 == 0 && (p.N * 4) % 16 == 0;
     kp.status = p.status;
 
     CUtensorMap ma, mb, mb2;
@@ -464,6 +573,8 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
         case TC_EPI_BF16_BIAS: return launch<TC_EPI_BF16_BIAS>(ma, mb, mb2, kp, grid, stream);
         case TC_EPI_GELU_BIAS: return launch<TC_EPI_GELU_BIAS>(ma, mb, mb2, kp, grid, stream);
         case TC_EPI_SWIGLU: return launch<TC_EPI_SWIGLU>(ma, mb, mb2, kp, grid, stream);
+        case TC_EPI_F32_DUAL: return launch<TC_EPI_F32_DUAL>(ma, mb, mb2, kp, grid, stream);
+        case TC_EPI_SWIGLU_BWD: return launch<TC_EPI_SWIGLU_BWD>(ma, mb, mb2, kp, grid, stream);
         default: return MOE_ERR_INVALID_ARG;
     }
 }

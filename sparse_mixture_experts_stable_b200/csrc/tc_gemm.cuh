@@ -20,7 +20,10 @@ enum TcEpilogue : int {
     TC_EPI_BF16 = 1,       // bf16 out                                    -- linear / down
     TC_EPI_BF16_BIAS = 2,  // bf16 out, + bf16 bias                       -- GELU MLP fc2
     TC_EPI_GELU_BIAS = 3,  // bf16 gelu(acc + bias)                       -- GELU MLP fc1
-    TC_EPI_SWIGLU = 4      // dual B: bf16 silu(acc_gate) * acc_up        -- SwiGLU gate/up
+    TC_EPI_SWIGLU = 4,     // dual B: bf16 silu(acc_gate) * acc_up        -- SwiGLU gate/up
+    TC_EPI_F32_DUAL = 5,   // dual B: fp32 acc_gate -> out[., n], acc_up -> out[., N + n]   -- [a | b] recompute
+    TC_EPI_SWIGLU_BWD = 6  // acc = dh; with (a, b) from aux (fp32, row stride aux_ld, b at + N):
+                           //   out (bf16) = h = silu(a) b; out2 (bf16, row stride ldo2) = [da | db]
 };
 
 struct TcGemmProblem {
@@ -38,11 +41,16 @@ struct TcGemmProblem {
     int64_t N;                // output columns per group
     int64_t K;
     const int32_t* rows;      // device (G) valid rows per group, or NULL (= M)
+    const int32_t* k_rows;    // device (G) valid K per group (operands zero past it), or NULL (= K)
     void* out;                // fp32 or bf16 per epilogue
     int64_t ldo;
     int64_t out_rows_per_group;
     const void* bias;         // fp32 (TC_EPI_F32) or bf16, per output column
     int64_t bias_group_stride;
+    const float* aux;         // TC_EPI_SWIGLU_BWD: [a | b] rows (same row index as out)
+    int64_t aux_ld;
+    void* out2;               // TC_EPI_SWIGLU_BWD: [da | db] rows (same row index as out)
+    int64_t ldo2;
     int epilogue;
     int32_t* status;
 };
