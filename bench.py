@@ -448,7 +448,7 @@ def _time_steps(step, steps, warmup, flush, stream, inner=None):
     return step_ms, inner_ms
 
 
-def run_other_workloads(steps, warmup, flush, stream, dev):
+def run_other_workloads(steps, warmup, flush, stream, dev, only=None):
     import sparse_mixture_experts_stable_b200 as moe
     from sparse_mixture_experts_stable_b200 import binding as B
     from sparse_mixture_experts_stable_b200 import inputs as I
@@ -456,270 +456,280 @@ def run_other_workloads(steps, warmup, flush, stream, dev):
     pk = measured_peaks()
     out = {}
 
+    def want(name):  # the tiny fp32 block also times its training-step line
+        return only is None or name == only or (name == "tiny_gelu_fp32" and only == "tiny_gelu_fp32_train")
+
     def events(lst):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         lst.append((e0, e1))
         return e0, e1
 
-    # router-only with load statistics (router GEMM + softmax/top-k/gates + statistics)
-    c = I.router_bf16(seed=0)
-    T, D, E, k = c["T"], c["D"], c["E"], c["k"]
-    x, w = c["x"].to(dev), c["w_router"].to(dev)
-    ro = dict(selected=torch.empty(T, k, dtype=torch.int64, device=dev),
-              gates=torch.empty(T, k, dtype=torch.bfloat16, device=dev),
-              gates_f32=torch.empty(T, k, dtype=torch.float32, device=dev),
-              counts=torch.empty(E, dtype=torch.int32, device=dev), prob_sum=torch.empty(E, device=dev))
-    ws = torch.empty(B.moe_route_workspace_size(T, D, E, B.MOE_BF16, True, "ED"), dtype=torch.uint8, device=dev)
-    inner = []
+    if want("router_bf16"):
+        # router-only with load statistics (router GEMM + softmax/top-k/gates + statistics)
+        c = I.router_bf16(seed=0)
+        T, D, E, k = c["T"], c["D"], c["E"], c["k"]
+        x, w = c["x"].to(dev), c["w_router"].to(dev)
+        ro = dict(selected=torch.empty(T, k, dtype=torch.int64, device=dev),
+                  gates=torch.empty(T, k, dtype=torch.bfloat16, device=dev),
+                  gates_f32=torch.empty(T, k, dtype=torch.float32, device=dev),
+                  counts=torch.empty(E, dtype=torch.int32, device=dev), prob_sum=torch.empty(E, device=dev))
+        ws = torch.empty(B.moe_route_workspace_size(T, D, E, B.MOE_BF16, True, "ED"), dtype=torch.uint8, device=dev)
+        inner = []
 
-    def step_router():
-        e0, e1 = events(inner)
-        e0.record(stream)
-        moe.moe_route(x, k, w_router=w, out=ro, workspace=ws)
-        e1.record(stream)
-        moe.moe_aux_stats(ro["counts"], ro["prob_sum"], T, k, out_dtype=torch.bfloat16)
+        def step_router():
+            e0, e1 = events(inner)
+            e0.record(stream)
+            moe.moe_route(x, k, w_router=w, out=ro, workspace=ws)
+            e1.record(stream)
+            moe.moe_aux_stats(ro["counts"], ro["prob_sum"], T, k, out_dtype=torch.bfloat16)
 
-    sm, im = _time_steps(step_router, steps, warmup, flush, stream, inner)
-    r_s = statistics.mean(im) / 1e3
-    bytes_alg = T * D * 2 + E * D * 2 + T * k * (8 + 2 + 4) + E * 8
-    flops = 2.0 * T * D * E
-    out["router_bf16"] = dict(
-        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
-        config=dict(T=T, D=D, E=E, k=k),
-        roofline=dict(bound="hbm/tensor ridge", kernel="moe_route: tc_gemm_kernel<F32> scores + route_topk_kernel + route_reduce_kernel",
-                      achieved=bytes_alg / r_s / 1e9, peak=pk["hbm"], unit="GB/s", frac=bytes_alg / r_s / 1e9 / pk["hbm"],
-                      tflops=flops / r_s / 1e12, frac_tensor=flops / r_s / 1e12 / pk["bf16"], traffic=None,
-                      bytes_per_launch=bytes_alg, flops_per_launch=flops, avg_launch_ms=1e3 * r_s))
-    del x, w, ws, ro
+        sm, im = _time_steps(step_router, steps, warmup, flush, stream, inner)
+        r_s = statistics.mean(im) / 1e3
+        bytes_alg = T * D * 2 + E * D * 2 + T * k * (8 + 2 + 4) + E * 8
+        flops = 2.0 * T * D * E
+        out["router_bf16"] = dict(
+            value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+            config=dict(T=T, D=D, E=E, k=k),
+            roofline=dict(bound="hbm/tensor ridge", kernel="moe_route: tc_gemm_kernel<F32> scores + route_topk_kernel + route_reduce_kernel",
+                          achieved=bytes_alg / r_s / 1e9, peak=pk["hbm"], unit="GB/s", frac=bytes_alg / r_s / 1e9 / pk["hbm"],
+                          tflops=flops / r_s / 1e12, frac_tensor=flops / r_s / 1e12 / pk["bf16"], traffic=None,
+                          bytes_per_launch=bytes_alg, flops_per_launch=flops, avg_launch_ms=1e3 * r_s))
+        del x, w, ws, ro
 
-    # capacity-limited top-1 dispatch/combine with linear experts
-    c = I.dispatch_top1_bf16(seed=0)
-    T, D, E = c["T"], c["D"], c["E"]
-    C = moe.moe_capacity(T, 1, E, c["capacity_factor"])
-    idx = c["expert_idx"].view(T, 1).to(dev)
-    x, w, gate = c["x"].to(dev), c["w"].to(dev), c["gate"].view(T, 1).to(dev)
-    do = dict(slot=torch.empty(T, 1, dtype=torch.int64, device=dev), kept=torch.empty(T, 1, dtype=torch.uint8, device=dev),
-              used=torch.empty(E, dtype=torch.int32, device=dev), overflow=torch.empty(E, dtype=torch.int32, device=dev),
-              drops=torch.empty(T, dtype=torch.int32, device=dev),
-              token_of_slot=torch.empty(E, C, dtype=torch.int32, device=dev),
-              xbuf=torch.empty(E, C, D, dtype=torch.bfloat16, device=dev))
-    ybuf = torch.empty(E, C, D, dtype=torch.bfloat16, device=dev)
-    y = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
-    wsd = torch.empty(B.moe_dispatch_workspace_size(T, 1, E), dtype=torch.uint8, device=dev)
-    inner = []
+    if want("dispatch_top1_bf16"):
+        # capacity-limited top-1 dispatch/combine with linear experts
+        c = I.dispatch_top1_bf16(seed=0)
+        T, D, E = c["T"], c["D"], c["E"]
+        C = moe.moe_capacity(T, 1, E, c["capacity_factor"])
+        idx = c["expert_idx"].view(T, 1).to(dev)
+        x, w, gate = c["x"].to(dev), c["w"].to(dev), c["gate"].view(T, 1).to(dev)
+        do = dict(slot=torch.empty(T, 1, dtype=torch.int64, device=dev), kept=torch.empty(T, 1, dtype=torch.uint8, device=dev),
+                  used=torch.empty(E, dtype=torch.int32, device=dev), overflow=torch.empty(E, dtype=torch.int32, device=dev),
+                  drops=torch.empty(T, dtype=torch.int32, device=dev),
+                  token_of_slot=torch.empty(E, C, dtype=torch.int32, device=dev),
+                  xbuf=torch.empty(E, C, D, dtype=torch.bfloat16, device=dev))
+        ybuf = torch.empty(E, C, D, dtype=torch.bfloat16, device=dev)
+        y = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
+        wsd = torch.empty(B.moe_dispatch_workspace_size(T, 1, E), dtype=torch.uint8, device=dev)
+        inner = []
 
-    def step_top1():
-        moe.moe_dispatch(idx, E, C, x=x, out=do, workspace=wsd)
-        e0, e1 = events(inner)
-        e0.record(stream)
-        moe.moe_expert_ffn("linear", do["xbuf"], do["used"], w, ybuf=ybuf)
-        e1.record(stream)
-        moe.moe_combine(ybuf, idx, do["slot"], gate, y=y)
+        def step_top1():
+            moe.moe_dispatch(idx, E, C, x=x, out=do, workspace=wsd)
+            e0, e1 = events(inner)
+            e0.record(stream)
+            moe.moe_expert_ffn("linear", do["xbuf"], do["used"], w, ybuf=ybuf)
+            e1.record(stream)
+            moe.moe_combine(ybuf, idx, do["slot"], gate, y=y)
 
-    sm, im = _time_steps(step_top1, steps, warmup, flush, stream, inner)
-    used = do["used"].cpu()
-    kept = int(used.sum())
-    active = int((used > 0).sum())
-    f_s = statistics.mean(im) / 1e3
-    bytes_alg = kept * D * 2 + active * D * D * 2 + kept * D * 2
-    out["dispatch_top1_bf16"] = dict(
-        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
-        config=dict(T=T, D=D, E=E, k=1, capacity=C, kept=kept),
-        roofline=dict(bound="hbm", kernel="tcx_kernel: linear experts (moe_expert_ffn)", achieved=bytes_alg / f_s / 1e9,
-                      peak=pk["hbm"], unit="GB/s", frac=bytes_alg / f_s / 1e9 / pk["hbm"], traffic=None,
-                      tflops=2.0 * kept * D * D / f_s / 1e12, bytes_per_launch=bytes_alg, avg_launch_ms=1e3 * f_s))
-    del x, w, gate, do, ybuf, y
+        sm, im = _time_steps(step_top1, steps, warmup, flush, stream, inner)
+        used = do["used"].cpu()
+        kept = int(used.sum())
+        active = int((used > 0).sum())
+        f_s = statistics.mean(im) / 1e3
+        bytes_alg = kept * D * 2 + active * D * D * 2 + kept * D * 2
+        out["dispatch_top1_bf16"] = dict(
+            value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+            config=dict(T=T, D=D, E=E, k=1, capacity=C, kept=kept),
+            roofline=dict(bound="hbm", kernel="tcx_kernel: linear experts (moe_expert_ffn)", achieved=bytes_alg / f_s / 1e9,
+                          peak=pk["hbm"], unit="GB/s", frac=bytes_alg / f_s / 1e9 / pk["hbm"], traffic=None,
+                          tflops=2.0 * kept * D * D / f_s / 1e12, bytes_per_launch=bytes_alg, avg_launch_ms=1e3 * f_s))
+        del x, w, gate, do, ybuf, y
 
-    # tiny top-2 GELU layer, fp32
-    c = I.tiny_gelu_fp32(seed=0)
-    T, D, E, F, k = c["T"], c["D"], c["E"], c["F"], c["k"]
-    C = moe.moe_capacity(T, k, E, c["capacity_factor"])
-    dv = {n: c[n].to(dev) for n in ("x", "w_router", "w1", "b1", "w2", "b2")}
-    inner = []
+    if want("tiny_gelu_fp32"):
+        # tiny top-2 GELU layer, fp32
+        c = I.tiny_gelu_fp32(seed=0)
+        T, D, E, F, k = c["T"], c["D"], c["E"], c["F"], c["k"]
+        C = moe.moe_capacity(T, k, E, c["capacity_factor"])
+        dv = {n: c[n].to(dev) for n in ("x", "w_router", "w1", "b1", "w2", "b2")}
+        inner = []
 
-    def step_tiny():
-        r = moe.moe_route(dv["x"], k, w_router=dv["w_router"])
-        d = moe.moe_dispatch(r["selected"], E, C, x=dv["x"])
-        e0, e1 = events(inner)
-        e0.record(stream)
-        yb = moe.moe_expert_ffn("gelu_mlp", d["xbuf"], d["used"], dv["w1"], b1=dv["b1"], w2=dv["w2"], b2=dv["b2"])
-        e1.record(stream)
-        moe.moe_combine(yb, r["selected"], d["slot"], r["gates_f32"], base_kind="input", base=dv["x"])
-        moe.moe_aux_stats(r["counts"], r["prob_sum"], T, k, True, 0.01)
+        def step_tiny():
+            r = moe.moe_route(dv["x"], k, w_router=dv["w_router"])
+            d = moe.moe_dispatch(r["selected"], E, C, x=dv["x"])
+            e0, e1 = events(inner)
+            e0.record(stream)
+            yb = moe.moe_expert_ffn("gelu_mlp", d["xbuf"], d["used"], dv["w1"], b1=dv["b1"], w2=dv["w2"], b2=dv["b2"])
+            e1.record(stream)
+            moe.moe_combine(yb, r["selected"], d["slot"], r["gates_f32"], base_kind="input", base=dv["x"])
+            moe.moe_aux_stats(r["counts"], r["prob_sum"], T, k, True, 0.01)
 
-    sm, im = _time_steps(step_tiny, steps, warmup, flush, stream, inner)
-    f_s = statistics.mean(im) / 1e3
-    flops = 2.0 * T * k * (D * F + F * D)
-    out["tiny_gelu_fp32"] = dict(
-        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
-        config=dict(T=T, D=D, E=E, F=F, k=k, capacity=C),
-        roofline=dict(bound="tensor", kernel="tf32x3_kernel: GELU MLP experts (moe_expert_ffn, split-tf32)",
-                      achieved=3 * flops / f_s / 1e12, peak=tf32_peak(pk), unit="TFLOP/s",
-                      frac=3 * flops / f_s / 1e12 / tf32_peak(pk), traffic=None, avg_launch_ms=1e3 * f_s,
-                      fp32_tflops=flops / f_s / 1e12, peak_source=TF32_PEAK_SOURCE,
-                      note="three tf32 MMAs per fp32 product; launch-latency bound at this size"))
+        sm, im = _time_steps(step_tiny, steps, warmup, flush, stream, inner)
+        f_s = statistics.mean(im) / 1e3
+        flops = 2.0 * T * k * (D * F + F * D)
+        out["tiny_gelu_fp32"] = dict(
+            value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+            config=dict(T=T, D=D, E=E, F=F, k=k, capacity=C),
+            roofline=dict(bound="tensor", kernel="tf32x3_kernel: GELU MLP experts (moe_expert_ffn, split-tf32)",
+                          achieved=3 * flops / f_s / 1e12, peak=tf32_peak(pk), unit="TFLOP/s",
+                          frac=3 * flops / f_s / 1e12 / tf32_peak(pk), traffic=None, avg_launch_ms=1e3 * f_s,
+                          fp32_tflops=flops / f_s / 1e12, peak_source=TF32_PEAK_SOURCE,
+                          note="three tf32 MMAs per fp32 product; launch-latency bound at this size"))
 
-    # the same layer's training step: forward, GELU-expert backward, router backward (fp32)
-    dyg = torch.randn(T, D, generator=torch.Generator().manual_seed(2)).to(dev)
-    wsg = torch.empty(B.moe_backward_gelu_workspace_size(E, C, D, F, D), dtype=torch.uint8, device=dev)
-    inner = []
-    kept_box = {}
+        # the same layer's training step: forward, GELU-expert backward, router backward (fp32)
+        dyg = torch.randn(T, D, generator=torch.Generator().manual_seed(2)).to(dev)
+        wsg = torch.empty(B.moe_backward_gelu_workspace_size(E, C, D, F, D), dtype=torch.uint8, device=dev)
+        inner = []
+        kept_box = {}
 
-    def step_tiny_train():
-        r = moe.moe_route(dv["x"], k, w_router=dv["w_router"], want_logits=True)
-        d = moe.moe_dispatch(r["selected"], E, C, x=dv["x"])
-        yb = moe.moe_expert_ffn("gelu_mlp", d["xbuf"], d["used"], dv["w1"], b1=dv["b1"], w2=dv["w2"], b2=dv["b2"])
-        moe.moe_combine(yb, r["selected"], d["slot"], r["gates_f32"], base_kind="input", base=dv["x"])
-        e0, e1 = events(inner)
-        e0.record(stream)
-        g = moe.moe_backward_gelu(dyg, r["logits"], r["selected"], r["gates_f32"], d["slot"], d["used"], d["xbuf"],
-                                  yb, dv["w1"], dv["b1"], dv["w2"], C, use_residual=True, workspace=wsg)
-        e1.record(stream)
-        moe.moe_router_backward(dv["x"], dv["w_router"], g[5])
-        kept_box["used"] = d["used"]
+        def step_tiny_train():
+            r = moe.moe_route(dv["x"], k, w_router=dv["w_router"], want_logits=True)
+            d = moe.moe_dispatch(r["selected"], E, C, x=dv["x"])
+            yb = moe.moe_expert_ffn("gelu_mlp", d["xbuf"], d["used"], dv["w1"], b1=dv["b1"], w2=dv["w2"], b2=dv["b2"])
+            moe.moe_combine(yb, r["selected"], d["slot"], r["gates_f32"], base_kind="input", base=dv["x"])
+            e0, e1 = events(inner)
+            e0.record(stream)
+            g = moe.moe_backward_gelu(dyg, r["logits"], r["selected"], r["gates_f32"], d["slot"], d["used"], d["xbuf"],
+                                      yb, dv["w1"], dv["b1"], dv["w2"], C, use_residual=True, workspace=wsg)
+            e1.record(stream)
+            moe.moe_router_backward(dv["x"], dv["w_router"], g[5])
+            kept_box["used"] = d["used"]
 
-    sm, im = _time_steps(step_tiny_train, steps, warmup, flush, stream, inner)
-    kept = int(kept_box["used"].sum())
-    b_s = statistics.mean(im) / 1e3
-    flops_b = 2.0 * kept * D * F * 5  # recomputed z, dh, dW2, dW1, dx: 2*kept*D*F each
-    out["tiny_gelu_fp32_train"] = dict(
-        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
-        config=dict(T=T, D=D, E=E, F=F, k=k, capacity=C, kept=kept,
-                    step="forward + moe_backward_gelu + moe_router_backward"),
-        roofline=dict(bound="tensor", kernel="moe_backward_gelu (tf32x3_kernel x5, elementwise, sums, combine)",
-                      achieved=3 * flops_b / b_s / 1e12, peak=tf32_peak(pk), unit="TFLOP/s",
-                      frac=3 * flops_b / b_s / 1e12 / tf32_peak(pk), traffic=None, avg_launch_ms=1e3 * b_s,
-                      fp32_tflops=flops_b / b_s / 1e12, peak_source=TF32_PEAK_SOURCE,
-                      note="launch-latency bound at this size"))
-    del dv, dyg, wsg
+        sm, im = _time_steps(step_tiny_train, steps, warmup, flush, stream, inner)
+        kept = int(kept_box["used"].sum())
+        b_s = statistics.mean(im) / 1e3
+        flops_b = 2.0 * kept * D * F * 5  # recomputed z, dh, dW2, dW1, dx: 2*kept*D*F each
+        out["tiny_gelu_fp32_train"] = dict(
+            value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+            config=dict(T=T, D=D, E=E, F=F, k=k, capacity=C, kept=kept,
+                        step="forward + moe_backward_gelu + moe_router_backward"),
+            roofline=dict(bound="tensor", kernel="moe_backward_gelu (tf32x3_kernel x5, elementwise, sums, combine)",
+                          achieved=3 * flops_b / b_s / 1e12, peak=tf32_peak(pk), unit="TFLOP/s",
+                          frac=3 * flops_b / b_s / 1e12 / tf32_peak(pk), traffic=None, avg_launch_ms=1e3 * b_s,
+                          fp32_tflops=flops_b / b_s / 1e12, peak_source=TF32_PEAK_SOURCE,
+                          note="launch-latency bound at this size"))
+        del dv, dyg, wsg
 
-    # forward + backward, fp32, linear experts with residual
-    c = I.fwd_bwd_fp32(seed=0)
-    T, D, E, k = c["T"], c["D"], c["E"], c["k"]
-    C = moe.moe_capacity(T, k, E, c["capacity_factor"])
-    lg, x, w, dy = (c[n].to(dev) for n in ("logits", "x", "w", "dy"))
-    inner = []
-    wsb = torch.empty(B.moe_backward_workspace_size(E, C, D, D), dtype=torch.uint8, device=dev)
-    state = {}
+    if want("fwd_bwd_fp32"):
+        # forward + backward, fp32, linear experts with residual
+        c = I.fwd_bwd_fp32(seed=0)
+        T, D, E, k = c["T"], c["D"], c["E"], c["k"]
+        C = moe.moe_capacity(T, k, E, c["capacity_factor"])
+        lg, x, w, dy = (c[n].to(dev) for n in ("logits", "x", "w", "dy"))
+        inner = []
+        wsb = torch.empty(B.moe_backward_workspace_size(E, C, D, D), dtype=torch.uint8, device=dev)
+        state = {}
 
-    def step_fb():
-        r = moe.moe_route(lg, k)
-        d = moe.moe_dispatch(r["selected"], E, C, x=x)
-        yb = moe.moe_expert_ffn("linear", d["xbuf"], d["used"], w)
-        moe.moe_combine(yb, r["selected"], d["slot"], r["gates_f32"], base_kind="input", base=x)
-        e0, e1 = events(inner)
-        e0.record(stream)
-        moe.moe_backward(dy, x, lg, r["selected"], r["gates_f32"], d["slot"], d["used"], d["token_of_slot"],
-                         d["xbuf"], yb, w, C, workspace=wsb)
-        e1.record(stream)
-        state["used"] = d["used"]
+        def step_fb():
+            r = moe.moe_route(lg, k)
+            d = moe.moe_dispatch(r["selected"], E, C, x=x)
+            yb = moe.moe_expert_ffn("linear", d["xbuf"], d["used"], w)
+            moe.moe_combine(yb, r["selected"], d["slot"], r["gates_f32"], base_kind="input", base=x)
+            e0, e1 = events(inner)
+            e0.record(stream)
+            moe.moe_backward(dy, x, lg, r["selected"], r["gates_f32"], d["slot"], d["used"], d["token_of_slot"],
+                             d["xbuf"], yb, w, C, workspace=wsb)
+            e1.record(stream)
+            state["used"] = d["used"]
 
-    sm, im = _time_steps(step_fb, steps, warmup, flush, stream, inner)
-    kept = int(state["used"].sum())
-    b_s = statistics.mean(im) / 1e3
-    flops_b = 2.0 * kept * D * D * 2 + 2.0 * kept * D
-    out["fwd_bwd_fp32"] = dict(
-        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
-        config=dict(T=T, D=D, E=E, k=k, capacity=C, kept=kept),
-        roofline=dict(bound="tensor", kernel="moe_backward (tf32x3_kernel dW + dx, dgate/dlogits, combine)",
-                      achieved=3 * flops_b / b_s / 1e12, peak=tf32_peak(pk), unit="TFLOP/s",
-                      frac=3 * flops_b / b_s / 1e12 / tf32_peak(pk), traffic=None, avg_launch_ms=1e3 * b_s,
-                      fp32_tflops=flops_b / b_s / 1e12, peak_source=TF32_PEAK_SOURCE))
-    del lg, x, w, dy, wsb, state
+        sm, im = _time_steps(step_fb, steps, warmup, flush, stream, inner)
+        kept = int(state["used"].sum())
+        b_s = statistics.mean(im) / 1e3
+        flops_b = 2.0 * kept * D * D * 2 + 2.0 * kept * D
+        out["fwd_bwd_fp32"] = dict(
+            value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+            config=dict(T=T, D=D, E=E, k=k, capacity=C, kept=kept),
+            roofline=dict(bound="tensor", kernel="moe_backward (tf32x3_kernel dW + dx, dgate/dlogits, combine)",
+                          achieved=3 * flops_b / b_s / 1e12, peak=tf32_peak(pk), unit="TFLOP/s",
+                          frac=3 * flops_b / b_s / 1e12 / tf32_peak(pk), traffic=None, avg_launch_ms=1e3 * b_s,
+                          fp32_tflops=flops_b / b_s / 1e12, peak_source=TF32_PEAK_SOURCE))
+        del lg, x, w, dy, wsb, state
 
-    # expert parallelism, 4 ranks emulated on this GPU: the full-layer batch split over the ranks, every rank's
-    # rows written into and read from the other ranks' buffers through the peer-pointer tables
-    from sparse_mixture_experts_stable_b200 import ep
-    c = I.full_layer_bf16(seed=0)
-    T, H, E, F, k = c["T"], c["H"], c["E"], c["F"], c["k"]
-    R, epr = 4, c["E"] // 4
-    C = moe.moe_capacity(T, k, E, c["capacity_factor"])
-    dv = {n: c[n].to(dev) for n in ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down")}
-    xs = [t.contiguous() for t in torch.chunk(dv["x"], R)]
-    wr = [{"w1": dv["w_gate"][q * epr:(q + 1) * epr], "w3": dv["w_up"][q * epr:(q + 1) * epr],
-           "w2": dv["w_down"][q * epr:(q + 1) * epr]} for q in range(R)]
-    xbufs = [torch.empty(epr, C, H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
-    ybufs = [torch.empty(epr, C, H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
-    ys = [torch.empty_like(t) for t in xs]
-    tb = ep.token_bases([t.shape[0] for t in xs])
-    wsd = torch.empty(B.moe_dispatch_workspace_size(T // R, k, E), dtype=torch.uint8, device=dev)
-    inner_d, inner_c = [], []
-    kept_box = {}
+    if want("full_layer_bf16_ep4_one_device"):
+        # expert parallelism, 4 ranks emulated on this GPU: the full-layer batch split over the ranks, every rank's
+        # rows written into and read from the other ranks' buffers through the peer-pointer tables
+        from sparse_mixture_experts_stable_b200 import ep
+        c = I.full_layer_bf16(seed=0)
+        T, H, E, F, k = c["T"], c["H"], c["E"], c["F"], c["k"]
+        R, epr = 4, c["E"] // 4
+        C = moe.moe_capacity(T, k, E, c["capacity_factor"])
+        dv = {n: c[n].to(dev) for n in ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down")}
+        xs = [t.contiguous() for t in torch.chunk(dv["x"], R)]
+        wr = [{"w1": dv["w_gate"][q * epr:(q + 1) * epr], "w3": dv["w_up"][q * epr:(q + 1) * epr],
+               "w2": dv["w_down"][q * epr:(q + 1) * epr]} for q in range(R)]
+        xbufs = [torch.empty(epr, C, H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
+        ybufs = [torch.empty(epr, C, H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
+        ys = [torch.empty_like(t) for t in xs]
+        tb = ep.token_bases([t.shape[0] for t in xs])
+        wsd = torch.empty(B.moe_dispatch_workspace_size(T // R, k, E), dtype=torch.uint8, device=dev)
+        inner_d, inner_c = [], []
+        kept_box = {}
 
-    def step_ep():
-        routes = [moe.moe_route(xs[q], k, w_router=dv["w_router"], logit_bias=dv["router_bias"]) for q in range(R)]
-        counts_all = torch.stack([r["counts"] for r in routes])
-        plans = [moe.moe_ep_plan(counts_all, q, C) for q in range(R)]
-        e0, e1 = events(inner_d)
-        e0.record(stream)
-        disp = [moe.moe_ep_dispatch(routes[q]["selected"], E, C, plans[q]["rank_base"], tb[q], xs[q], xbufs,
-                                    workspace=wsd) for q in range(R)]
-        e1.record(stream)
-        for q in range(R):
-            moe.moe_expert_ffn("swiglu", xbufs[q], plans[q]["used"][q * epr:(q + 1) * epr], wr[q]["w1"],
-                               w2=wr[q]["w2"], w3=wr[q]["w3"], ybuf=ybufs[q])
-        e0, e1 = events(inner_c)
-        e0.record(stream)
-        for q in range(R):
-            moe.moe_ep_combine(ybufs, routes[q]["selected"], disp[q]["slot"], routes[q]["gates_f32"], E, C, H,
-                               torch.bfloat16, base_kind="input", base=xs[q], y=ys[q])
-        e1.record(stream)
-        kept_box["used"] = plans[0]["used"]
+        def step_ep():
+            routes = [moe.moe_route(xs[q], k, w_router=dv["w_router"], logit_bias=dv["router_bias"]) for q in range(R)]
+            counts_all = torch.stack([r["counts"] for r in routes])
+            plans = [moe.moe_ep_plan(counts_all, q, C) for q in range(R)]
+            e0, e1 = events(inner_d)
+            e0.record(stream)
+            disp = [moe.moe_ep_dispatch(routes[q]["selected"], E, C, plans[q]["rank_base"], tb[q], xs[q], xbufs,
+                                        workspace=wsd) for q in range(R)]
+            e1.record(stream)
+            for q in range(R):
+                moe.moe_expert_ffn("swiglu", xbufs[q], plans[q]["used"][q * epr:(q + 1) * epr], wr[q]["w1"],
+                                   w2=wr[q]["w2"], w3=wr[q]["w3"], ybuf=ybufs[q])
+            e0, e1 = events(inner_c)
+            e0.record(stream)
+            for q in range(R):
+                moe.moe_ep_combine(ybufs, routes[q]["selected"], disp[q]["slot"], routes[q]["gates_f32"], E, C, H,
+                                   torch.bfloat16, base_kind="input", base=xs[q], y=ys[q])
+            e1.record(stream)
+            kept_box["used"] = plans[0]["used"]
 
-    sm, _ = _time_steps(step_ep, steps, warmup, flush, stream)
-    kept = int(kept_box["used"].sum())
-    d_s = statistics.mean(a.elapsed_time(b) for a, b in inner_d[-steps:]) / 1e3
-    c_s = statistics.mean(a.elapsed_time(b) for a, b in inner_c[-steps:]) / 1e3
-    moved = 2 * kept * H * 2  # kept rows out to their owner ranks and back (bf16)
-    bytes_alg = (T * H * 2 + kept * H * 2) + (kept * H * 2 + 2 * T * H * 2)  # dispatch + combine (x and y base/out)
-    out["full_layer_bf16_ep4_one_device"] = dict(
-        value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
-        config=dict(T=T, H=H, E=E, F=F, k=k, capacity=C, kept=kept, ranks=R, experts_per_rank=epr,
-                    step="4 ranks on one GPU: route, counts, moe_ep_plan, moe_ep_dispatch, experts, moe_ep_combine",
-                    shared_experts=0),
-        roofline=dict(bound="hbm", kernel="moe_ep_dispatch gather + moe_ep_combine (peer-pointer row exchange)",
-                      achieved=bytes_alg / (d_s + c_s) / 1e9, peak=pk["hbm"], unit="GB/s",
-                      frac=bytes_alg / (d_s + c_s) / 1e9 / pk["hbm"], traffic=None,
-                      dispatch_ms=1e3 * d_s, combine_ms=1e3 * c_s, bytes_per_step=bytes_alg,
-                      exchanged_bytes=moved, payload_bytes_no_drops=ep.payload_bytes(T, H, k, 2),
-                      note="on one GPU the peer buffers are local HBM; across GPUs the exchanged bytes cross NVLink"))
-    del dv, xs, wr, xbufs, ybufs, ys, wsd
+        sm, _ = _time_steps(step_ep, steps, warmup, flush, stream)
+        kept = int(kept_box["used"].sum())
+        d_s = statistics.mean(a.elapsed_time(b) for a, b in inner_d[-steps:]) / 1e3
+        c_s = statistics.mean(a.elapsed_time(b) for a, b in inner_c[-steps:]) / 1e3
+        moved = 2 * kept * H * 2  # kept rows out to their owner ranks and back (bf16)
+        bytes_alg = (T * H * 2 + kept * H * 2) + (kept * H * 2 + 2 * T * H * 2)  # dispatch + combine (x and y base/out)
+        out["full_layer_bf16_ep4_one_device"] = dict(
+            value=T * steps / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / steps, steps=steps,
+            config=dict(T=T, H=H, E=E, F=F, k=k, capacity=C, kept=kept, ranks=R, experts_per_rank=epr,
+                        step="4 ranks on one GPU: route, counts, moe_ep_plan, moe_ep_dispatch, experts, moe_ep_combine",
+                        shared_experts=0),
+            roofline=dict(bound="hbm", kernel="moe_ep_dispatch gather + moe_ep_combine (peer-pointer row exchange)",
+                          achieved=bytes_alg / (d_s + c_s) / 1e9, peak=pk["hbm"], unit="GB/s",
+                          frac=bytes_alg / (d_s + c_s) / 1e9 / pk["hbm"], traffic=None,
+                          dispatch_ms=1e3 * d_s, combine_ms=1e3 * c_s, bytes_per_step=bytes_alg,
+                          exchanged_bytes=moved, payload_bytes_no_drops=ep.payload_bytes(T, H, k, 2),
+                          note="on one GPU the peer buffers are local HBM; across GPUs the exchanged bytes cross NVLink"))
+        del dv, xs, wr, xbufs, ybufs, ys, wsd
 
-    # training step of the full layer: forward, SwiGLU-expert backward and router backward (bf16)
-    from sparse_mixture_experts_stable_b200.layer import SwiGLUMoE
-    c = I.full_layer_bf16(seed=0)
-    T, H, E, F, k = c["T"], c["H"], c["E"], c["F"], c["k"]
-    dv = {n: c[n].to(dev) for n in ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down")}
-    dyt = (torch.randn(T, H, generator=torch.Generator().manual_seed(1)) * 0.1).to(torch.bfloat16).to(dev)
-    layer = SwiGLUMoE(T, H, E, F, k, c["capacity_factor"], F_shared=0, aux_coef=c["aux_coef"], device=dev)
-    wsbs = torch.empty(B.moe_backward_swiglu_workspace_size(E, layer.C, H, F), dtype=torch.uint8, device=dev)
-    kept_box = {}
-    inner = []
+    if want("full_layer_bf16_train"):
+        # training step of the full layer: forward, SwiGLU-expert backward and router backward (bf16)
+        from sparse_mixture_experts_stable_b200.layer import SwiGLUMoE
+        c = I.full_layer_bf16(seed=0)
+        T, H, E, F, k = c["T"], c["H"], c["E"], c["F"], c["k"]
+        dv = {n: c[n].to(dev) for n in ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down")}
+        dyt = (torch.randn(T, H, generator=torch.Generator().manual_seed(1)) * 0.1).to(torch.bfloat16).to(dev)
+        layer = SwiGLUMoE(T, H, E, F, k, c["capacity_factor"], F_shared=0, aux_coef=c["aux_coef"], device=dev)
+        wsbs = torch.empty(B.moe_backward_swiglu_workspace_size(E, layer.C, H, F), dtype=torch.uint8, device=dev)
+        kept_box = {}
+        inner = []
 
-    def step_train():
-        o = layer.forward(dv["x"], dv["w_router"], dv["router_bias"], dv["w_gate"], dv["w_up"], dv["w_down"])
-        lg_t = layer.route_out.get("logits")
-        e0, e1 = events(inner)
-        e0.record(stream)
-        dxe, dwg, dwu, dwd, dl, dg = moe.moe_backward_swiglu(
-            dyt, lg_t, o["selected"], o["gates_f32"], o["slot"], o["used"], o["xbuf"], layer.ybuf, dv["w_gate"],
-            dv["w_up"], dv["w_down"], layer.C, aux_coef=c["aux_coef"], counts=o["counts"], workspace=wsbs)
-        e1.record(stream)
-        moe.moe_router_backward(dv["x"], dv["w_router"], dl)
-        kept_box["used"] = o["used"]
+        def step_train():
+            o = layer.forward(dv["x"], dv["w_router"], dv["router_bias"], dv["w_gate"], dv["w_up"], dv["w_down"])
+            lg_t = layer.route_out.get("logits")
+            e0, e1 = events(inner)
+            e0.record(stream)
+            dxe, dwg, dwu, dwd, dl, dg = moe.moe_backward_swiglu(
+                dyt, lg_t, o["selected"], o["gates_f32"], o["slot"], o["used"], o["xbuf"], layer.ybuf, dv["w_gate"],
+                dv["w_up"], dv["w_down"], layer.C, aux_coef=c["aux_coef"], counts=o["counts"], workspace=wsbs)
+            e1.record(stream)
+            moe.moe_router_backward(dv["x"], dv["w_router"], dl)
+            kept_box["used"] = o["used"]
 
-    layer.route_out["logits"] = torch.empty(T, E, dtype=torch.float32, device=dev)
-    sm, im = _time_steps(step_train, max(steps // 5, 3), warmup, flush, stream, inner)
-    kept = int(kept_box["used"].sum())
-    bw_s = statistics.mean(im) / 1e3
-    flops_bw = 16.0 * kept * H * F  # recomputed gate/up (4), dh (2), three weight gradients (6), dx (4): x kept*H*F
-    out["full_layer_bf16_train"] = dict(
-        value=T * len(sm) / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / len(sm), steps=len(sm),
-        config=dict(T=T, H=H, E=E, F=F, k=k, capacity=layer.C, kept=kept, shared_experts=0,
-                    step="forward + moe_backward_swiglu + moe_router_backward"),
-        roofline=dict(bound="tensor", kernel="moe_backward_swiglu (tcgen05 GEMMs + transposes)",
-                      achieved=flops_bw / bw_s / 1e12, peak=pk["bf16_sustained"], unit="TFLOP/s",
-                      frac=flops_bw / bw_s / 1e12 / pk["bf16_sustained"], traffic=None, avg_launch_ms=1e3 * bw_s))
+        layer.route_out["logits"] = torch.empty(T, E, dtype=torch.float32, device=dev)
+        sm, im = _time_steps(step_train, max(steps // 5, 3), warmup, flush, stream, inner)
+        kept = int(kept_box["used"].sum())
+        bw_s = statistics.mean(im) / 1e3
+        flops_bw = 16.0 * kept * H * F  # recomputed gate/up (4), dh (2), three weight gradients (6), dx (4): x kept*H*F
+        out["full_layer_bf16_train"] = dict(
+            value=T * len(sm) / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / len(sm), steps=len(sm),
+            config=dict(T=T, H=H, E=E, F=F, k=k, capacity=layer.C, kept=kept, shared_experts=0,
+                        step="forward + moe_backward_swiglu + moe_router_backward"),
+            roofline=dict(bound="tensor", kernel="moe_backward_swiglu (tcgen05 GEMMs + transposes)",
+                          achieved=flops_bw / bw_s / 1e12, peak=pk["bf16_sustained"], unit="TFLOP/s",
+                          frac=flops_bw / bw_s / 1e12 / pk["bf16_sustained"], traffic=None, avg_launch_ms=1e3 * bw_s))
+
     return out
 
 
@@ -736,10 +746,25 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="skip timing the router-only, top-1, tiny fp32 and fp32 fwd+bwd workloads")
+    ap.add_argument("--workload", default=None,
+                    help="time only this secondary workload (e.g. full_layer_bf16_train) and print its line; "
+                         "for profiling captures")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:
-        if args.impl == "reference":
+        if args.workload is not None:
+            import sparse_mixture_experts_stable_b200 as moe
+
+            dev = torch.device("cuda", local)
+            torch.cuda.set_device(dev)
+            moe.lib()
+            flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+            out = run_other_workloads(args.steps, args.warmup, flush, torch.cuda.current_stream(dev), dev,
+                                      only=args.workload)
+            if args.workload not in out:
+                raise SystemExit(f"unknown workload {args.workload}; known: {sorted(out)}")
+            print(json.dumps(dict(workload=args.workload, **out[args.workload])), flush=True)
+        elif args.impl == "reference":
             run_reference(args, world, rank)
         else:
             run_ours(args, world, rank, local)

@@ -274,9 +274,8 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
 //   1. dgate / dlogits                       as above, on bf16 rows
 //   2. dybuf[e,c] = gate * dy[token]         scaled gather (bf16)
 //   3. [a | b] = xbuf [Wg; Wu]^T             one tensor-core GEMM (both weights), fp32 out
-//   4. dh = dybuf Wd -> h, da, db            tensor-core GEMM on Wd^T whose epilogue takes
-//                                            a, b and forms h = silu(a) b and the
-//                                            derivatives (dh never leaves the SM)
+//   4. dh = dybuf Wd                         tensor-core GEMM on Wd^T, fp32 out
+//   5. h, da, db from (a, b, dh)             elementwise (silu and its derivative)
 //   6. dWd = dybuf^T h, dWg = da^T xbuf, dWu = db^T xbuf
 //                                            tensor-core GEMMs on zero-padded,
 //                                            token-transposed operands, fp32 out
@@ -383,6 +382,49 @@ int transpose_valid(const __nv_bfloat16* src, int64_t lds, int64_t sgs, int G, i
     return launch_status();
 }
 
+// h, da, db from a, b (ab rows: [a | b], fp32) and dh (fp32), for c < used[e]:
+//   s = sigmoid(a), h = a s b, da = dh b s (1 + a (1 - s)), db = dh a s.
+// Eight consecutive f per thread (F a multiple of 8): 32-byte fp32 loads,
+// 16-byte bf16 stores.
+__global__ void swiglu_bwd_elem_kernel(const float* __restrict__ ab, const float* __restrict__ dh,
+                                       const int32_t* __restrict__ used, int64_t C, int64_t F,
+                                       __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ dab) {
+    const int e = blockIdx.y;
+    const int64_t u = used[e] < 0 ? 0 : (used[e] < C ? used[e] : C);
+    const int64_t F8 = F / 8;
+    const int64_t n = u * F8;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t c = i / F8, f = (i - c * F8) * 8;
+        const int64_t row = (int64_t)e * C + c;
+        const float4* pa = reinterpret_cast<const float4*>(ab + row * 2 * F + f);
+        const float4* pb = reinterpret_cast<const float4*>(ab + row * 2 * F + F + f);
+        const float4* pg = reinterpret_cast<const float4*>(dh + row * F + f);
+        const float4 a0 = pa[0], a1 = pa[1], b0 = pb[0], b1 = pb[1], g0 = pg[0], g1 = pg[1];
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        uint32_t ph[4], pda[4], pdb[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float hv[2], dav[2], dbv[2];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const float a = av[2 * j + m], b = bv[2 * j + m], g = gv[2 * j + m];
+                const float s = 1.0f / (1.0f + expf(-a));
+                hv[m] = a * s * b;
+                dav[m] = g * b * s * (1.0f + a * (1.0f - s));
+                dbv[m] = g * a * s;
+            }
+            ph[j] = tc::pack_bf16x2(hv[0], hv[1]);
+            pda[j] = tc::pack_bf16x2(dav[0], dav[1]);
+            pdb[j] = tc::pack_bf16x2(dbv[0], dbv[1]);
+        }
+        *reinterpret_cast<uint4*>(h + row * F + f) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(dab + row * 2 * F + f) = make_uint4(pda[0], pda[1], pda[2], pda[3]);
+        *reinterpret_cast<uint4*>(dab + row * 2 * F + F + f) = make_uint4(pdb[0], pdb[1], pdb[2], pdb[3]);
+    }
+}
+
 // Grouped bf16 GEMM out[g] (M x N, fp32 or bf16) = A[g] (M x K) B[g]^T, K-major operands.
 int gemm(const void* a, int64_t lda, int64_t a_rows_total, int64_t a_rows_per_group, const void* b, int64_t ldb,
          int64_t b_rows_total, int64_t b_rows_per_group, int G, int64_t M, int64_t N, int64_t K, const int32_t* rows,
@@ -412,7 +454,7 @@ int gemm(const void* a, int64_t lda, int64_t a_rows_total, int64_t a_rows_per_gr
 }
 
 struct SwigluBwdWs {
-    size_t dybuf, ab, h, dab, wdT, wguT, dybufT, hT, dabT, xbufT, dxbuf, total;
+    size_t dybuf, ab, dh, h, dab, wdT, wguT, dybufT, hT, dabT, xbufT, dxbuf, total;
     int64_t Cp;
 };
 
@@ -427,6 +469,7 @@ SwigluBwdWs swiglu_bwd_layout(int32_t E, int64_t C, int64_t H, int64_t F) {
     };
     w.dybuf = take((size_t)E * C * H * 2);
     w.ab = take((size_t)E * C * 2 * F * 4);
+    w.dh = take((size_t)E * C * F * 4);
     w.h = take((size_t)E * C * F * 2);
     w.dab = take((size_t)E * C * 2 * F * 2);
     w.wdT = take((size_t)E * F * H * 2);
@@ -490,6 +533,7 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     bf16* dybuf = reinterpret_cast<bf16*>(ws + l.dybuf);
     float* ab = reinterpret_cast<float*>(ws + l.ab);
+    float* dh = reinterpret_cast<float*>(ws + l.dh);
     bf16* h = reinterpret_cast<bf16*>(ws + l.h);
     bf16* dab = reinterpret_cast<bf16*>(ws + l.dab);
     bf16* wdT = reinterpret_cast<bf16*>(ws + l.wdT);
@@ -530,34 +574,19 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
         rc = tc_gemm_run(p, stream);
         if (rc != MOE_OK) return rc;
     }
-    // 4. dh = dybuf Wd (Wd (E, H, F) transposed to (E, F, H)); the epilogue turns dh and [a | b] into h, [da | db]
+    // 4. dh = dybuf Wd, with Wd (E, H, F) transposed to (E, F, H)
     rc = transpose_valid(static_cast<const bf16*>(w_down), F, H * F, E, H, F, nullptr, H, wdT, H, F * H, stream);
     if (rc != MOE_OK) return rc;
+    rc = gemm(dybuf, H, (int64_t)E * C, C, wdT, H, (int64_t)E * F, F, E, C, F, H, used, dh, F, C, TC_EPI_F32,
+              dev_status, stream);
+    if (rc != MOE_OK) return rc;
+    // 5. h, da, db
     {
-        TcGemmProblem p{};
-        p.a = dybuf;
-        p.lda = H;
-        p.a_rows_total = (int64_t)E * C;
-        p.a_rows_per_group = C;
-        p.b = wdT;
-        p.ldb = H;
-        p.b_rows_total = (int64_t)E * F;
-        p.b_rows_per_group = F;
-        p.G = E;
-        p.M = C;
-        p.N = F;
-        p.K = H;
-        p.rows = used;
-        p.out = h;
-        p.ldo = F;
-        p.out_rows_per_group = C;
-        p.aux = ab;
-        p.aux_ld = F2;
-        p.out2 = dab;
-        p.ldo2 = F2;
-        p.epilogue = TC_EPI_SWIGLU_BWD;
-        p.status = dev_status;
-        rc = tc_gemm_run(p, stream);
+        const int64_t nb = (C * (F / 8) + 255) / 256;
+        const dim3 g2((unsigned)(nb < 1024 ? nb : 1024), (unsigned)E);
+        MOE_REQUIRE(E <= 65535, MOE_ERR_UNSUPPORTED);
+        swiglu_bwd_elem_kernel<<<g2, 256, 0, stream>>>(ab, dh, used, C, F, h, dab);
+        rc = launch_status();
         if (rc != MOE_OK) return rc;
     }
     // 6. weight gradients over the token index: transposed operands, zeros past used[e]

@@ -52,10 +52,6 @@ struct KParams {
     int64_t out_rows_per_group;
     const void* bias;
     int64_t bias_group_stride;
-    const float* aux;
-    int64_t aux_ld;
-    void* out2;
-    int64_t ldo2;
     int vec_ok;
     int32_t* status;
 };
@@ -92,6 +88,36 @@ __device__ __forceinline__ int group_k_blocks(const KParams& p, int g) {
     return kb < p.k_blocks ? kb : p.k_blocks;
 }
 
+// Warp-cooperative store of one 32 x 32 output chunk.  Lane i holds row i's
+// 32 values as W 32-bit words (W = 16: bf16 pairs, W = 32: fp32).  The rows
+// are staged in shared memory (16-byte quads XOR-swizzled by row, so neither
+// phase has bank conflicts) and written back row-contiguous, W / 4 lanes per
+// row, so every store instruction covers whole 32-byte sectors instead of 32
+// rows' 16-byte pieces.  Row r goes to row0 + r * pitch bytes, if r < nrows.
+template <int W>
+__device__ __forceinline__ int stage_swz(int r) {
+    return W == 16 ? ((r >> 1) & 3) : (r & 7);
+}
+
+template <int W>
+__device__ __forceinline__ void warp_store_chunk(uint32_t* stg, const uint32_t (&w)[W], uint8_t* row0, int64_t pitch,
+                                                 int nrows, int lane) {
+    constexpr int Q = W / 4;  // 16-byte quads per row
+#pragma unroll
+    for (int m = 0; m < Q; ++m)
+        *reinterpret_cast<uint4*>(stg + lane * W + 4 * (m ^ stage_swz<W>(lane))) =
+            make_uint4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
+    __syncwarp();
+    constexpr int RPI = 32 / Q;  // rows per store instruction
+#pragma unroll
+    for (int it = 0; it < Q; ++it) {
+        const int r = it * RPI + lane / Q, m = lane % Q;
+        const uint4 v = *reinterpret_cast<const uint4*>(stg + r * W + 4 * (m ^ stage_swz<W>(r)));
+        if (r < nrows) *reinterpret_cast<uint4*>(row0 + r * pitch + 16 * m) = v;
+    }
+    __syncwarp();
+}
+
 // Store 32 bf16 values (already packed in pairs) for columns n0..n0+31 of one row.
 __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* row, int64_t n0, int64_t N, const uint32_t (&pk)[16],
                                               bool vec) {
@@ -117,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmB2, const KParams p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_prefix[kMaxGroups + 1];
+    __shared__ __align__(16) uint32_t s_stage[4][32 * 32];  // epilogue staging, one 32 x 32 chunk per warp
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
 
@@ -267,6 +294,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_ok = m < rows_g;
             const int64_t out_row = (int64_t)g * p.out_rows_per_group + m;
             const uint32_t t_row = tmem_base + acc * kBN + ((uint32_t)(q * 32) << 16);
+            // this warp's 32 rows for the staged stores
+            const int64_t wrow0 = (int64_t)mt * kBM + q * 32;
+            const int wrows = (int)(rows_g - wrow0 < 0 ? 0 : (rows_g - wrow0 > 32 ? 32 : rows_g - wrow0));
+            const int64_t out_wrow0 = (int64_t)g * p.out_rows_per_group + wrow0;
+            uint32_t* stg = s_stage[q];
 
             if (EPI == TC_EPI_SWIGLU) {
                 __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * p.ldo;
@@ -285,7 +317,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pk[i] = pack_bf16x2(h0, h1);
                     }
                     const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
-                    if (row_ok) store_bf16_32(orow, n0, p.N, pk, p.vec_ok);
+                    if (p.vec_ok && n0 + 32 <= p.N)
+                        warp_store_chunk<16>(stg, pk,
+                                             reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                                                        out_wrow0 * p.ldo + n0),
+                                             p.ldo * 2, wrows, lane);
+                    else if (row_ok)
+                        store_bf16_32(orow, n0, p.N, pk, p.vec_ok);
                 }
             } else if (EPI == TC_EPI_F32_DUAL) {
                 // gate half of the accumulator -> columns [0, N), up half -> [N, 2N)
@@ -312,57 +350,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-            } else if (EPI == TC_EPI_SWIGLU_BWD) {
-                // dh in the accumulator; a, b from aux:
-                //   h = silu(a) b, da = dh b s (1 + a (1 - s)), db = dh a s,  s = sigmoid(a)
-                __nv_bfloat16* hrow = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * p.ldo;
-                __nv_bfloat16* drow = reinterpret_cast<__nv_bfloat16*>(p.out2) + out_row * p.ldo2;
-                const float* arow = p.aux + out_row * p.aux_ld;
-                for (int c = 0; c < p.n_mma / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(t_row + c * 32, r);
-                    tmem_ld_wait(r);
-                    const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
-                    if (!row_ok || n0 >= p.N) continue;
-                    float av[32], bv[32];
-                    if (p.vec_ok && n0 + 32 <= p.N) {
-                        const float4* a4 = reinterpret_cast<const float4*>(arow + n0);
-                        const float4* b4 = reinterpret_cast<const float4*>(arow + p.N + n0);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 x = a4[i], y = b4[i];
-                            av[4 * i] = x.x; av[4 * i + 1] = x.y; av[4 * i + 2] = x.z; av[4 * i + 3] = x.w;
-                            bv[4 * i] = y.x; bv[4 * i + 1] = y.y; bv[4 * i + 2] = y.z; bv[4 * i + 3] = y.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const bool in = n0 + i < p.N;
-                            av[i] = in ? arow[n0 + i] : 0.f;
-                            bv[i] = in ? arow[p.N + n0 + i] : 0.f;
-                        }
-                    }
-                    uint32_t ph[16], pa[16], pb[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float hv[2], dav[2], dbv[2];
-#pragma unroll
-                        for (int m = 0; m < 2; ++m) {
-                            const float a = av[2 * i + m], b = bv[2 * i + m];
-                            const float g = __uint_as_float(r[2 * i + m]);
-                            const float s = 1.0f / (1.0f + expf(-a));
-                            hv[m] = a * s * b;
-                            dav[m] = g * b * s * (1.0f + a * (1.0f - s));
-                            dbv[m] = g * a * s;
-                        }
-                        ph[i] = pack_bf16x2(hv[0], hv[1]);
-                        pa[i] = pack_bf16x2(dav[0], dav[1]);
-                        pb[i] = pack_bf16x2(dbv[0], dbv[1]);
-                    }
-                    store_bf16_32(hrow, n0, p.N, ph, p.vec_ok);
-                    store_bf16_32(drow, n0, p.N, pa, p.vec_ok);
-                    store_bf16_32(drow + p.N, n0, p.N, pb, p.vec_ok);
-                }
             } else if (EPI == TC_EPI_F32) {
                 float* orow = reinterpret_cast<float*>(p.out) + out_row * p.ldo;
                 const float* bias = reinterpret_cast<const float*>(p.bias);
@@ -371,23 +358,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(t_row + c * 32, r);
                     tmem_ld_wait(r);
                     const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
-                    if (row_ok) {
-                        if (p.vec_ok && n0 + 32 <= p.N) {
-                            float4* dst = reinterpret_cast<float4*>(orow + n0);
+                    if (p.vec_ok && n0 + 32 <= p.N) {
+                        uint32_t w[32];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                float4 v;
-                                v.x = __uint_as_float(r[4 * i + 0]) + (bias ? bias[n0 + 4 * i + 0] : 0.f);
-                                v.y = __uint_as_float(r[4 * i + 1]) + (bias ? bias[n0 + 4 * i + 1] : 0.f);
-                                v.z = __uint_as_float(r[4 * i + 2]) + (bias ? bias[n0 + 4 * i + 2] : 0.f);
-                                v.w = __uint_as_float(r[4 * i + 3]) + (bias ? bias[n0 + 4 * i + 3] : 0.f);
-                                dst[i] = v;
-                            }
-                        } else {
+                        for (int i = 0; i < 32; ++i)
+                            w[i] = __float_as_uint(__uint_as_float(r[i]) + (bias ? bias[n0 + i] : 0.f));
+                        warp_store_chunk<32>(stg, w,
+                                             reinterpret_cast<uint8_t*>(reinterpret_cast<float*>(p.out) +
+                                                                        out_wrow0 * p.ldo + n0),
+                                             p.ldo * 4, wrows, lane);
+                    } else if (row_ok) {
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (n0 + i < p.N) orow[n0 + i] = __uint_as_float(r[i]) + (bias ? bias[n0 + i] : 0.f);
-                        }
+                        for (int i = 0; i < 32; ++i)
+                            if (n0 + i < p.N) orow[n0 + i] = __uint_as_float(r[i]) + (bias ? bias[n0 + i] : 0.f);
                     }
                 }
             } else {
@@ -415,7 +398,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         pk[i] = pack_bf16x2(v0, v1);
                     }
-                    if (row_ok) store_bf16_32(orow, n0, p.N, pk, p.vec_ok);
+                    if (p.vec_ok && n0 + 32 <= p.N)
+                        warp_store_chunk<16>(stg, pk,
+                                             reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                                                        out_wrow0 * p.ldo + n0),
+                                             p.ldo * 2, wrows, lane);
+                    else if (row_ok)
+                        store_bf16_32(orow, n0, p.N, pk, p.vec_ok);
                 }
             }
             tc_fence_before();
@@ -510,8 +499,6 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
                 MOE_ERR_UNSUPPORTED);
     MOE_REQUIRE(p.lda >= p.K && p.ldb >= p.K, MOE_ERR_INVALID_ARG);
     const bool dual = p.epilogue == TC_EPI_SWIGLU || p.epilogue == TC_EPI_F32_DUAL;
-    if (p.epilogue == TC_EPI_SWIGLU_BWD)
-        MOE_REQUIRE(p.aux && p.out2 && p.aux_ld >= 2 * p.N && p.ldo2 >= 2 * p.N, MOE_ERR_INVALID_ARG);
     if (dual) MOE_REQUIRE(p.b2 && aligned16(p.b2), MOE_ERR_INVALID_ARG);
     // TMA coordinates are 32-bit.
     MOE_REQUIRE(p.a_rows_total < (int64_t(1) << 31) && p.b_rows_total < (int64_t(1) << 31), MOE_ERR_UNSUPPORTED);
@@ -542,17 +529,10 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     kp.out_rows_per_group = p.out_rows_per_group;
     kp.bias = p.bias;
     kp.bias_group_stride = p.bias_group_stride;
-    kp.aux = p.aux;
-    kp.aux_ld = p.aux_ld;
-    kp.out2 = p.out2;
-    kp.ldo2 = p.ldo2;
     const bool f32_out = p.epilogue == TC_EPI_F32 || p.epilogue == TC_EPI_F32_DUAL;
     const size_t esz = f32_out ? 4 : 2;
     kp.vec_ok = aligned16(p.out) && (p.ldo * (int64_t)esz) % 16 == 0;
     if (p.epilogue == TC_EPI_F32_DUAL) kp.vec_ok = kp.vec_ok && (p.N * 4) % 16 == 0;
-    if (p.epilogue == TC_EPI_SWIGLU_BWD)
-        kp.vec_ok = kp.vec_ok && aligned16(p.out2) && (p.ldo2 * 2) % 16 == 0 && (p.N * 2) % 16 == 0 &&
-                    aligned16(p.aux) && (p.aux_ld * 4) % 16 == 0 && (p.N * 4) % 16 == 0;
     kp.status = p.status;
 
     CUtensorMap ma, mb, mb2;
@@ -574,7 +554,6 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
         case TC_EPI_GELU_BIAS: return launch<TC_EPI_GELU_BIAS>(ma, mb, mb2, kp, grid, stream);
         case TC_EPI_SWIGLU: return launch<TC_EPI_SWIGLU>(ma, mb, mb2, kp, grid, stream);
         case TC_EPI_F32_DUAL: return launch<TC_EPI_F32_DUAL>(ma, mb, mb2, kp, grid, stream);
-        case TC_EPI_SWIGLU_BWD: return launch<TC_EPI_SWIGLU_BWD>(ma, mb, mb2, kp, grid, stream);
         default: return MOE_ERR_INVALID_ARG;
     }
 }

@@ -21,9 +21,7 @@ enum TcEpilogue : int {
     TC_EPI_BF16_BIAS = 2,  // bf16 out, + bf16 bias                       -- GELU MLP fc2
     TC_EPI_GELU_BIAS = 3,  // bf16 gelu(acc + bias)                       -- GELU MLP fc1
     TC_EPI_SWIGLU = 4,     // dual B: bf16 silu(acc_gate) * acc_up        -- SwiGLU gate/up
-    TC_EPI_F32_DUAL = 5,   // dual B: fp32 acc_gate -> out[., n], acc_up -> out[., N + n]   -- [a | b] recompute
-    TC_EPI_SWIGLU_BWD = 6  // acc = dh; with (a, b) from aux (fp32, row stride aux_ld, b at + N):
-                           //   out (bf16) = h = silu(a) b; out2 (bf16, row stride ldo2) = [da | db]
+    TC_EPI_F32_DUAL = 5    // dual B: fp32 acc_gate -> out[., n], acc_up -> out[., N + n]   -- [a | b] recompute
 };
 
 struct TcGemmProblem {
@@ -47,10 +45,6 @@ struct TcGemmProblem {
     int64_t out_rows_per_group;
     const void* bias;         // fp32 (TC_EPI_F32) or bf16, per output column
     int64_t bias_group_stride;
-    const float* aux;         // TC_EPI_SWIGLU_BWD: [a | b] rows (same row index as out)
-    int64_t aux_ld;
-    void* out2;               // TC_EPI_SWIGLU_BWD: [da | db] rows (same row index as out)
-    int64_t ldo2;
     int epilogue;
     int32_t* status;
 };
