@@ -472,8 +472,9 @@ SwigluBwdWs swiglu_bwd_layout(int32_t E, int64_t C, int64_t H, int64_t F) {
     w.dh = take((size_t)E * C * F * 4);
     w.h = take((size_t)E * C * F * 2);
     w.dab = take((size_t)E * C * 2 * F * 2);
-    w.wdT = take((size_t)E * F * H * 2);
-    w.wguT = take((size_t)E * H * 2 * F * 2);
+    const bool mn = H % 64 == 0 && F % 64 == 0;  // weights read in place (MN-major): no transposed copies
+    w.wdT = take(mn ? 0 : (size_t)E * F * H * 2);
+    w.wguT = take(mn ? 0 : (size_t)E * H * 2 * F * 2);
     w.dybufT = take((size_t)E * H * w.Cp * 2);
     w.hT = take((size_t)E * F * w.Cp * 2);
     w.dabT = take((size_t)E * 2 * F * w.Cp * 2);
@@ -574,11 +575,38 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
         rc = tc_gemm_run(p, stream);
         if (rc != MOE_OK) return rc;
     }
-    // 4. dh = dybuf Wd, with Wd (E, H, F) transposed to (E, F, H)
-    rc = transpose_valid(static_cast<const bf16*>(w_down), F, H * F, E, H, F, nullptr, H, wdT, H, F * H, stream);
-    if (rc != MOE_OK) return rc;
-    rc = gemm(dybuf, H, (int64_t)E * C, C, wdT, H, (int64_t)E * F, F, E, C, F, H, used, dh, F, C, TC_EPI_F32,
-              dev_status, stream);
+    // With H and F multiples of 64 the weights are read in their own layout as MN-major
+    // operands; otherwise transposed copies feed the K-major form.
+    const bool mn = H % 64 == 0 && F % 64 == 0;
+    // 4. dh = dybuf Wd: B(k = h, n = f) = Wd[e][h][f]
+    if (mn) {
+        TcGemmProblem p{};
+        p.a = dybuf;
+        p.lda = H;
+        p.a_rows_total = (int64_t)E * C;
+        p.a_rows_per_group = C;
+        p.b = w_down;
+        p.ldb = F;
+        p.b_rows_total = (int64_t)E * H;
+        p.b_rows_per_group = H;
+        p.b_mn_major = true;
+        p.G = E;
+        p.M = C;
+        p.N = F;
+        p.K = H;
+        p.rows = used;
+        p.out = dh;
+        p.ldo = F;
+        p.out_rows_per_group = C;
+        p.epilogue = TC_EPI_F32;
+        p.status = dev_status;
+        rc = tc_gemm_run(p, stream);
+    } else {
+        rc = transpose_valid(static_cast<const bf16*>(w_down), F, H * F, E, H, F, nullptr, H, wdT, H, F * H, stream);
+        if (rc != MOE_OK) return rc;
+        rc = gemm(dybuf, H, (int64_t)E * C, C, wdT, H, (int64_t)E * F, F, E, C, F, H, used, dh, F, C, TC_EPI_F32,
+                  dev_status, stream);
+    }
     if (rc != MOE_OK) return rc;
     // 5. h, da, db
     {
@@ -608,13 +636,41 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     rc = gemm(dabT + F * Cp, Cp, (int64_t)E * F2 - F, F2, xbufT, Cp, (int64_t)E * H, H, E, F, H, Cp, nullptr, dw_up,
               H, F, TC_EPI_F32, dev_status, stream, used);
     if (rc != MOE_OK) return rc;
-    // 7. dxbuf = [da | db] [Wg; Wu], with the stacked weights transposed to (E, H, 2F)
-    rc = transpose_valid(static_cast<const bf16*>(w_gate), H, F * H, E, F, H, nullptr, F, wguT, F2, H * F2, stream);
-    if (rc != MOE_OK) return rc;
-    rc = transpose_valid(static_cast<const bf16*>(w_up), H, F * H, E, F, H, nullptr, F, wguT + F, F2, H * F2, stream);
-    if (rc != MOE_OK) return rc;
-    rc = gemm(dab, F2, (int64_t)E * C, C, wguT, F2, (int64_t)E * H, H, E, C, H, F2, used, dxbuf, H, C, TC_EPI_BF16,
-              dev_status, stream);
+    // 7. dxbuf = [da | db] [Wg; Wu]: B(k, n = h) = Wg[e][k][h] for k < F, Wu[e][k - F][h] after
+    if (mn) {
+        TcGemmProblem p{};
+        p.a = dab;
+        p.lda = F2;
+        p.a_rows_total = (int64_t)E * C;
+        p.a_rows_per_group = C;
+        p.b = w_gate;
+        p.b2 = w_up;
+        p.k_split = F;
+        p.ldb = H;
+        p.b_rows_total = (int64_t)E * F;
+        p.b_rows_per_group = F;
+        p.b_mn_major = true;
+        p.G = E;
+        p.M = C;
+        p.N = H;
+        p.K = F2;
+        p.rows = used;
+        p.out = dxbuf;
+        p.ldo = H;
+        p.out_rows_per_group = C;
+        p.epilogue = TC_EPI_BF16;
+        p.status = dev_status;
+        rc = tc_gemm_run(p, stream);
+    } else {
+        rc = transpose_valid(static_cast<const bf16*>(w_gate), H, F * H, E, F, H, nullptr, F, wguT, F2, H * F2,
+                             stream);
+        if (rc != MOE_OK) return rc;
+        rc = transpose_valid(static_cast<const bf16*>(w_up), H, F * H, E, F, H, nullptr, F, wguT + F, F2, H * F2,
+                             stream);
+        if (rc != MOE_OK) return rc;
+        rc = gemm(dab, F2, (int64_t)E * C, C, wguT, F2, (int64_t)E * H, H, E, C, H, F2, used, dxbuf, H, C,
+                  TC_EPI_BF16, dev_status, stream);
+    }
     if (rc != MOE_OK) return rc;
     // 8. dx
     return combine_rows(dxbuf, selected, slot, nullptr, MOE_F32, T, k, E, C, H, use_residual ? dy : nullptr, H, dx,

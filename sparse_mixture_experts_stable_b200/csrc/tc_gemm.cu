@@ -44,6 +44,7 @@ struct KParams {
     int tile_n_out;   // output columns produced per tile
     int b_box_rows;   // rows per B TMA box (n_mma, or n_mma/2 for the dual form)
     int k_blocks;
+    int k_split_blocks;  // MN-major B: K blocks from the first map before switching to the second (0: none)
     uint32_t tx_bytes;
     const int32_t* rows;
     const int32_t* k_rows;
@@ -137,7 +138,7 @@ __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* row, int64_t n0, in
     }
 }
 
-template <int EPI>
+template <int EPI, bool BMN>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const KParams p) {
@@ -216,7 +217,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* a_dst = smA + stage * kABytes;
                     uint8_t* b_dst = smB + stage * kBBytes;
                     tma_load_2d(a_dst, &tmA, kb * kBK, a_y, &full[stage]);
-                    tma_load_2d(b_dst, &tmB, kb * kBK, b_y, &full[stage]);
+                    if (BMN) {
+                        // K rows kb*64 .. +63 of the (K, N) weight, in 64-column boxes of 8 KB
+                        const bool second = p.k_split_blocks > 0 && kb >= p.k_split_blocks;
+                        const int32_t k_y = (int32_t)(g * p.b_rows_per_group +
+                                                      (int64_t)(kb - (second ? p.k_split_blocks : 0)) * kBK);
+                        for (int i = 0; i < p.n_mma / 64; ++i)
+                            tma_load_2d(b_dst + i * 8192, second ? &tmB2 : &tmB, nt * p.n_mma + 64 * i, k_y,
+                                        &full[stage]);
+                    } else {
+                        tma_load_2d(b_dst, &tmB, kb * kBK, b_y, &full[stage]);
+                    }
                     if (is_dual(EPI))
                         tma_load_2d(b_dst + p.b_box_rows * (kBK * 2), &tmB2, kb * kBK, b_y, &full[stage]);
                     if (++stage == kStages) {
@@ -230,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------- MMA issuer -------------------------------
         if (lane == 0) {
-            const uint32_t idesc = make_idesc(kBM, p.n_mma);
+            const uint32_t idesc = make_idesc(kBM, p.n_mma) | (BMN ? (1u << 16) : 0u);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t it = 0;
@@ -255,10 +266,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint64_t ad = sw128_desc(smem_u32(smA + stage * kABytes));
-                    const uint64_t bd = sw128_desc(smem_u32(smB + stage * kBBytes));
+                    const uint64_t bd = BMN ? sw128_mn_desc(smem_u32(smB + stage * kBBytes), 8192)
+                                            : sw128_desc(smem_u32(smB + stage * kBBytes));
+                    // a K step of 16: 32 bytes along a K-major row, or two 1024-byte groups of 8 K rows
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        tc_mma(d_tmem, ad + 2 * kk, bd + (BMN ? 128 : 2) * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
                         stage = 0;
@@ -336,18 +349,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool up = c * 32 >= half;
                     const int64_t n0 = (int64_t)nt * p.tile_n_out + (up ? c * 32 - half : c * 32);
                     float* dst = orow + (up ? p.N : 0);
-                    if (row_ok) {
-                        if (p.vec_ok && n0 + 32 <= p.N) {
-                            float4* d4 = reinterpret_cast<float4*>(dst + n0);
+                    if (p.vec_ok && n0 + 32 <= p.N) {
+                        warp_store_chunk<32>(stg, r,
+                                             reinterpret_cast<uint8_t*>(reinterpret_cast<float*>(p.out) +
+                                                                        out_wrow0 * p.ldo + (up ? p.N : 0) + n0),
+                                             p.ldo * 4, wrows, lane);
+                    } else if (row_ok) {
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                    __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (n0 + i < p.N) dst[n0 + i] = __uint_as_float(r[i]);
-                        }
+                        for (int i = 0; i < 32; ++i)
+                            if (n0 + i < p.N) dst[n0 + i] = __uint_as_float(r[i]);
                     }
                 }
             } else if (EPI == TC_EPI_F32) {
@@ -473,18 +483,18 @@ bool make_map_f32(CUtensorMap* m, const void* base, int64_t inner, int64_t rows,
 
 namespace {
 
-template <int EPI>
+template <int EPI, bool BMN = false>
 int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const KParams& kp, int grid,
            cudaStream_t stream) {
     static bool attr_set[64] = {false};
     int dev = 0;
     MOE_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 64 && !attr_set[dev]) {
-        MOE_CUDA_TRY(cudaFuncSetAttribute(tc_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        MOE_CUDA_TRY(cudaFuncSetAttribute(tc_gemm_kernel<EPI, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)kSmemBytes));
         attr_set[dev] = true;
     }
-    tc_gemm_kernel<EPI><<<grid, kThreads, kSmemBytes, stream>>>(a, b, b2, kp);
+    tc_gemm_kernel<EPI, BMN><<<grid, kThreads, kSmemBytes, stream>>>(a, b, b2, kp);
     return launch_status();
 }
 
@@ -497,7 +507,13 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     // TMA: 16-byte aligned bases, row strides a multiple of 16 bytes.
     MOE_REQUIRE(aligned16(p.a) && aligned16(p.b) && (p.lda * 2) % 16 == 0 && (p.ldb * 2) % 16 == 0,
                 MOE_ERR_UNSUPPORTED);
-    MOE_REQUIRE(p.lda >= p.K && p.ldb >= p.K, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(p.lda >= p.K && (p.b_mn_major ? p.ldb >= p.N : p.ldb >= p.K), MOE_ERR_INVALID_ARG);
+    if (p.b_mn_major) {
+        MOE_REQUIRE(p.epilogue == TC_EPI_F32 || p.epilogue == TC_EPI_BF16, MOE_ERR_UNSUPPORTED);
+        MOE_REQUIRE(p.k_split % kBK == 0 && p.k_split >= 0 && p.k_split < p.K, MOE_ERR_UNSUPPORTED);
+        MOE_REQUIRE(p.k_split == 0 || (p.b2 && aligned16(p.b2)), MOE_ERR_INVALID_ARG);
+        MOE_REQUIRE(p.b_rows_per_group >= (p.k_split > 0 ? p.k_split : p.K), MOE_ERR_INVALID_ARG);
+    }
     const bool dual = p.epilogue == TC_EPI_SWIGLU || p.epilogue == TC_EPI_F32_DUAL;
     if (dual) MOE_REQUIRE(p.b2 && aligned16(p.b2), MOE_ERR_INVALID_ARG);
     // TMA coordinates are 32-bit.
@@ -519,8 +535,10 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
         kp.tile_n_out = kp.n_mma;
         kp.b_box_rows = kp.n_mma;
     }
+    if (p.b_mn_major) MOE_REQUIRE(kp.n_mma % 64 == 0, MOE_ERR_UNSUPPORTED);
     kp.n_tiles = (int)((p.N + kp.tile_n_out - 1) / kp.tile_n_out);
     kp.k_blocks = (int)((p.K + kBK - 1) / kBK);
+    kp.k_split_blocks = p.b_mn_major ? (int)(p.k_split / kBK) : 0;
     kp.tx_bytes = (uint32_t)(kABytes + kp.n_mma * kBK * 2);
     kp.rows = p.rows;
     kp.k_rows = p.k_rows;
@@ -537,9 +555,16 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
 
     CUtensorMap ma, mb, mb2;
     MOE_REQUIRE(make_map(&ma, p.a, p.K, p.a_rows_total, p.lda, kBM), MOE_ERR_CUDA);
-    MOE_REQUIRE(make_map(&mb, p.b, p.K, p.b_rows_total, p.ldb, kp.b_box_rows), MOE_ERR_CUDA);
-    if (dual) MOE_REQUIRE(make_map(&mb2, p.b2, p.K, p.b_rows_total, p.ldb, kp.b_box_rows), MOE_ERR_CUDA);
-    else mb2 = mb;
+    if (p.b_mn_major) {
+        // (K rows, N columns) with 64 x 64 boxes: rows past b_rows_total and columns past N read as zero
+        MOE_REQUIRE(make_map(&mb, p.b, p.N, p.b_rows_total, p.ldb, kBK), MOE_ERR_CUDA);
+        if (p.k_split > 0) MOE_REQUIRE(make_map(&mb2, p.b2, p.N, p.b_rows_total, p.ldb, kBK), MOE_ERR_CUDA);
+        else mb2 = mb;
+    } else {
+        MOE_REQUIRE(make_map(&mb, p.b, p.K, p.b_rows_total, p.ldb, kp.b_box_rows), MOE_ERR_CUDA);
+        if (dual) MOE_REQUIRE(make_map(&mb2, p.b2, p.K, p.b_rows_total, p.ldb, kp.b_box_rows), MOE_ERR_CUDA);
+        else mb2 = mb;
+    }
 
     const int64_t max_tiles = (int64_t)p.G * ((p.M + kBM - 1) / kBM) * kp.n_tiles;
     MOE_REQUIRE(max_tiles < (int64_t(1) << 30), MOE_ERR_UNSUPPORTED);
@@ -547,6 +572,9 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     if (max_tiles < grid) grid = (int)max_tiles;
     if (grid < 1) grid = 1;
 
+    if (p.b_mn_major)
+        return p.epilogue == TC_EPI_F32 ? launch<TC_EPI_F32, true>(ma, mb, mb2, kp, grid, stream)
+                                        : launch<TC_EPI_BF16, true>(ma, mb, mb2, kp, grid, stream);
     switch (p.epilogue) {
         case TC_EPI_F32: return launch<TC_EPI_F32>(ma, mb, mb2, kp, grid, stream);
         case TC_EPI_BF16: return launch<TC_EPI_BF16>(ma, mb, mb2, kp, grid, stream);

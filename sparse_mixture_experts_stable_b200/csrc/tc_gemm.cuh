@@ -3,7 +3,8 @@
 // out[g, m, n] = epilogue( sum_k A[g, m, k] * B[g, n, k] )     for m < rows[g]
 //
 // Both operands are K-major bf16 (A: activations (rows, K); B: weights in the
-// (out, in) layout), fp32 accumulation in tensor memory.  One persistent CTA per
+// (out, in) layout), or B is MN-major (b_mn_major: B stored (K, N), N
+// contiguous, e.g. a weight read transposed), fp32 accumulation in tensor memory.  One persistent CTA per
 // SM walks a static list of (group, m-tile, n-tile) tiles whose length depends on
 // the per-group row counts read on the device.
 #pragma once
@@ -30,10 +31,14 @@ struct TcGemmProblem {
     int64_t a_rows_total;
     int64_t a_rows_per_group; // row offset of group g in A
     const void* b;            // bf16 (b_rows_total, K), row stride ldb
-    const void* b2;           // second B for TC_EPI_SWIGLU (same shape), else NULL
+    const void* b2;           // second B for TC_EPI_SWIGLU (same shape), else NULL; with b_mn_major
+                              // and k_split > 0: the rows of K positions >= k_split (row k - k_split)
     int64_t ldb;
     int64_t b_rows_total;
-    int64_t b_rows_per_group; // row offset of group g in B
+    int64_t b_rows_per_group; // row offset of group g in B (b_mn_major: K rows per group)
+    bool b_mn_major;          // B(k, n) = b[(g * b_rows_per_group + k) * ldb + n]; epilogues F32 / BF16 only,
+                              // UMMA N a multiple of 64, k_split a multiple of 64
+    int64_t k_split;
     int G;                    // groups
     int64_t M;                // max rows per group
     int64_t N;                // output columns per group

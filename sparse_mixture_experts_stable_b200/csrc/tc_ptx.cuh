@@ -100,6 +100,20 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory descriptor of an MN-major operand in 128-byte-swizzle atoms:
+// each K row of an atom holds 64 consecutive MN elements (128 bytes), eight K
+// rows form a 1024-byte swizzle group (the stride between K groups), and the
+// next 64 MN elements start lbo_bytes further on.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t lbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);          // start address (16-byte units)
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset: next 64 MN elements
+    d |= (uint64_t)(1024 >> 4) << 32;                   // stride byte offset: next 8 K rows
+    d |= (uint64_t)1 << 46;                             // descriptor version for tcgen05
+    d |= (uint64_t)2 << 61;                             // layout: 128-byte swizzle
+    return d;
+}
+
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major.
 __device__ __forceinline__ uint32_t make_idesc(int m, int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);

@@ -28,6 +28,8 @@ def _close(got, want, what):
     (300, 128, 96, 6, 2, 0.8, False, 0.0),   # capacity binds: drops
     (517, 64, 48, 4, 3, 1.5, True, 0.1),     # ragged token count, residual, aux term
     (64, 72, 40, 3, 1, 2.0, False, 0.0),     # top-1; H, F not multiples of 64
+    (400, 128, 128, 6, 2, 1.0, True, 0.0),   # H, F multiples of 64: weights read MN-major, no transposed copies
+    (333, 256, 64, 5, 3, 0.7, False, 0.05),  # the same with drops and the aux term
 ])
 def test_backward_swiglu_matches_oracle(T, H, F, E, k, cf, residual, aux):
     g = torch.Generator().manual_seed(T + H)
