@@ -448,7 +448,7 @@ def _time_steps(step, steps, warmup, flush, stream, inner=None):
     return step_ms, inner_ms
 
 
-def run_other_workloads(steps, warmup, flush, stream, dev, only=None):
+def run_other_workloads(steps, warmup, flush, stream, dev, only=None, layer_sizes=None):
     import sparse_mixture_experts_stable_b200 as moe
     from sparse_mixture_experts_stable_b200 import binding as B
     from sparse_mixture_experts_stable_b200 import inputs as I
@@ -638,7 +638,7 @@ def run_other_workloads(steps, warmup, flush, stream, dev, only=None):
         # expert parallelism, 4 ranks emulated on this GPU: the full-layer batch split over the ranks, every rank's
         # rows written into and read from the other ranks' buffers through the peer-pointer tables
         from sparse_mixture_experts_stable_b200 import ep
-        c = I.full_layer_bf16(seed=0)
+        c = I.full_layer_bf16(seed=0, **(layer_sizes or {}))
         T, H, E, F, k = c["T"], c["H"], c["E"], c["F"], c["k"]
         R, epr = 4, c["E"] // 4
         C = moe.moe_capacity(T, k, E, c["capacity_factor"])
@@ -696,7 +696,7 @@ def run_other_workloads(steps, warmup, flush, stream, dev, only=None):
     if want("full_layer_bf16_train"):
         # training step of the full layer: forward, SwiGLU-expert backward and router backward (bf16)
         from sparse_mixture_experts_stable_b200.layer import SwiGLUMoE
-        c = I.full_layer_bf16(seed=0)
+        c = I.full_layer_bf16(seed=0, **(layer_sizes or {}))
         T, H, E, F, k = c["T"], c["H"], c["E"], c["F"], c["k"]
         dv = {n: c[n].to(dev) for n in ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down")}
         dyt = (torch.randn(T, H, generator=torch.Generator().manual_seed(1)) * 0.1).to(torch.bfloat16).to(dev)
@@ -759,8 +759,11 @@ def main():
             torch.cuda.set_device(dev)
             moe.lib()
             flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+            sizes = None
+            if args.tokens != WORKLOAD["T"] or args.experts != WORKLOAD["experts"]:
+                sizes = dict(T=args.tokens, E=args.experts)  # smaller full-layer shapes for profiling captures
             out = run_other_workloads(args.steps, args.warmup, flush, torch.cuda.current_stream(dev), dev,
-                                      only=args.workload)
+                                      only=args.workload, layer_sizes=sizes)
             if args.workload not in out:
                 raise SystemExit(f"unknown workload {args.workload}; known: {sorted(out)}")
             print(json.dumps(dict(workload=args.workload, **out[args.workload])), flush=True)
