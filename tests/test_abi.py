@@ -115,3 +115,27 @@ def test_backward_gelu_host_checks():
     assert call(B.MOE_F32, k=5) == B.MOE_ERR_INVALID_ARG     # k > E
     assert call(B.MOE_F32, residual=1, Dout=8) == B.MOE_ERR_INVALID_ARG  # residual needs Dout == D
     assert call(B.MOE_F32, ws_bytes=64) == B.MOE_ERR_WORKSPACE
+
+
+def test_expert_parallel_host_checks():
+    L = moe.lib()
+    p, nul = ctypes.c_void_p(16), None
+    tab2 = (ctypes.c_void_p * 2)(16, 32)
+    # E not a multiple of the rank count
+    rc = L.moe_ep_dispatch(p, 8, 2, 6, 4, p, 0, nul, 0, 0, 0, tab2, 4, p, p, p, nul, nul, p, 1 << 20, nul)
+    assert rc == B.MOE_ERR_INVALID_ARG
+    # more ranks than the peer-pointer table holds
+    rc = L.moe_ep_dispatch(p, 8, 2, 128, 4, p, 0, nul, 0, 0, 0, tab2, 128, p, p, p, nul, nul, p, 1 << 20, nul)
+    assert rc == B.MOE_ERR_UNSUPPORTED
+    # a NULL entry in the table when rows are moved
+    bad = (ctypes.c_void_p * 2)(16, 0)
+    rc = L.moe_ep_dispatch(p, 8, 2, 4, 4, p, 0, p, 1, 8, 8, bad, 2, p, p, p, nul, nul, p, 1 << 20, nul)
+    assert rc == B.MOE_ERR_INVALID_ARG
+    # combine: rank out of range for the plan, missing table
+    assert L.moe_ep_plan(p, 2, 2, 4, 4, p, nul, nul, nul, nul) == B.MOE_ERR_INVALID_ARG
+    rc = L.moe_ep_combine(nul, 2, p, p, nul, 0, 8, 2, 4, 4, 8, 0, nul, 0, p, 8, 1, nul, nul)
+    assert rc == B.MOE_ERR_INVALID_ARG
+    # IPC calls reject NULL arguments before touching the driver
+    assert L.moe_ipc_export(nul, nul, nul) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_ipc_import(nul, nul) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_ipc_close(nul) == B.MOE_ERR_INVALID_ARG
