@@ -22,7 +22,11 @@ namespace {
 constexpr int kRouteWarps = 8;
 constexpr int kRouteThreads = kRouteWarps * 32;
 constexpr int kMaxRouteBlocks = 1024;  // bound on the per-block partials (workspace sizing)
-constexpr int kRouteBlocksPerSm = 4;    // blocks launched per SM; each warp then walks several tokens
+// Blocks launched per SM (each warp then walks several tokens): the top-k kernel
+// uses 80 registers, so three 256-thread blocks are resident per SM; a fourth
+// only added a second partial wave (moe_route 197.6-198.6 against 201.0 us on
+// the 65536-token router workload).
+constexpr int kRouteBlocksPerSm = 3;
 constexpr int kMaxK = 64;
 constexpr int kMaxE = 1024;
 
