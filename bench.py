@@ -700,7 +700,8 @@ def run_other_workloads(steps, warmup, flush, stream, dev, only=None, layer_size
         T, H, E, F, k = c["T"], c["H"], c["E"], c["F"], c["k"]
         dv = {n: c[n].to(dev) for n in ("x", "w_router", "router_bias", "w_gate", "w_up", "w_down")}
         dyt = (torch.randn(T, H, generator=torch.Generator().manual_seed(1)) * 0.1).to(torch.bfloat16).to(dev)
-        layer = SwiGLUMoE(T, H, E, F, k, c["capacity_factor"], F_shared=0, aux_coef=c["aux_coef"], device=dev)
+        layer = SwiGLUMoE(T, H, E, F, k, c["capacity_factor"], F_shared=0, aux_coef=c["aux_coef"], device=dev,
+                          save_for_backward=True)
         wsbs = torch.empty(B.moe_backward_swiglu_workspace_size(E, layer.C, H, F), dtype=torch.uint8, device=dev)
         kept_box = {}
         inner = []
@@ -712,7 +713,8 @@ def run_other_workloads(steps, warmup, flush, stream, dev, only=None, layer_size
             e0.record(stream)
             dxe, dwg, dwu, dwd, dl, dg = moe.moe_backward_swiglu(
                 dyt, lg_t, o["selected"], o["gates_f32"], o["slot"], o["used"], o["xbuf"], layer.ybuf, dv["w_gate"],
-                dv["w_up"], dv["w_down"], layer.C, aux_coef=c["aux_coef"], counts=o["counts"], workspace=wsbs)
+                dv["w_up"], dv["w_down"], layer.C, aux_coef=c["aux_coef"], counts=o["counts"], workspace=wsbs,
+                saved_ab=layer.saved_ab)
             e1.record(stream)
             moe.moe_router_backward(dv["x"], dv["w_router"], dl)
             kept_box["used"] = o["used"]
@@ -725,7 +727,7 @@ def run_other_workloads(steps, warmup, flush, stream, dev, only=None, layer_size
         out["full_layer_bf16_train"] = dict(
             value=T * len(sm) / (sum(sm) / 1e3), unit=UNIT, ms_per_step=sum(sm) / len(sm), steps=len(sm),
             config=dict(T=T, H=H, E=E, F=F, k=k, capacity=layer.C, kept=kept, shared_experts=0,
-                        step="forward + moe_backward_swiglu + moe_router_backward"),
+                        step="forward (moe_expert_ffn_save) + moe_backward_swiglu + moe_router_backward"),
             roofline=dict(bound="tensor", kernel="moe_backward_swiglu (tcgen05 GEMMs + transposes)",
                           achieved=flops_bw / bw_s / 1e12, peak=pk["bf16_sustained"], unit="TFLOP/s",
                           frac=flops_bw / bw_s / 1e12 / pk["bf16_sustained"], traffic=None, avg_launch_ms=1e3 * bw_s))

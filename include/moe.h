@@ -351,6 +351,23 @@ MOE_API int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const vo
                                     size_t workspace_bytes, moe_stream_t stream);
 
 /*
+ * moe_expert_ffn_save -- moe_expert_ffn for bf16 SwiGLU experts that also
+ * keeps what the backward needs: saved_ab[e, c] = [a | b] with a = xbuf[e,c]
+ * Wg_e^T and b = xbuf[e,c] Wu_e^T (the gate and up pre-activations, fp32
+ * accumulation rounded to bf16), for c < used[e] (other rows are not
+ * written).  Pass it to moe_backward_swiglu, which then skips recomputing
+ * them.  ([P3] swiglu_expert; the usual store-for-backward trade of memory
+ * for a GEMM.)
+ *   xbuf bf16 (E, C, D); used int32 (E) (required); w_gate, w_up bf16 (E, F, D);
+ *   w_down bf16 (E, Dout, F); ybuf bf16 (E, C, Dout); saved_ab bf16 (E, C, 2F).
+ *   workspace >= moe_expert_ffn_workspace_size(MOE_FFN_SWIGLU, MOE_BF16, E, C, D, F, Dout).
+ */
+MOE_API int moe_expert_ffn_save(const void* xbuf, const int32_t* used, int32_t E, int64_t C, int64_t D, int64_t F,
+                                int64_t Dout, const void* w_gate, const void* w_down, const void* w_up, void* ybuf,
+                                void* saved_ab, int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                                moe_stream_t stream);
+
+/*
  * moe_combine -- gate-weighted combine back to token order.
  *   y[t,:] = base[t,:] + sum_{j : slot[t,j] >= 0} gate[t,j] * ybuf[e_{t,j}, slot[t,j], :]
  * ([P1] section 1 item 4: y = x + sum over kept; [P2] y = shared + sum;
@@ -440,12 +457,14 @@ MOE_API int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, con
  *   dw_gate[e] += da^T x_t       (E, F, H)
  *   dw_up[e]   += db^T x_t       (E, F, H)
  *   dx[t]      = [dy_t] + sum_kept (da Wg_e + db Wu_e)     (T, H), bf16
- * a and b are recomputed from xbuf; h, da, db are rounded to bf16 before the
- * weight-gradient and dx products.
+ * a and b are recomputed from xbuf (fp32), or read from saved_ab when the
+ * forward ran moe_expert_ffn_save (bf16, which saves that GEMM); h, da, db are
+ * rounded to bf16 before the weight-gradient and dx products.
  *
  * Arguments (device): dy bf16 (T, H); logits fp32 (T, E); selected int64,
  *   gates fp32, slot int64 (T, k); used int32 (E); xbuf bf16 (E, C, H) and
- *   ybuf bf16 (E, C, H) from the forward; w_gate, w_up bf16 (E, F, H);
+ *   ybuf bf16 (E, C, H) from the forward; saved_ab bf16 (E, C, 2F) from
+ *   moe_expert_ffn_save, or NULL; w_gate, w_up bf16 (E, F, H);
  *   w_down bf16 (E, H, F); counts int32 (E) when aux_coef != 0.
  *   H and F multiples of 8, k <= 64, dtype MOE_BF16 (else MOE_ERR_UNSUPPORTED).
  *   Outputs: dx bf16 (T, H); dw_gate, dw_up fp32 (E, F, H); dw_down fp32
@@ -455,7 +474,7 @@ MOE_API int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, con
 MOE_API size_t moe_backward_swiglu_workspace_size(int32_t E, int64_t C, int64_t H, int64_t F);
 MOE_API int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float* logits, const int64_t* selected,
                                 const float* gates, const int64_t* slot, const int32_t* used, const void* xbuf,
-                                const void* ybuf, const void* w_gate, const void* w_up, const void* w_down,
+                                const void* ybuf, const void* saved_ab, const void* w_gate, const void* w_up, const void* w_down,
                                 int64_t T, int32_t k, int32_t E, int64_t C, int64_t H, int64_t F, int use_residual,
                                 float aux_coef, int normalize_by_k, const int32_t* counts, void* dx,
                                 float* dw_gate, float* dw_up, float* dw_down, float* dlogits, float* dgate,

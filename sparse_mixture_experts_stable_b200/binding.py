@@ -40,7 +40,7 @@ EXPORTED = [
     "moe_route_ex", "moe_renormalize_kept_gates", "moe_expert_ffn_gathered", "moe_backward_swiglu_workspace_size",
     "moe_backward_swiglu", "moe_router_backward_workspace_size", "moe_router_backward",
     "moe_backward_gelu_workspace_size", "moe_backward_gelu", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine",
-    "moe_ipc_export", "moe_ipc_import", "moe_ipc_close",
+    "moe_ipc_export", "moe_ipc_import", "moe_ipc_close", "moe_expert_ffn_save",
 ]
 IPC_HANDLE_BYTES = 64
 SCORING = {"softmax": 0, "sigmoid": 1}
@@ -100,7 +100,10 @@ def lib():
                                           _vp, _vp, _vp, _vp, _sz, _vp]
         L.moe_backward_swiglu_workspace_size.restype = _sz
         L.moe_backward_swiglu_workspace_size.argtypes = [_i32, _i64, _i64, _i64]
-        L.moe_backward_swiglu.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+        L.moe_expert_ffn_save.argtypes = [_vp, _vp, _i32, _i64, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _sz, _vp]
+        L.moe_backward_swiglu.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _i64,
                                           _i32, _i32, _i64, _i64, _i64, ctypes.c_int, _f32, ctypes.c_int, _vp, _vp,
                                           _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
         L.moe_backward_gelu_workspace_size.restype = _sz
@@ -373,6 +376,28 @@ def moe_expert_ffn_gathered(x: torch.Tensor, token_of_slot: torch.Tensor, used: 
     return ybuf
 
 
+def moe_expert_ffn_save(xbuf: torch.Tensor, used: torch.Tensor, w_gate: torch.Tensor, w_down: torch.Tensor,
+                        w_up: torch.Tensor, saved_ab: Optional[torch.Tensor] = None, ybuf: Optional[torch.Tensor] = None,
+                        dev_status: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                        stream=None):
+    """bf16 SwiGLU experts that also keep the gate/up pre-activations [a | b] (E, C, 2F) for the backward.
+
+    Returns (ybuf, saved_ab).
+    """
+    dev = _dev(xbuf)
+    E, C, D = xbuf.shape
+    F, Dout = w_gate.shape[1], w_down.shape[1]
+    if ybuf is None:
+        ybuf = torch.empty(E, C, Dout, dtype=xbuf.dtype, device=dev)
+    if saved_ab is None:
+        saved_ab = torch.empty(E, C, 2 * F, dtype=xbuf.dtype, device=dev)
+    ws = _workspace(moe_expert_ffn_workspace_size("swiglu", MOE_BF16, E, C, D, F, Dout), dev, workspace)
+    rc = lib().moe_expert_ffn_save(_p(xbuf), _p(used), E, C, D, F, Dout, _p(w_gate), _p(w_down), _p(w_up), _p(ybuf),
+                                   _p(saved_ab), _p(dev_status), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_expert_ffn_save", rc)
+    return ybuf, saved_ab
+
+
 def moe_combine(ybuf: torch.Tensor, selected: torch.Tensor, slot: torch.Tensor, gates: Optional[torch.Tensor],
                 base_kind: str = "zero", base: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
                 dev_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
@@ -459,7 +484,7 @@ def moe_backward_swiglu_workspace_size(E: int, C: int, H: int, F: int) -> int:
 
 def moe_backward_swiglu(dy, logits, selected, gates_f32, slot, used, xbuf, ybuf, w_gate, w_up, w_down, C: int,
                         use_residual: bool = False, aux_coef: float = 0.0, normalize_by_k: bool = True, counts=None,
-                        dev_status=None, workspace=None, stream=None):
+                        dev_status=None, workspace=None, stream=None, saved_ab=None):
     """Backward of the bf16 SwiGLU-expert layer.
 
     Returns (dx bf16 (T,H), dw_gate fp32 (E,F,H), dw_up fp32 (E,F,H), dw_down fp32 (E,H,F),
@@ -477,7 +502,7 @@ def moe_backward_swiglu(dy, logits, selected, gates_f32, slot, used, xbuf, ybuf,
     dg = torch.empty(T, k, dtype=torch.float32, device=dev)
     ws = _workspace(moe_backward_swiglu_workspace_size(E, C, H, F), dev, workspace)
     rc = lib().moe_backward_swiglu(_dt(dy), _p(dy), _p(logits), _p(selected), _p(gates_f32), _p(slot), _p(used),
-                                   _p(xbuf), _p(ybuf), _p(w_gate), _p(w_up), _p(w_down), T, k, E, C, H, F,
+                                   _p(xbuf), _p(ybuf), _p(saved_ab), _p(w_gate), _p(w_up), _p(w_down), T, k, E, C, H, F,
                                    int(bool(use_residual)), float(aux_coef), int(bool(normalize_by_k)), _p(counts),
                                    _p(dx), _p(dwg), _p(dwu), _p(dwd), _p(dl), _p(dg), _p(dev_status), _p(ws),
                                    ws.numel(), _stream(stream))

@@ -382,11 +382,27 @@ int transpose_valid(const __nv_bfloat16* src, int64_t lds, int64_t sgs, int G, i
     return launch_status();
 }
 
-// h, da, db from a, b (ab rows: [a | b], fp32) and dh (fp32), for c < used[e]:
+// h, da, db from a, b (ab rows: [a | b], fp32, or bf16 when saved by the forward) and dh
+// (fp32), for c < used[e]:
 //   s = sigmoid(a), h = a s b, da = dh b s (1 + a (1 - s)), db = dh a s.
-// Eight consecutive f per thread (F a multiple of 8): 32-byte fp32 loads,
-// 16-byte bf16 stores.
-__global__ void swiglu_bwd_elem_kernel(const float* __restrict__ ab, const float* __restrict__ dh,
+// Eight consecutive f per thread (F a multiple of 8): vector loads, 16-byte bf16 stores.
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 x = reinterpret_cast<const float4*>(p)[0], y = reinterpret_cast<const float4*>(p)[1];
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 x = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+template <typename AB>
+__global__ void swiglu_bwd_elem_kernel(const AB* __restrict__ ab, const float* __restrict__ dh,
                                        const int32_t* __restrict__ used, int64_t C, int64_t F,
                                        __nv_bfloat16* __restrict__ h, __nv_bfloat16* __restrict__ dab) {
     const int e = blockIdx.y;
@@ -396,13 +412,10 @@ __global__ void swiglu_bwd_elem_kernel(const float* __restrict__ ab, const float
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t c = i / F8, f = (i - c * F8) * 8;
         const int64_t row = (int64_t)e * C + c;
-        const float4* pa = reinterpret_cast<const float4*>(ab + row * 2 * F + f);
-        const float4* pb = reinterpret_cast<const float4*>(ab + row * 2 * F + F + f);
-        const float4* pg = reinterpret_cast<const float4*>(dh + row * F + f);
-        const float4 a0 = pa[0], a1 = pa[1], b0 = pb[0], b1 = pb[1], g0 = pg[0], g1 = pg[1];
-        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        float av[8], bv[8], gv[8];
+        load8(ab + row * 2 * F + f, av);
+        load8(ab + row * 2 * F + F + f, bv);
+        load8(dh + row * F + f, gv);
         uint32_t ph[4], pda[4], pdb[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -494,7 +507,7 @@ extern "C" size_t moe_backward_swiglu_workspace_size(int32_t E, int64_t C, int64
 
 extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float* logits, const int64_t* selected,
                                    const float* gates, const int64_t* slot, const int32_t* used, const void* xbuf,
-                                   const void* ybuf, const void* w_gate, const void* w_up, const void* w_down,
+                                   const void* ybuf, const void* saved_ab, const void* w_gate, const void* w_up, const void* w_down,
                                    int64_t T, int32_t k, int32_t E, int64_t C, int64_t H, int64_t F, int use_residual,
                                    float aux_coef, int normalize_by_k, const int32_t* counts, void* dx,
                                    float* dw_gate, float* dw_up, float* dw_down, float* dlogits, float* dgate,
@@ -550,8 +563,9 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     // 2. dybuf[e,c] = gate * dy[token]
     rc = gather_rows(dy, H, T, k, selected, slot, E, C, gates, dybuf, H, MOE_BF16, dev_status, stream);
     if (rc != MOE_OK) return rc;
-    // 3. [a | b] = xbuf [Wg; Wu]^T  (fp32), both weights in one pass over xbuf
-    {
+    // 3. [a | b] = xbuf [Wg; Wu]^T  (fp32), both weights in one pass over xbuf, unless the
+    //    forward saved them (bf16, moe_expert_ffn_save)
+    if (saved_ab == nullptr) {
         TcGemmProblem p{};
         p.a = xbuf;
         p.lda = H;
@@ -613,7 +627,11 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
         const int64_t nb = (C * (F / 8) + 255) / 256;
         const dim3 g2((unsigned)(nb < 1024 ? nb : 1024), (unsigned)E);
         MOE_REQUIRE(E <= 65535, MOE_ERR_UNSUPPORTED);
-        swiglu_bwd_elem_kernel<<<g2, 256, 0, stream>>>(ab, dh, used, C, F, h, dab);
+        if (saved_ab)
+            swiglu_bwd_elem_kernel<bf16><<<g2, 256, 0, stream>>>(static_cast<const bf16*>(saved_ab), dh, used, C, F,
+                                                                 h, dab);
+        else
+            swiglu_bwd_elem_kernel<float><<<g2, 256, 0, stream>>>(ab, dh, used, C, F, h, dab);
         rc = launch_status();
         if (rc != MOE_OK) return rc;
     }

@@ -88,11 +88,38 @@ int down_projection(moe_ffn_kind kind, const void* h, const int32_t* used, int32
 
 }  // namespace
 
+namespace moe {
+namespace {
+int expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32_t* used, int32_t E, int64_t C,
+               int64_t D, int64_t F, int64_t Dout, const void* w1, const void* b1, const void* w2, const void* b2,
+               const void* w3, void* ybuf, void* saved_ab, int32_t* dev_status, void* workspace,
+               size_t workspace_bytes, cudaStream_t stream);
+}  // namespace
+}  // namespace moe
+
 extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32_t* used, int32_t E,
                               int64_t C, int64_t D, int64_t F, int64_t Dout, const void* w1, const void* b1,
                               const void* w2, const void* b2, const void* w3, void* ybuf, int32_t* dev_status,
-                              void* workspace, size_t workspace_bytes, moe_stream_t stream_) {
-    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+                              void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+    return expert_ffn(kind, dtype, xbuf, used, E, C, D, F, Dout, w1, b1, w2, b2, w3, ybuf, nullptr, dev_status,
+                      workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int moe_expert_ffn_save(const void* xbuf, const int32_t* used, int32_t E, int64_t C, int64_t D, int64_t F,
+                                   int64_t Dout, const void* w_gate, const void* w_down, const void* w_up,
+                                   void* ybuf, void* saved_ab, int32_t* dev_status, void* workspace,
+                                   size_t workspace_bytes, moe_stream_t stream) {
+    MOE_REQUIRE(used != nullptr && saved_ab != nullptr, MOE_ERR_INVALID_ARG);
+    return expert_ffn(MOE_FFN_SWIGLU, MOE_BF16, xbuf, used, E, C, D, F, Dout, w_gate, nullptr, w_down, nullptr, w_up,
+                      ybuf, saved_ab, dev_status, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace moe {
+namespace {
+int expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32_t* used, int32_t E, int64_t C,
+               int64_t D, int64_t F, int64_t Dout, const void* w1, const void* b1, const void* w2, const void* b2,
+               const void* w3, void* ybuf, void* saved_ab, int32_t* dev_status, void* workspace,
+               size_t workspace_bytes, cudaStream_t stream) {
     MOE_REQUIRE(valid_dtype(dtype), MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(kind == MOE_FFN_LINEAR || kind == MOE_FFN_GELU_MLP || kind == MOE_FFN_SWIGLU, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(xbuf && ybuf && w1 && E >= 1 && C >= 0 && D >= 1 && Dout >= 1, MOE_ERR_INVALID_ARG);
@@ -136,6 +163,8 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
             p.out_rows_per_group = C;
             p.epilogue = TC_EPI_SWIGLU;
             p.status = dev_status;
+            p.save_ab = saved_ab;
+            p.ld_save = 2 * F;
             rc = tcx_gemm_run(p, stream);
         } else {
             // first GEMM: xbuf (E*C, D) x W^T
@@ -254,6 +283,8 @@ extern "C" int moe_expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xb
     }
     return run(d);
 }
+}  // namespace
+}  // namespace moe
 
 extern "C" int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const void* x, int64_t T, int64_t ldx,
                                        const int32_t* token_of_slot, const int32_t* used, int32_t E, int64_t C,

@@ -69,6 +69,8 @@ struct XParams {
     int64_t kdim;             // K (gathered mode: chunks past K are zero-filled)
     int64_t xrows;            // gathered mode: rows of the source matrix
     const int32_t* gidx;      // gathered mode: (G, max_tokens) source row per token slot
+    __nv_bfloat16* save_ab;   // SwiGLU: the pre-activations a (gate) and b (up) in bf16, or NULL
+    int64_t ld_save;
 };
 
 __device__ __forceinline__ int64_t group_rows(const XParams& p, int g) {
@@ -346,6 +348,17 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
                         tmem_ld_wait(u);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = silu_f(__uint_as_float(r[i])) * __uint_as_float(u[i]);
+                        if (p.save_ab && f < p.features) {  // [a | b] rows for the backward
+                            const int64_t row0 = (int64_t)g * p.out_rows_per_group + n0 + c * 32;
+                            const int i_end = (int)((n_valid - c * 32) < 32 ? (n_valid - c * 32) : 32);
+                            __nv_bfloat16* sa = p.save_ab + row0 * p.ld_save + f;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < i_end) {
+                                    sa[(int64_t)i * p.ld_save] = __float2bfloat16_rn(__uint_as_float(r[i]));
+                                    sa[(int64_t)i * p.ld_save + p.features] = __float2bfloat16_rn(__uint_as_float(u[i]));
+                                }
+                        }
                     } else {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
@@ -433,6 +446,8 @@ int tcx_gemm_run(const TcxProblem& p, cudaStream_t stream) {
     kp.rows = p.rows;
     kp.out = p.out;
     kp.ldo = p.ldo;
+    kp.save_ab = static_cast<__nv_bfloat16*>(p.save_ab);
+    kp.ld_save = p.ld_save;
     kp.out_rows_per_group = p.out_rows_per_group;
     kp.bias = p.bias;
     kp.bias_group_stride = p.bias_group_stride;

@@ -35,6 +35,10 @@ struct TcxProblem {
     int64_t bias_group_stride;
     int epilogue;              // TcEpilogue
     int32_t* status;
+    // TC_EPI_SWIGLU: when non-NULL, the bf16 pre-activations are also stored, row for row
+    // like out: a (gate) at column f, b (up) at column features + f, row stride ld_save.
+    void* save_ab;
+    int64_t ld_save;
 };
 
 // Single-CTA kernel: 256 weight rows x up to 128 tokens per tile.

@@ -18,7 +18,8 @@ class SwiGLUMoE:
     """
 
     def __init__(self, T: int, H: int, E: int, F: int, k: int, capacity_factor: float, F_shared: int = 0,
-                 aux_coef: float = 0.0, dtype=torch.bfloat16, device="cuda", gathered: bool = False):
+                 aux_coef: float = 0.0, dtype=torch.bfloat16, device="cuda", gathered: bool = False,
+                 save_for_backward: bool = False):
         self.T, self.H, self.E, self.F, self.k = T, H, E, F, k
         self.F_shared, self.aux_coef, self.dtype = F_shared, aux_coef, dtype
         self.C = B.moe_capacity(T, k, E, capacity_factor)
@@ -47,6 +48,10 @@ class SwiGLUMoE:
         if not self.gathered:
             self.disp_out["xbuf"] = torch.empty(E, C, H, dtype=dtype, device=dev)
         self.ybuf = torch.empty(E, C, H, dtype=dtype, device=dev)
+        # save_for_backward (bf16, not gathered): the routed experts also keep their gate/up
+        # pre-activations (E, C, 2F) for moe_backward_swiglu, which then skips recomputing them
+        self.saved_ab = (torch.empty(E, C, 2 * F, dtype=dtype, device=dev)
+                         if save_for_backward and dtype == torch.bfloat16 and not self.gathered else None)
         self.y = torch.empty(T, H, dtype=dtype, device=dev)
         self.shared = torch.empty(T, H, dtype=dtype, device=dev) if F_shared else None
         self.status = B.new_status(dev)
@@ -89,8 +94,12 @@ class SwiGLUMoE:
         else:
             d = B.moe_dispatch(r["selected"], self.E, self.C, x=x, out=self.disp_out, dev_status=self.status,
                                workspace=self.ws_disp)
-            B.moe_expert_ffn("swiglu", d["xbuf"], d["used"], w_gate, w2=w_down, w3=w_up, ybuf=self.ybuf,
-                             dev_status=self.status, workspace=self.ws_ffn)
+            if self.saved_ab is not None:
+                B.moe_expert_ffn_save(d["xbuf"], d["used"], w_gate, w_down, w_up, self.saved_ab, ybuf=self.ybuf,
+                                      dev_status=self.status, workspace=self.ws_ffn)
+            else:
+                B.moe_expert_ffn("swiglu", d["xbuf"], d["used"], w_gate, w2=w_down, w3=w_up, ybuf=self.ybuf,
+                                 dev_status=self.status, workspace=self.ws_ffn)
         if self.F_shared:
             main.wait_event(self.ev_shared)
         B.moe_combine(self.ybuf, r["selected"], d["slot"], r["gates_f32"], base_kind=base_kind, base=base, y=self.y,

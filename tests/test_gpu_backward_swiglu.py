@@ -31,7 +31,8 @@ def _close(got, want, what):
     (400, 128, 128, 6, 2, 1.0, True, 0.0),   # H, F multiples of 64: weights read MN-major, no transposed copies
     (333, 256, 64, 5, 3, 0.7, False, 0.05),  # the same with drops and the aux term
 ])
-def test_backward_swiglu_matches_oracle(T, H, F, E, k, cf, residual, aux):
+@pytest.mark.parametrize("saved", [False, True])
+def test_backward_swiglu_matches_oracle(T, H, F, E, k, cf, residual, aux, saved):
     g = torch.Generator().manual_seed(T + H)
 
     def rnd(*shape, scale=1.0):
@@ -48,10 +49,23 @@ def test_backward_swiglu_matches_oracle(T, H, F, E, k, cf, residual, aux):
     r = moe.moe_route(lgd, k)
     d = moe.moe_dispatch(r["selected"], E, C, x=xd)
     st = moe.new_status()
-    ybuf = moe.moe_expert_ffn("swiglu", d["xbuf"], d["used"], wgd, w2=wdd, w3=wud, dev_status=st)
+    saved_ab = None
+    if saved:  # the forward keeps [a | b] (bf16) and the backward skips recomputing them
+        ybuf, saved_ab = moe.moe_expert_ffn_save(d["xbuf"], d["used"], wgd, wdd, wud, dev_status=st)
+        ref = moe.moe_expert_ffn("swiglu", d["xbuf"], d["used"], wgd, w2=wdd, w3=wud, dev_status=st)
+        used_h = cpu(d["used"])
+        for e in range(E):  # the same expert outputs as without saving
+            assert torch.equal(ybuf[e, :int(used_h[e])], ref[e, :int(used_h[e])])
+        # the saved pre-activations are x W^T rounded to bf16
+        e0 = int(np.argmax(used_h))
+        a_ref = (d["xbuf"][e0, :int(used_h[e0])].float() @ wgd[e0].float().T)
+        np.testing.assert_allclose(cpu64(saved_ab[e0, :int(used_h[e0]), :F]), cpu64(a_ref), rtol=2e-2,
+                                   atol=2e-2 * float(a_ref.abs().max()))
+    else:
+        ybuf = moe.moe_expert_ffn("swiglu", d["xbuf"], d["used"], wgd, w2=wdd, w3=wud, dev_status=st)
     dx, dwg, dwu, dwd, dl, dg = moe.moe_backward_swiglu(
         dyd, lgd, r["selected"], r["gates_f32"], d["slot"], d["used"], d["xbuf"], ybuf, wgd, wud, wdd, C,
-        use_residual=residual, aux_coef=aux, counts=r["counts"], dev_status=st)
+        use_residual=residual, aux_coef=aux, counts=r["counts"], dev_status=st, saved_ab=saved_ab)
     assert moe.moe_read_status(st) == 0
 
     s64 = cpu64(lg)
