@@ -488,10 +488,11 @@ SwigluBwdWs swiglu_bwd_layout(int32_t E, int64_t C, int64_t H, int64_t F) {
     const bool mn = H % 64 == 0 && F % 64 == 0;  // weights read in place (MN-major): no transposed copies
     w.wdT = take(mn ? 0 : (size_t)E * F * H * 2);
     w.wguT = take(mn ? 0 : (size_t)E * H * 2 * F * 2);
-    w.dybufT = take((size_t)E * H * w.Cp * 2);
-    w.hT = take((size_t)E * F * w.Cp * 2);
-    w.dabT = take((size_t)E * 2 * F * w.Cp * 2);
-    w.xbufT = take((size_t)E * H * w.Cp * 2);
+    // token-transposed operands of the weight gradients (not needed when both operands are read MN-major)
+    w.dybufT = take(mn ? 0 : (size_t)E * H * w.Cp * 2);
+    w.hT = take(mn ? 0 : (size_t)E * F * w.Cp * 2);
+    w.dabT = take(mn ? 0 : (size_t)E * 2 * F * w.Cp * 2);
+    w.xbufT = take(mn ? 0 : (size_t)E * H * w.Cp * 2);
     w.dxbuf = take((size_t)E * C * H * 2);
     w.total = off;
     return w;
@@ -635,25 +636,58 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
         rc = launch_status();
         if (rc != MOE_OK) return rc;
     }
-    // 6. weight gradients over the token index: transposed operands, zeros past used[e]
-    rc = transpose_valid(dybuf, H, C * H, E, C, H, used, Cp, dybufT, Cp, H * Cp, stream);
-    if (rc != MOE_OK) return rc;
-    rc = transpose_valid(h, F, C * F, E, C, F, used, Cp, hT, Cp, F * Cp, stream);
-    if (rc != MOE_OK) return rc;
-    rc = transpose_valid(dab, F2, C * F2, E, C, F2, used, Cp, dabT, Cp, F2 * Cp, stream);
-    if (rc != MOE_OK) return rc;
-    rc = transpose_valid(xb, H, C * H, E, C, H, used, Cp, xbufT, Cp, H * Cp, stream);
-    if (rc != MOE_OK) return rc;
-    // K = the expert's kept tokens only (the transposed operands are zero past used[e])
-    rc = gemm(dybufT, Cp, (int64_t)E * H, H, hT, Cp, (int64_t)E * F, F, E, H, F, Cp, nullptr, dw_down, F, H,
-              TC_EPI_F32, dev_status, stream, used);
-    if (rc != MOE_OK) return rc;
-    rc = gemm(dabT, Cp, (int64_t)E * F2, F2, xbufT, Cp, (int64_t)E * H, H, E, F, H, Cp, nullptr, dw_gate, H, F,
-              TC_EPI_F32, dev_status, stream, used);
-    if (rc != MOE_OK) return rc;
-    rc = gemm(dabT + F * Cp, Cp, (int64_t)E * F2 - F, F2, xbufT, Cp, (int64_t)E * H, H, E, F, H, Cp, nullptr, dw_up,
-              H, F, TC_EPI_F32, dev_status, stream, used);
-    if (rc != MOE_OK) return rc;
+    // 6. weight gradients over the token index, K = the expert's kept tokens.  With H and F multiples
+    //    of 64 both operands are read in place with the token on their rows (MN-major A and B; the
+    //    GEMM clears the rows past used[e] of an expert's last K block); otherwise from transposed
+    //    copies that are zero past used[e].
+    if (mn) {
+        auto wgrad = [&](const void* a, int64_t lda, int64_t M, const void* b, int64_t ldb, int64_t N, float* out) {
+            TcGemmProblem p{};
+            p.a = a;
+            p.lda = lda;
+            p.a_rows_total = (int64_t)E * C;
+            p.a_rows_per_group = C;
+            p.a_mn_major = true;
+            p.b = b;
+            p.ldb = ldb;
+            p.b_rows_total = (int64_t)E * C;
+            p.b_rows_per_group = C;
+            p.b_mn_major = true;
+            p.G = E;
+            p.M = M;
+            p.N = N;
+            p.K = C;
+            p.k_rows = used;
+            p.out = out;
+            p.ldo = N;
+            p.out_rows_per_group = M;
+            p.epilogue = TC_EPI_F32;
+            p.status = dev_status;
+            return tc_gemm_run(p, stream);
+        };
+        if ((rc = wgrad(dybuf, H, H, h, F, F, dw_down)) != MOE_OK) return rc;  // dWd[e] (H, F) = dybuf^T h
+        if ((rc = wgrad(dab, F2, F, xb, H, H, dw_gate)) != MOE_OK) return rc;  // dWg[e] (F, H) = da^T x
+        if ((rc = wgrad(dab + F, F2, F, xb, H, H, dw_up)) != MOE_OK) return rc;  // dWu[e] (F, H) = db^T x
+    } else {
+        rc = transpose_valid(dybuf, H, C * H, E, C, H, used, Cp, dybufT, Cp, H * Cp, stream);
+        if (rc != MOE_OK) return rc;
+        rc = transpose_valid(h, F, C * F, E, C, F, used, Cp, hT, Cp, F * Cp, stream);
+        if (rc != MOE_OK) return rc;
+        rc = transpose_valid(dab, F2, C * F2, E, C, F2, used, Cp, dabT, Cp, F2 * Cp, stream);
+        if (rc != MOE_OK) return rc;
+        rc = transpose_valid(xb, H, C * H, E, C, H, used, Cp, xbufT, Cp, H * Cp, stream);
+        if (rc != MOE_OK) return rc;
+        // K = the expert's kept tokens only (the transposed operands are zero past used[e])
+        rc = gemm(dybufT, Cp, (int64_t)E * H, H, hT, Cp, (int64_t)E * F, F, E, H, F, Cp, nullptr, dw_down, F, H,
+                  TC_EPI_F32, dev_status, stream, used);
+        if (rc != MOE_OK) return rc;
+        rc = gemm(dabT, Cp, (int64_t)E * F2, F2, xbufT, Cp, (int64_t)E * H, H, E, F, H, Cp, nullptr, dw_gate, H, F,
+                  TC_EPI_F32, dev_status, stream, used);
+        if (rc != MOE_OK) return rc;
+        rc = gemm(dabT + F * Cp, Cp, (int64_t)E * F2 - F, F2, xbufT, Cp, (int64_t)E * H, H, E, F, H, Cp, nullptr, dw_up,
+                  H, F, TC_EPI_F32, dev_status, stream, used);
+        if (rc != MOE_OK) return rc;
+    }
     // 7. dxbuf = [da | db] [Wg; Wu]: B(k, n = h) = Wg[e][k][h] for k < F, Wu[e][k - F][h] after
     if (mn) {
         TcGemmProblem p{};

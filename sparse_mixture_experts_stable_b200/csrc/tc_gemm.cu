@@ -138,7 +138,7 @@ __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* row, int64_t n0, in
     }
 }
 
-template <int EPI, bool BMN>
+template <int EPI, bool AMN, bool BMN>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const KParams p) {
@@ -216,7 +216,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_expect_tx(&full[stage], p.tx_bytes);
                     uint8_t* a_dst = smA + stage * kABytes;
                     uint8_t* b_dst = smB + stage * kBBytes;
-                    tma_load_2d(a_dst, &tmA, kb * kBK, a_y, &full[stage]);
+                    if (AMN) {
+                        // K rows kb*64 .. +63 of the group's (K, M) matrix, two 64-column boxes of 8 KB
+                        const int32_t k_y = (int32_t)(g * p.a_rows_per_group + (int64_t)kb * kBK);
+                        tma_load_2d(a_dst, &tmA, mt * kBM, k_y, &full[stage]);
+                        tma_load_2d(a_dst + 8192, &tmA, mt * kBM + 64, k_y, &full[stage]);
+                    } else {
+                        tma_load_2d(a_dst, &tmA, kb * kBK, a_y, &full[stage]);
+                    }
                     if (BMN) {
                         // K rows kb*64 .. +63 of the (K, N) weight, in 64-column boxes of 8 KB
                         const bool second = p.k_split_blocks > 0 && kb >= p.k_split_blocks;
@@ -240,49 +247,94 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------- MMA issuer -------------------------------
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc(kBM, p.n_mma) | (BMN ? (1u << 16) : 0u);
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t it = 0;
-            for (int tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x, ++it) {
-                const uint32_t acc = it & 1u;
-                const uint32_t acc_phase = (it >> 1) & 1u;
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status)) {
+        // Lane 0 issues the MMAs.  When the K range of a group ends inside a block
+        // and an operand is MN-major (K on its rows), the whole warp first clears
+        // that block's rows past the valid K in shared memory (they hold whatever
+        // follows the group in memory), so garbage never meets a zero.
+        constexpr bool kMask = AMN || BMN;
+        const uint32_t idesc = make_idesc(kBM, p.n_mma) | (AMN ? (1u << 15) : 0u) | (BMN ? (1u << 16) : 0u);
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t it = 0;
+        for (int tile = blockIdx.x;; tile += gridDim.x, ++it) {
+            // one decision for the whole warp (s_abort may be raised by another warp meanwhile)
+            if (!__shfl_sync(0xffffffffu, (tile < total && !s_abort) ? 1 : 0, 0)) break;
+            const uint32_t acc = it & 1u;
+            const uint32_t acc_phase = (it >> 1) & 1u;
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                s_abort = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * kBN;
+            int g_, mt_, nt_;
+            decode_tile(tile, s_prefix, p.G, p.n_tiles, g_, mt_, nt_);
+            const int kbg = group_k_blocks(p, g_);
+            int kvalid_last = kBK;  // valid K rows in the group's last block
+            if (kMask && p.k_rows) {
+                const int v = p.k_rows[g_];
+                kvalid_last = v <= 0 ? 0 : v - (kbg - 1) * kBK;
+                if (kvalid_last > kBK) kvalid_last = kBK;
+            }
+            for (int kb = 0; kb < kbg; ++kb) {
+                const bool clear = kMask && kb == kbg - 1 && kvalid_last < kBK;
+                int okf = 1;
+                if (lane == 0 || clear) okf = mbar_wait(&full[stage], phase, p.status) ? 1 : 0;
+                okf = __all_sync(0xffffffffu, okf);
+                if (!okf) {
                     s_abort = 1;
+                    ok = 0;
                     break;
                 }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * kBN;
-                bool ok = true;
-                int g_, mt_, nt_;
-                decode_tile(tile, s_prefix, p.G, p.n_tiles, g_, mt_, nt_);
-                const int kbg = group_k_blocks(p, g_);
-                for (int kb = 0; kb < kbg; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, p.status)) {
-                        s_abort = 1;
-                        ok = false;
-                        break;
+                if (clear) {
+                    // rows [kvalid_last, 64) of every 8 KB MN-major box: 128 bytes per row
+                    const int nrow = kBK - kvalid_last;
+                    if (AMN) {
+                        uint8_t* base = smA + stage * kABytes;
+                        for (int i = lane; i < 2 * nrow * 8; i += 32) {
+                            const int box = i / (nrow * 8), rem = i - box * nrow * 8;
+                            *reinterpret_cast<uint4*>(base + box * 8192 + (kvalid_last + rem / 8) * 128 + (rem & 7) * 16) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
                     }
+                    if (BMN) {
+                        uint8_t* base = smB + stage * kBBytes;
+                        const int nbox = p.n_mma / 64;
+                        for (int i = lane; i < nbox * nrow * 8; i += 32) {
+                            const int box = i / (nrow * 8), rem = i - box * nrow * 8;
+                            *reinterpret_cast<uint4*>(base + box * 8192 + (kvalid_last + rem / 8) * 128 + (rem & 7) * 16) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                if (lane == 0) {
                     tc_fence_after();
-                    const uint64_t ad = sw128_desc(smem_u32(smA + stage * kABytes));
+                    const uint64_t ad = AMN ? sw128_mn_desc(smem_u32(smA + stage * kABytes), 8192)
+                                            : sw128_desc(smem_u32(smA + stage * kABytes));
                     const uint64_t bd = BMN ? sw128_mn_desc(smem_u32(smB + stage * kBBytes), 8192)
                                             : sw128_desc(smem_u32(smB + stage * kBBytes));
                     // a K step of 16: 32 bytes along a K-major row, or two 1024-byte groups of 8 K rows
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma(d_tmem, ad + 2 * kk, bd + (BMN ? 128 : 2) * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        tc_mma(d_tmem, ad + (AMN ? 128 : 2) * kk, bd + (BMN ? 128 : 2) * kk, idesc,
+                               (kb > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&empty[stage]);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
                 }
-                if (!ok) break;
-                tc_commit(&tfull[acc]);
+                __syncwarp();
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
+            if (!ok) break;
+            if (lane == 0) tc_commit(&tfull[acc]);
+            __syncwarp();
         }
-        __syncwarp();
     } else {
         // -------------------------------- epilogue --------------------------------
         const int q = warp & 3;
@@ -483,18 +535,18 @@ bool make_map_f32(CUtensorMap* m, const void* base, int64_t inner, int64_t rows,
 
 namespace {
 
-template <int EPI, bool BMN = false>
+template <int EPI, bool AMN = false, bool BMN = false>
 int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const KParams& kp, int grid,
            cudaStream_t stream) {
     static bool attr_set[64] = {false};
     int dev = 0;
     MOE_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 64 && !attr_set[dev]) {
-        MOE_CUDA_TRY(cudaFuncSetAttribute(tc_gemm_kernel<EPI, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        MOE_CUDA_TRY(cudaFuncSetAttribute(tc_gemm_kernel<EPI, AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)kSmemBytes));
         attr_set[dev] = true;
     }
-    tc_gemm_kernel<EPI, BMN><<<grid, kThreads, kSmemBytes, stream>>>(a, b, b2, kp);
+    tc_gemm_kernel<EPI, AMN, BMN><<<grid, kThreads, kSmemBytes, stream>>>(a, b, b2, kp);
     return launch_status();
 }
 
@@ -507,7 +559,12 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     // TMA: 16-byte aligned bases, row strides a multiple of 16 bytes.
     MOE_REQUIRE(aligned16(p.a) && aligned16(p.b) && (p.lda * 2) % 16 == 0 && (p.ldb * 2) % 16 == 0,
                 MOE_ERR_UNSUPPORTED);
-    MOE_REQUIRE(p.lda >= p.K && (p.b_mn_major ? p.ldb >= p.N : p.ldb >= p.K), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE((p.a_mn_major ? p.lda >= p.M : p.lda >= p.K) && (p.b_mn_major ? p.ldb >= p.N : p.ldb >= p.K),
+                MOE_ERR_INVALID_ARG);
+    // MN-major A is built for the weight-gradient products: fp32 out, MN-major B, K rows per group
+    if (p.a_mn_major)
+        MOE_REQUIRE(p.b_mn_major && p.epilogue == TC_EPI_F32 && p.k_split == 0 && p.rows == nullptr,
+                    MOE_ERR_UNSUPPORTED);
     if (p.b_mn_major) {
         MOE_REQUIRE(p.epilogue == TC_EPI_F32 || p.epilogue == TC_EPI_BF16, MOE_ERR_UNSUPPORTED);
         MOE_REQUIRE(p.k_split % kBK == 0 && p.k_split >= 0 && p.k_split < p.K, MOE_ERR_UNSUPPORTED);
@@ -554,7 +611,10 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     kp.status = p.status;
 
     CUtensorMap ma, mb, mb2;
-    MOE_REQUIRE(make_map(&ma, p.a, p.K, p.a_rows_total, p.lda, kBM), MOE_ERR_CUDA);
+    if (p.a_mn_major)  // (K rows, M columns) with 64 x 64 boxes
+        MOE_REQUIRE(make_map(&ma, p.a, p.M, p.a_rows_total, p.lda, kBK), MOE_ERR_CUDA);
+    else
+        MOE_REQUIRE(make_map(&ma, p.a, p.K, p.a_rows_total, p.lda, kBM), MOE_ERR_CUDA);
     if (p.b_mn_major) {
         // (K rows, N columns) with 64 x 64 boxes: rows past b_rows_total and columns past N read as zero
         MOE_REQUIRE(make_map(&mb, p.b, p.N, p.b_rows_total, p.ldb, kBK), MOE_ERR_CUDA);
@@ -572,9 +632,10 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     if (max_tiles < grid) grid = (int)max_tiles;
     if (grid < 1) grid = 1;
 
+    if (p.a_mn_major) return launch<TC_EPI_F32, true, true>(ma, mb, mb2, kp, grid, stream);
     if (p.b_mn_major)
-        return p.epilogue == TC_EPI_F32 ? launch<TC_EPI_F32, true>(ma, mb, mb2, kp, grid, stream)
-                                        : launch<TC_EPI_BF16, true>(ma, mb, mb2, kp, grid, stream);
+        return p.epilogue == TC_EPI_F32 ? launch<TC_EPI_F32, false, true>(ma, mb, mb2, kp, grid, stream)
+                                        : launch<TC_EPI_BF16, false, true>(ma, mb, mb2, kp, grid, stream);
     switch (p.epilogue) {
         case TC_EPI_F32: return launch<TC_EPI_F32>(ma, mb, mb2, kp, grid, stream);
         case TC_EPI_BF16: return launch<TC_EPI_BF16>(ma, mb, mb2, kp, grid, stream);

@@ -39,6 +39,9 @@ struct TcGemmProblem {
     bool b_mn_major;          // B(k, n) = b[(g * b_rows_per_group + k) * ldb + n]; epilogues F32 / BF16 only,
                               // UMMA N a multiple of 64, k_split a multiple of 64
     int64_t k_split;
+    bool a_mn_major;          // A(m, k) = a[(g * a_rows_per_group + k) * lda + m] (with b_mn_major, F32 out):
+                              // both operands hold K on their rows; with k_rows the rows of a group's last
+                              // K block past k_rows[g] are cleared in shared memory before the MMAs
     int G;                    // groups
     int64_t M;                // max rows per group
     int64_t N;                // output columns per group
