@@ -280,7 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (kvalid_last > kBK) kvalid_last = kBK;
             }
             for (int kb = 0; kb < kbg; ++kb) {
-                const bool clear = kMask && kb == kbg - 1 && kvalid_last < kBK;
+                // the group's last block: only the K steps of 16 that hold valid rows (at least one),
+                // and only the rows between the last valid one and the end of those steps are cleared
+                const bool last = kMask && kb == kbg - 1 && kvalid_last < kBK;
+                const int nkk = last ? (kvalid_last <= 0 ? 1 : (kvalid_last + 15) / 16) : kBK / 16;
+                const int kend = nkk * 16;
+                const bool clear = last && kvalid_last < kend;
                 int okf = 1;
                 if (lane == 0 || clear) okf = mbar_wait(&full[stage], phase, p.status) ? 1 : 0;
                 okf = __all_sync(0xffffffffu, okf);
@@ -290,13 +295,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 if (clear) {
-                    // rows [kvalid_last, 64) of every 8 KB MN-major box: 128 bytes per row
-                    const int nrow = kBK - kvalid_last;
+                    // rows [kvalid_last, kend) of every 8 KB MN-major box: 128 bytes per row
+                    const int nrow = kend - (kvalid_last < 0 ? 0 : kvalid_last);
+                    const int r0 = kend - nrow;
                     if (AMN) {
                         uint8_t* base = smA + stage * kABytes;
                         for (int i = lane; i < 2 * nrow * 8; i += 32) {
                             const int box = i / (nrow * 8), rem = i - box * nrow * 8;
-                            *reinterpret_cast<uint4*>(base + box * 8192 + (kvalid_last + rem / 8) * 128 + (rem & 7) * 16) =
+                            *reinterpret_cast<uint4*>(base + box * 8192 + (r0 + rem / 8) * 128 + (rem & 7) * 16) =
                                 make_uint4(0u, 0u, 0u, 0u);
                         }
                     }
@@ -305,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int nbox = p.n_mma / 64;
                         for (int i = lane; i < nbox * nrow * 8; i += 32) {
                             const int box = i / (nrow * 8), rem = i - box * nrow * 8;
-                            *reinterpret_cast<uint4*>(base + box * 8192 + (kvalid_last + rem / 8) * 128 + (rem & 7) * 16) =
+                            *reinterpret_cast<uint4*>(base + box * 8192 + (r0 + rem / 8) * 128 + (rem & 7) * 16) =
                                 make_uint4(0u, 0u, 0u, 0u);
                         }
                     }
@@ -321,8 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // a K step of 16: 32 bytes along a K-major row, or two 1024-byte groups of 8 K rows
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma(d_tmem, ad + (AMN ? 128 : 2) * kk, bd + (BMN ? 128 : 2) * kk, idesc,
-                               (kb > 0 || kk > 0) ? 1u : 0u);
+                        if (kk < nkk)
+                            tc_mma(d_tmem, ad + (AMN ? 128 : 2) * kk, bd + (BMN ? 128 : 2) * kk, idesc,
+                                   (kb > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&empty[stage]);
                 }
                 __syncwarp();
