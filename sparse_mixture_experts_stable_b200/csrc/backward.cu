@@ -273,17 +273,19 @@ extern "C" int moe_backward(moe_ffn_kind kind, moe_dtype dtype, const void* dy, 
 // moe_backward_swiglu: bf16 SwiGLU experts, the kept mask held constant.
 //   1. dgate / dlogits                       as above, on bf16 rows
 //   2. dybuf[e,c] = gate * dy[token]         scaled gather (bf16)
-//   3. [a | b] = xbuf [Wg; Wu]^T             one tensor-core GEMM (both weights), fp32 out
-//   4. dh = dybuf Wd                         tensor-core GEMM on Wd^T, fp32 out
+//   3. [a | b] = xbuf [Wg; Wu]^T             one tensor-core GEMM (both weights), fp32 out,
+//                                            unless the forward saved them (bf16)
+//   4. dh = dybuf Wd                         tensor-core GEMM, fp32 out
 //   5. h, da, db from (a, b, dh)             elementwise (silu and its derivative)
 //   6. dWd = dybuf^T h, dWg = da^T xbuf, dWu = db^T xbuf
-//                                            tensor-core GEMMs on zero-padded,
-//                                            token-transposed operands, fp32 out
-//   7. dxbuf = [da | db] [Wg; Wu]            tensor-core GEMM on the transposed
-//                                            stacked weights, bf16 out
+//                                            tensor-core GEMMs over each expert's kept
+//                                            tokens, fp32 out
+//   7. dxbuf = [da | db] [Wg; Wu]            tensor-core GEMM, bf16 out
 //   8. dx[t] = [dy[t]] + sum_kept dxbuf[e, slot]
-// All GEMMs are the K-major tcgen05 kernel; operands that the products need
-// with the token index as K are transposed (with zeros past used[e]) first.
+// All products run on the tcgen05 kernel.  With H and F multiples of 64 every
+// operand is read in place (the weights and, for step 6, both token-major
+// operands as MN-major operands); otherwise the operands that need another
+// major order are transposed first (zero past used[e] for the token-major ones).
 // ---------------------------------------------------------------------------
 namespace moe {
 namespace {
