@@ -89,36 +89,6 @@ __device__ __forceinline__ int group_k_blocks(const KParams& p, int g) {
     return kb < p.k_blocks ? kb : p.k_blocks;
 }
 
-// Warp-cooperative store of one 32 x 32 output chunk.  Lane i holds row i's
-// 32 values as W 32-bit words (W = 16: bf16 pairs, W = 32: fp32).  The rows
-// are staged in shared memory (16-byte quads XOR-swizzled by row, so neither
-// phase has bank conflicts) and written back row-contiguous, W / 4 lanes per
-// row, so every store instruction covers whole 32-byte sectors instead of 32
-// rows' 16-byte pieces.  Row r goes to row0 + r * pitch bytes, if r < nrows.
-template <int W>
-__device__ __forceinline__ int stage_swz(int r) {
-    return W == 16 ? ((r >> 1) & 3) : (r & 7);
-}
-
-template <int W>
-__device__ __forceinline__ void warp_store_chunk(uint32_t* stg, const uint32_t (&w)[W], uint8_t* row0, int64_t pitch,
-                                                 int nrows, int lane) {
-    constexpr int Q = W / 4;  // 16-byte quads per row
-#pragma unroll
-    for (int m = 0; m < Q; ++m)
-        *reinterpret_cast<uint4*>(stg + lane * W + 4 * (m ^ stage_swz<W>(lane))) =
-            make_uint4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
-    __syncwarp();
-    constexpr int RPI = 32 / Q;  // rows per store instruction
-#pragma unroll
-    for (int it = 0; it < Q; ++it) {
-        const int r = it * RPI + lane / Q, m = lane % Q;
-        const uint4 v = *reinterpret_cast<const uint4*>(stg + r * W + 4 * (m ^ stage_swz<W>(r)));
-        if (r < nrows) *reinterpret_cast<uint4*>(row0 + r * pitch + 16 * m) = v;
-    }
-    __syncwarp();
-}
-
 // Store 32 bf16 values (already packed in pairs) for columns n0..n0+31 of one row.
 __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* row, int64_t n0, int64_t N, const uint32_t (&pk)[16],
                                               bool vec) {

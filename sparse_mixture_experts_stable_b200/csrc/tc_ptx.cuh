@@ -171,6 +171,36 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Warp-cooperative store of one 32 x 32 output chunk.  Lane i holds row i's
+// 32 values as W 32-bit words (W = 16: bf16 pairs, W = 32: fp32).  The rows
+// are staged in shared memory (16-byte quads XOR-swizzled by row, so neither
+// phase has bank conflicts) and written back row-contiguous, W / 4 lanes per
+// row, so every store instruction covers whole 32-byte sectors instead of 32
+// rows' 16-byte pieces.  Row r goes to row0 + r * pitch bytes, if r < nrows.
+template <int W>
+__device__ __forceinline__ int stage_swz(int r) {
+    return W == 16 ? ((r >> 1) & 3) : (r & 7);
+}
+
+template <int W>
+__device__ __forceinline__ void warp_store_chunk(uint32_t* stg, const uint32_t (&w)[W], uint8_t* row0, int64_t pitch,
+                                                 int nrows, int lane) {
+    constexpr int Q = W / 4;  // 16-byte quads per row
+#pragma unroll
+    for (int m = 0; m < Q; ++m)
+        *reinterpret_cast<uint4*>(stg + lane * W + 4 * (m ^ stage_swz<W>(lane))) =
+            make_uint4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]);
+    __syncwarp();
+    constexpr int RPI = 32 / Q;  // rows per store instruction
+#pragma unroll
+    for (int it = 0; it < Q; ++it) {
+        const int r = it * RPI + lane / Q, m = lane % Q;
+        const uint4 v = *reinterpret_cast<const uint4*>(stg + r * W + 4 * (m ^ stage_swz<W>(r)));
+        if (r < nrows) *reinterpret_cast<uint4*>(row0 + r * pitch + 16 * m) = v;
+    }
+    __syncwarp();
+}
+
 // Ask the TMA unit to bring a box into L2 (no shared-memory destination).
 __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
     asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),

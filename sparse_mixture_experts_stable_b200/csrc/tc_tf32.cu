@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const T3Params p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_prefix[kMaxGroups + 1];
+    __shared__ __align__(16) uint32_t s_stage[4][32 * 32];  // epilogue staging, one 32 x 32 chunk per warp
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
 
@@ -288,7 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const int64_t m = (int64_t)mt * kBM + q * 32 + lane;
-            const bool row_ok = m < group_m(p, g);
+            const int64_t gm = group_m(p, g);
+            const bool row_ok = m < gm;
+            // this warp's 32 rows for the staged stores
+            const int64_t wrow0 = (int64_t)mt * kBM + q * 32;
+            const int wrows = (int)(gm - wrow0 < 0 ? 0 : (gm - wrow0 > 32 ? 32 : gm - wrow0));
+            float* cw = p.C + g * p.c_group_stride + wrow0 * p.ldc;
             float* crow = p.C + g * p.c_group_stride + m * p.ldc;
             const float* bias = p.bias ? p.bias + g * p.bias_group_stride : nullptr;
             const uint32_t t_row = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
@@ -297,6 +303,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(t_row + c * 32, r);
                 tmem_ld_wait(r);
                 const int64_t n0 = (int64_t)nt * p.n_mma + c * 32;
+                if (p.epilogue != F32_EPI_SILU_MUL && p.vec_ok && n0 + 32 <= p.N) {
+                    // row-contiguous stores through shared memory (see warp_store_chunk)
+                    uint32_t w[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float v = __uint_as_float(r[i]);
+                        if ((p.epilogue == F32_EPI_BIAS || p.epilogue == F32_EPI_BIAS_GELU) && bias) v += bias[n0 + i];
+                        if (p.epilogue == F32_EPI_BIAS_GELU) v = gelu_f(v);
+                        w[i] = __float_as_uint(v);
+                    }
+                    warp_store_chunk<32>(s_stage[q], w, reinterpret_cast<uint8_t*>(cw + n0), p.ldc * 4, wrows, lane);
+                    continue;
+                }
                 if (!row_ok) continue;
                 if (p.vec_ok && n0 + 32 <= p.N) {
 #pragma unroll
