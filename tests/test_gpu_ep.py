@@ -156,3 +156,17 @@ def test_ipc_mapping_in_a_second_process():
         got = torch.load(outp)
     assert torch.equal(got, want.cpu())
     del pad
+
+
+def test_ep_with_zero_capacity_keeps_every_row_as_its_base():
+    # C = 0 (the numpy-layer page, section 3 edge checks): every assignment is dropped on every rank and y = x
+    E, k, D, F = 8, 2, 64, 64
+    g = torch.Generator().manual_seed(9)
+    xs = [torch.randn(t, D, generator=g).to(torch.bfloat16).to(DEV) for t in (40, 24)]
+    w_router = (torch.randn(E, D, generator=g) * D ** -0.5).to(torch.bfloat16).to(DEV)
+    w = _weights("swiglu", E, D, F, g, torch.bfloat16)
+    out = ep.run_ranks_on_one_device(xs, E, k, 0, "swiglu", w_router, [_slice(w, q * 4, (q + 1) * 4) for q in range(2)])
+    for q in range(2):
+        assert (out["dispatch"][q]["slot"] == -1).all()
+        assert (out["plan"][q]["used"] == 0).all()
+        assert torch.equal(out["y"][q], xs[q])
