@@ -20,8 +20,8 @@ namespace {
 
 constexpr int kWarps = 8;
 
-// This lane's part of the dot product of two rows of n elements: 16-byte
-// vectors when VEC (n a multiple of the vector width, rows 16-byte aligned).
+// Dot products of rows of n elements, this lane's part: 16-byte vectors when
+// VEC (n a multiple of the vector width, rows 16-byte aligned).
 __device__ __forceinline__ float dot16(const uint4& a, const uint4& b, float acc, const float*) {
     acc = fmaf(__uint_as_float(a.x), __uint_as_float(b.x), acc);
     acc = fmaf(__uint_as_float(a.y), __uint_as_float(b.y), acc);
@@ -40,20 +40,30 @@ __device__ __forceinline__ float dot16(const uint4& a, const uint4& b, float acc
     return acc;
 }
 
+// Two rows b0, b1 against one row a (a read once; a NULL row is skipped).
 template <typename In, bool VEC>
-__device__ __forceinline__ float row_dot_part(const In* __restrict__ a, const In* __restrict__ b, int64_t n,
-                                              int lane) {
-    float part = 0.f;
+__device__ __forceinline__ void row_dot_part2(const In* __restrict__ a, const In* __restrict__ b0,
+                                              const In* __restrict__ b1, int64_t n, int lane, float& p0, float& p1) {
+    p0 = 0.f;
+    p1 = 0.f;
     if (VEC) {
         constexpr int EPV = 16 / sizeof(In);
         const int64_t nv = n / EPV;
         const uint4* va = reinterpret_cast<const uint4*>(a);
-        const uint4* vb = reinterpret_cast<const uint4*>(b);
-        for (int64_t v = lane; v < nv; v += 32) part = dot16(va[v], vb[v], part, a);
+        const uint4* v0 = reinterpret_cast<const uint4*>(b0);
+        const uint4* v1 = reinterpret_cast<const uint4*>(b1);
+        for (int64_t v = lane; v < nv; v += 32) {
+            const uint4 x = va[v];
+            if (b0) p0 = dot16(x, v0[v], p0, a);
+            if (b1) p1 = dot16(x, v1[v], p1, a);
+        }
     } else {
-        for (int64_t i = lane; i < n; i += 32) part = fmaf(to_f32(a[i]), to_f32(b[i]), part);
+        for (int64_t i = lane; i < n; i += 32) {
+            const float x = to_f32(a[i]);
+            if (b0) p0 = fmaf(x, to_f32(b0[i]), p0);
+            if (b1) p1 = fmaf(x, to_f32(b1[i]), p1);
+        }
     }
-    return part;
 }
 
 template <typename In, bool VEC>
@@ -70,21 +80,34 @@ __global__ void __launch_bounds__(kWarps * 32)
     // dgate_j (all lanes end up with every dgate_j through the warp sums)
     float gdot = 0.f;
     float my_dg0 = 0.f, my_dg1 = 0.f;  // dgate for j = lane, lane + 32
-    for (int j = 0; j < k; ++j) {
-        const int64_t e = selected[t * k + j];
-        const int64_t s = slot[t * k + j];
-        float dg = 0.f;
-        if (s >= 0) {
-            if (e < 0 || e >= E || s >= C) {
-                if (lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
-            } else {
-                const In* yr = ybuf + (e * C + s) * Dout;
-                dg = warp_sum(row_dot_part<In, VEC>(dyr, yr, Dout, lane));
+    // two assignments at a time: the dy row is read once for both, and both rows' loads are in flight
+    for (int j = 0; j < k; j += 2) {
+        const In* yr[2] = {nullptr, nullptr};
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (j + u >= k) break;
+            const int64_t e = selected[t * k + j + u];
+            const int64_t s = slot[t * k + j + u];
+            if (s >= 0) {
+                if (e < 0 || e >= E || s >= C) {
+                    if (lane == 0) set_status(status, MOE_ERR_BAD_INDEX);
+                } else {
+                    yr[u] = ybuf + (e * C + s) * Dout;
+                }
             }
         }
-        gdot = fmaf(gates[t * k + j], dg, gdot);
-        if (j == lane) my_dg0 = dg;
-        if (j == lane + 32) my_dg1 = dg;
+        float p0, p1;
+        row_dot_part2<In, VEC>(dyr, yr[0], yr[1], Dout, lane, p0, p1);
+        const float dg0 = yr[0] ? warp_sum(p0) : 0.f;
+        const float dg1 = yr[1] ? warp_sum(p1) : 0.f;
+        gdot = fmaf(gates[t * k + j], dg0, gdot);
+        if (j == lane) my_dg0 = dg0;
+        if (j == lane + 32) my_dg1 = dg0;
+        if (j + 1 < k) {
+            gdot = fmaf(gates[t * k + j + 1], dg1, gdot);
+            if (j + 1 == lane) my_dg0 = dg1;
+            if (j + 1 == lane + 32) my_dg1 = dg1;
+        }
     }
     if (lane < k) dgate[t * k + lane] = my_dg0;
     if (lane + 32 < k) dgate[t * k + lane + 32] = my_dg1;
