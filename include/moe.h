@@ -302,9 +302,10 @@ MOE_API int moe_dispatch_static(const int64_t* selected, int64_t T, int32_t k, i
  * split-tf32 operands (x = hi + lo, three tf32 products per term, fp32
  * accumulation), which keeps fp32 accuracy; the split operands live in the
  * workspace.
- * Rows c >= rows(e) of ybuf are not written.  An always-on shared expert
- * ([P3] EducationalMoE) is this call with E = 1, C = T, used = NULL and the
- * token matrix as xbuf.
+ * Rows c >= rows(e) of ybuf are not written.  With C = 0 nothing is read or
+ * written (the buffer and weight pointers may then be NULL).  An always-on
+ * shared expert ([P3] EducationalMoE) is this call with E = 1, C = T,
+ * used = NULL and the token matrix as xbuf.
  *
  * Arguments:
  *   xbuf      device (E, C, D) contiguous, dtype `dtype`.

@@ -109,7 +109,7 @@ extern "C" int moe_expert_ffn_save(const void* xbuf, const int32_t* used, int32_
                                    int64_t Dout, const void* w_gate, const void* w_down, const void* w_up,
                                    void* ybuf, void* saved_ab, int32_t* dev_status, void* workspace,
                                    size_t workspace_bytes, moe_stream_t stream) {
-    MOE_REQUIRE(used != nullptr && saved_ab != nullptr, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(C == 0 || (used != nullptr && saved_ab != nullptr), MOE_ERR_INVALID_ARG);
     return expert_ffn(MOE_FFN_SWIGLU, MOE_BF16, xbuf, used, E, C, D, F, Dout, w_gate, nullptr, w_down, nullptr, w_up,
                       ybuf, saved_ab, dev_status, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -122,8 +122,9 @@ int expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32
                size_t workspace_bytes, cudaStream_t stream) {
     MOE_REQUIRE(valid_dtype(dtype), MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(kind == MOE_FFN_LINEAR || kind == MOE_FFN_GELU_MLP || kind == MOE_FFN_SWIGLU, MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(xbuf && ybuf && w1 && E >= 1 && C >= 0 && D >= 1 && Dout >= 1, MOE_ERR_INVALID_ARG);
-    if (C == 0) return MOE_OK;
+    MOE_REQUIRE(E >= 1 && C >= 0 && D >= 1 && Dout >= 1, MOE_ERR_INVALID_ARG);
+    if (C == 0) return MOE_OK;  // no rows: nothing is read or written
+    MOE_REQUIRE(xbuf && ybuf && w1, MOE_ERR_INVALID_ARG);
     if (kind == MOE_FFN_GELU_MLP) MOE_REQUIRE(b1 && w2 && b2 && F >= 1, MOE_ERR_INVALID_ARG);
     if (kind == MOE_FFN_SWIGLU) MOE_REQUIRE(w2 && w3 && F >= 1, MOE_ERR_INVALID_ARG);
     void* h = nullptr;
@@ -293,9 +294,9 @@ extern "C" int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const
                                        size_t workspace_bytes, moe_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     MOE_REQUIRE(kind == MOE_FFN_SWIGLU && dtype == MOE_BF16, MOE_ERR_UNSUPPORTED);
-    MOE_REQUIRE(x && token_of_slot && used && ybuf && w1 && w2 && w3, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(T >= 1 && ldx >= D && E >= 1 && C >= 0 && D >= 1 && F >= 1 && Dout >= 1, MOE_ERR_INVALID_ARG);
-    if (C == 0) return MOE_OK;
+    if (C == 0) return MOE_OK;  // no rows: nothing is read or written
+    MOE_REQUIRE(x && token_of_slot && used && ybuf && w1 && w2 && w3, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(workspace && workspace_bytes >= moe_expert_ffn_workspace_size(kind, dtype, E, C, D, F, Dout),
                 MOE_ERR_WORKSPACE);
     void* h = workspace;
