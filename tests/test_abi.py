@@ -139,3 +139,18 @@ def test_expert_parallel_host_checks():
     assert L.moe_ipc_export(nul, nul, nul) == B.MOE_ERR_INVALID_ARG
     assert L.moe_ipc_import(nul, nul) == B.MOE_ERR_INVALID_ARG
     assert L.moe_ipc_close(nul) == B.MOE_ERR_INVALID_ARG
+
+
+def test_expert_ffn_with_zero_capacity_touches_nothing():
+    # C = 0: nothing is read or written, so NULL buffers are accepted and no kernel is launched
+    L = moe.lib()
+    nul = None
+    for kind in (0, 1, 2):
+        for dtype in (B.MOE_F32, B.MOE_BF16):
+            rc = L.moe_expert_ffn(kind, dtype, nul, nul, 4, 0, 64, 32, 64, nul, nul, nul, nul, nul, nul, nul, nul, 0,
+                                  nul)
+            assert rc == B.MOE_OK, (kind, dtype)
+    assert L.moe_expert_ffn_save(nul, nul, 4, 0, 64, 32, 64, nul, nul, nul, nul, nul, nul, nul, 0, nul) == B.MOE_OK
+    # with rows to compute the buffers are required
+    rc = L.moe_expert_ffn(2, B.MOE_BF16, nul, nul, 4, 8, 64, 32, 64, nul, nul, nul, nul, nul, nul, nul, nul, 0, nul)
+    assert rc == B.MOE_ERR_INVALID_ARG
