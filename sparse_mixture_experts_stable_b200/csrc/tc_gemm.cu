@@ -3,10 +3,14 @@
 //
 // Warp roles in a 192-thread persistent CTA (one per SM):
 //   warp 0      : TMA producer (one lane), 4-stage smem ring
-//   warp 1      : TMEM allocator and MMA issuer (one lane)
-//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4) .. 32*(w%4)+31
+//   warp 1      : TMEM allocator and MMA issuer (lane 0 issues; the whole warp
+//                 clears the rows past a group's K in MN-major stages)
+//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4) .. 32*(w%4)+31 and
+//                 stores each 32 x 32 chunk row-contiguous through shared memory
 // The accumulator is double-buffered in TMEM (2 x 256 fp32 columns), so the
-// epilogue of one tile overlaps the main loop of the next.
+// epilogue of one tile overlaps the main loop of the next.  Operands are
+// K-major, or MN-major (B, and A with B) when K lies on the rows of the stored
+// matrix: 64 x 64 TMA boxes and MN-major shared-memory descriptors.
 //
 // Every wait on an mbarrier is bounded (kWaitLimitNs); on expiry the kernel
 // records MOE_ERR_TIMEOUT, every role leaves its loop, and TMEM is freed.
