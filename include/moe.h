@@ -623,6 +623,16 @@ MOE_API int moe_ipc_close(void* mapping);
 MOE_API int moe_transpose_weights(const void* src, void* dst, int32_t E, int64_t K_in, int64_t N_out,
                           moe_dtype dtype, moe_stream_t stream);
 
+/*
+ * moe_wait_probe -- the failure-detection path of the library's device-side
+ * waits (slot-scan look-back, GEMM pipeline barriers), on a flag the caller
+ * controls: one thread waits until the device word *flag becomes non-zero,
+ * or records MOE_ERR_TIMEOUT in dev_status once limit_ns nanoseconds have
+ * passed and returns, leaving the context usable.  0 < limit_ns <= 4e9.
+ *   flag, dev_status: device.
+ */
+MOE_API int moe_wait_probe(const uint32_t* flag, int64_t limit_ns, int32_t* dev_status, moe_stream_t stream);
+
 /* Set the device status word to MOE_OK (stream-ordered). */
 MOE_API int moe_clear_status(int32_t* dev_status, moe_stream_t stream);
 

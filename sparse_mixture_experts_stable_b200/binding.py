@@ -40,7 +40,7 @@ EXPORTED = [
     "moe_route_ex", "moe_renormalize_kept_gates", "moe_expert_ffn_gathered", "moe_backward_swiglu_workspace_size",
     "moe_backward_swiglu", "moe_router_backward_workspace_size", "moe_router_backward",
     "moe_backward_gelu_workspace_size", "moe_backward_gelu", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine",
-    "moe_ipc_export", "moe_ipc_import", "moe_ipc_close", "moe_expert_ffn_save",
+    "moe_ipc_export", "moe_ipc_import", "moe_ipc_close", "moe_expert_ffn_save", "moe_wait_probe",
 ]
 IPC_HANDLE_BYTES = 64
 SCORING = {"softmax": 0, "sigmoid": 1}
@@ -125,6 +125,7 @@ def lib():
         L.moe_ipc_import.argtypes = [_vp, ctypes.POINTER(_vp)]
         L.moe_ipc_close.argtypes = [_vp]
         L.moe_transpose_weights.argtypes = [_vp, _vp, _i32, _i64, _i64, ctypes.c_int, _vp]
+        L.moe_wait_probe.argtypes = [_vp, _i64, _vp, _vp]
         L.moe_clear_status.argtypes = [_vp, _vp]
         L.moe_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_i32)]
         _lib = L
@@ -641,6 +642,11 @@ def moe_transpose_weights(src: torch.Tensor, stream=None) -> torch.Tensor:
     rc = lib().moe_transpose_weights(_p(src.contiguous()), _p(dst), E, K, N, _dt(src), _stream(stream))
     _check("moe_transpose_weights", rc)
     return dst
+
+
+def moe_wait_probe(flag: torch.Tensor, limit_ns: int, dev_status: torch.Tensor, stream=None):
+    """Bounded device wait on ``flag`` (int32, device): MOE_ERR_TIMEOUT in dev_status after limit_ns."""
+    _check("moe_wait_probe", lib().moe_wait_probe(_p(flag), int(limit_ns), _p(dev_status), _stream(stream)))
 
 
 def moe_clear_status(dev_status: torch.Tensor, stream=None):

@@ -92,3 +92,33 @@ extern "C" int moe_read_status(const int32_t* dev_status, moe_stream_t stream, i
     MOE_CUDA_TRY(cudaMemcpy(host_status, dev_status, sizeof(int32_t), cudaMemcpyDeviceToHost));
     return MOE_OK;
 }
+
+// ---------------------------------------------------------------------------
+// moe_wait_probe: the library's bounded device wait, on a caller's flag
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+// One thread polls *flag (at most every microsecond) until it is non-zero or
+// limit_ns has passed on the global timer; in the second case it records
+// MOE_ERR_TIMEOUT and returns, as every wait inside the library does.
+__global__ void wait_probe_kernel(const volatile uint32_t* flag, uint64_t limit_ns, int32_t* status) {
+    if (blockIdx.x != 0 || threadIdx.x != 0) return;
+    const uint64_t t0 = globaltimer_ns();
+    while (*flag == 0u) {
+        if (globaltimer_ns() - t0 > limit_ns) {
+            set_status(status, MOE_ERR_TIMEOUT);
+            return;
+        }
+        __nanosleep(1000);
+    }
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_wait_probe(const uint32_t* flag, int64_t limit_ns, int32_t* dev_status, moe_stream_t stream) {
+    MOE_REQUIRE(flag && dev_status && limit_ns > 0 && (uint64_t)limit_ns <= kWaitLimitNs, MOE_ERR_INVALID_ARG);
+    wait_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(flag, (uint64_t)limit_ns, dev_status);
+    return launch_status();
+}

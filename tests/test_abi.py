@@ -154,3 +154,11 @@ def test_expert_ffn_with_zero_capacity_touches_nothing():
     # with rows to compute the buffers are required
     rc = L.moe_expert_ffn(2, B.MOE_BF16, nul, nul, 4, 8, 64, 32, 64, nul, nul, nul, nul, nul, nul, nul, nul, 0, nul)
     assert rc == B.MOE_ERR_INVALID_ARG
+
+
+def test_wait_probe_host_checks():
+    L = moe.lib()
+    p, nul = ctypes.c_void_p(16), None
+    assert L.moe_wait_probe(nul, 1000, p, nul) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_wait_probe(p, 0, p, nul) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_wait_probe(p, 5_000_000_000, p, nul) == B.MOE_ERR_INVALID_ARG  # above the library's wait bound
