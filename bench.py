@@ -14,7 +14,11 @@ N > 1 runs under torchrun, one rank per GPU, each rank on its own batch
 launch stream around every step, an L2 flush (a 256 MiB write) between steps,
 a barrier + synchronize on both sides of the timed loop, max over ranks.
 ``--impl reference`` times the fp64 CPU oracle on a bounded token sample of the
-same workload (rank 0 only).
+same workload (rank 0 only).  The JSON line also carries the other workloads
+(router only, top-1 dispatch/combine, tiny fp32 GELU layer and its training
+step, fp32 fwd+bwd, the expert-parallel step with 4 ranks on one GPU, and the
+full-layer training step); ``--workload NAME`` times one of them alone (with
+``--tokens/--experts`` for smaller full-layer shapes), for profiling captures.
 """
 from __future__ import annotations
 
