@@ -714,3 +714,137 @@ def test_module7_survivor_renormalisation():
     d2 = O.dispatch(sel2, 2, O.capacity(4, a["top_k"], 2, a["capacity_factor"]))
     r2 = O.renormalize_kept(gates2, d2["kept"])
     assert (r2[1:] == 0).all() and r2[0, 0] == 1.0
+
+
+# --------------------------------------------------------------------------
+# expert-major combine against the Dispatch page's one-hot contraction (step 6),
+# and the Module 7 single-expert / shared-expert invariants of EducationalMoE
+# --------------------------------------------------------------------------
+def _one_hot_tec(selected, slot, kept, E, C):
+    """The Dispatch page's (T, E, C) address tensor: 1 where token t sits in expert e at slot c."""
+    T, k = selected.shape
+    disp = np.zeros((T, E, C))
+    for t in range(T):
+        for j in range(k):
+            if kept[t, j]:
+                disp[t, selected[t, j], slot[t, j]] = 1.0
+    return disp
+
+
+@pytest.mark.parametrize("seed", range(3))
+@pytest.mark.parametrize("base", ["zero", "input", "tensor"])
+def test_combine_slots_equals_dispatch_page_einsum(seed, base):
+    rng = np.random.default_rng(900 + seed)
+    T, E, k, N = 23, 5, 2, 6
+    C = O.capacity(T, k, E, 0.7)  # tight capacity: drops occur
+    x = rng.standard_normal((T, N))
+    s = rng.standard_normal((T, E))
+    _, sel, gates, _, _ = O.route(s, k)
+    d = O.dispatch(sel, E, C)
+    assert (~d["kept"]).any() and d["kept"].any()
+    disp = _one_hot_tec(sel, d["slot"], d["kept"], E, C)
+    # the page's gather: expert_inputs = einsum("tec,td->ecd", dispatch, x) equals the rows that
+    # the inverse map names; empty slots are all zero
+    xbuf = np.einsum("tec,td->ecd", disp, x)
+    for e in range(E):
+        for c in range(C):
+            t = d["token_of_slot"][e, c]
+            np.testing.assert_array_equal(xbuf[e, c], x[t] if t >= 0 else np.zeros(N))
+    # expert outputs, with the empty slots holding values that must never be read
+    ybuf = rng.standard_normal((E, C, N))
+    ybuf[d["token_of_slot"] < 0] = 1e6
+    comb = disp * np.einsum("tj,tje->tje", gates, np.eye(E)[sel]).sum(1)[:, :, None]
+    want = np.einsum("tec,ecd->td", comb, ybuf)
+    base_t = {"zero": None, "input": x, "tensor": rng.standard_normal((T, N))}[base]
+    if base_t is not None:
+        want = want + base_t
+    got = O.combine_slots(ybuf, sel, d["slot"], d["kept"], gates, base=base_t)
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
+    # dropped-everywhere tokens get exactly the base row (the page: all-zero dispatch row)
+    full = np.flatnonzero(d["drops"] == k)
+    for t in full:
+        np.testing.assert_array_equal(got[t], np.zeros(N) if base_t is None else base_t[t])
+
+
+def test_combine_slots_hand_worked_two_tokens():
+    # T=2, E=2, k=2, C=1. Token 0 ranks [0, 1] and takes slot 0 of both experts; token 1 ranks
+    # [1, 0] and finds both experts full, so it keeps only its base row.
+    s = np.array([[1.0, 0.0], [0.0, 1.0]])
+    _, sel, gates, _, _ = O.route(s, 2)
+    d = O.dispatch(sel, 2, 1)
+    assert sel.tolist() == [[0, 1], [1, 0]]
+    assert d["kept"].tolist() == [[True, True], [False, False]]
+    ybuf = np.array([[[2.0, -1.0]], [[4.0, 3.0]]])  # (E=2, C=1, N=2)
+    base = np.array([[0.5, 0.25], [-7.0, 9.0]])
+    g0 = math.e / (1.0 + math.e)  # softmax([1, 0])[0]
+    want0 = base[0] + g0 * np.array([2.0, -1.0]) + (1.0 - g0) * np.array([4.0, 3.0])
+    got = O.combine_slots(ybuf, sel, d["slot"], d["kept"], gates, base=base)
+    np.testing.assert_allclose(got[0], want0, rtol=1e-15)
+    np.testing.assert_array_equal(got[1], base[1])
+
+
+def test_combine_slots_identity_expert_equals_layer():
+    # with the identity as every expert, expert-major combine of the dispatched rows equals the
+    # token-major layer sum  base + sum_kept gate * x_t
+    rng = np.random.default_rng(31)
+    T, E, k, D = 17, 4, 2, 5
+    x = rng.standard_normal((T, D))
+    _, sel, gates, _, _ = O.route(rng.standard_normal((T, E)), k)
+    C = O.capacity(T, k, E, 0.8)
+    d = O.dispatch(sel, E, C)
+    xbuf = np.zeros((E, C, D))
+    for e in range(E):
+        for c in range(C):
+            if d["token_of_slot"][e, c] >= 0:
+                xbuf[e, c] = x[d["token_of_slot"][e, c]]
+    eye = np.tile(np.eye(D), (E, 1, 1))
+    want = O.layer_rows("linear", x, sel, d["kept"], gates, {"w1": eye}, base_kind="input")
+    got = O.combine_slots(xbuf, sel, d["slot"], d["kept"], gates, base=x)
+    np.testing.assert_allclose(got, want, rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(want, x * (1.0 + (gates * d["kept"]).sum(1))[:, None], rtol=1e-14)
+
+
+def _swiglu_np(x, g, u, dn):
+    """Module 7 swiglu_expert written out: (a * sigmoid(a) * b) @ down with a = x@g, b = x@u."""
+    a, b = x @ g, x @ u
+    return (a / (1.0 + np.exp(-a)) * b) @ dn
+
+
+def test_module7_single_expert_and_shared_expert_invariants():
+    # The invariant cell after EducationalMoE: one routed expert with k=1 is the dense SwiGLU
+    # expert (atol 1e-12 as on the page); an always-on shared expert adds its own output.
+    rng = np.random.default_rng(60)
+    H, I, T = 8, 12, 16
+    x = rng.standard_normal((T, H))
+    router_w = rng.standard_normal((H, 1)) / math.sqrt(H)
+    gate = rng.standard_normal((1, H, I)) / math.sqrt(H)
+    up = rng.standard_normal((1, H, I)) / math.sqrt(H)
+    down = rng.standard_normal((1, I, H)) / math.sqrt(I)
+    w = {"w1": gate, "w3": up, "w2": down}
+    s = O.router_logits(x, router_w)
+    out = O.forward("swiglu", x, s, 1, T, w, base_kind="zero")
+    dense = _swiglu_np(x, gate[0], up[0], down[0])
+    np.testing.assert_allclose(out["y"], dense, rtol=0, atol=1e-12)
+    sg = rng.standard_normal((1, H, I)) / math.sqrt(H)
+    su = rng.standard_normal((1, H, I)) / math.sqrt(H)
+    sd = rng.standard_normal((1, I, H)) / math.sqrt(I)
+    shared = _swiglu_np(x, sg[0], su[0], sd[0])
+    y = O.layer_rows("swiglu", x, out["selected"], out["kept"], out["gates"], w, base_kind="tensor",
+                     base=shared)
+    np.testing.assert_allclose(y, dense + shared, rtol=0, atol=1e-12)
+    # a subset of tokens in scrambled order reads each token's own base row
+    toks = rng.permutation(T)[:7]
+    ys = O.layer_rows("swiglu", x, out["selected"], out["kept"], out["gates"], w, base_kind="tensor",
+                      base=shared, tokens=toks)
+    np.testing.assert_allclose(ys, (dense + shared)[toks], rtol=0, atol=1e-12)
+    # the shared expert computed by the oracle's own expert path is the same function
+    sh = O.expert_rows("swiglu", x, np.arange(T), np.zeros(T, np.int64), {"w1": sg, "w3": su, "w2": sd})
+    np.testing.assert_allclose(sh, shared, rtol=0, atol=1e-12)
+    # with drops (capacity 5 of 16 tokens), dropped tokens keep exactly the shared row
+    d = O.dispatch(out["selected"], 1, 5)
+    yd = O.layer_rows("swiglu", x, out["selected"], d["kept"], out["gates"], w, base_kind="tensor",
+                      base=shared)
+    dropped = np.flatnonzero(~d["kept"][:, 0])
+    assert len(dropped) == T - 5
+    np.testing.assert_array_equal(yd[dropped], shared[dropped])
+    np.testing.assert_allclose(yd[:5], (dense + shared)[:5], rtol=0, atol=1e-12)
