@@ -60,6 +60,7 @@ extern "C" {
 #endif
 
 typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+typedef struct CUevent_st* moe_event_t;   /* identical to cudaEvent_t */
 
 typedef enum {
     MOE_OK = 0,
@@ -272,8 +273,11 @@ MOE_API int moe_dispatch(const int64_t* selected, int64_t T, int32_t k, int32_t 
  * the array (E = 256 allows T <= 524160); a larger problem returns
  * MOE_ERR_UNSUPPORTED and enqueues nothing.
  * Set-up: the first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.
+ * (cudaGetSymbolAddress) with that device current and keeps it for the life
+ * of the process; make that first call before any stream capture.  A device
+ * reset (cudaDeviceReset, or anything else that destroys the device's primary
+ * context) makes the kept address stale: do not call this entry point on that
+ * device after such a reset.
  * Sharing: all calls on a device use the same array; each call clears, in
  * stream order, the part it uses before the scan, so a later call never sees
  * an earlier call's state.  Calls that can overlap on the GPU (different
@@ -406,6 +410,75 @@ MOE_API int moe_combine(const void* ybuf, const int64_t* selected, const int64_t
 MOE_API int moe_aux_stats(const int32_t* counts, const float* prob_sum, int64_t T, int32_t E, int32_t k,
                   int normalize_by_k, float aux_coef, void* f, void* P, moe_dtype out_dtype,
                   float* aux, moe_stream_t stream);
+
+/*
+ * moe_swiglu_layer_forward -- the whole layer forward in one call: [P3]
+ * EducationalMoE with SwiGLU routed experts and an optional always-on shared
+ * SwiGLU expert, softmax router with a per-expert logit bias ([P2] problem
+ * statement), capacity-limited greedy dispatch ([P1] section 2
+ * position_priority_dispatch), gate-weighted combine onto the shared output
+ * ([P2] y = shared + sum), and the load statistics with the Switch aux loss.
+ * It runs moe_route, moe_dispatch, moe_expert_ffn (routed, and shared on the
+ * side stream), moe_combine and moe_aux_stats on buffers carved from one
+ * workspace; the results equal that sequence of calls exactly.
+ *
+ * Layer description (all weights device bf16, (out, in) layout):
+ *   T, H          tokens and hidden size; E experts, k per token, C capacity
+ *                 (moe_capacity; 0 drops everything), F / F_shared the routed
+ *                 and shared intermediate sizes (F_shared = 0: no shared
+ *                 expert, y = sum of the gated outputs).
+ *   w_router (E, H); router_bias fp32 (E) or NULL; w_gate, w_up (E, F, H);
+ *   w_down (E, H, F); s_gate, s_up (1, F_shared, H); s_down (1, H, F_shared).
+ *   aux_coef      scales aux[1].
+ *
+ * Arguments:
+ *   x     (T, H) bf16, contiguous: device memory, or host memory (pinned for
+ *         an asynchronous copy) that the call copies into the workspace with
+ *         one cudaMemcpyAsync on copy_in_stream.
+ *   y     (T, H) bf16 output, device or host; a host y is copied back with one
+ *         cudaMemcpyAsync on copy_out_stream after the layer.
+ *   aux   fp32 (2): {aux loss, aux_coef * aux loss}, device or host, or NULL.
+ *   dev_status   device status word or NULL (as for the calls above).
+ *   workspace    device, >= moe_swiglu_layer_workspace_size(L) bytes.  It
+ *         holds the device copies of x and y, every routing and dispatch
+ *         output and the expert buffers; the call owns it until it is done.
+ *   stream       the layer's kernels; side_stream (or NULL: stream) the
+ *         shared expert; copy_in_stream / copy_out_stream (or NULL: stream)
+ *         the host copies.
+ *   x_free, y_free  cudaEvent_t handles or NULL, one pair per workspace.
+ *         x_free: the call waits for it before its first use of the workspace
+ *         (the copy-in of a host x, else the first kernel) and records it on
+ *         `stream` after its last kernel.  y_free: before writing the y
+ *         staging of a host y the call waits for it, and records it after the
+ *         copy-out.  With two workspaces used in turn, each with its own pair,
+ *         one batch's copy-in, the previous batch's copy-out and the kernels
+ *         in between overlap.  When x_free is NULL, a host copy-in waits for
+ *         all work already on `stream`.
+ * Results: with host outputs, y and aux are complete when copy_out_stream
+ * (or `stream`) reaches the end of the call's work; synchronise it (or the
+ * event) before reading them.  Returns MOE_ERR_WORKSPACE / _INVALID_ARG /
+ * _UNSUPPORTED / _CUDA for host-detected problems, nothing enqueued then
+ * except possibly the copy-in.
+ */
+typedef struct moe_swiglu_layer {
+    int64_t T, H, F, F_shared, C;
+    int32_t E, k;
+    float aux_coef;
+    const void* w_router;
+    const float* router_bias;
+    const void* w_gate;
+    const void* w_up;
+    const void* w_down;
+    const void* s_gate;
+    const void* s_up;
+    const void* s_down;
+} moe_swiglu_layer;
+
+MOE_API size_t moe_swiglu_layer_workspace_size(const moe_swiglu_layer* L);
+MOE_API int moe_swiglu_layer_forward(const moe_swiglu_layer* L, const void* x, void* y, float* aux,
+                                     int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                                     moe_stream_t stream, moe_stream_t side_stream, moe_stream_t copy_in_stream,
+                                     moe_stream_t copy_out_stream, moe_event_t x_free, moe_event_t y_free);
 
 /*
  * moe_backward -- backward of the linear-expert layer, the kept mask and the

@@ -11,5 +11,5 @@ from .binding import (  # noqa: F401
     moe_capacity, moe_clear_status, moe_combine, moe_dispatch, moe_dispatch_static, moe_ep_combine, moe_ep_dispatch,
     moe_ep_plan, moe_expert_ffn, moe_expert_ffn_gathered, moe_expert_ffn_save, moe_ipc_close, moe_ipc_export, moe_ipc_import,
     moe_read_status, moe_renormalize_kept_gates, moe_route, moe_router_backward, moe_transpose_weights, new_status,
-    status_string,
+    status_string, moe_swiglu_layer_forward, moe_swiglu_layer_workspace_size, SwiGLULayerDesc,
 )

@@ -41,9 +41,20 @@ EXPORTED = [
     "moe_backward_swiglu", "moe_router_backward_workspace_size", "moe_router_backward",
     "moe_backward_gelu_workspace_size", "moe_backward_gelu", "moe_ep_plan", "moe_ep_dispatch", "moe_ep_combine",
     "moe_ipc_export", "moe_ipc_import", "moe_ipc_close", "moe_expert_ffn_save", "moe_wait_probe",
+    "moe_swiglu_layer_workspace_size", "moe_swiglu_layer_forward",
 ]
 IPC_HANDLE_BYTES = 64
 SCORING = {"softmax": 0, "sigmoid": 1}
+
+
+class SwiGLULayerDesc(ctypes.Structure):
+    """``moe_swiglu_layer`` of include/moe.h (sizes and device weight pointers)."""
+
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int64), ("F", ctypes.c_int64), ("F_shared", ctypes.c_int64),
+                ("C", ctypes.c_int64), ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("aux_coef", ctypes.c_float),
+                ("w_router", ctypes.c_void_p), ("router_bias", ctypes.c_void_p), ("w_gate", ctypes.c_void_p),
+                ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p), ("s_gate", ctypes.c_void_p),
+                ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p)]
 
 
 class MoeError(RuntimeError):
@@ -126,6 +137,10 @@ def lib():
         L.moe_ipc_close.argtypes = [_vp]
         L.moe_transpose_weights.argtypes = [_vp, _vp, _i32, _i64, _i64, ctypes.c_int, _vp]
         L.moe_wait_probe.argtypes = [_vp, _i64, _vp, _vp]
+        L.moe_swiglu_layer_workspace_size.restype = _sz
+        L.moe_swiglu_layer_workspace_size.argtypes = [ctypes.POINTER(SwiGLULayerDesc)]
+        L.moe_swiglu_layer_forward.argtypes = [ctypes.POINTER(SwiGLULayerDesc), _vp, _vp, _vp, _vp, _vp, _sz, _vp,
+                                               _vp, _vp, _vp, _vp, _vp]
         L.moe_clear_status.argtypes = [_vp, _vp]
         L.moe_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_i32)]
         _lib = L
@@ -642,6 +657,40 @@ def moe_transpose_weights(src: torch.Tensor, stream=None) -> torch.Tensor:
     rc = lib().moe_transpose_weights(_p(src.contiguous()), _p(dst), E, K, N, _dt(src), _stream(stream))
     _check("moe_transpose_weights", rc)
     return dst
+
+
+def moe_swiglu_layer_workspace_size(desc: SwiGLULayerDesc) -> int:
+    return int(lib().moe_swiglu_layer_workspace_size(ctypes.byref(desc)))
+
+
+def moe_swiglu_layer_forward(desc: SwiGLULayerDesc, x: torch.Tensor, y: torch.Tensor, aux: Optional[torch.Tensor],
+                             workspace: torch.Tensor, dev_status: Optional[torch.Tensor] = None, stream=None,
+                             side_stream=None, copy_in_stream=None, copy_out_stream=None,
+                             x_free: Optional[torch.cuda.Event] = None, y_free: Optional[torch.cuda.Event] = None):
+    """The whole SwiGLU layer forward in one C call; x, y and aux may be host (pinned) or device tensors."""
+    if x.dtype != torch.bfloat16 or y.dtype != torch.bfloat16 or not x.is_contiguous() or not y.is_contiguous():
+        raise TypeError("x and y must be contiguous bf16")
+    if tuple(x.shape) != (desc.T, desc.H) or tuple(y.shape) != (desc.T, desc.H):
+        raise ValueError("x and y must be (T, H)")
+    if aux is not None and (aux.dtype != torch.float32 or aux.numel() < 2):
+        raise TypeError("aux must hold two fp32 values")
+    nbytes = workspace.numel() * workspace.element_size()
+
+    def st(s):
+        return None if s is None else ctypes.c_void_p(s.cuda_stream)
+
+    def ev(e):
+        if e is None:
+            return None
+        if not e.cuda_event:  # PyTorch creates the CUDA event at its first record
+            e.record()
+        return ctypes.c_void_p(e.cuda_event)
+
+    rc = lib().moe_swiglu_layer_forward(ctypes.byref(desc), _p(x), _p(y), _p(aux), _p(dev_status), _p(workspace),
+                                        nbytes, _stream(stream), st(side_stream), st(copy_in_stream),
+                                        st(copy_out_stream), ev(x_free), ev(y_free))
+    _check("moe_swiglu_layer_forward", rc)
+    return y
 
 
 def moe_wait_probe(flag: torch.Tensor, limit_ns: int, dev_status: torch.Tensor, stream=None):

@@ -42,6 +42,10 @@ size_t fp32_split_bytes(moe_ffn_kind kind, int32_t E, int64_t C, int64_t D, int6
 
 }  // namespace
 
+namespace {
+constexpr size_t kTileCounterBytes = 256;  // after the intermediate h: scratch words of the wide GEMMs' schedulers
+}
+
 extern "C" size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dtype, int32_t E, int64_t C, int64_t D,
                                                 int64_t F, int64_t Dout) {
     if (E < 1 || C < 1) return 0;
@@ -49,15 +53,41 @@ extern "C" size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dty
     if (kind != MOE_FFN_LINEAR && F >= 1) h = align_up((size_t)E * C * F * dtype_size(dtype), 1024);
     if (dtype == MOE_F32 && D >= 1 && Dout >= 1 && (kind == MOE_FFN_LINEAR || F >= 1))
         return h + fp32_split_bytes(kind, E, C, D, F, Dout);
+    if (kind == MOE_FFN_SWIGLU && F >= 1) h += kTileCounterBytes;  // tile counters of the wide GEMMs
     return h;
 }
 
 namespace {
 
-// Second GEMM of the bf16 MLP experts: ybuf = h (E*C, F) x W2^T (+ b2).
+// Second GEMM of the bf16 MLP experts: ybuf = h (E*C, F) x W2^T (+ b2).  tile_counter:
+// a device word of scratch for the routed SwiGLU form (tcw_gemm_run).
 int down_projection(moe_ffn_kind kind, const void* h, const int32_t* used, int32_t E, int64_t C, int64_t F,
                     int64_t Dout, const void* w2, const void* b2, void* ybuf, int32_t* dev_status,
-                    cudaStream_t stream) {
+                    cudaStream_t stream, uint32_t* tile_counter = nullptr) {
+    if (kind == MOE_FFN_SWIGLU && used != nullptr) {
+        // routed experts: 256 output features x up to 256 tokens per tile (tc_wide_gemm.cu)
+        TcxProblem p{};
+        p.w = w2;
+        p.ldw = F;
+        p.w_rows_total = (int64_t)E * Dout;
+        p.w_rows_per_group = Dout;
+        p.x = h;
+        p.ldx = F;
+        p.x_rows_total = (int64_t)E * C;
+        p.x_rows_per_group = C;
+        p.G = E;
+        p.features = Dout;
+        p.max_tokens = C;
+        p.K = F;
+        p.rows = used;
+        p.out = ybuf;
+        p.ldo = Dout;
+        p.out_rows_per_group = C;
+        p.epilogue = TC_EPI_BF16;
+        p.status = dev_status;
+        p.tile_counter = tile_counter;
+        return tcw_gemm_run(p, stream);
+    }
     TcGemmProblem q{};
     q.a = h;
     q.lda = F;
@@ -138,10 +168,10 @@ int expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32
 
     if (dtype == MOE_BF16) {
         // Kernel choice (measured on B200): the SwiGLU gate/up GEMM over ragged
-        // experts runs with weights on the MMA's M side (tcx_gemm_run: at most
-        // 15 padded token rows per expert); every other bf16 GEMM runs with
-        // token rows on the M side and a single N=256 weight operand
-        // (tc_gemm_run), which reads the fewest shared-memory operand bytes.
+        // experts runs with weights on the MMA's M side and up to 256 tokens on N
+        // (tcw_gemm_run: at most 15 padded token rows per expert, and the fewest
+        // operand bytes per FLOP through the TMA); every other bf16 GEMM runs with
+        // token rows on the M side and a single N=256 weight operand (tc_gemm_run).
         int rc;
         if (kind == MOE_FFN_SWIGLU && used != nullptr) {
             TcxProblem p{};
@@ -166,7 +196,8 @@ int expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32
             p.status = dev_status;
             p.save_ab = saved_ab;
             p.ld_save = 2 * F;
-            rc = tcx_gemm_run(p, stream);
+            p.tile_counter = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + h_bytes);
+            rc = tcw_gemm_run(p, stream);
         } else {
             // first GEMM: xbuf (E*C, D) x W^T
             TcGemmProblem p{};
@@ -210,7 +241,11 @@ int expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32
             rc = tc_gemm_run(p, stream);
         }
         if (rc != MOE_OK) return rc;
-        return down_projection(kind, h, used, E, C, F, Dout, w2, b2, ybuf, dev_status, stream);
+        uint32_t* counters = kind == MOE_FFN_SWIGLU
+                                 ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + h_bytes)
+                                 : nullptr;
+        return down_projection(kind, h, used, E, C, F, Dout, w2, b2, ybuf, dev_status, stream,
+                               counters ? counters + 1 : nullptr);
     }
 
     // fp32: split-tf32 tensor-core GEMMs, B = weights in (out, in) layout -> transposed operand
@@ -324,5 +359,7 @@ extern "C" int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const
     p.status = dev_status;
     const int rc = tcx_gemm_run(p, stream);
     if (rc != MOE_OK) return rc;
-    return down_projection(kind, h, used, E, C, F, Dout, w2, nullptr, ybuf, dev_status, stream);
+    uint32_t* counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) +
+                                                     align_up((size_t)E * C * F * 2, 1024));
+    return down_projection(kind, h, used, E, C, F, Dout, w2, nullptr, ybuf, dev_status, stream, counters + 1);
 }

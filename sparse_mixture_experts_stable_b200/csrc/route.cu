@@ -10,6 +10,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "route_fused.cuh"
 #include "route_scores.cuh"
 #include "f32_gemm.cuh"
 #include "tc_gemm.cuh"
@@ -384,6 +385,28 @@ extern "C" int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D
     const int epl = epl_for(E);
     const int gates_bf16 = dtype == MOE_BF16;
     int rc = MOE_OK;
+    int nb = topk_grid(T);
+
+    // bf16 softmax router without the variants: scores, softmax, top-k and gates in one kernel
+    if (has_w && dtype == MOE_BF16 && sc == 0 && selection_bias == nullptr && z_loss == nullptr &&
+        (logits_out == nullptr || aligned16(logits_out))) {
+        const void* w_ed = w_router;
+        if (layout == MOE_ROUTER_DE) w_ed = ws + wl.wt_off;
+        if (route_fused_supported(T, D, ldx, x, w_ed, E, k)) {
+            if (layout == MOE_ROUTER_DE) {
+                rc = transpose_matrices(w_router, ws + wl.wt_off, 1, D, E, MOE_BF16, stream);
+                if (rc != MOE_OK) return rc;
+            }
+            rc = route_fused_run(x, T, D, ldx, w_ed, E, logit_bias, k, logits_out, selected, gates, gates_bf16,
+                                 gates_f32, part_counts, part_psum, dev_status, stream);
+            if (rc != MOE_OK) return rc;
+            nb = route_fused_grid(T);
+            route_reduce_kernel<<<(E + 31) / 32, kReduceWarps * 32, 0, stream>>>(part_counts, part_psum, nb, E,
+                                                                                 counts, prob_sum, nullptr, T,
+                                                                                 nullptr);
+            return launch_status();
+        }
+    }
 
     if (has_w) {
         // scores s = x . W (+ bias) into fp32 logits
@@ -450,7 +473,6 @@ extern "C" int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D
                                 dev_status, stream);
     }
     if (rc != MOE_OK) return rc;
-    const int nb = topk_grid(T);
     route_reduce_kernel<<<(E + 31) / 32, kReduceWarps * 32, 0, stream>>>(part_counts, part_psum, nb, E, counts,
                                                                          prob_sum, part_z, T, z_loss);
     return launch_status();

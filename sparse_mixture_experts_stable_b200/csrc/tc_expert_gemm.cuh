@@ -39,10 +39,16 @@ struct TcxProblem {
     // like out: a (gate) at column f, b (up) at column features + f, row stride ld_save.
     void* save_ab;
     int64_t ld_save;
+    // tcw_gemm_run only: one device word of scratch for its tile counter (zeroed by the call, in stream order)
+    uint32_t* tile_counter;
 };
 
 // Single-CTA kernel: 256 weight rows x up to 128 tokens per tile.
 int tcx_gemm_run(const TcxProblem& p, cudaStream_t stream);
+
+// SwiGLU gate/up (TC_EPI_SWIGLU) without gathered rows: 128 features (gate and
+// up) x up to 256 tokens per tile, single-buffered TMEM (tc_wide_gemm.cu).
+int tcw_gemm_run(const TcxProblem& p, cudaStream_t stream);
 
 
 }  // namespace moe

@@ -107,3 +107,40 @@ class SwiGLUMoE:
         f, P, aux = B.moe_aux_stats(r["counts"], r["prob_sum"], self.T, self.k, True, self.aux_coef,
                                     out_dtype=self.dtype)
         return dict(y=self.y, f=f, P=P, aux=aux, **r, **d)
+
+
+class SwiGLULayer:
+    """The same layer as SwiGLUMoE through the single C call moe_swiglu_layer_forward.
+
+    Holds the layer description (sizes and device weight pointers) and one
+    workspace per in-flight batch; ``forward`` accepts x and y on the device or
+    in (pinned) host memory, in which case the library does the copies.
+    """
+
+    def __init__(self, T: int, H: int, E: int, F: int, k: int, capacity_factor: float, w_router, router_bias, w_gate,
+                 w_up, w_down, s_gate=None, s_up=None, s_down=None, aux_coef: float = 0.0, n_workspaces: int = 1,
+                 device="cuda"):
+        self.C = B.moe_capacity(T, k, E, capacity_factor)
+        F_shared = 0 if s_gate is None else int(s_gate.shape[1])
+        self._keep = [w_router, router_bias, w_gate, w_up, w_down, s_gate, s_up, s_down]
+        d = B.SwiGLULayerDesc()
+        d.T, d.H, d.F, d.F_shared, d.C, d.E, d.k, d.aux_coef = T, H, F, F_shared, self.C, E, k, aux_coef
+        for name, t in (("w_router", w_router), ("router_bias", router_bias), ("w_gate", w_gate), ("w_up", w_up),
+                        ("w_down", w_down), ("s_gate", s_gate), ("s_up", s_up), ("s_down", s_down)):
+            setattr(d, name, None if t is None else t.data_ptr())
+        self.desc = d
+        nbytes = B.moe_swiglu_layer_workspace_size(d)
+        if nbytes == 0:
+            raise ValueError("invalid layer description")
+        self.workspaces = [torch.empty(nbytes, dtype=torch.uint8, device=device) for _ in range(n_workspaces)]
+        self.x_free = [torch.cuda.Event() for _ in range(n_workspaces)]
+        self.y_free = [torch.cuda.Event() for _ in range(n_workspaces)]
+        self.status = B.new_status(device)
+
+    def forward(self, x, y, aux=None, slot: int = 0, stream=None, side_stream=None, copy_in_stream=None,
+                copy_out_stream=None):
+        """Enqueue one batch on workspace ``slot``; returns y (complete once the copy-out stream gets there)."""
+        return B.moe_swiglu_layer_forward(self.desc, x, y, aux, self.workspaces[slot], dev_status=self.status,
+                                          stream=stream, side_stream=side_stream, copy_in_stream=copy_in_stream,
+                                          copy_out_stream=copy_out_stream, x_free=self.x_free[slot],
+                                          y_free=self.y_free[slot])

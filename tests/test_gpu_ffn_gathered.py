@@ -1,6 +1,10 @@
 """moe_expert_ffn_gathered: SwiGLU experts reading their rows from x through
-token_of_slot, against the gather + moe_expert_ffn path (bit for bit: the same
-tensor-core products over the same row values) and the fp64 oracle.
+token_of_slot, against the gather + moe_expert_ffn path and the fp64 oracle.
+
+The two paths run different gate/up kernels (the gathered one fills its token
+tiles with cp.async, 128 tokens per tile; the other takes 256-token tiles
+through TMA and a faster SiLU exponential), so they agree to the bf16
+tolerance, not bit for bit.
 
 Shapes cover ragged experts (empty, one row, exactly one tile, full C), a K
 tail (D not a multiple of 64), several tiles per expert and the full-layer
@@ -52,7 +56,7 @@ def test_gathered_matches_gather_then_ffn(T, D, E, k, cf):
     used = d["used"].cpu().tolist()
     for e in range(E):
         u = used[e]
-        assert torch.equal(got[e, :u], ref[e, :u]), f"expert {e}"
+        assert_close(cpu64(got[e, :u]), cpu64(ref[e, :u]), BF16_RTOL, BF16_ATOL, f"expert {e}")
         # rows past used stay untouched
         assert torch.isnan(got[e, u:].float()).all()
     # against the oracle on the rows the dispatch chose
@@ -95,4 +99,4 @@ def test_gathered_full_layer_size_sampled():
     assert moe.moe_read_status(st) == 0
     used = d["used"].cpu().tolist()
     for e in range(E):
-        assert torch.equal(got[e, :used[e]], ref[e, :used[e]]), f"expert {e}"
+        assert_close(cpu64(got[e, :used[e]]), cpu64(ref[e, :used[e]]), BF16_RTOL, BF16_ATOL, f"expert {e}")

@@ -81,28 +81,75 @@ def test_dispatch_combine_top1_linear_bf16(full_size):
     assert_close(yc[sample], want, BF16_RTOL, BF16_ATOL, "top-1 y")
 
 
-def _swiglu_oracle_rows(cfg, o, tokens, shared_rows):
-    """Oracle y for the listed tokens, with only the experts those tokens use."""
-    ys = []
+def _expert_weights64(cfg, e, prefix="w"):
+    """One expert's SwiGLU weights in the pages' x @ W layout (float64)."""
+    sl = slice(e, e + 1)
+    return {"w1": pages_layout(cfg[prefix + "_gate"][sl]), "w3": pages_layout(cfg[prefix + "_up"][sl]),
+            "w2": pages_layout(cfg[prefix + "_down"][sl])}
+
+
+def _check_swiglu_layer(cfg, out, sel, kept, gates, token_of_slot, used, tokens, experts):
+    """Compare the GPU's expert outputs and layer output with the oracle.
+
+    ``experts``: every kept row of these experts is compared in the expert-major
+    output buffer.  ``tokens``: y of these tokens is compared; the oracle forms
+    each kept (token, expert) output and combines them with the gates and the
+    shared-expert row.  The oracle converts each expert's weights once.
+    """
+    x64 = cpu64(cfg["x"])
+    k = sel.shape[1]
+    H = x64.shape[1]
+    ybuf = out["ybuf"]
+    pairs = {}  # expert -> list of (position in tokens, j)
     for i, t in enumerate(tokens):
-        sel = o["selected"][t]
-        idx = torch.from_numpy(sel)
-        sub = {
-            "w1": pages_layout(cfg["w_gate"][idx]),
-            "w3": pages_layout(cfg["w_up"][idx]),
-            "w2": pages_layout(cfg["w_down"][idx]),
-        }
-        ys.append(O.layer_rows("swiglu", cpu64(cfg["x"][t:t + 1]), np.arange(len(sel))[None], o["kept"][t][None],
-                               o["gates"][t][None], sub, base_kind="tensor", base=shared_rows[i:i + 1])[0])
-    return np.stack(ys)
+        for j in range(k):
+            if kept[t, j]:
+                pairs.setdefault(int(sel[t, j]), []).append((i, j))
+    u = np.zeros((len(tokens), k, H))
+    for e in sorted(set(pairs) | set(int(e) for e in experts)):
+        w = _expert_weights64(cfg, e)
+        if e in experts and used[e]:
+            rows = token_of_slot[e, :used[e]]
+            want = O.expert_rows("swiglu", x64, rows, np.zeros(len(rows), np.int64), w)
+            assert_close(cpu64(ybuf[e, :used[e]]), want, BF16_RTOL, BF16_ATOL, f"ybuf rows of expert {e}")
+        if e in pairs:
+            ij = pairs[e]
+            toks = np.array([tokens[i] for i, _ in ij], np.int64)
+            rows = O.expert_rows("swiglu", x64, toks, np.zeros(len(toks), np.int64), w)
+            for (i, j), r in zip(ij, rows):
+                u[i, j] = r
+    shared = O.expert_rows("swiglu", x64, tokens, np.zeros(len(tokens), np.int64), _expert_weights64(cfg, 0, "s"))
+    local = np.tile(np.arange(k), (len(tokens), 1))
+    want_y = O.combine_precomputed(u, local, kept[tokens], gates[tokens], base=shared)
+    assert_close(cpu64(out["y"])[tokens], want_y, BF16_RTOL, BF16_ATOL, "swiglu y")
+    return want_y
 
 
-@pytest.mark.parametrize("full_size,gathered", [(False, False), (False, True), (True, False), (True, True)])
-def test_full_swiglu_layer_bf16(full_size, gathered):
+def _unit_scale(cfg):
+    """Expert weights rescaled so that gate/up pre-activations and expert outputs are O(1):
+    then |y| is about 1 and the stated atol would catch one missing expert term."""
+    c = dict(cfg)
+    xs = float(cfg["x"].float().std())
+    H, F = cfg["H"], cfg["F"]
+    for pre, f_in in (("w", F), ("s", cfg["F_shared"])):
+        for n in ("_gate", "_up"):
+            t = cfg[pre + n].float()
+            c[pre + n] = (t * (H ** -0.5 / xs / float(t.std()))).to(torch.bfloat16)
+        t = cfg[pre + "_down"].float()
+        c[pre + "_down"] = (t * (f_in ** -0.5 / float(t.std()))).to(torch.bfloat16)
+    return c
+
+
+@pytest.mark.parametrize("full_size,gathered,unit", [(False, False, False), (False, True, False),
+                                                     (True, False, False), (True, True, False),
+                                                     (True, False, True)])
+def test_full_swiglu_layer_bf16(full_size, gathered, unit):
     if full_size:
         cfg = I.full_layer_bf16(seed=0)
     else:
         cfg = I.full_layer_bf16(seed=7, T=2048, H=512, E=32, F=256, k=8, F_shared=256)
+    if unit:
+        cfg = _unit_scale(cfg)
     T, H, E, F, k = cfg["T"], cfg["H"], cfg["E"], cfg["F"], cfg["k"]
     layer = SwiGLUMoE(T, H, E, F, k, cfg["capacity_factor"], F_shared=cfg["F_shared"], aux_coef=cfg["aux_coef"],
                       gathered=gathered)
@@ -128,17 +175,20 @@ def test_full_swiglu_layer_bf16(full_size, gathered):
     assert math.isclose(float(out["aux"][1]), cfg["aux_coef"] * auxo, rel_tol=1e-5)
 
     rng = np.random.default_rng(1)
-    tokens = np.sort(rng.choice(T, 12, replace=False)) if full_size else np.arange(0, T, 7)
-    # include a token with a dropped assignment when there is one
-    dropped_t = np.flatnonzero(o["drops"] > 0)
-    if len(dropped_t):
-        tokens = np.unique(np.concatenate([tokens, dropped_t[:2]]))
-    shared = O.expert_rows("swiglu", x64, tokens, np.zeros(len(tokens), np.int64),
-                           {"w1": pages_layout(cfg["s_gate"]), "w3": pages_layout(cfg["s_up"]),
-                            "w2": pages_layout(cfg["s_down"])})
-    od = dict(selected=sel, kept=o["kept"], gates=gates)
-    want = _swiglu_oracle_rows(cfg, od, tokens, shared)
-    assert_close(cpu64(out["y"])[tokens], want, BF16_RTOL, BF16_ATOL, "swiglu y")
+    if full_size:
+        tokens = np.sort(rng.choice(T, 512, replace=False))
+        # every token with a dropped assignment among the first ones, and the fullest and emptiest experts
+        tokens = np.unique(np.concatenate([tokens, np.flatnonzero(o["drops"] > 0)[:32]]))
+        order = np.argsort(o["used"], kind="stable")
+        experts = np.unique(np.concatenate([order[-4:], order[:4], rng.choice(E, 8, replace=False)]))
+        assert len(experts) >= 16
+    else:
+        tokens, experts = np.arange(0, T, 3), np.arange(E)
+    out["ybuf"] = layer.ybuf
+    want = _check_swiglu_layer(cfg, out, sel, o["kept"], gates, o["token_of_slot"], o["used"], tokens, experts)
+    if unit:
+        # at unit scale the output is O(1): one expert term (gate ~ 1/k of an O(1) row) exceeds the tolerance
+        assert float(np.abs(want).mean()) > 0.3
 
 
 def test_full_layer_is_deterministic():
