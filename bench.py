@@ -42,12 +42,12 @@ UNIT = "tokens/s"
 WORKLOAD = dict(workload="full_layer_bf16", T=16384, hidden=2048, experts=256, top_k=8, expert_intermediate=512,
                 shared_experts=1, shared_intermediate=512, capacity_factor=1.25, capacity=640, aux_coef=0.001)
 KERNELS_PER_STEP = 10  # fused router, reduce, scan, gather, 2 routed GEMMs, 2 shared GEMMs, combine, aux
-# DRAM bytes (read + write) per launch of the two routed expert-FFN kernels,
-# from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum on this
-# workload (profiles/expert_gemm_dram_traffic.md; a one-pass metric set).  For
-# other sizes the same capture's ratio to the algorithmic bytes is applied.
-TRAFFIC_MEASURED = {"gate_up": 1600.2e6, "down": 986.5e6}
-TRAFFIC_PER_ALG_BYTE = {"gate_up": 1.036, "down": 0.978}
+# DRAM bytes (read + write) per algorithmic byte of the two routed expert-FFN kernels (the SwiGLU
+# gate/up tcw_kernel and the down projection tc_gemm_kernel<BF16>), from one ncu capture of
+# dram__bytes_read.sum + dram__bytes_write.sum on the T=8192, E=128 case (one kernel, a few
+# launches); the bench scales it by its own algorithmic bytes.  None until measured for the
+# current kernels.
+TRAFFIC_PER_ALG_BYTE = None
 
 
 def measured_peaks():
@@ -348,14 +348,14 @@ def run_ours(args, world, rank, local):
     achieved = flops / ffn_avg_s / 1e12
     alg_gate_up = E * 2 * F * H * 2 + kept * H * 2 + kept * F * 2  # weights, gathered rows, h written
     alg_down = E * H * F * 2 + kept * F * 2 + kept * H * 2
-    if T == WORKLOAD["T"] and E == WORKLOAD["experts"]:
-        traffic = TRAFFIC_MEASURED["gate_up"] + TRAFFIC_MEASURED["down"]
-        traffic_source = "ncu dram__bytes_read.sum + dram__bytes_write.sum of both launches, this workload"
+    if TRAFFIC_PER_ALG_BYTE is None:
+        traffic, traffic_source = None, "not captured for the current kernels"
     else:
         traffic = TRAFFIC_PER_ALG_BYTE["gate_up"] * alg_gate_up + TRAFFIC_PER_ALG_BYTE["down"] * alg_down
-        traffic_source = "full-workload ncu DRAM bytes per algorithmic byte, times this size's algorithmic bytes"
+        traffic_source = ("ncu DRAM bytes per algorithmic byte of each kernel on the T=8192, E=128 case, "
+                          "times this workload's algorithmic bytes")
     # the routed FFN is timed inside ~1 ms steps, so the burst peak (a kernel timed alone) applies
-    roof = dict(bound="tensor", kernel="routed expert FFN: tcx_kernel<SWIGLU> gate/up + tc_gemm_kernel<BF16> down",
+    roof = dict(bound="tensor", kernel="routed expert FFN: tcw_kernel<SWIGLU> gate/up + tc_gemm_kernel<BF16> down",
                 achieved=achieved, peak=pk["bf16"], unit="TFLOP/s", frac=achieved / pk["bf16"],
                 traffic=traffic, traffic_source=traffic_source, bytes_alg=alg_gate_up + alg_down,
                 peak_source=f"{pk['source']} bf16 burst (cuBLAS)", frac_of_sustained=achieved / pk["bf16_sustained"],

@@ -44,6 +44,10 @@ size_t fp32_split_bytes(moe_ffn_kind kind, int32_t E, int64_t C, int64_t D, int6
 
 namespace {
 constexpr size_t kTileCounterBytes = 256;  // after the intermediate h: scratch words of the wide GEMMs' schedulers
+// The routed down projection (K = F = 512) through the 256 x 256 single-buffered tile measured
+// slower than tc_gemm's double-buffered 128-token tiles (186 against ~118 us at T = 8192, E = 128):
+// with a short K loop the TMEM drain is a large share of each tile.  tc_gemm keeps it.
+constexpr bool kWideDown = false;
 }
 
 extern "C" size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dtype, int32_t E, int64_t C, int64_t D,
@@ -64,7 +68,7 @@ namespace {
 int down_projection(moe_ffn_kind kind, const void* h, const int32_t* used, int32_t E, int64_t C, int64_t F,
                     int64_t Dout, const void* w2, const void* b2, void* ybuf, int32_t* dev_status,
                     cudaStream_t stream, uint32_t* tile_counter = nullptr) {
-    if (kind == MOE_FFN_SWIGLU && used != nullptr) {
+    if (kind == MOE_FFN_SWIGLU && used != nullptr && tile_counter != nullptr && kWideDown) {
         // routed experts: 256 output features x up to 256 tokens per tile (tc_wide_gemm.cu)
         TcxProblem p{};
         p.w = w2;

@@ -34,6 +34,11 @@
 // fixed butterfly, kept in registers across tiles and added in a fixed order
 // at the end, so prob_sum stays bitwise reproducible for a given grid.
 //
+// The exponentials use the fast intrinsic __expf.  Its documented error bound
+// grows with |argument|; the arguments here are score differences (at most 0),
+// so the error is largest on the smallest probabilities, whose absolute error
+// stays far below the tolerances of the probability sums and the gates.
+//
 // Every mbarrier wait is bounded; after a timeout the producers and the MMA
 // issuer stop, and the epilogue runs its remaining tiles without writing
 // anything, so the named barriers between its warps always complete.
@@ -324,14 +329,19 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 tmem_ld32(tmem_base + acc * E + lane_off + (uint32_t)(c * CQ + 32 * h), r);
                 tmem_ld_wait(r);
                 float v[32];
+                const float4* b4 = reinterpret_cast<const float4*>(s_bias + c * CQ + 32 * h);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    float xv = __uint_as_float(r[j]) + s_bias[c * CQ + 32 * h + j];
-                    if (!isfinite(xv)) {
-                        finite = false;
-                        xv = -INFINITY;
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 b = b4[j4];
+                    const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = 4 * j4 + u;
+                        const float xv = __uint_as_float(r[j]) + bb[u];
+                        const bool ok = fabsf(xv) < INFINITY;  // false for +-inf and NaN
+                        finite = finite && ok;
+                        v[j] = ok ? xv : -INFINITY;
                     }
-                    v[j] = xv;
                 }
                 if (p.logits_out && write) {
                     float4* dst = reinterpret_cast<float4*>(p.logits_out + t * E + c * CQ + 32 * h);
@@ -344,7 +354,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     // branch-free: one exponential of -|xv - m_run| rescales the sum or adds the term
                     const float xv = v[j];
                     const float d = xv - m_run;
-                    const float ed = xv == -INFINITY ? 0.f : expf(-fabsf(d));
+                    const float ed = xv == -INFINITY ? 0.f : __expf(-fabsf(d));
                     const bool up = d > 0.f;
                     ls = up ? fmaf(ls, ed, 1.0f) : ls + ed;
                     m_run = up ? xv : m_run;
@@ -365,8 +375,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
             const float mx = fmaxf(fmaxf(s_red[0][0][row], s_red[0][1][row]), fmaxf(s_red[0][2][row], s_red[0][3][row]));
             float tot = 0.f;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) tot += s_red[1][cc][row] * expf(s_red[0][cc][row] - mx);
-            const float scale = valid ? expf(m_run - mx) / tot : 0.f;
+            for (int cc = 0; cc < 4; ++cc) tot += s_red[1][cc][row] * __expf(s_red[0][cc][row] - mx);
+            const float scale = valid ? __expf(m_run - mx) / tot : 0.f;
 
             // pass 2: probabilities, summed over the warp's 32 tokens per expert
             auto pass2 = [&](const int h) {
@@ -374,10 +384,18 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 tmem_ld32(tmem_base + acc * E + lane_off + (uint32_t)(c * CQ + 32 * h), r);
                 tmem_ld_wait(r);
                 float pr[32];
+                const float4* b4 = reinterpret_cast<const float4*>(s_bias + c * CQ + 32 * h);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float xv = __uint_as_float(r[j]) + s_bias[c * CQ + 32 * h + j];
-                    pr[j] = valid && isfinite(xv) ? expf(xv - m_run) * scale : 0.f;
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 b = b4[j4];
+                    const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = 4 * j4 + u;
+                        const float xv = __uint_as_float(r[j]) + bb[u];
+                        // scale is 0 for rows outside the run; a non-finite score contributes 0
+                        pr[j] = fabsf(xv) < INFINITY ? __expf(xv - m_run) * scale : 0.f;
+                    }
                 }
                 const float cs = transpose_sum32(pr, lane);
 #pragma unroll
@@ -423,7 +441,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     float es = 0.f;
 #pragma unroll
                     for (int j = 0; j < kRTopK; ++j) {
-                        ex[j] = j < p.k ? expf(tv[j] - tv[0]) : 0.f;
+                        ex[j] = j < p.k ? __expf(tv[j] - tv[0]) : 0.f;
                         es += ex[j];
                     }
                     const float ginv = 1.0f / es;

@@ -112,6 +112,26 @@ __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* row, int64_t n0, in
     }
 }
 
+// Drain n 32-column chunks of this thread's TMEM lane starting at t_row, with the
+// load of chunk c + 1 in flight while chunk c is processed (its stores overlap the
+// TMEM read latency).
+template <typename F>
+__device__ __forceinline__ void pipelined_chunks(uint32_t t_row, int n, F&& process) {
+    uint32_t ra[32], rb[32];
+    tmem_ld32(t_row, ra);
+    tmem_ld_wait(ra);
+    for (int c = 0; c < n; c += 2) {
+        if (c + 1 < n) tmem_ld32(t_row + (c + 1) * 32, rb);
+        process(c, ra);
+        if (c + 1 < n) {
+            tmem_ld_wait(rb);
+            if (c + 2 < n) tmem_ld32(t_row + (c + 2) * 32, ra);
+            process(c + 1, rb);
+            if (c + 2 < n) tmem_ld_wait(ra);
+        }
+    }
+}
+
 template <int EPI, bool AMN, bool BMN>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -396,10 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (EPI == TC_EPI_F32) {
                 float* orow = reinterpret_cast<float*>(p.out) + out_row * p.ldo;
                 const float* bias = reinterpret_cast<const float*>(p.bias);
-                for (int c = 0; c < p.n_mma / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(t_row + c * 32, r);
-                    tmem_ld_wait(r);
+                auto process = [&](const int c, const uint32_t (&r)[32]) {
                     const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
                     if (p.vec_ok && n0 + 32 <= p.N) {
                         uint32_t w[32];
@@ -415,15 +432,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 32; ++i)
                             if (n0 + i < p.N) orow[n0 + i] = __uint_as_float(r[i]) + (bias ? bias[n0 + i] : 0.f);
                     }
-                }
+                };
+                pipelined_chunks(t_row, p.n_mma / 32, process);
             } else {
                 __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * p.ldo;
                 const __nv_bfloat16* bias =
                     reinterpret_cast<const __nv_bfloat16*>(p.bias) + (p.bias ? g * p.bias_group_stride : 0);
-                for (int c = 0; c < p.n_mma / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(t_row + c * 32, r);
-                    tmem_ld_wait(r);
+                auto process = [&](const int c, const uint32_t (&r)[32]) {
                     const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
                     uint32_t pk[16];
 #pragma unroll
@@ -448,7 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              p.ldo * 2, wrows, lane);
                     else if (row_ok)
                         store_bf16_32(orow, n0, p.N, pk, p.vec_ok);
-                }
+                };
+                pipelined_chunks(t_row, p.n_mma / 32, process);
             }
             tc_fence_before();
             mbar_arrive(&tempty[acc]);

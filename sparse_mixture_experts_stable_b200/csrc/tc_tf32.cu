@@ -1,5 +1,13 @@
 // fp32 grouped GEMM as split-tf32 products on sm_100a (see tc_tf32.cuh).
 //
+// An operand that is already fp32 and K-major in memory (a_trans false / b_trans
+// true, contiguous groups, no per-group K limit) is not split beforehand: the
+// TMA brings its raw fp32 tile into the stage's "hi" slot and four converter
+// warps write lo = x - trunc(x) into the "lo" slot.  The tf32 MMA reads a raw
+// fp32 operand as its value truncated to tf32 (its low 13 mantissa bits
+// ignored; checked on the hardware), so the raw tile is exactly the hi part
+// and lo is exact in fp32.  (With truncation |lo| < 2^-10 |x|, so the dropped
+// lo*lo product stays below 2^-20 |a*b|.)  Other operands go through:
 // 1. split_kernel writes hi/lo of A as (G, M, Kp) and of B as (G, N, Kp),
 //    K-major, Kp = K rounded up to 32 (one 128-byte swizzle row of fp32), with
 //    zeros for k >= the group's valid K; transposed source forms go through a
@@ -30,6 +38,9 @@ constexpr int kBN = 128;                 // max rows of B per tile (UMMA N)
 constexpr int kBK = 32;                  // fp32 elements per 128-byte swizzle row
 constexpr int kStages = 3;
 constexpr int kThreads = 192;
+constexpr int kConvThreads = 128;  // converter warps for raw operands (after the 192 threads above)
+// MN-major raw operands (tf32 MMA with the transpose bits): off until checked on the hardware.
+constexpr bool kRawMnMajor = false;
 constexpr int kMaxGroups = 1024;
 constexpr int kTileBytes = 128 * kBK * 4;   // 16 KB per operand tile
 constexpr int kStageBytes = 4 * kTileBytes;  // A hi, A lo, B hi, B lo
@@ -98,6 +109,14 @@ struct T3Params {
     int n_mma;
     int k_blocks;
     uint32_t tx_bytes;
+    int a_raw;  // A's hi slot holds the raw fp32 tile; the converter warps write its lo slot
+    int b_raw;
+    int a_mn;   // the raw tile is MN-major (4 KB atoms of 32 K rows x 32 fp32 along M or N)
+    int b_mn;
+    int64_t a_rows_per_group;  // MN-major raw operands: rows (K positions) of a group in memory
+    int64_t b_rows_per_group;
+    const int32_t* krows;      // per-group valid K (rows past it are zeroed in the stage), or NULL
+    int64_t K;
     const int32_t* rows;
     int rows_mode;
     float* C;
@@ -146,7 +165,7 @@ __device__ __forceinline__ void decode_tile(int tile, const int* prefix, int G, 
     mt = local - nt * mtiles;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads + kConvThreads, 1)
     tf32x3_kernel(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CUtensorMap tmAl,
                   const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmBl,
                   const T3Params p) {
@@ -162,6 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* empty = bars + kStages;
     uint64_t* tfull = bars + 2 * kStages;
     uint64_t* tempty = bars + 2 * kStages + 2;
+    uint64_t* conv = bars + 2 * kStages + 4;  // the converter warps have written the stage's lo slots
+    const bool any_raw = p.a_raw || p.b_raw;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -170,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&conv[s], kConvThreads);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
@@ -214,10 +236,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     mbar_expect_tx(&full[stage], p.tx_bytes);
                     uint8_t* st = smem + stage * kStageBytes;
-                    tma_load_2d(st, &tmAh, kb * kBK, a_y, &full[stage]);
-                    tma_load_2d(st + kTileBytes, &tmAl, kb * kBK, a_y, &full[stage]);
-                    tma_load_2d(st + 2 * kTileBytes, &tmBh, kb * kBK, b_y, &full[stage]);
-                    tma_load_2d(st + 3 * kTileBytes, &tmBl, kb * kBK, b_y, &full[stage]);
+                    if (p.a_mn) {  // four 32 x 32 atoms along M
+                        const int32_t ky = (int32_t)(g * p.a_rows_per_group + (int64_t)kb * kBK);
+                        for (int i = 0; i < kBM / 32; ++i)
+                            tma_load_2d(st + i * 4096, &tmAh, mt * kBM + 32 * i, ky, &full[stage]);
+                    } else {
+                        tma_load_2d(st, &tmAh, kb * kBK, a_y, &full[stage]);
+                        if (!p.a_raw) tma_load_2d(st + kTileBytes, &tmAl, kb * kBK, a_y, &full[stage]);
+                    }
+                    if (p.b_mn) {
+                        const int32_t ky = (int32_t)(g * p.b_rows_per_group + (int64_t)kb * kBK);
+                        for (int i = 0; i < p.n_mma / 32; ++i)
+                            tma_load_2d(st + 2 * kTileBytes + i * 4096, &tmBh, nt * p.n_mma + 32 * i, ky,
+                                        &full[stage]);
+                    } else {
+                        tma_load_2d(st + 2 * kTileBytes, &tmBh, kb * kBK, b_y, &full[stage]);
+                        if (!p.b_raw) tma_load_2d(st + 3 * kTileBytes, &tmBl, kb * kBK, b_y, &full[stage]);
+                    }
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -229,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------- MMA issuer -------------------------------
         if (lane == 0) {
-            const uint32_t idesc = make_idesc_tf32(kBM, p.n_mma);
+            const uint32_t idesc =
+                make_idesc_tf32(kBM, p.n_mma) | (p.a_mn ? (1u << 15) : 0u) | (p.b_mn ? (1u << 16) : 0u);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t it = 0;
@@ -244,21 +280,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d_tmem = tmem_base + acc * kAccCols;
                 bool ok = true;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, p.status)) {
+                    if (!mbar_wait(any_raw ? &conv[stage] : &full[stage], phase, p.status)) {
                         s_abort = 1;
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + stage * kStageBytes);
-                    const uint64_t ah = sw128_desc(st), al = sw128_desc(st + kTileBytes);
-                    const uint64_t bh = sw128_desc(st + 2 * kTileBytes), bl = sw128_desc(st + 3 * kTileBytes);
+                    // K-major: a K step of 8 is 32 bytes along the row (2 descriptor units); MN-major:
+                    // 8 K rows of 128 bytes (64 units), atoms 4 KB apart
+                    const uint64_t ah = p.a_mn ? sw128_mn_desc(st, 4096) : sw128_desc(st);
+                    const uint64_t al = p.a_mn ? sw128_mn_desc(st + kTileBytes, 4096) : sw128_desc(st + kTileBytes);
+                    const uint64_t bh = p.b_mn ? sw128_mn_desc(st + 2 * kTileBytes, 4096) : sw128_desc(st + 2 * kTileBytes);
+                    const uint64_t bl =
+                        p.b_mn ? sw128_mn_desc(st + 3 * kTileBytes, 4096) : sw128_desc(st + 3 * kTileBytes);
+                    const uint32_t sa = p.a_mn ? 64u : 2u, sb = p.b_mn ? 64u : 2u;
 #pragma unroll
-                    for (int ks = 0; ks < kBK / 8; ++ks) {  // K step 8 = 32 bytes = 2 descriptor units
+                    for (int ks = 0; ks < kBK / 8; ++ks) {
                         const uint32_t first = (kb == 0 && ks == 0) ? 0u : 1u;
-                        mma_tf32(d_tmem, al + 2 * ks, bh + 2 * ks, idesc, first);
-                        mma_tf32(d_tmem, ah + 2 * ks, bl + 2 * ks, idesc, 1u);
-                        mma_tf32(d_tmem, ah + 2 * ks, bh + 2 * ks, idesc, 1u);
+                        mma_tf32(d_tmem, al + sa * ks, bh + sb * ks, idesc, first);
+                        mma_tf32(d_tmem, ah + sa * ks, bl + sb * ks, idesc, 1u);
+                        mma_tf32(d_tmem, ah + sa * ks, bh + sb * ks, idesc, 1u);
                     }
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
@@ -268,6 +310,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
                 tc_commit(&tfull[acc]);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= kThreads / 32) {
+        // -------------------------- raw-operand converters --------------------------
+        // For each stage: lo = x - trunc(x) of every raw fp32 tile element, written
+        // at the same position of the lo slot (the swizzled layout is elementwise).
+        if (any_raw) {
+            const int ct = threadIdx.x - kThreads;
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
+                int g, mt_, nt_;
+                decode_tile(tile, s_prefix, p.G, p.n_tiles, g, mt_, nt_);
+                int64_t kv = p.krows ? (int64_t)p.krows[g] : p.K;  // MN-major rows past it read the next group
+                if (kv > p.K) kv = p.K;
+                const int kval = (int)kv;
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    int ok = 1;
+                    if (lane == 0) ok = mbar_wait(&full[stage], phase, p.status) ? 1 : 0;
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) {
+                        s_abort = 1;
+                        break;
+                    }
+                    uint8_t* st = smem + stage * kStageBytes;
+#pragma unroll
+                    for (int op = 0; op < 2; ++op) {
+                        if (op == 0 ? !p.a_raw : !p.b_raw) continue;
+                        float4* src = reinterpret_cast<float4*>(st + 2 * op * kTileBytes);
+                        float4* dst = reinterpret_cast<float4*>(st + (2 * op + 1) * kTileBytes);
+                        const bool mn = op == 0 ? p.a_mn : p.b_mn;
+                        const int k_lim = kval - kb * kBK;  // MN-major: rows at or past it are zero
+#pragma unroll 4
+                        for (int i = ct; i < kTileBytes / 16; i += kConvThreads) {
+                            float4 x = src[i];
+                            if (mn && ((i >> 3) & 31) >= k_lim) {  // row (i / 8) % 32 of its 4 KB atom
+                                x = make_float4(0.f, 0.f, 0.f, 0.f);
+                                src[i] = x;
+                            }
+                            float4 lo;
+                            lo.x = x.x - __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
+                            lo.y = x.y - __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
+                            lo.z = x.z - __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
+                            lo.w = x.w - __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
+                            dst[i] = lo;
+                        }
+                    }
+                    fence_proxy_async_smem();  // the lo tiles are read by the tensor core
+                    mbar_arrive(&conv[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
             }
         }
         __syncwarp();
@@ -426,13 +523,32 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
     float* b_lo = reinterpret_cast<float*>(ws + 2 * l.a_bytes + l.b_bytes);
     const int32_t* krows = g.rows_mode == 2 ? g.rows : nullptr;
 
-    // K-major split operands: A as (groups, M, Kp), B^T as (groups, N, Kp)
-    int rc = launch_split(g.a_trans, g.a_bf16, g.A, g.lda, g.a_group_stride, g.groups, g.M, g.K, l.Kp, krows, a_hi,
+    // Raw operands (no split pass): fp32 with 16-byte aligned rows, and either K-major with contiguous
+    // groups and no per-group K limit, or MN-major with a whole number of rows per group (rows past a
+    // group's K limit are zeroed in the stage by the converter warps).
+    const bool a_rawk = !g.a_bf16 && !g.a_trans && krows == nullptr && aligned16(g.A) && g.lda % 4 == 0 &&
+                        g.lda >= g.K && (g.groups == 1 || g.a_group_stride == g.M * g.lda);
+    const bool b_rawk = !g.b_bf16 && g.b_trans && krows == nullptr && aligned16(g.B) && g.ldb % 4 == 0 &&
+                        g.ldb >= g.K && (g.groups == 1 || g.b_group_stride == g.N * g.ldb);
+    const int64_t a_rpg = g.groups == 1 ? g.K : (g.lda > 0 ? g.a_group_stride / g.lda : 0);
+    const int64_t b_rpg = g.groups == 1 ? g.K : (g.ldb > 0 ? g.b_group_stride / g.ldb : 0);
+    const bool a_mn = kRawMnMajor && !g.a_bf16 && g.a_trans && aligned16(g.A) && g.lda % 4 == 0 && g.lda >= g.M &&
+                      (g.groups == 1 || g.a_group_stride % g.lda == 0) && a_rpg >= g.K;
+    const bool b_mn = kRawMnMajor && !g.b_bf16 && !g.b_trans && aligned16(g.B) && g.ldb % 4 == 0 && g.ldb >= g.N &&
+                      (g.groups == 1 || g.b_group_stride % g.ldb == 0) && b_rpg >= g.K;
+    const bool a_raw = a_rawk || a_mn, b_raw = b_rawk || b_mn;
+    // The other operands are split beforehand, K-major: A as (groups, M, Kp), B^T as (groups, N, Kp)
+    int rc = MOE_OK;
+    if (!a_raw) {
+        rc = launch_split(g.a_trans, g.a_bf16, g.A, g.lda, g.a_group_stride, g.groups, g.M, g.K, l.Kp, krows, a_hi,
                           a_lo, stream);
-    if (rc != MOE_OK) return rc;
-    rc = launch_split(!g.b_trans, g.b_bf16, g.B, g.ldb, g.b_group_stride, g.groups, g.N, g.K, l.Kp, krows, b_hi,
-                      b_lo, stream);
-    if (rc != MOE_OK) return rc;
+        if (rc != MOE_OK) return rc;
+    }
+    if (!b_raw) {
+        rc = launch_split(!g.b_trans, g.b_bf16, g.B, g.ldb, g.b_group_stride, g.groups, g.N, g.K, l.Kp, krows, b_hi,
+                          b_lo, stream);
+        if (rc != MOE_OK) return rc;
+    }
 
     T3Params kp{};
     kp.G = g.groups;
@@ -442,7 +558,15 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
     kp.n_mma = (int)(n32 < kBN ? n32 : kBN);
     kp.n_tiles = (int)((g.N + kp.n_mma - 1) / kp.n_mma);
     kp.k_blocks = (int)(l.Kp / kBK);
-    kp.tx_bytes = (uint32_t)(2 * kTileBytes + 2 * kp.n_mma * kBK * 4);
+    kp.tx_bytes = (uint32_t)((a_raw ? 1 : 2) * kTileBytes + (b_raw ? 1 : 2) * kp.n_mma * kBK * 4);
+    kp.a_raw = a_raw;
+    kp.b_raw = b_raw;
+    kp.a_mn = a_mn;
+    kp.b_mn = b_mn;
+    kp.a_rows_per_group = a_rpg;
+    kp.b_rows_per_group = b_rpg;
+    kp.krows = (a_mn || b_mn) ? krows : nullptr;
+    kp.K = g.K;
     kp.rows = g.rows;
     kp.rows_mode = g.rows_mode;
     kp.C = g.C;
@@ -456,10 +580,26 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
     kp.status = status;
 
     CUtensorMap mah, mal, mbh, mbl;
-    MOE_REQUIRE(make_map_f32(&mah, a_hi, l.Kp, (int64_t)g.groups * g.M, l.Kp, kBM), MOE_ERR_CUDA);
-    MOE_REQUIRE(make_map_f32(&mal, a_lo, l.Kp, (int64_t)g.groups * g.M, l.Kp, kBM), MOE_ERR_CUDA);
-    MOE_REQUIRE(make_map_f32(&mbh, b_hi, l.Kp, (int64_t)g.groups * g.N, l.Kp, kp.n_mma), MOE_ERR_CUDA);
-    MOE_REQUIRE(make_map_f32(&mbl, b_lo, l.Kp, (int64_t)g.groups * g.N, l.Kp, kp.n_mma), MOE_ERR_CUDA);
+    if (a_mn) {  // the (K rows, M columns) operand in 32 x 32 boxes
+        MOE_REQUIRE(make_map_f32(&mah, g.A, g.M, (int64_t)g.groups * a_rpg, g.lda, 32), MOE_ERR_CUDA);
+        mal = mah;
+    } else if (a_raw) {  // the operand itself: K columns (zero fill up to Kp), row stride lda
+        MOE_REQUIRE(make_map_f32(&mah, g.A, g.K, (int64_t)g.groups * g.M, g.lda, kBM), MOE_ERR_CUDA);
+        mal = mah;
+    } else {
+        MOE_REQUIRE(make_map_f32(&mah, a_hi, l.Kp, (int64_t)g.groups * g.M, l.Kp, kBM), MOE_ERR_CUDA);
+        MOE_REQUIRE(make_map_f32(&mal, a_lo, l.Kp, (int64_t)g.groups * g.M, l.Kp, kBM), MOE_ERR_CUDA);
+    }
+    if (b_mn) {
+        MOE_REQUIRE(make_map_f32(&mbh, g.B, g.N, (int64_t)g.groups * b_rpg, g.ldb, 32), MOE_ERR_CUDA);
+        mbl = mbh;
+    } else if (b_raw) {
+        MOE_REQUIRE(make_map_f32(&mbh, g.B, g.K, (int64_t)g.groups * g.N, g.ldb, kp.n_mma), MOE_ERR_CUDA);
+        mbl = mbh;
+    } else {
+        MOE_REQUIRE(make_map_f32(&mbh, b_hi, l.Kp, (int64_t)g.groups * g.N, l.Kp, kp.n_mma), MOE_ERR_CUDA);
+        MOE_REQUIRE(make_map_f32(&mbl, b_lo, l.Kp, (int64_t)g.groups * g.N, l.Kp, kp.n_mma), MOE_ERR_CUDA);
+    }
 
     const int64_t max_tiles = (int64_t)g.groups * ((g.M + kBM - 1) / kBM) * kp.n_tiles;
     MOE_REQUIRE(max_tiles < (int64_t(1) << 30), MOE_ERR_UNSUPPORTED);
@@ -474,7 +614,7 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
         MOE_CUDA_TRY(cudaFuncSetAttribute(tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes));
         if (dev < 64) attr_set[dev] = true;
     }
-    tf32x3_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mah, mal, mbh, mbl, kp);
+    tf32x3_kernel<<<grid, kThreads + kConvThreads, kSmemBytes, stream>>>(mah, mal, mbh, mbl, kp);
     return launch_status();
 }
 
