@@ -14,30 +14,52 @@
 // 32-row TMA boxes that hold the run's own rows are loaded.
 //
 // Warp roles (608 threads):
-//   warp 0      TMA producer of the token rows: a 6-stage ring of 16 KB stages
-//               (the deep ring keeps ~96 KB of activations in flight per SM,
-//               what HBM latency needs at this SM's share of the bandwidth)
-//   warp 1      TMA producer of the router weight: a 3-stage ring of E x 64
-//               (the weight is re-read from L2 for every tile)
+//   warp 0      TMA producer of the token rows: 5 stages of 16 KB (~80 KB of
+//               activations in flight per SM, what HBM latency needs at this
+//               SM's share of the bandwidth)
+//   warp 1      TMA producer of the router weight: 3 stages of E x 64 (the
+//               weight is re-read from L2 for every tile)
 //   warp 2      TMEM owner and MMA issuer (one lane): two E-column
 //               accumulators, so a tile's epilogue overlaps the next tile's
 //               main loop
+// The two producers feed one ring of barriers: k-block g waits on full[g % 5]
+// (both loads land on it) and releases empty[g % 5] with one commit; the
+// weight producer reuses its stage g % 3 once k-block g - 3 is released.  One
+// wait and one commit per k-block keep the issuing thread's work between two
+// k-blocks short, and the next k-block's barrier is tested while the current
+// one's MMAs are being accepted, since the tensor core takes new MMAs only as
+// it finishes old ones: a late look at the barrier leaves it idle.
 //   warps 3-18  epilogue: warp w reads TMEM lanes 32*(w%4).. (its 32 tokens)
 //               and one quarter of the E columns, 32 columns per TMEM load.
-//               Pass 1 keeps the quarter's sorted top-8 (score desc, expert
-//               index asc) and an online softmax sum; the four quarters' (max,
-//               sum) pairs are combined through shared memory; pass 2 re-reads
-//               the accumulator for the probabilities and then releases it.
-//               The four top-8 lists are merged in two rounds, and the warp of
-//               the first quarter writes selected, the gates and the counts.
+//
+// The epilogue finds the top-8 without ranking every score against a list:
+//   pass 1  each 32-score chunk is sorted in groups of eight by a 19-comparator
+//           network and the groups are merged by bitonic half-cleaners, so the
+//           chunk's eight largest VALUES cost about eight min/max operations
+//           per score; the quarter keeps its eight largest values and an
+//           online softmax sum (the chunk maximum is the largest group head).
+//   exchange  the four quarters of a token publish their value lists and sums
+//           through shared memory; every thread merges them in a fixed order,
+//           which gives the token's exact eighth-largest score tau, its maximum
+//           and its softmax denominator.
+//   pass 2  re-reads the accumulator for the probabilities (summed over the
+//           warp's 32 tokens per expert) and collects the candidates: a score
+//           above tau (at most seven per token) goes to a value slot, a score
+//           equal to tau only sets a bit, since its value is known.
+//   select  each thread inserts its candidates into a list ordered by (score
+//           descending, expert index ascending), the slots first and then the
+//           tied experts in ascending order; the four lists are merged in two
+//           rounds and the first quarter writes selected, gates and counts.
+// Every score below tau is outside the top-8 and every score above it inside,
+// so the candidates hold the whole answer and the ordered insertion makes the
+// tie-break exact.
 // Per-expert probability sums are reduced over the 32 tokens of a warp with a
 // fixed butterfly, kept in registers across tiles and added in a fixed order
 // at the end, so prob_sum stays bitwise reproducible for a given grid.
 //
-// The exponentials use the fast intrinsic __expf.  Its documented error bound
-// grows with |argument|; the arguments here are score differences (at most 0),
-// so the error is largest on the smallest probabilities, whose absolute error
-// stays far below the tolerances of the probability sums and the gates.
+// The exponentials are ex2.approx of (score - max) * log2(e) (a fused
+// multiply-add); its documented relative error is a few ulp, far below the
+// tolerances of the probability sums and the gates.
 //
 // Every mbarrier wait is bounded; after a timeout the producers and the MMA
 // issuer stop, and the epilogue runs its remaining tiles without writing
@@ -59,17 +81,40 @@ using namespace tc;
 
 constexpr int kRM = 128;       // tokens per tile (UMMA M)
 constexpr int kRBK = 64;       // K per stage (64 bf16 = one 128-byte swizzle row)
-constexpr int kRAStages = 6;
+constexpr int kRAStages = 5;
 constexpr int kRBStages = 3;
 constexpr int kRBox = 32;      // token rows per TMA box
 constexpr int kREpiWarps = 16;
 constexpr int kRThreads = (3 + kREpiWarps) * 32;
 constexpr int kRABytes = kRM * kRBK * 2;  // 16 KB
 constexpr int kRTopK = 8;
+constexpr int kRE = 256;                  // experts (the fused path's only width)
+constexpr int kRCQ = kRE / 4;             // columns per epilogue quarter
+constexpr int kRBBytes = kRE * kRBK * 2;  // 32 KB
 
-size_t fused_dyn_smem(int E) {
-    return 1024 + (size_t)kRAStages * kRABytes + (size_t)kRBStages * E * kRBK * 2 + 256;
-}
+// Shared memory of one lane-quarter group (the 4 epilogue warps that read the
+// same 32 TMEM lanes): an 8 KB area that holds first the exchange of the
+// quarters' (top-8 values, softmax sum, finiteness) and then the value slots
+// of the candidates above tau, and a 4 KB area for the two lists in transit
+// of the final merge.
+constexpr int kExWords = kRTopK + 2;         // per (quarter, token): 8 values, sum, finite flag
+constexpr int kSlots = kRTopK;               // 7 candidates at most, plus one scratch slot
+constexpr int kGroupUnion = kSlots * 128 * 8;  // 8 KB
+constexpr int kGroupMerge = 2 * kRTopK * 32 * 8;  // 4 KB
+static_assert(4 * kExWords * 32 * 4 <= kGroupUnion, "exchange must fit the union area");
+
+// dynamic shared memory layout (offsets from a 1024-byte aligned base)
+constexpr size_t kOffA = 0;
+constexpr size_t kOffB = kOffA + (size_t)kRAStages * kRABytes;
+constexpr size_t kOffBars = kOffB + (size_t)kRBStages * kRBBytes;
+constexpr size_t kOffMisc = kOffBars + 256;
+constexpr size_t kOffBias = kOffMisc + 64;
+constexpr size_t kOffCounts = kOffBias + kRE * 4;
+constexpr size_t kOffUnion = kOffCounts + kRE * 4;
+constexpr size_t kOffMerge = kOffUnion + 4 * (size_t)kGroupUnion;
+constexpr size_t kSmemBytes = kOffMerge + 4 * (size_t)kGroupMerge;
+static_assert(kSmemBytes <= 232448, "the router kernel must fit one SM's shared memory");
+static_assert(4 * kRE * 4 <= 4 * kGroupUnion, "final per-group sums reuse the union area");
 
 struct RFParams {
     int64_t T;
@@ -89,6 +134,12 @@ struct RFParams {
 
 __device__ __forceinline__ void named_bar(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // Insert (v, idx) into a list sorted by (score descending, index ascending).
@@ -111,6 +162,37 @@ __device__ __forceinline__ void topk_insert(float (&tv)[kRTopK], int (&ti)[kRTop
     ti[0] = p[0] ? idx : ti[0];
 }
 
+// compare-exchange for a descending order (values only)
+__device__ __forceinline__ void cx(float& a, float& b) {
+    const float hi = fmaxf(a, b);
+    b = fminf(a, b);
+    a = hi;
+}
+
+// sorts a[0..7] descending: the 19-comparator, depth-6 network of Knuth's
+// Sorting and Searching (section 5.3.4), checked on all 0-1 inputs
+__device__ __forceinline__ void sort8_desc(float* a) {
+    cx(a[0], a[2]); cx(a[1], a[3]); cx(a[4], a[6]); cx(a[5], a[7]);
+    cx(a[0], a[4]); cx(a[1], a[5]); cx(a[2], a[6]); cx(a[3], a[7]);
+    cx(a[0], a[1]); cx(a[2], a[3]); cx(a[4], a[5]); cx(a[6], a[7]);
+    cx(a[2], a[4]); cx(a[3], a[5]);
+    cx(a[1], a[4]); cx(a[3], a[6]);
+    cx(a[1], a[2]); cx(a[3], a[4]); cx(a[5], a[6]);
+}
+
+// a <- the eight largest of a and b (both sorted descending), sorted
+// descending: max(a_i, b_(7-i)) is bitonic and holds the eight largest, and
+// three half-cleaner stages sort it
+__device__ __forceinline__ void merge8_desc(float* a, const float* b) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], b[7 - i]);
+#pragma unroll
+    for (int d = 4; d >= 1; d >>= 1)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (!(i & d)) cx(a[i], a[i + d]);
+}
+
 // Lane l returns the sum over the warp's lanes of a[l] (a is overwritten).
 __device__ __forceinline__ float transpose_sum32(float* a, int lane) {
 #pragma unroll
@@ -126,33 +208,28 @@ __device__ __forceinline__ float transpose_sum32(float* a, int lane) {
     return a[0];
 }
 
-template <int CQ>
 __global__ void __launch_bounds__(kRThreads, 1)
     route_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                        const RFParams p) {
-    constexpr int E = 4 * CQ;
-    constexpr int kBBytes = E * kRBK * 2;
-    constexpr int NH = CQ / 32;  // 32-column chunks per quarter
-    extern __shared__ uint8_t smem_raw[];
-    __shared__ float s_red[2][4][kRM];          // per-quarter max and sum of each token
-    __shared__ float s_cv[2][kRM][kRTopK];      // top-8 lists in transit: scores
-    __shared__ int s_ci[2][kRM][kRTopK];        //                         indices
-    __shared__ float s_bias[E];
-    __shared__ int s_counts[E];
-    __shared__ float s_psum[4][E];
-    __shared__ uint32_t s_tmem;
-    __shared__ volatile int s_abort;
-
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* smA = smem;
-    uint8_t* smB = smA + kRAStages * kRABytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smB + kRBStages * kBBytes);
-    uint64_t* a_full = bars;
-    uint64_t* a_empty = bars + kRAStages;
-    uint64_t* b_full = bars + 2 * kRAStages;
-    uint64_t* b_empty = bars + 2 * kRAStages + kRBStages;
-    uint64_t* tfull = bars + 2 * kRAStages + 2 * kRBStages;
+    constexpr int E = kRE;
+    constexpr int CQ = kRCQ;
+    constexpr float kLog2e = 1.4426950408889634f;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    if ((smem_u32(smem_raw) & 1023u) != 0) {  // the layout needs a 1024-byte aligned base (swizzled stages)
+        if (threadIdx.x == 0) set_status(p.status, MOE_ERR_CUDA);
+        return;
+    }
+    uint8_t* smA = smem_raw + kOffA;
+    uint8_t* smB = smem_raw + kOffB;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kOffBars);
+    uint64_t* full = bars;                  // k-block g's A and W have landed (two arrivals + bytes)
+    uint64_t* empty = bars + kRAStages;     // k-block g's MMAs are done
+    uint64_t* tfull = bars + 2 * kRAStages;
     uint64_t* tempty = tfull + 2;
+    uint32_t* s_tmem_p = reinterpret_cast<uint32_t*>(smem_raw + kOffMisc);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem_raw + kOffMisc + 4);
+    float* s_bias = reinterpret_cast<float*>(smem_raw + kOffBias);
+    int* s_counts = reinterpret_cast<int*>(smem_raw + kOffCounts);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -166,24 +243,20 @@ __global__ void __launch_bounds__(kRThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRAStages; ++s) {
-            mbar_init(&a_full[s], 1);
-            mbar_init(&a_empty[s], 1);
-        }
-        for (int s = 0; s < kRBStages; ++s) {
-            mbar_init(&b_full[s], 1);
-            mbar_init(&b_empty[s], 1);
+            mbar_init(&full[s], 2);
+            mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], kREpiWarps * 32);
         }
-        s_abort = 0;
+        *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmX)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
     }
     if (warp == 2) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem_p)),
                      "r"(2 * E)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -195,27 +268,27 @@ __global__ void __launch_bounds__(kRThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = s_tmem;
+    const uint32_t tmem_base = *s_tmem_p;
 
     if (warp == 0) {
         // ------------------------- token-row producer -------------------------
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            for (int i = 0; i < n_tiles && !s_abort; ++i) {
+            for (int i = 0; i < n_tiles && !*s_abort; ++i) {
                 const int64_t r0 = row_begin + (int64_t)i * kRM;
                 const int64_t nrows = row_end - r0 < kRM ? row_end - r0 : kRM;
                 const int nbox = (int)((nrows + kRBox - 1) / kRBox);
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!mbar_wait(&a_empty[stage], phase ^ 1u, p.status)) {
-                        s_abort = 1;
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) {  // k-block g - 5 is done
+                        *s_abort = 1;
                         break;
                     }
-                    mbar_expect_tx(&a_full[stage], (uint32_t)(nbox * kRBox * kRBK * 2));
+                    mbar_expect_tx(&full[stage], (uint32_t)(nbox * kRBox * kRBK * 2));
                     uint8_t* dst = smA + stage * kRABytes;
                     for (int b = 0; b < nbox; ++b)
                         tma_load_2d(dst + b * (kRBox * kRBK * 2), &tmX, kb * kRBK, (int32_t)(r0 + b * kRBox),
-                                    &a_full[stage]);
+                                    &full[stage]);
                     if (++stage == kRAStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -227,20 +300,21 @@ __global__ void __launch_bounds__(kRThreads, 1)
     } else if (warp == 1) {
         // ------------------------ router-weight producer -----------------------
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int i = 0; i < n_tiles && !s_abort; ++i) {
-                for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!mbar_wait(&b_empty[stage], phase ^ 1u, p.status)) {
-                        s_abort = 1;
-                        break;
+            static_assert(kRAStages >= kRBStages, "the weight stages are released through the A ring");
+            uint32_t g = 0;  // k-block counter over the whole run
+            int wstage = 0;
+            for (int i = 0; i < n_tiles && !*s_abort; ++i) {
+                for (int kb = 0; kb < p.k_blocks; ++kb, ++g) {
+                    if (g >= (uint32_t)kRBStages) {  // stage g % 3 was last read by k-block g - 3
+                        const uint32_t pg = g - kRBStages;
+                        if (!mbar_wait(&empty[pg % kRAStages], (pg / kRAStages) & 1u, p.status)) {
+                            *s_abort = 1;
+                            break;
+                        }
                     }
-                    mbar_expect_tx(&b_full[stage], (uint32_t)kBBytes);
-                    tma_load_2d(smB + stage * kBBytes, &tmW, kb * kRBK, 0, &b_full[stage]);
-                    if (++stage == kRBStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    mbar_expect_tx(&full[g % kRAStages], (uint32_t)kRBBytes);
+                    tma_load_2d(smB + wstage * kRBBytes, &tmW, kb * kRBK, 0, &full[g % kRAStages]);
+                    if (++wstage == kRBStages) wstage = 0;
                 }
             }
         }
@@ -250,40 +324,40 @@ __global__ void __launch_bounds__(kRThreads, 1)
         if (lane == 0) {
             const uint32_t idesc = make_idesc(kRM, E);
             int sa = 0, sb = 0;
-            uint32_t pa = 0, pb = 0;
-            for (int i = 0; i < n_tiles && !s_abort; ++i) {
+            uint32_t pa = 0;
+            const uint32_t full0 = smem_u32(full);
+            bool ready = mbar_test(full0, 0u);
+            for (int i = 0; i < n_tiles && !*s_abort; ++i) {
                 const uint32_t acc = (uint32_t)i & 1u;
                 if (!mbar_wait(&tempty[acc], (((uint32_t)i >> 1) & 1u) ^ 1u, p.status)) {
-                    s_abort = 1;
+                    *s_abort = 1;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * E;
                 bool ok = true;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!mbar_wait(&a_full[sa], pa, p.status) || !mbar_wait(&b_full[sb], pb, p.status)) {
+                    if (!ready && !mbar_wait(&full[sa], pa, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint64_t ad = sw128_desc(smem_u32(smA + sa * kRABytes));
-                    const uint64_t bd = sw128_desc(smem_u32(smB + sb * kBBytes));
-#pragma unroll
-                    for (int kk = 0; kk < kRBK / 16; ++kk)
-                        tc_mma(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(&a_empty[sa]);
-                    tc_commit(&b_empty[sb]);
-                    if (++sa == kRAStages) {
-                        sa = 0;
-                        pa ^= 1u;
-                    }
-                    if (++sb == kRBStages) {
-                        sb = 0;
-                        pb ^= 1u;
-                    }
+                    const uint64_t bd = sw128_desc(smem_u32(smB + sb * kRBBytes));
+                    const int sn = sa + 1 == kRAStages ? 0 : sa + 1;
+                    const uint32_t pn = sa + 1 == kRAStages ? pa ^ 1u : pa;
+                    tc_mma(d_tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);
+                    tc_mma(d_tmem, ad + 2, bd + 2, idesc, 1u);
+                    ready = mbar_test(full0 + 8u * (uint32_t)sn, pn);  // the next k-block, early
+                    tc_mma(d_tmem, ad + 4, bd + 4, idesc, 1u);
+                    tc_mma(d_tmem, ad + 6, bd + 6, idesc, 1u);
+                    tc_commit(&empty[sa]);
+                    sa = sn;
+                    pa = pn;
+                    if (++sb == kRBStages) sb = 0;
                 }
                 if (!ok) {
-                    s_abort = 1;
+                    *s_abort = 1;
                     break;
                 }
                 tc_commit(&tfull[acc]);
@@ -295,53 +369,53 @@ __global__ void __launch_bounds__(kRThreads, 1)
         const int q = warp & 3;         // TMEM lane quarter this warp may read
         const int c = (warp - 3) >> 2;  // column quarter
         const int row = q * 32 + lane;
+        const int tig = c * 32 + lane;  // thread within the lane-quarter group
         const int bar_id = 1 + q;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        float acc_ps[NH];
-#pragma unroll
-        for (int h = 0; h < NH; ++h) acc_ps[h] = 0.f;
+        float* s_ex = reinterpret_cast<float*>(smem_raw + kOffUnion + (size_t)q * kGroupUnion);  // [c][word][lane]
+        uint8_t* s_slot = smem_raw + kOffUnion + (size_t)q * kGroupUnion;  // [slot][tig] x (value, index)
+        float* s_mv = reinterpret_cast<float*>(smem_raw + kOffMerge + (size_t)q * kGroupMerge);  // [list][j][lane]
+        int* s_mi = reinterpret_cast<int*>(smem_raw + kOffMerge + (size_t)q * kGroupMerge + kGroupMerge / 2);
+        const uint32_t slot_base = smem_u32(s_slot) + (uint32_t)tig * 8u;
+        const uint32_t slot_last = slot_base + (uint32_t)(kSlots - 1) * 1024u;  // the scratch slot
+        float acc_ps[2] = {0.f, 0.f};
 
         for (int i = 0; i < n_tiles; ++i) {
             const uint32_t acc = (uint32_t)i & 1u;
             int ok = 1;
             if (lane == 0) ok = mbar_wait(&tfull[acc], ((uint32_t)i >> 1) & 1u, p.status) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) s_abort = 1;
+            if (!ok) *s_abort = 1;
             tc_fence_after();
             const int64_t r0 = row_begin + (int64_t)i * kRM;
             const bool valid = r0 + row < row_end;
             const int64_t t = r0 + row;
+            const bool write = valid && !*s_abort;
+            const uint32_t tcol = tmem_base + acc * E + lane_off + (uint32_t)(c * CQ);
 
-            // pass 1, 32 columns at a time: bias, the quarter's top-8 (its experts in
-            // ascending order) and an online softmax sum against the running max
-            float tv[kRTopK];
-            int ti[kRTopK];
+            // ---- pass 1: the quarter's eight largest values and its softmax sum ----
+            float qt[kRTopK];
+            float m_run = -INFINITY, ssum = 0.f, fin0 = 0.f, fin1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < kRTopK; ++j) {
-                tv[j] = -INFINITY;
-                ti[j] = c * CQ + j;
-            }
-            float m_run = -INFINITY, ls = 0.f;
-            bool finite = true;
-            const bool write = valid && !s_abort;
-            auto pass1 = [&](const int h) {
+            for (int h = 0; h < 2; ++h) {
                 uint32_t r[32];
-                tmem_ld32(tmem_base + acc * E + lane_off + (uint32_t)(c * CQ + 32 * h), r);
+                tmem_ld32(tcol + 32 * h, r);
                 tmem_ld_wait(r);
                 float v[32];
                 const float4* b4 = reinterpret_cast<const float4*>(s_bias + c * CQ + 32 * h);
 #pragma unroll
                 for (int j4 = 0; j4 < 8; ++j4) {
                     const float4 b = b4[j4];
-                    const float bb[4] = {b.x, b.y, b.z, b.w};
+                    v[4 * j4 + 0] = __uint_as_float(r[4 * j4 + 0]) + b.x;
+                    v[4 * j4 + 1] = __uint_as_float(r[4 * j4 + 1]) + b.y;
+                    v[4 * j4 + 2] = __uint_as_float(r[4 * j4 + 2]) + b.z;
+                    v[4 * j4 + 3] = __uint_as_float(r[4 * j4 + 3]) + b.w;
+                }
+                // x * 0 is 0 for finite x and NaN for an infinity or a NaN
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int j = 4 * j4 + u;
-                        const float xv = __uint_as_float(r[j]) + bb[u];
-                        const bool ok = fabsf(xv) < INFINITY;  // false for +-inf and NaN
-                        finite = finite && ok;
-                        v[j] = ok ? xv : -INFINITY;
-                    }
+                for (int j = 0; j < 32; j += 2) {
+                    fin0 = fmaf(v[j], 0.f, fin0);
+                    fin1 = fmaf(v[j + 1], 0.f, fin1);
                 }
                 if (p.logits_out && write) {
                     float4* dst = reinterpret_cast<float4*>(p.logits_out + t * E + c * CQ + 32 * h);
@@ -349,41 +423,83 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
                 }
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    topk_insert(tv, ti, v[j], c * CQ + 32 * h + j);
-                    // branch-free: one exponential of -|xv - m_run| rescales the sum or adds the term
-                    const float xv = v[j];
-                    const float d = xv - m_run;
-                    const float ed = xv == -INFINITY ? 0.f : __expf(-fabsf(d));
-                    const bool up = d > 0.f;
-                    ls = up ? fmaf(ls, ed, 1.0f) : ls + ed;
-                    m_run = up ? xv : m_run;
-                }
-            };
-            if constexpr (NH == 1) {
-                pass1(0);
-            } else {
-#pragma unroll 1
-                for (int h = 0; h < NH; ++h) pass1(h);
-            }
-            if (!finite && valid) set_status(p.status, MOE_ERR_NONFINITE);
-
-            // softmax over all E: the quarters' (max, sum) pairs combined in a fixed order
-            s_red[0][c][row] = m_run;
-            s_red[1][c][row] = ls;
-            named_bar(bar_id, 128);
-            const float mx = fmaxf(fmaxf(s_red[0][0][row], s_red[0][1][row]), fmaxf(s_red[0][2][row], s_red[0][3][row]));
-            float tot = 0.f;
+                for (int g = 0; g < 4; ++g) sort8_desc(v + 8 * g);
+                // online softmax: the chunk maximum is the largest group head
+                const float cm = fmaxf(fmaxf(v[0], v[8]), fmaxf(v[16], v[24]));
+                const float m_new = fmaxf(m_run, cm);
+                const float mL = m_new == -INFINITY ? 0.f : m_new * kLog2e;
+                float e0 = 0.f, e1 = 0.f;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) tot += s_red[1][cc][row] * __expf(s_red[0][cc][row] - mx);
-            const float scale = valid ? __expf(m_run - mx) / tot : 0.f;
+                for (int j = 0; j < 32; j += 2) {
+                    e0 += ex2_approx(fmaf(v[j], kLog2e, -mL));
+                    e1 += ex2_approx(fmaf(v[j + 1], kLog2e, -mL));
+                }
+                ssum = (m_run == m_new ? ssum : ssum * ex2_approx(fmaf(m_run, kLog2e, -mL))) + (e0 + e1);
+                m_run = m_new;
+                merge8_desc(v, v + 8);
+                merge8_desc(v + 16, v + 24);
+                merge8_desc(v, v + 16);
+                if (h == 0) {
+#pragma unroll
+                    for (int j = 0; j < kRTopK; ++j) qt[j] = v[j];
+                } else {
+                    merge8_desc(qt, v);
+                }
+            }
+            const bool q_finite = (fin0 + fin1) == 0.f;
+            if (!q_finite && valid) set_status(p.status, MOE_ERR_NONFINITE);
 
-            // pass 2: probabilities, summed over the warp's 32 tokens per expert
-            auto pass2 = [&](const int h) {
+            // ---- exchange: every thread merges the four lists in the same order ----
+#pragma unroll
+            for (int j = 0; j < kRTopK; ++j) s_ex[(c * kExWords + j) * 32 + lane] = qt[j];
+            s_ex[(c * kExWords + kRTopK) * 32 + lane] = ssum;
+            s_ex[(c * kExWords + kRTopK + 1) * 32 + lane] = q_finite ? 1.f : 0.f;
+            named_bar(bar_id, 128);
+            float l0[kRTopK], l1[kRTopK], sq[4];
+            bool row_finite = true;
+#pragma unroll
+            for (int j = 0; j < kRTopK; ++j) {
+                l0[j] = s_ex[(0 * kExWords + j) * 32 + lane];
+                l1[j] = s_ex[(1 * kExWords + j) * 32 + lane];
+            }
+            merge8_desc(l0, l1);
+            float l2[kRTopK], l3[kRTopK];
+#pragma unroll
+            for (int j = 0; j < kRTopK; ++j) {
+                l2[j] = s_ex[(2 * kExWords + j) * 32 + lane];
+                l3[j] = s_ex[(3 * kExWords + j) * 32 + lane];
+            }
+            merge8_desc(l2, l3);
+            float qmax[4];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                qmax[cc] = s_ex[(cc * kExWords + 0) * 32 + lane];
+                sq[cc] = s_ex[(cc * kExWords + kRTopK) * 32 + lane];
+                row_finite = row_finite && s_ex[(cc * kExWords + kRTopK + 1) * 32 + lane] != 0.f;
+            }
+            merge8_desc(l0, l2);  // l0: the token's eight largest scores
+            named_bar(bar_id, 128);  // the exchange area becomes the candidate slots
+            const float tau = l0[kRTopK - 1];
+            const float mx = l0[0];
+            const float mxL = mx * kLog2e;
+            float den = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) den += sq[cc] * ex2_approx(fmaf(qmax[cc], kLog2e, -mxL));
+            // p = 2^(s log2e - (max log2e + log2 den)); rows outside the run or with a
+            // non-finite score contribute nothing to the probability sums
+            const float cL = mxL + log2f(den);
+            const float pcap = (valid && row_finite) ? INFINITY : 0.f;
+
+            // ---- pass 2: probabilities and the candidates ----
+            uint32_t slot = slot_base;
+            uint32_t eq_bits[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
                 uint32_t r[32];
-                tmem_ld32(tmem_base + acc * E + lane_off + (uint32_t)(c * CQ + 32 * h), r);
+                tmem_ld32(tcol + 32 * h, r);
                 tmem_ld_wait(r);
                 float pr[32];
+                uint32_t eqb = 0;
                 const float4* b4 = reinterpret_cast<const float4*>(s_bias + c * CQ + 32 * h);
 #pragma unroll
                 for (int j4 = 0; j4 < 8; ++j4) {
@@ -393,48 +509,74 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     for (int u = 0; u < 4; ++u) {
                         const int j = 4 * j4 + u;
                         const float xv = __uint_as_float(r[j]) + bb[u];
-                        // scale is 0 for rows outside the run; a non-finite score contributes 0
-                        pr[j] = fabsf(xv) < INFINITY ? __expf(xv - m_run) * scale : 0.f;
+                        pr[j] = fminf(ex2_approx(fmaf(xv, kLog2e, -cL)), pcap);  // fminf drops a NaN
+                        // a score above tau goes to the next slot; one equal to tau sets its bit
+                        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(slot), "f"(xv),
+                                     "f"(__int_as_float(c * CQ + 32 * h + j)));
+                        slot = min(slot + (xv > tau ? 1024u : 0u), slot_last);  // seven at most, capped anyway
+                        eqb |= xv == tau ? (1u << j) : 0u;
                     }
                 }
+                eq_bits[h] = eqb;
                 const float cs = transpose_sum32(pr, lane);
-#pragma unroll
-                for (int hh = 0; hh < NH; ++hh) acc_ps[hh] += hh == h ? cs : 0.f;
-            };
-            if constexpr (NH == 1) {
-                pass2(0);
-            } else {
-#pragma unroll 1
-                for (int h = 0; h < NH; ++h) pass2(h);
+                acc_ps[h] += cs;
             }
             tc_fence_before();
             mbar_arrive(&tempty[acc]);  // the accumulator is no longer read: the next tile may use it
 
-            // merge the four lists: (1 into 0, 3 into 2), then (2 into 0)
+            // ---- select: the quarter's candidates in (score desc, index asc) order ----
+            float tv[kRTopK];
+            int ti[kRTopK];
+#pragma unroll
+            for (int j = 0; j < kRTopK; ++j) {
+                tv[j] = -INFINITY;
+                ti[j] = c * CQ + j;
+            }
+            const int n_gt = (int)((slot - slot_base) >> 10);
+            for (int s = 0; s < n_gt; ++s) {
+                float2 e;
+                asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(e.x), "=f"(e.y) : "r"(slot_base + 1024u * (uint32_t)s));
+                topk_insert(tv, ti, e.x, __float_as_int(e.y));
+            }
+            // the experts tied at tau, ascending; no list needs more than eight of them
+#pragma unroll 1
+            for (int h = 0, n_eq = 0; h < 2; ++h) {
+                uint32_t b = eq_bits[h];
+                while (b != 0u && n_eq < kRTopK) {
+                    const int j = __ffs(b) - 1;
+                    b &= b - 1u;
+                    topk_insert(tv, ti, tau, c * CQ + 32 * h + j);
+                    ++n_eq;
+                }
+            }
+
+            // ---- merge the four lists: (1 into 0, 3 into 2), then (2 into 0) ----
             if (c & 1) {
 #pragma unroll
                 for (int j = 0; j < kRTopK; ++j) {
-                    s_cv[c >> 1][row][j] = tv[j];
-                    s_ci[c >> 1][row][j] = ti[j];
+                    s_mv[((c >> 1) * kRTopK + j) * 32 + lane] = tv[j];
+                    s_mi[((c >> 1) * kRTopK + j) * 32 + lane] = ti[j];
                 }
             }
             named_bar(bar_id, 128);
             if (!(c & 1)) {
 #pragma unroll
-                for (int j = 0; j < kRTopK; ++j) topk_insert(tv, ti, s_cv[c >> 1][row][j], s_ci[c >> 1][row][j]);
+                for (int j = 0; j < kRTopK; ++j)
+                    topk_insert(tv, ti, s_mv[((c >> 1) * kRTopK + j) * 32 + lane],
+                                s_mi[((c >> 1) * kRTopK + j) * 32 + lane]);
             }
-            named_bar(bar_id, 128);
-            if (c == 2) {
+            if (c == 2) {  // list 1 was read by this thread only
 #pragma unroll
                 for (int j = 0; j < kRTopK; ++j) {
-                    s_cv[0][row][j] = tv[j];
-                    s_ci[0][row][j] = ti[j];
+                    s_mv[(kRTopK + j) * 32 + lane] = tv[j];
+                    s_mi[(kRTopK + j) * 32 + lane] = ti[j];
                 }
             }
             named_bar(bar_id, 128);
             if (c == 0) {
 #pragma unroll
-                for (int j = 0; j < kRTopK; ++j) topk_insert(tv, ti, s_cv[0][row][j], s_ci[0][row][j]);
+                for (int j = 0; j < kRTopK; ++j)
+                    topk_insert(tv, ti, s_mv[(kRTopK + j) * 32 + lane], s_mi[(kRTopK + j) * 32 + lane]);
                 if (write) {
                     // gates: softmax of the selected scores (the first is the largest)
                     float ex[kRTopK];
@@ -464,11 +606,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
             }
         }
         // per-CTA partials: the four lane quarters of each expert in a fixed order
+        named_bar(5, kREpiWarps * 32);  // every group is done with its union area
+        float* s_psum = reinterpret_cast<float*>(smem_raw + kOffUnion);  // [q][E]
 #pragma unroll
-        for (int h = 0; h < NH; ++h) s_psum[q][c * CQ + 32 * h + lane] = acc_ps[h];
+        for (int h = 0; h < 2; ++h) s_psum[q * E + c * CQ + 32 * h + lane] = acc_ps[h];
         named_bar(5, kREpiWarps * 32);
         for (int e = threadIdx.x - 96; e < E; e += kREpiWarps * 32) {
-            p.part_psum[(int64_t)blockIdx.x * E + e] = ((s_psum[0][e] + s_psum[1][e]) + s_psum[2][e]) + s_psum[3][e];
+            p.part_psum[(int64_t)blockIdx.x * E + e] =
+                ((s_psum[0 * E + e] + s_psum[1 * E + e]) + s_psum[2 * E + e]) + s_psum[3 * E + e];
             p.part_counts[(int64_t)blockIdx.x * E + e] = s_counts[e];
         }
     }
@@ -481,18 +626,16 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
 }
 
-template <int CQ>
 int launch_fused(const CUtensorMap& mx, const CUtensorMap& mw, const RFParams& rp, int grid, cudaStream_t stream) {
     static bool attr_set[64] = {false};
     int dev = 0;
     MOE_CUDA_TRY(cudaGetDevice(&dev));
-    const size_t smem = fused_dyn_smem(4 * CQ);
     if (dev < 64 && !attr_set[dev]) {
-        MOE_CUDA_TRY(cudaFuncSetAttribute(route_fused_kernel<CQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)smem));
+        MOE_CUDA_TRY(cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)kSmemBytes));
         attr_set[dev] = true;
     }
-    route_fused_kernel<CQ><<<grid, kRThreads, smem, stream>>>(mx, mw, rp);
+    route_fused_kernel<<<grid, kRThreads, kSmemBytes, stream>>>(mx, mw, rp);
     return launch_status();
 }
 
@@ -532,7 +675,7 @@ int route_fused_run(const void* x, int64_t T, int64_t D, int64_t ldx, const void
     rp.part_psum = part_psum;
     rp.status = status;
     const int grid = route_fused_grid(T);
-    return launch_fused<64>(mx, mw, rp, grid, stream);
+    return launch_fused(mx, mw, rp, grid, stream);
 }
 
 }  // namespace moe

@@ -40,19 +40,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity to complete.
-static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
-    const uint32_t a = smem_u32(bar);
-    if (mbar_try_wait(a, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
+// Non-blocking test of the phase with the given parity (acquire semantics,
+// like try_wait); lets an issuing thread look at the next stage's barrier
+// while its current MMAs are still being accepted by the tensor core.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// The slow path of mbar_wait: polls in bursts of 64 and reads the global
+// timer only between bursts, so a wait that is about to complete does not pay
+// for a timer read.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, int32_t* status) {
+    uint64_t t0 = 0;
+    for (uint32_t n = 0;; ++n) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(a, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        const uint64_t now = globaltimer_ns();
+        if (n == 0) {
+            t0 = now;
+        } else if (now - t0 > kWaitLimitNs) {
             set_status(status, MOE_ERR_TIMEOUT);
             return false;
         }
     }
+}
+
+// Bounded wait for the phase with the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    return mbar_wait_slow(a, parity, status);
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
