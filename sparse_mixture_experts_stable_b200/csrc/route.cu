@@ -33,6 +33,7 @@ constexpr int kMaxE = 1024;
 
 int route_blocks(int64_t T) {
     int64_t b = (T + kRouteWarps - 1) / kRouteWarps;
+    if (b < 2) b = 2;  // the fused kernel runs in CTA pairs
     return (int)(b < kMaxRouteBlocks ? b : kMaxRouteBlocks);
 }
 

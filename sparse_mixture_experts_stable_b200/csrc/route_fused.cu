@@ -8,27 +8,31 @@
 // 128 x E fp32 accumulator in TMEM, and sixteen epilogue warps take it apart
 // in registers.
 //
-// Work split: every CTA (one per SM) owns one contiguous run of tokens whose
-// length is balanced to 32 rows across the grid, so no SM idles in a last
-// partial wave; a run is processed in tiles of up to 128 tokens, and only the
-// 32-row TMA boxes that hold the run's own rows are loaded.
+// Work split: CTAs run in pairs (a two-CTA cluster on two SMs) that share one
+// tcgen05 MMA of 256 tokens x E experts: each CTA stages its own 128 token
+// rows and half of the router weight's rows, and receives its tokens' 128 x E
+// scores in its own tensor memory.  Sharing the weight halves the bytes each
+// SM pulls from L2 per k-block (16 KB of weight beside 16 KB of activations,
+// against 32 KB + 16 KB for a CTA alone), and one thread issues the MMAs of
+// two SMs.  Every pair owns one contiguous run of tokens balanced to 32 rows
+// across the grid; a run is processed in pair tiles of up to 256 tokens, and
+// only the 32-row TMA boxes that hold the run's own rows are loaded.
 //
-// Warp roles (608 threads):
-//   warp 0      TMA producer of the token rows: 5 stages of 16 KB (~80 KB of
-//               activations in flight per SM, what HBM latency needs at this
-//               SM's share of the bandwidth)
-//   warp 1      TMA producer of the router weight: 3 stages of E x 64 (the
-//               weight is re-read from L2 for every tile)
-//   warp 2      TMEM owner and MMA issuer (one lane): two E-column
-//               accumulators, so a tile's epilogue overlaps the next tile's
-//               main loop
-// The two producers feed one ring of barriers: k-block g waits on full[g % 5]
-// (both loads land on it) and releases empty[g % 5] with one commit; the
-// weight producer reuses its stage g % 3 once k-block g - 3 is released.  One
-// wait and one commit per k-block keep the issuing thread's work between two
-// k-blocks short, and the next k-block's barrier is tested while the current
-// one's MMAs are being accepted, since the tensor core takes new MMAs only as
-// it finishes old ones: a late look at the barrier leaves it idle.
+// Warp roles (608 threads per CTA):
+//   warp 0      TMA producer of the CTA's token rows
+//   warp 1      TMA producer of the CTA's half of the router weight (re-read
+//               from L2 for every tile)
+//   warp 2      TMEM owner (both CTAs) and MMA issuer (one lane of the even
+//               CTA): two E-column accumulators, so a tile's epilogue overlaps
+//               the next tile's main loop
+// Both CTAs' producers feed one ring of five 32 KB stages: k-block g's four
+// loads land on the even CTA's full[g % 5], whose two producers arm it with
+// the bytes of both CTAs (the odd CTA's producers only issue their loads), and
+// the MMA commit releases empty[g % 5] in both CTAs.  One wait and one commit per k-block keep the
+// issuing thread's work between two k-blocks short, and the next k-block's
+// barrier is tested while the current one's MMAs are being accepted, since
+// the tensor core takes new MMAs only as it finishes old ones: a late look at
+// the barrier leaves it idle.
 //   warps 3-18  epilogue: warp w reads TMEM lanes 32*(w%4).. (its 32 tokens)
 //               and one quarter of the E columns, 32 columns per TMEM load.
 //
@@ -63,7 +67,8 @@
 //
 // Every mbarrier wait is bounded; after a timeout the producers and the MMA
 // issuer stop, and the epilogue runs its remaining tiles without writing
-// anything, so the named barriers between its warps always complete.
+// anything, so the named barriers between its warps and the closing cluster
+// barrier always complete.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -81,8 +86,7 @@ using namespace tc;
 
 constexpr int kRM = 128;       // tokens per tile (UMMA M)
 constexpr int kRBK = 64;       // K per stage (64 bf16 = one 128-byte swizzle row)
-constexpr int kRAStages = 5;
-constexpr int kRBStages = 3;
+constexpr int kRStages = 5;
 constexpr int kRBox = 32;      // token rows per TMA box
 constexpr int kREpiWarps = 16;
 constexpr int kRThreads = (3 + kREpiWarps) * 32;
@@ -90,7 +94,8 @@ constexpr int kRABytes = kRM * kRBK * 2;  // 16 KB
 constexpr int kRTopK = 8;
 constexpr int kRE = 256;                  // experts (the fused path's only width)
 constexpr int kRCQ = kRE / 4;             // columns per epilogue quarter
-constexpr int kRBBytes = kRE * kRBK * 2;  // 32 KB
+constexpr int kRBBytes = (kRE / 2) * kRBK * 2;  // this CTA's half of the weight: 16 KB
+constexpr int kRStageBytes = kRABytes + kRBBytes;
 
 // Shared memory of one lane-quarter group (the 4 epilogue warps that read the
 // same 32 TMEM lanes): an 8 KB area that holds first the exchange of the
@@ -98,15 +103,14 @@ constexpr int kRBBytes = kRE * kRBK * 2;  // 32 KB
 // of the candidates above tau, and a 4 KB area for the two lists in transit
 // of the final merge.
 constexpr int kExWords = kRTopK + 2;         // per (quarter, token): 8 values, sum, finite flag
-constexpr int kSlots = kRTopK;               // 7 candidates at most, plus one scratch slot
+constexpr int kSlots = kRTopK;               // 7 candidates at most (one spare)
 constexpr int kGroupUnion = kSlots * 128 * 8;  // 8 KB
 constexpr int kGroupMerge = 2 * kRTopK * 32 * 8;  // 4 KB
 static_assert(4 * kExWords * 32 * 4 <= kGroupUnion, "exchange must fit the union area");
 
 // dynamic shared memory layout (offsets from a 1024-byte aligned base)
-constexpr size_t kOffA = 0;
-constexpr size_t kOffB = kOffA + (size_t)kRAStages * kRABytes;
-constexpr size_t kOffBars = kOffB + (size_t)kRBStages * kRBBytes;
+constexpr size_t kOffStages = 0;  // stage s: A at s * 32 KB, the weight half 16 KB after it
+constexpr size_t kOffBars = kOffStages + (size_t)kRStages * kRStageBytes;
 constexpr size_t kOffMisc = kOffBars + 256;
 constexpr size_t kOffBias = kOffMisc + 64;
 constexpr size_t kOffCounts = kOffBias + kRE * 4;
@@ -208,7 +212,7 @@ __device__ __forceinline__ float transpose_sum32(float* a, int lane) {
     return a[0];
 }
 
-__global__ void __launch_bounds__(kRThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRThreads, 1)
     route_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                        const RFParams p) {
     constexpr int E = kRE;
@@ -219,13 +223,12 @@ __global__ void __launch_bounds__(kRThreads, 1)
         if (threadIdx.x == 0) set_status(p.status, MOE_ERR_CUDA);
         return;
     }
-    uint8_t* smA = smem_raw + kOffA;
-    uint8_t* smB = smem_raw + kOffB;
+    uint8_t* stages = smem_raw + kOffStages;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + kOffBars);
-    uint64_t* full = bars;                  // k-block g's A and W have landed (two arrivals + bytes)
-    uint64_t* empty = bars + kRAStages;     // k-block g's MMAs are done
-    uint64_t* tfull = bars + 2 * kRAStages;
-    uint64_t* tempty = tfull + 2;
+    uint64_t* full = bars;                 // even CTA: k-block g's four loads have landed
+    uint64_t* empty = bars + kRStages;     // both CTAs: k-block g's MMAs are done
+    uint64_t* tfull = bars + 2 * kRStages; // both CTAs: the accumulator holds a finished tile
+    uint64_t* tempty = tfull + 2;          // even CTA: both CTAs' epilogues released the accumulator
     uint32_t* s_tmem_p = reinterpret_cast<uint32_t*>(smem_raw + kOffMisc);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem_raw + kOffMisc + 4);
     float* s_bias = reinterpret_cast<float*>(smem_raw + kOffBias);
@@ -233,22 +236,29 @@ __global__ void __launch_bounds__(kRThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();  // 0: issues the MMAs; 1: its partner
+    const bool leader = rank == 0;
 
-    // this CTA's run of tokens, balanced in 32-row units
-    const int64_t u0 = (int64_t)blockIdx.x * p.units / gridDim.x;
-    const int64_t u1 = (int64_t)(blockIdx.x + 1) * p.units / gridDim.x;
+    // the pair's run of tokens, balanced in 32-row units; pair tile i holds rows
+    // row_begin + 256 i .. + 256, this CTA the half starting at 128 * rank
+    const int64_t pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int64_t u0 = pair * p.units / n_pairs;
+    const int64_t u1 = (pair + 1) * p.units / n_pairs;
     const int64_t row_begin = u0 * kRBox;
     const int64_t row_end = u1 * kRBox < p.T ? u1 * kRBox : p.T;
-    const int n_tiles = row_end > row_begin ? (int)((row_end - row_begin + kRM - 1) / kRM) : 0;
+    const int n_tiles = row_end > row_begin ? (int)((row_end - row_begin + 2 * kRM - 1) / (2 * kRM)) : 0;
+    // the even CTA's barriers, as shared::cluster addresses
+    const uint32_t full_l = mapa_shared(smem_u32(full), 0);
+    const uint32_t tempty_l = mapa_shared(smem_u32(tempty), 0);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kRAStages; ++s) {
-            mbar_init(&full[s], 2);
+        for (int s = 0; s < kRStages; ++s) {
+            mbar_init(&full[s], 2);  // the even CTA's A and weight producers
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], kREpiWarps * 32);
+            mbar_init(&tempty[a], 2 * kREpiWarps);  // one arrival per epilogue warp of either CTA
         }
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -256,17 +266,17 @@ __global__ void __launch_bounds__(kRThreads, 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
     }
     if (warp == 2) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem_p)),
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem_p)),
                      "r"(2 * E)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         s_bias[e] = p.bias ? p.bias[e] : 0.f;
         s_counts[e] = 0;
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other's
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem_p;
 
@@ -276,20 +286,25 @@ __global__ void __launch_bounds__(kRThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             for (int i = 0; i < n_tiles && !*s_abort; ++i) {
-                const int64_t r0 = row_begin + (int64_t)i * kRM;
-                const int64_t nrows = row_end - r0 < kRM ? row_end - r0 : kRM;
-                const int nbox = (int)((nrows + kRBox - 1) / kRBox);
+                const int64_t rp = row_begin + (int64_t)i * 2 * kRM;  // the pair tile's first row
+                auto boxes = [&](int64_t r) {  // 32-row boxes of the half starting at row r
+                    const int64_t n = row_end - r < kRM ? (row_end > r ? row_end - r : 0) : kRM;
+                    return (int)((n + kRBox - 1) / kRBox);
+                };
+                const int64_t r0 = rp + (int64_t)rank * kRM;
+                const int nbox = boxes(r0);
+                const uint32_t pair_bytes = (uint32_t)((boxes(rp) + boxes(rp + kRM)) * kRBox * kRBK * 2);
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) {  // k-block g - 5 is done
                         *s_abort = 1;
                         break;
                     }
-                    mbar_expect_tx(&full[stage], (uint32_t)(nbox * kRBox * kRBK * 2));
-                    uint8_t* dst = smA + stage * kRABytes;
+                    const uint32_t fb = full_l + 8u * (uint32_t)stage;
+                    if (leader) mbar_expect_tx(&full[stage], pair_bytes);
+                    uint8_t* dst = stages + stage * kRStageBytes;
                     for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(dst + b * (kRBox * kRBK * 2), &tmX, kb * kRBK, (int32_t)(r0 + b * kRBox),
-                                    &full[stage]);
-                    if (++stage == kRAStages) {
+                        tma_load_2d_pair(dst + b * (kRBox * kRBK * 2), &tmX, kb * kRBK, (int32_t)(r0 + b * kRBox), fb);
+                    if (++stage == kRStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -300,30 +315,31 @@ __global__ void __launch_bounds__(kRThreads, 1)
     } else if (warp == 1) {
         // ------------------------ router-weight producer -----------------------
         if (lane == 0) {
-            static_assert(kRAStages >= kRBStages, "the weight stages are released through the A ring");
-            uint32_t g = 0;  // k-block counter over the whole run
-            int wstage = 0;
+            int stage = 0;
+            uint32_t phase = 0;
             for (int i = 0; i < n_tiles && !*s_abort; ++i) {
-                for (int kb = 0; kb < p.k_blocks; ++kb, ++g) {
-                    if (g >= (uint32_t)kRBStages) {  // stage g % 3 was last read by k-block g - 3
-                        const uint32_t pg = g - kRBStages;
-                        if (!mbar_wait(&empty[pg % kRAStages], (pg / kRAStages) & 1u, p.status)) {
-                            *s_abort = 1;
-                            break;
-                        }
+                for (int kb = 0; kb < p.k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) {
+                        *s_abort = 1;
+                        break;
                     }
-                    mbar_expect_tx(&full[g % kRAStages], (uint32_t)kRBBytes);
-                    tma_load_2d(smB + wstage * kRBBytes, &tmW, kb * kRBK, 0, &full[g % kRAStages]);
-                    if (++wstage == kRBStages) wstage = 0;
+                    const uint32_t fb = full_l + 8u * (uint32_t)stage;
+                    if (leader) mbar_expect_tx(&full[stage], 2u * (uint32_t)kRBBytes);
+                    tma_load_2d_pair(stages + stage * kRStageBytes + kRABytes, &tmW, kb * kRBK,
+                                     (int32_t)(rank * (kRE / 2)), fb);
+                    if (++stage == kRStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
         }
         __syncwarp();
     } else if (warp == 2) {
         // ------------------------------ MMA issuer -----------------------------
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc(kRM, E);
-            int sa = 0, sb = 0;
+        if (lane == 0 && leader) {
+            const uint32_t idesc = make_idesc(2 * kRM, E);
+            int sa = 0;
             uint32_t pa = 0;
             const uint32_t full0 = smem_u32(full);
             bool ready = mbar_test(full0, 0u);
@@ -342,25 +358,24 @@ __global__ void __launch_bounds__(kRThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t ad = sw128_desc(smem_u32(smA + sa * kRABytes));
-                    const uint64_t bd = sw128_desc(smem_u32(smB + sb * kRBBytes));
-                    const int sn = sa + 1 == kRAStages ? 0 : sa + 1;
-                    const uint32_t pn = sa + 1 == kRAStages ? pa ^ 1u : pa;
-                    tc_mma(d_tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);
-                    tc_mma(d_tmem, ad + 2, bd + 2, idesc, 1u);
+                    const uint64_t ad = sw128_desc(smem_u32(stages + sa * kRStageBytes));
+                    const uint64_t bd = sw128_desc(smem_u32(stages + sa * kRStageBytes + kRABytes));
+                    const int sn = sa + 1 == kRStages ? 0 : sa + 1;
+                    const uint32_t pn = sa + 1 == kRStages ? pa ^ 1u : pa;
+                    tc_mma_pair(d_tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);
+                    tc_mma_pair(d_tmem, ad + 2, bd + 2, idesc, 1u);
                     ready = mbar_test(full0 + 8u * (uint32_t)sn, pn);  // the next k-block, early
-                    tc_mma(d_tmem, ad + 4, bd + 4, idesc, 1u);
-                    tc_mma(d_tmem, ad + 6, bd + 6, idesc, 1u);
-                    tc_commit(&empty[sa]);
+                    tc_mma_pair(d_tmem, ad + 4, bd + 4, idesc, 1u);
+                    tc_mma_pair(d_tmem, ad + 6, bd + 6, idesc, 1u);
+                    tc_commit_pair(&empty[sa]);
                     sa = sn;
                     pa = pn;
-                    if (++sb == kRBStages) sb = 0;
                 }
                 if (!ok) {
                     *s_abort = 1;
                     break;
                 }
-                tc_commit(&tfull[acc]);
+                tc_commit_pair(&tfull[acc]);
             }
         }
         __syncwarp();
@@ -377,7 +392,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         float* s_mv = reinterpret_cast<float*>(smem_raw + kOffMerge + (size_t)q * kGroupMerge);  // [list][j][lane]
         int* s_mi = reinterpret_cast<int*>(smem_raw + kOffMerge + (size_t)q * kGroupMerge + kGroupMerge / 2);
         const uint32_t slot_base = smem_u32(s_slot) + (uint32_t)tig * 8u;
-        const uint32_t slot_last = slot_base + (uint32_t)(kSlots - 1) * 1024u;  // the scratch slot
+        const uint32_t slot_last = slot_base + (uint32_t)(kSlots - 1) * 1024u;
         float acc_ps[2] = {0.f, 0.f};
 
         for (int i = 0; i < n_tiles; ++i) {
@@ -387,7 +402,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) *s_abort = 1;
             tc_fence_after();
-            const int64_t r0 = row_begin + (int64_t)i * kRM;
+            const int64_t r0 = row_begin + (int64_t)i * 2 * kRM + (int64_t)rank * kRM;
             const bool valid = r0 + row < row_end;
             const int64_t t = r0 + row;
             const bool write = valid && !*s_abort;
@@ -511,9 +526,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
                         const float xv = __uint_as_float(r[j]) + bb[u];
                         pr[j] = fminf(ex2_approx(fmaf(xv, kLog2e, -cL)), pcap);  // fminf drops a NaN
                         // a score above tau goes to the next slot; one equal to tau sets its bit
-                        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(slot), "f"(xv),
-                                     "f"(__int_as_float(c * CQ + 32 * h + j)));
-                        slot = min(slot + (xv > tau ? 1024u : 0u), slot_last);  // seven at most, capped anyway
+                        if (xv > tau && slot <= slot_last) {  // seven at most; the bound only guards the area
+                            asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(slot), "f"(xv),
+                                         "f"(__int_as_float(c * CQ + 32 * h + j)));
+                            slot += 1024u;
+                        }
                         eqb |= xv == tau ? (1u << j) : 0u;
                     }
                 }
@@ -522,7 +539,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 acc_ps[h] += cs;
             }
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);  // the accumulator is no longer read: the next tile may use it
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_l + 8u * acc);  // the next tile may use the accumulator
 
             // ---- select: the quarter's candidates in (score desc, index asc) order ----
             float tv[kRTopK];
@@ -532,7 +550,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 tv[j] = -INFINITY;
                 ti[j] = c * CQ + j;
             }
-            const int n_gt = (int)((slot - slot_base) >> 10);
+            const int n_gt = (int)((slot - slot_base) >> 10);  // <= kSlots
             for (int s = 0; s < n_gt; ++s) {
                 float2 e;
                 asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(e.x), "=f"(e.y) : "r"(slot_base + 1024u * (uint32_t)s));
@@ -619,10 +637,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // neither CTA leaves while the other may still signal its barriers or read its stages
     if (warp == 2) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(2 * E) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(2 * E) : "memory");
     }
 }
 
@@ -649,8 +667,8 @@ bool route_fused_supported(int64_t T, int64_t D, int64_t ldx, const void* x, con
 
 int route_fused_grid(int64_t T) {
     const int64_t units = (T + kRBox - 1) / kRBox;
-    const int sms = device_sm_count();
-    return (int)(units < sms ? units : sms);
+    const int64_t pairs = device_sm_count() / 2;
+    return 2 * (int)(units < pairs ? units : pairs);
 }
 
 int route_fused_run(const void* x, int64_t T, int64_t D, int64_t ldx, const void* w_ed, int32_t E,
@@ -659,7 +677,7 @@ int route_fused_run(const void* x, int64_t T, int64_t D, int64_t ldx, const void
     MOE_REQUIRE(route_fused_supported(T, D, ldx, x, w_ed, E, k), MOE_ERR_UNSUPPORTED);
     CUtensorMap mx, mw;
     MOE_REQUIRE(make_map(&mx, x, D, T, ldx, kRBox), MOE_ERR_CUDA);
-    MOE_REQUIRE(make_map(&mw, w_ed, D, E, D, E), MOE_ERR_CUDA);
+    MOE_REQUIRE(make_map(&mw, w_ed, D, E, D, E / 2), MOE_ERR_CUDA);
     RFParams rp{};
     rp.T = T;
     rp.units = (T + kRBox - 1) / kRBox;
