@@ -43,11 +43,7 @@ size_t fp32_split_bytes(moe_ffn_kind kind, int32_t E, int64_t C, int64_t D, int6
 }  // namespace
 
 namespace {
-constexpr size_t kTileCounterBytes = 256;  // after the intermediate h: scratch words of the wide GEMMs' schedulers
-// The routed down projection (K = F = 512) through the 256 x 256 single-buffered tile measured
-// slower than tc_gemm's double-buffered 128-token tiles (186 against ~118 us at T = 8192, E = 128):
-// with a short K loop the TMEM drain is a large share of each tile.  tc_gemm keeps it.
-constexpr bool kWideDown = false;
+constexpr size_t kTileCounterBytes = 256;  // after the intermediate h: scratch words of the wide GEMM's scheduler
 }
 
 extern "C" size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dtype, int32_t E, int64_t C, int64_t D,
@@ -57,41 +53,16 @@ extern "C" size_t moe_expert_ffn_workspace_size(moe_ffn_kind kind, moe_dtype dty
     if (kind != MOE_FFN_LINEAR && F >= 1) h = align_up((size_t)E * C * F * dtype_size(dtype), 1024);
     if (dtype == MOE_F32 && D >= 1 && Dout >= 1 && (kind == MOE_FFN_LINEAR || F >= 1))
         return h + fp32_split_bytes(kind, E, C, D, F, Dout);
-    if (kind == MOE_FFN_SWIGLU && F >= 1) h += kTileCounterBytes;  // tile counters of the wide GEMMs
+    if (kind == MOE_FFN_SWIGLU && F >= 1) h += kTileCounterBytes;  // the wide GEMM's tile counter
     return h;
 }
 
 namespace {
 
-// Second GEMM of the bf16 MLP experts: ybuf = h (E*C, F) x W2^T (+ b2).  tile_counter:
-// a device word of scratch for the routed SwiGLU form (tcw_gemm_run).
+// Second GEMM of the bf16 MLP experts: ybuf = h (E*C, F) x W2^T (+ b2).
 int down_projection(moe_ffn_kind kind, const void* h, const int32_t* used, int32_t E, int64_t C, int64_t F,
                     int64_t Dout, const void* w2, const void* b2, void* ybuf, int32_t* dev_status,
-                    cudaStream_t stream, uint32_t* tile_counter = nullptr) {
-    if (kind == MOE_FFN_SWIGLU && used != nullptr && tile_counter != nullptr && kWideDown) {
-        // routed experts: 256 output features x up to 256 tokens per tile (tc_wide_gemm.cu)
-        TcxProblem p{};
-        p.w = w2;
-        p.ldw = F;
-        p.w_rows_total = (int64_t)E * Dout;
-        p.w_rows_per_group = Dout;
-        p.x = h;
-        p.ldx = F;
-        p.x_rows_total = (int64_t)E * C;
-        p.x_rows_per_group = C;
-        p.G = E;
-        p.features = Dout;
-        p.max_tokens = C;
-        p.K = F;
-        p.rows = used;
-        p.out = ybuf;
-        p.ldo = Dout;
-        p.out_rows_per_group = C;
-        p.epilogue = TC_EPI_BF16;
-        p.status = dev_status;
-        p.tile_counter = tile_counter;
-        return tcw_gemm_run(p, stream);
-    }
+                    cudaStream_t stream) {
     TcGemmProblem q{};
     q.a = h;
     q.lda = F;
@@ -245,11 +216,7 @@ int expert_ffn(moe_ffn_kind kind, moe_dtype dtype, const void* xbuf, const int32
             rc = tc_gemm_run(p, stream);
         }
         if (rc != MOE_OK) return rc;
-        uint32_t* counters = kind == MOE_FFN_SWIGLU
-                                 ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + h_bytes)
-                                 : nullptr;
-        return down_projection(kind, h, used, E, C, F, Dout, w2, b2, ybuf, dev_status, stream,
-                               counters ? counters + 1 : nullptr);
+        return down_projection(kind, h, used, E, C, F, Dout, w2, b2, ybuf, dev_status, stream);
     }
 
     // fp32: split-tf32 tensor-core GEMMs, B = weights in (out, in) layout -> transposed operand
@@ -363,7 +330,5 @@ extern "C" int moe_expert_ffn_gathered(moe_ffn_kind kind, moe_dtype dtype, const
     p.status = dev_status;
     const int rc = tcx_gemm_run(p, stream);
     if (rc != MOE_OK) return rc;
-    uint32_t* counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) +
-                                                     align_up((size_t)E * C * F * 2, 1024));
-    return down_projection(kind, h, used, E, C, F, Dout, w2, nullptr, ybuf, dev_status, stream, counters + 1);
+    return down_projection(kind, h, used, E, C, F, Dout, w2, nullptr, ybuf, dev_status, stream);
 }

@@ -345,7 +345,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRThreads, 1)
             bool ready = mbar_test(full0, 0u);
             for (int i = 0; i < n_tiles && !*s_abort; ++i) {
                 const uint32_t acc = (uint32_t)i & 1u;
-                if (!mbar_wait(&tempty[acc], (((uint32_t)i >> 1) & 1u) ^ 1u, p.status)) {
+                if (!mbar_wait_cluster(&tempty[acc], (((uint32_t)i >> 1) & 1u) ^ 1u, p.status)) {
                     *s_abort = 1;
                     break;
                 }

@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
             int stage = 0;
             uint32_t phase = 0;
             uint32_t it = 0;
+            bool ready = false;  // full[stage] was seen complete by an early test
             for (int tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x, ++it) {
                 int g, ft, tt;
                 decode(tile, s_prefix, p.G, p.f_tiles, g, ft, tt);
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
                 const uint32_t d = tmem_base + acc * kAccCols;
                 bool ok = true;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, p.status)) {
+                    if (!ready && !mbar_wait(&full[stage], phase, p.status)) {
                         s_abort = 1;
                         ok = false;
                         break;
@@ -210,17 +211,20 @@ __global__ void __launch_bounds__(GATHER ? kThreads + kGatherThreads : kThreads,
                     const uint32_t st = smem_u32(stages + stage * kStageBytes);
                     const uint64_t wd = sw128_desc(st);
                     const uint64_t xd = sw128_desc(st + x_off);
+                    const int ns = stage + 1 == kStages ? 0 : stage + 1;
+                    const uint32_t np = stage + 1 == kStages ? phase ^ 1u : phase;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
                         tc_mma(d, wd + 2 * kk, xd + 2 * kk, idesc, accum);
                         tc_mma(d + 128, sw128_desc(st + 16 * 1024) + 2 * kk, xd + 2 * kk, idesc, accum);
+                        // the tensor core takes new MMAs only as it finishes old ones: look at the
+                        // next stage while this one's MMAs are being accepted
+                        if (kk == 1) ready = mbar_test(smem_u32(&full[ns]), np);
                     }
                     tc_commit(&empty[stage]);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    stage = ns;
+                    phase = np;
                 }
                 if (!ok) break;
                 tc_commit(&tfull[acc]);

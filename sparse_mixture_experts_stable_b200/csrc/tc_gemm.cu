@@ -250,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         uint32_t it = 0;
+        bool ready = false;  // lane 0: full[stage] was seen complete by an early test
         for (int tile = blockIdx.x;; tile += gridDim.x, ++it) {
             // one decision for the whole warp (s_abort may be raised by another warp meanwhile)
             if (!__shfl_sync(0xffffffffu, (tile < total && !s_abort) ? 1 : 0, 0)) break;
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int kend = nkk * 16;
                 const bool clear = last && kvalid_last < kend;
                 int okf = 1;
-                if (lane == 0 || clear) okf = mbar_wait(&full[stage], phase, p.status) ? 1 : 0;
+                if ((lane == 0 && !ready) || (lane != 0 && clear)) okf = mbar_wait(&full[stage], phase, p.status) ? 1 : 0;
                 okf = __all_sync(0xffffffffu, okf);
                 if (!okf) {
                     s_abort = 1;
@@ -319,11 +320,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = BMN ? sw128_mn_desc(smem_u32(smB + stage * kBBytes), 8192)
                                             : sw128_desc(smem_u32(smB + stage * kBBytes));
                     // a K step of 16: 32 bytes along a K-major row, or two 1024-byte groups of 8 K rows
+                    const int ns = stage + 1 == kStages ? 0 : stage + 1;
+                    const uint32_t np = stage + 1 == kStages ? phase ^ 1u : phase;
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
                         if (kk < nkk)
                             tc_mma(d_tmem, ad + (AMN ? 128 : 2) * kk, bd + (BMN ? 128 : 2) * kk, idesc,
                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                        // the tensor core takes new MMAs only as it finishes old ones: look at the
+                        // next stage while this one's MMAs are being accepted
+                        if (kk == 1) ready = mbar_test(smem_u32(&full[ns]), np);
+                    }
                     tc_commit(&empty[stage]);
                 }
                 __syncwarp();

@@ -73,6 +73,40 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, 
     }
 }
 
+// Bounded wait with acquire semantics at cluster scope, for a barrier that
+// the other CTA of a pair arrives on (its writes before a release.cluster
+// arrive are visible after this returns).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+static __device__ __noinline__ bool mbar_wait_cluster_slow(uint32_t a, uint32_t parity, int32_t* status) {
+    uint64_t t0 = 0;
+    for (uint32_t n = 0;; ++n) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_cluster(a, parity)) return true;
+        const uint64_t now = globaltimer_ns();
+        if (n == 0) {
+            t0 = now;
+        } else if (now - t0 > kWaitLimitNs) {
+            set_status(status, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int32_t* status) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    return mbar_wait_cluster_slow(a, parity, status);
+}
+
 // Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
     const uint32_t a = smem_u32(bar);

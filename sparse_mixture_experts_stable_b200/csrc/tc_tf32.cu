@@ -269,6 +269,7 @@ __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             uint32_t it = 0;
+            bool ready = false;  // the next stage was seen complete by an early test
             for (int tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x, ++it) {
                 const uint32_t acc = it & 1u;
                 const uint32_t acc_phase = (it >> 1) & 1u;
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
                 const uint32_t d_tmem = tmem_base + acc * kAccCols;
                 bool ok = true;
                 for (int kb = 0; kb < p.k_blocks; ++kb) {
-                    if (!mbar_wait(any_raw ? &conv[stage] : &full[stage], phase, p.status)) {
+                    if (!ready && !mbar_wait(any_raw ? &conv[stage] : &full[stage], phase, p.status)) {
                         s_abort = 1;
                         ok = false;
                         break;
@@ -295,18 +296,21 @@ __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
                     const uint64_t bl =
                         p.b_mn ? sw128_mn_desc(st + 3 * kTileBytes, 4096) : sw128_desc(st + 3 * kTileBytes);
                     const uint32_t sa = p.a_mn ? 64u : 2u, sb = p.b_mn ? 64u : 2u;
+                    const int ns = stage + 1 == kStages ? 0 : stage + 1;
+                    const uint32_t np = stage + 1 == kStages ? phase ^ 1u : phase;
 #pragma unroll
                     for (int ks = 0; ks < kBK / 8; ++ks) {
                         const uint32_t first = (kb == 0 && ks == 0) ? 0u : 1u;
                         mma_tf32(d_tmem, al + sa * ks, bh + sb * ks, idesc, first);
                         mma_tf32(d_tmem, ah + sa * ks, bl + sb * ks, idesc, 1u);
                         mma_tf32(d_tmem, ah + sa * ks, bh + sb * ks, idesc, 1u);
+                        // the tensor core takes new MMAs only as it finishes old ones: look at the
+                        // next stage while this one's MMAs are being accepted
+                        if (ks == 1) ready = mbar_test(smem_u32(any_raw ? &conv[ns] : &full[ns]), np);
                     }
                     tc_commit(&empty[stage]);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    stage = ns;
+                    phase = np;
                 }
                 if (!ok) break;
                 tc_commit(&tfull[acc]);
