@@ -58,6 +58,7 @@ struct KParams {
     const void* bias;
     int64_t bias_group_stride;
     int vec_ok;
+    int tma_out;  // fp32 output through TMA stores (every tile row valid, N a multiple of 32)
     int32_t* status;
 };
 
@@ -135,10 +136,12 @@ __device__ __forceinline__ void pipelined_chunks(uint32_t t_row, int n, F&& proc
 template <int EPI, bool AMN, bool BMN>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB2, const KParams p) {
+                   const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
+                   const KParams p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_prefix[kMaxGroups + 1];
-    __shared__ __align__(16) uint32_t s_stage[4][32 * 32];  // epilogue staging, one 32 x 32 chunk per warp
+    // epilogue staging, one 32 x 32 chunk per warp (1024-aligned: the TMA store reads it 128-byte swizzled)
+    __shared__ __align__(1024) uint32_t s_stage[4][32 * 32];
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
 
@@ -420,6 +423,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (n0 + i < p.N) dst[n0 + i] = __uint_as_float(r[i]);
                     }
                 }
+            } else if (EPI == TC_EPI_F32 && AMN && BMN && p.tma_out) {
+                // the weight-gradient form: every row valid, full 32-column chunks.  Each chunk goes
+                // to the warp's staging buffer in the map's 128-byte swizzled layout (conflict-free:
+                // lane = row) and one lane hands it to the TMA, which streams it out while the warp
+                // drains the next chunk; the buffer is rewritten only once the TMA has read it.
+                auto process = [&](const int c, const uint32_t (&r)[32]) {
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+#pragma unroll
+                    for (int m = 0; m < 8; ++m)
+                        *reinterpret_cast<uint4*>(stg + lane * 32 + 4 * (m ^ (lane & 7))) =
+                            make_uint4(r[4 * m], r[4 * m + 1], r[4 * m + 2], r[4 * m + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmOut, stg, (int32_t)(nt * p.tile_n_out + c * 32), (int32_t)out_wrow0);
+                        bulk_commit();
+                    }
+                };
+                pipelined_chunks(t_row, p.n_mma / 32, process);
             } else if (EPI == TC_EPI_F32) {
                 float* orow = reinterpret_cast<float*>(p.out) + out_row * p.ldo;
                 const float* bias = reinterpret_cast<const float*>(p.bias);
@@ -477,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&tempty[acc]);
             if (s_abort) break;
         }
+        if (EPI == TC_EPI_F32 && AMN && BMN && p.tma_out && lane == 0) bulk_wait_all();  // stores done before exit
     }
 
     __syncthreads();
@@ -540,8 +564,8 @@ bool make_map_f32(CUtensorMap* m, const void* base, int64_t inner, int64_t rows,
 namespace {
 
 template <int EPI, bool AMN = false, bool BMN = false>
-int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const KParams& kp, int grid,
-           cudaStream_t stream) {
+int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const CUtensorMap& out,
+           const KParams& kp, int grid, cudaStream_t stream) {
     static bool attr_set[64] = {false};
     int dev = 0;
     MOE_CUDA_TRY(cudaGetDevice(&dev));
@@ -550,7 +574,7 @@ int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, co
                                           (int)kSmemBytes));
         attr_set[dev] = true;
     }
-    tc_gemm_kernel<EPI, AMN, BMN><<<grid, kThreads, kSmemBytes, stream>>>(a, b, b2, kp);
+    tc_gemm_kernel<EPI, AMN, BMN><<<grid, kThreads, kSmemBytes, stream>>>(a, b, b2, out, kp);
     return launch_status();
 }
 
@@ -613,8 +637,12 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     kp.vec_ok = aligned16(p.out) && (p.ldo * (int64_t)esz) % 16 == 0;
     if (p.epilogue == TC_EPI_F32_DUAL) kp.vec_ok = kp.vec_ok && (p.N * 4) % 16 == 0;
     kp.status = p.status;
+    // the weight-gradient form writes whole 32 x 32 fp32 boxes through the TMA
+    kp.tma_out = p.a_mn_major && p.epilogue == TC_EPI_F32 && p.rows == nullptr && p.bias == nullptr &&
+                 p.M % kBM == 0 && p.N % 32 == 0 && kp.vec_ok && p.out_rows_per_group >= p.M &&
+                 (int64_t)p.G * p.out_rows_per_group < (int64_t(1) << 31);
 
-    CUtensorMap ma, mb, mb2;
+    CUtensorMap ma, mb, mb2, mo;
     if (p.a_mn_major)  // (K rows, M columns) with 64 x 64 boxes
         MOE_REQUIRE(make_map(&ma, p.a, p.M, p.a_rows_total, p.lda, kBK), MOE_ERR_CUDA);
     else
@@ -636,17 +664,21 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     if (max_tiles < grid) grid = (int)max_tiles;
     if (grid < 1) grid = 1;
 
-    if (p.a_mn_major) return launch<TC_EPI_F32, true, true>(ma, mb, mb2, kp, grid, stream);
+    if (kp.tma_out)
+        MOE_REQUIRE(make_map_f32(&mo, p.out, p.N, (int64_t)p.G * p.out_rows_per_group, p.ldo, 32), MOE_ERR_CUDA);
+    else
+        mo = ma;  // unused
+    if (p.a_mn_major) return launch<TC_EPI_F32, true, true>(ma, mb, mb2, mo, kp, grid, stream);
     if (p.b_mn_major)
-        return p.epilogue == TC_EPI_F32 ? launch<TC_EPI_F32, false, true>(ma, mb, mb2, kp, grid, stream)
-                                        : launch<TC_EPI_BF16, false, true>(ma, mb, mb2, kp, grid, stream);
+        return p.epilogue == TC_EPI_F32 ? launch<TC_EPI_F32, false, true>(ma, mb, mb2, mo, kp, grid, stream)
+                                        : launch<TC_EPI_BF16, false, true>(ma, mb, mb2, mo, kp, grid, stream);
     switch (p.epilogue) {
-        case TC_EPI_F32: return launch<TC_EPI_F32>(ma, mb, mb2, kp, grid, stream);
-        case TC_EPI_BF16: return launch<TC_EPI_BF16>(ma, mb, mb2, kp, grid, stream);
-        case TC_EPI_BF16_BIAS: return launch<TC_EPI_BF16_BIAS>(ma, mb, mb2, kp, grid, stream);
-        case TC_EPI_GELU_BIAS: return launch<TC_EPI_GELU_BIAS>(ma, mb, mb2, kp, grid, stream);
-        case TC_EPI_SWIGLU: return launch<TC_EPI_SWIGLU>(ma, mb, mb2, kp, grid, stream);
-        case TC_EPI_F32_DUAL: return launch<TC_EPI_F32_DUAL>(ma, mb, mb2, kp, grid, stream);
+        case TC_EPI_F32: return launch<TC_EPI_F32>(ma, mb, mb2, mo, kp, grid, stream);
+        case TC_EPI_BF16: return launch<TC_EPI_BF16>(ma, mb, mb2, mo, kp, grid, stream);
+        case TC_EPI_BF16_BIAS: return launch<TC_EPI_BF16_BIAS>(ma, mb, mb2, mo, kp, grid, stream);
+        case TC_EPI_GELU_BIAS: return launch<TC_EPI_GELU_BIAS>(ma, mb, mb2, mo, kp, grid, stream);
+        case TC_EPI_SWIGLU: return launch<TC_EPI_SWIGLU>(ma, mb, mb2, mo, kp, grid, stream);
+        case TC_EPI_F32_DUAL: return launch<TC_EPI_F32_DUAL>(ma, mb, mb2, mo, kp, grid, stream);
         default: return MOE_ERR_INVALID_ARG;
     }
 }
