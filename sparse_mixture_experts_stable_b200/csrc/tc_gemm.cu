@@ -561,6 +561,21 @@ bool make_map_f32(CUtensorMap* m, const void* base, int64_t inner, int64_t rows,
     return r == CUDA_SUCCESS;
 }
 
+// 2-D fp32 map read MN-major by the tf32 MMA: box = box_rows x 32 elements (128
+// bytes), 128-byte swizzle of 32-byte chunks (the layout tf32 MN-major operands take).
+bool make_map_f32_mn(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld_elems, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld_elems * 4};
+    cuuint32_t box[2] = {32u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 template <int EPI, bool AMN = false, bool BMN = false>

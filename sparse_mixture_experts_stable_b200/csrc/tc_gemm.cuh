@@ -66,5 +66,7 @@ bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int
 
 // The same for fp32 elements: box = box_rows x 32 elements (128 bytes).
 bool make_map_f32(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld_elems, int box_rows);
+// fp32, box_rows x 32, 128-byte swizzle of 32-byte chunks: MN-major tf32 operands.
+bool make_map_f32_mn(CUtensorMap* m, const void* base, int64_t inner, int64_t rows, int64_t ld_elems, int box_rows);
 
 }  // namespace moe

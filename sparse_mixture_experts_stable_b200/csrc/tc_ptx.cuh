@@ -250,6 +250,21 @@ __device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t lbo_b
     return d;
 }
 
+// Shared-memory descriptor of an MN-major 32-bit operand (tf32) in the layout
+// of a TMA load with 128-byte swizzle on a 32-byte base: K rows of 128 bytes (32
+// elements along MN), the 32-byte chunks of row r permuted by r % 4, groups of
+// four K rows 512 bytes apart (layout type 1); the next 32 MN elements start
+// lbo_bytes further on.
+__device__ __forceinline__ uint64_t sw128b32_mn_desc(uint32_t saddr, uint32_t lbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);          // start address (16-byte units)
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset: next 32 MN elements
+    d |= (uint64_t)(512 >> 4) << 32;                    // stride byte offset: next 4 K rows
+    d |= (uint64_t)1 << 46;                             // descriptor version for tcgen05
+    d |= (uint64_t)1 << 61;                             // layout: 128-byte swizzle, 32-byte base
+    return d;
+}
+
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major.
 __device__ __forceinline__ uint32_t make_idesc(int m, int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);

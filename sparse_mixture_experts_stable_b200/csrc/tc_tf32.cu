@@ -39,8 +39,9 @@ constexpr int kBK = 32;                  // fp32 elements per 128-byte swizzle r
 constexpr int kStages = 3;
 constexpr int kThreads = 192;
 constexpr int kConvThreads = 128;  // converter warps for raw operands (after the 192 threads above)
-// MN-major raw operands (tf32 MMA with the transpose bits): off until checked on the hardware.
-constexpr bool kRawMnMajor = false;
+// MN-major raw operands: TMA-loaded with the 128-byte swizzle on a 32-byte base, the layout
+// the tf32 MMA reads with its transpose bits (layout type 1 in the shared-memory descriptor).
+constexpr bool kRawMnMajor = true;
 constexpr int kMaxGroups = 1024;
 constexpr int kTileBytes = 128 * kBK * 4;   // 16 KB per operand tile
 constexpr int kStageBytes = 4 * kTileBytes;  // A hi, A lo, B hi, B lo
@@ -290,11 +291,12 @@ __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
                     const uint32_t st = smem_u32(smem + stage * kStageBytes);
                     // K-major: a K step of 8 is 32 bytes along the row (2 descriptor units); MN-major:
                     // 8 K rows of 128 bytes (64 units), atoms 4 KB apart
-                    const uint64_t ah = p.a_mn ? sw128_mn_desc(st, 4096) : sw128_desc(st);
-                    const uint64_t al = p.a_mn ? sw128_mn_desc(st + kTileBytes, 4096) : sw128_desc(st + kTileBytes);
-                    const uint64_t bh = p.b_mn ? sw128_mn_desc(st + 2 * kTileBytes, 4096) : sw128_desc(st + 2 * kTileBytes);
+                    const uint64_t ah = p.a_mn ? sw128b32_mn_desc(st, 4096) : sw128_desc(st);
+                    const uint64_t al = p.a_mn ? sw128b32_mn_desc(st + kTileBytes, 4096) : sw128_desc(st + kTileBytes);
+                    const uint64_t bh =
+                        p.b_mn ? sw128b32_mn_desc(st + 2 * kTileBytes, 4096) : sw128_desc(st + 2 * kTileBytes);
                     const uint64_t bl =
-                        p.b_mn ? sw128_mn_desc(st + 3 * kTileBytes, 4096) : sw128_desc(st + 3 * kTileBytes);
+                        p.b_mn ? sw128b32_mn_desc(st + 3 * kTileBytes, 4096) : sw128_desc(st + 3 * kTileBytes);
                     const uint32_t sa = p.a_mn ? 64u : 2u, sb = p.b_mn ? 64u : 2u;
                     const int ns = stage + 1 == kStages ? 0 : stage + 1;
                     const uint32_t np = stage + 1 == kStages ? phase ^ 1u : phase;
@@ -585,7 +587,7 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
 
     CUtensorMap mah, mal, mbh, mbl;
     if (a_mn) {  // the (K rows, M columns) operand in 32 x 32 boxes
-        MOE_REQUIRE(make_map_f32(&mah, g.A, g.M, (int64_t)g.groups * a_rpg, g.lda, 32), MOE_ERR_CUDA);
+        MOE_REQUIRE(make_map_f32_mn(&mah, g.A, g.M, (int64_t)g.groups * a_rpg, g.lda, 32), MOE_ERR_CUDA);
         mal = mah;
     } else if (a_raw) {  // the operand itself: K columns (zero fill up to Kp), row stride lda
         MOE_REQUIRE(make_map_f32(&mah, g.A, g.K, (int64_t)g.groups * g.M, g.lda, kBM), MOE_ERR_CUDA);
@@ -595,7 +597,7 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
         MOE_REQUIRE(make_map_f32(&mal, a_lo, l.Kp, (int64_t)g.groups * g.M, l.Kp, kBM), MOE_ERR_CUDA);
     }
     if (b_mn) {
-        MOE_REQUIRE(make_map_f32(&mbh, g.B, g.N, (int64_t)g.groups * b_rpg, g.ldb, 32), MOE_ERR_CUDA);
+        MOE_REQUIRE(make_map_f32_mn(&mbh, g.B, g.N, (int64_t)g.groups * b_rpg, g.ldb, 32), MOE_ERR_CUDA);
         mbl = mbh;
     } else if (b_raw) {
         MOE_REQUIRE(make_map_f32(&mbh, g.B, g.K, (int64_t)g.groups * g.N, g.ldb, kp.n_mma), MOE_ERR_CUDA);
