@@ -188,8 +188,11 @@ MOE_API int moe_route_ex(const void* x, moe_dtype dtype, int64_t T, int64_t D, i
  *   db_router[e]   = sum_t dlogits[t,e]                   fp32 (E), fixed order
  * ([P2] s = x . w_e is linear in x, w and b.)  The layer's full input
  * gradient is the expert backward's dx plus dx_router.  Both products run on
- * the tensor cores as split-tf32 (fp32 accuracy; bf16 x and w are read as
- * they are).  Any of the three outputs may be NULL to skip it.
+ * the tensor cores with fp32 accuracy: for bf16 x and w with E and D multiples
+ * of 64, dlogits is split into three bf16 parts (24 mantissa bits; each
+ * product with a bf16 x or w is exact in the fp32 accumulator) and bf16 GEMMs
+ * take them; otherwise as split-tf32.  Any of the three outputs may be NULL to
+ * skip it.
  *   x          device (T, D), row stride ldx, dtype `dtype`.
  *   w_router   device, layout `layout`, dtype `dtype`.
  *   dlogits    device fp32 (T, E).

@@ -697,6 +697,157 @@ RouterBwdWs router_bwd_layout(const F32Gemm& gx, const F32Gemm& gw, int32_t E) {
     return l;
 }
 
+// ---- the bf16 router backward: dlogits in three bf16 parts on the bf16 tensor cores ----
+//
+// x and W_r in bf16 are exact in any wider format, so the only operand that
+// needs more than bf16 is dlogits (fp32).  It is split as g = g1 + g2 + g3
+// with g1 = bf16(g), g2 = bf16(g - g1), g3 = bf16(g - g1 - g2): 24 mantissa bits
+// in all, each product g_i * x (or g_i * W) exact in the fp32 accumulator.  So
+//   dx = [g1 | g2 | g3] . [W; W; W]     one bf16 GEMM with K = 3E
+//   dW = sum_i g_i^T x                  three bf16 GEMMs reading g_i in place,
+//                                       the reduction over the tokens split in S
+//                                       groups, all partials summed in a fixed order.
+
+__global__ void split3_bf16_kernel(const float* __restrict__ g, int64_t n, int E, __nv_bfloat16* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / E;
+        const int e = (int)(i - t * E);
+        const float v = g[i];
+        const __nv_bfloat16 h1 = __float2bfloat16_rn(v);
+        const float r1 = v - __bfloat162float(h1);
+        const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(h2);
+        __nv_bfloat16* row = out + t * 3 * E;
+        row[e] = h1;
+        row[E + e] = h2;
+        row[2 * E + e] = __float2bfloat16_rn(r2);
+    }
+}
+
+// token groups of the weight gradient (each a multiple of 64 tokens, so no group
+// reads into the next); one group when T is not a multiple of 64
+int router_bwd_bf16_groups(int64_t T) {
+    int s = 1;
+    while (s < 8 && T % (128 * s) == 0 && T / (2 * s) >= 1024) s *= 2;
+    return s;
+}
+
+bool router_bwd_bf16_shape_ok(int64_t D, int32_t E) { return E % 64 == 0 && D % 64 == 0; }
+
+struct RouterBwdBf16Ws {
+    size_t parts, wrep, partials, colsum, total;
+};
+
+RouterBwdBf16Ws router_bwd_bf16_layout(int64_t T, int64_t D, int32_t E) {
+    RouterBwdBf16Ws l{};
+    size_t off = 0;
+    l.parts = off;
+    off += align_up((size_t)T * 3 * E * 2, 256);
+    l.wrep = off;
+    off += align_up((size_t)3 * E * D * 2, 256);
+    l.partials = off;
+    off += align_up((size_t)3 * router_bwd_bf16_groups(T) * E * D * 4, 256);
+    l.colsum = off;
+    off += align_up((size_t)kColChunks * E * 4, 256);
+    l.total = off;
+    return l;
+}
+
+int router_backward_bf16(const void* x, int64_t T, int64_t D, int64_t ldx, const void* w, moe_router_layout layout,
+                         int32_t E, const float* dlogits, float* dx, float* dw, int32_t* status, uint8_t* ws,
+                         const RouterBwdBf16Ws& l, cudaStream_t stream) {
+    __nv_bfloat16* parts = reinterpret_cast<__nv_bfloat16*>(ws + l.parts);
+    {
+        const int64_t n = T * E;
+        const int64_t nb = (n + 255) / 256;
+        split3_bf16_kernel<<<(unsigned)(nb < 8192 ? nb : 8192), 256, 0, stream>>>(dlogits, n, E, parts);
+        const int rc = launch_status();
+        if (rc != MOE_OK) return rc;
+    }
+    const bool ed = layout == MOE_ROUTER_ED;
+    if (dx) {
+        // [W; W; W] along K in the weight's own orientation
+        __nv_bfloat16* wrep = reinterpret_cast<__nv_bfloat16*>(ws + l.wrep);
+        for (int i = 0; i < 3; ++i) {
+            if (ed)
+                MOE_CUDA_TRY(cudaMemcpyAsync(wrep + (int64_t)i * E * D, w, (size_t)E * D * 2, cudaMemcpyDeviceToDevice,
+                                             stream));
+            else
+                MOE_CUDA_TRY(cudaMemcpy2DAsync(wrep + (int64_t)i * E, (size_t)3 * E * 2, w, (size_t)E * 2,
+                                               (size_t)E * 2, (size_t)D, cudaMemcpyDeviceToDevice, stream));
+        }
+        TcGemmProblem q{};
+        q.a = parts;
+        q.lda = 3 * E;
+        q.a_rows_total = T;
+        q.b = wrep;
+        if (ed) {  // B(k, n) = wrep[k * D + n]
+            q.b_mn_major = true;
+            q.ldb = D;
+            q.b_rows_total = 3 * E;
+            q.b_rows_per_group = 3 * E;
+        } else {  // B(k, n) = wrep[n * 3E + k]
+            q.ldb = 3 * E;
+            q.b_rows_total = D;
+        }
+        q.G = 1;
+        q.M = T;
+        q.N = D;
+        q.K = 3 * E;
+        q.out = dx;
+        q.ldo = D;
+        q.out_rows_per_group = T;
+        q.epilogue = TC_EPI_F32;
+        q.status = status;
+        const int rc = tc_gemm_run(q, stream);
+        if (rc != MOE_OK) return rc;
+    }
+    if (dw) {
+        const int S = router_bwd_bf16_groups(T);
+        const int64_t tg = T / S;
+        float* part = reinterpret_cast<float*>(ws + l.partials);
+        for (int i = 0; i < 3; ++i) {
+            TcGemmProblem q{};
+            q.a_mn_major = true;
+            q.b_mn_major = true;
+            q.G = S;
+            q.K = tg;
+            if (ed) {  // dw[e, d] = sum_t g_i[t, e] x[t, d]
+                q.a = parts + (int64_t)i * E;
+                q.lda = 3 * E;
+                q.M = E;
+                q.b = x;
+                q.ldb = ldx;
+                q.N = D;
+            } else {  // dw[d, e] = sum_t x[t, d] g_i[t, e]
+                q.a = x;
+                q.lda = ldx;
+                q.M = D;
+                q.b = parts + (int64_t)i * E;
+                q.ldb = 3 * E;
+                q.N = E;
+            }
+            q.a_rows_total = T;
+            q.a_rows_per_group = tg;
+            q.b_rows_total = T;
+            q.b_rows_per_group = tg;
+            q.out = part + (int64_t)i * S * E * D;
+            q.ldo = q.N;
+            q.out_rows_per_group = q.M;
+            q.epilogue = TC_EPI_F32;
+            q.status = status;
+            const int rc = tc_gemm_run(q, stream);
+            if (rc != MOE_OK) return rc;
+        }
+        const int64_t len = (int64_t)E * D;
+        const int64_t nb = (len + 255) / 256;
+        sum_rows_kernel<<<(unsigned)(nb < 4096 ? nb : 4096), 256, 0, stream>>>(part, 3 * S, len, dw);
+        const int rc = launch_status();
+        if (rc != MOE_OK) return rc;
+    }
+    return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -705,7 +856,12 @@ extern "C" size_t moe_router_backward_workspace_size(int64_t T, int64_t D, int32
     if (T < 1 || D < 1 || E < 1) return 0;
     F32Gemm gx, gw;
     router_bwd_gemms(dtype, nullptr, T, D, D, nullptr, layout, E, nullptr, nullptr, nullptr, gx, gw);
-    return router_bwd_layout(gx, gw, E).total;
+    size_t total = router_bwd_layout(gx, gw, E).total;
+    if (dtype == MOE_BF16 && moe::router_bwd_bf16_shape_ok(D, E)) {  // room for either path
+        const size_t b = moe::router_bwd_bf16_layout(T, D, E).total;
+        if (b > total) total = b;
+    }
+    return total;
 }
 
 extern "C" int moe_router_backward(moe_dtype dtype, const void* x, int64_t T, int64_t D, int64_t ldx,
@@ -718,11 +874,32 @@ extern "C" int moe_router_backward(moe_dtype dtype, const void* x, int64_t T, in
     MOE_REQUIRE(x && w_router && dlogits && T >= 1 && D >= 1 && E >= 1 && ldx >= D, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(workspace_bytes >= moe_router_backward_workspace_size(T, D, E, dtype, layout) && workspace,
                 MOE_ERR_WORKSPACE);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int rc;
+    if (dtype == MOE_BF16 && router_bwd_bf16_shape_ok(D, E) && ldx % 8 == 0 && aligned16(x) && aligned16(w_router) &&
+        T < (int64_t(1) << 31) / 3) {
+        const RouterBwdBf16Ws lb = router_bwd_bf16_layout(T, D, E);
+        if (dx_router || dw_router) {
+            rc = router_backward_bf16(x, T, D, ldx, w_router, layout, E, dlogits, dx_router, dw_router, dev_status, ws,
+                                      lb, stream);
+            if (rc != MOE_OK) return rc;
+        }
+        if (db_router) {
+            float* part = reinterpret_cast<float*>(ws + lb.colsum);
+            const int64_t chunk = (T + kColChunks - 1) / kColChunks;
+            const int chunks = (int)((T + chunk - 1) / chunk);
+            column_sum_part_kernel<<<dim3((unsigned)((E + 31) / 32), (unsigned)chunks), 1024, 0, stream>>>(
+                dlogits, T, E, chunk, part);
+            rc = launch_status();
+            if (rc != MOE_OK) return rc;
+            sum_rows_kernel<<<(unsigned)((E + 255) / 256), 256, 0, stream>>>(part, chunks, E, db_router);
+            return launch_status();
+        }
+        return MOE_OK;
+    }
     F32Gemm gx, gw;
     router_bwd_gemms(dtype, x, T, D, ldx, w_router, layout, E, dlogits, dx_router, dw_router, gx, gw);
     const RouterBwdWs l = router_bwd_layout(gx, gw, E);
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    int rc;
     if (dx_router) {
         rc = tf32x3_gemm_run(gx, ws, l.split, dev_status, stream);
         if (rc != MOE_OK) return rc;

@@ -109,13 +109,17 @@ def test_backward_swiglu_with_nothing_kept():
     assert (dl == 0).all() and (dg == 0).all()
 
 
-@pytest.mark.parametrize("dtype,layout,T", [(torch.bfloat16, "ED", 700), (torch.bfloat16, "DE", 700),
-                                            (torch.float32, "ED", 700),
-                                            (torch.bfloat16, "ED", 4096),   # token reduction split 8 ways
-                                            (torch.float32, "DE", 4100)])   # split 4 ways
-def test_router_backward_matches_oracle(dtype, layout, T):
+@pytest.mark.parametrize("dtype,layout,T,E", [(torch.bfloat16, "ED", 700, 40), (torch.bfloat16, "DE", 700, 40),
+                                              (torch.float32, "ED", 700, 40),
+                                              (torch.bfloat16, "ED", 4096, 40),   # token reduction split 8 ways
+                                              (torch.float32, "DE", 4100, 40),    # split 4 ways
+                                              # bf16 with E a multiple of 64: dlogits in three bf16 parts on the
+                                              # bf16 tensor cores (one group at T = 700, four at T = 4096)
+                                              (torch.bfloat16, "ED", 700, 64), (torch.bfloat16, "DE", 4096, 128),
+                                              (torch.bfloat16, "ED", 4096, 256)])
+def test_router_backward_matches_oracle(dtype, layout, T, E):
     # s = x W (+ b): dx = dlogits W^T, dW = x^T dlogits, db = column sums (fp32 accuracy)
-    D, E = 192, 40
+    D = 192
     g = torch.Generator().manual_seed(5 + (layout == "DE"))
     x = torch.randn(T, D, generator=g).to(dtype)
     w_ed = (torch.randn(E, D, generator=g) * 0.1).to(dtype)
