@@ -577,11 +577,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRThreads, 1)
                 }
             }
             named_bar(bar_id, 128);
+            // a list holds its candidates first and fillers of -inf after them: insert up to the first
+            // filler (a row whose top-8 reaches -inf has a non-finite score and is flagged)
             if (!(c & 1)) {
-#pragma unroll
-                for (int j = 0; j < kRTopK; ++j)
-                    topk_insert(tv, ti, s_mv[((c >> 1) * kRTopK + j) * 32 + lane],
-                                s_mi[((c >> 1) * kRTopK + j) * 32 + lane]);
+#pragma unroll 1
+                for (int j = 0; j < kRTopK; ++j) {
+                    const float v = s_mv[((c >> 1) * kRTopK + j) * 32 + lane];
+                    if (!(v > -INFINITY)) break;
+                    topk_insert(tv, ti, v, s_mi[((c >> 1) * kRTopK + j) * 32 + lane]);
+                }
             }
             if (c == 2) {  // list 1 was read by this thread only
 #pragma unroll
@@ -592,9 +596,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kRThreads, 1)
             }
             named_bar(bar_id, 128);
             if (c == 0) {
-#pragma unroll
-                for (int j = 0; j < kRTopK; ++j)
-                    topk_insert(tv, ti, s_mv[(kRTopK + j) * 32 + lane], s_mi[(kRTopK + j) * 32 + lane]);
+#pragma unroll 1
+                for (int j = 0; j < kRTopK; ++j) {
+                    const float v = s_mv[(kRTopK + j) * 32 + lane];
+                    if (!(v > -INFINITY)) break;
+                    topk_insert(tv, ti, v, s_mi[(kRTopK + j) * 32 + lane]);
+                }
                 if (write) {
                     // gates: softmax of the selected scores (the first is the largest)
                     float ex[kRTopK];
