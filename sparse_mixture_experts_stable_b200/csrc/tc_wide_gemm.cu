@@ -121,9 +121,19 @@ __device__ __forceinline__ void decode(int tile, const int* prefix, int G, int f
     ft = local - tt * f_tiles;
 }
 
-// silu(a) * b with a fast exponential: the product is rounded to bf16, whose
-// spacing (2^-8 relative) is far above the exponential's error.
-__device__ __forceinline__ float swiglu_fast(float a, float b) { return __fdividef(a, 1.0f + __expf(-a)) * b; }
+// silu(a) * b = a * sigmoid(a) * b with sigmoid(a) = 1/2 + tanh(a/2)/2 through the
+// hardware tanh approximation (tanh.approx.f32, relative error about 2^-11): one
+// special-function operation per element where exp and a reciprocal took two, and
+// the drain of the accumulators, which holds up the next tile's MMAs, is bound by
+// that unit.  The product is rounded to bf16 (spacing 2^-8 relative).
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float swiglu_fast(float a, float b) {
+    return a * fmaf(0.5f, tanh_approx(0.5f * a), 0.5f) * b;
+}
 
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr, int v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");

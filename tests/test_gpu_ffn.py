@@ -127,3 +127,52 @@ def test_transpose_weights_roundtrip():
     assert torch.equal(dst, src.transpose(1, 2))
     src32 = torch.randn(2, 33, 65, device=DEV)
     assert torch.equal(moe.moe_transpose_weights(src32), src32.transpose(1, 2))
+
+
+def test_swiglu_gate_up_elementwise_error():
+    """The routed SwiGLU gate/up epilogue element by element.
+
+    With F == Dout and every down-projection matrix the identity, each output
+    element is h = silu(a) * b itself (one product with 1.0, accumulated in fp32
+    and rounded to bf16 again: exact).  The epilogue computes the sigmoid as
+    1/2 + tanh(a/2)/2 with the hardware tanh approximation, whose absolute error
+    is below 2^-11, so |sigmoid error| < 2^-12 and the bound per element is the
+    bf16 rounding of h, plus that error times |a * b|, plus the fp32 sums of a and
+    b (any order: at most D * 2^-24 * sum |x w| each) carried through
+    silu(a) * b (|silu'| < 1.1).  Pre-activations reach |a| ~ 9, where the
+    cancellation in 1 + tanh(a/2) matters most.
+    """
+    E, C, D, F = 3, 300, 256, 256
+    used = [300, 77, 0]
+    g = torch.Generator().manual_seed(29)
+    xbuf = torch.randn(E, C, D, generator=g).to(torch.bfloat16)
+    wg = (torch.randn(E, F, D, generator=g) * 3.0 * D ** -0.5).to(torch.bfloat16)
+    wu = (torch.randn(E, F, D, generator=g) * D ** -0.5).to(torch.bfloat16)
+    eye = torch.eye(F).to(torch.bfloat16).expand(E, F, F).contiguous()
+    ybuf = torch.full((E, C, F), float("nan"), dtype=torch.bfloat16, device=DEV)
+    st = moe.new_status()
+    moe.moe_expert_ffn("swiglu", xbuf.to(DEV), torch.tensor(used, dtype=torch.int32).to(DEV), wg.to(DEV),
+                       w2=eye.to(DEV), w3=wu.to(DEV), ybuf=ybuf, dev_status=st)
+    assert moe.moe_read_status(st) == 0
+    w = {"w1": wg, "w2": eye, "w3": wu}
+    want = _oracle("swiglu", xbuf, w, used)
+    yb = cpu64(ybuf)
+    n_neg = 0
+    for e in range(E):
+        u = used[e]
+        assert np.isnan(yb[e, u:]).all()
+        if not u:
+            continue
+        rows = cpu64(xbuf[e, :u])
+        a = rows @ cpu64(wg[e]).T  # magnitudes for the bound only
+        b = rows @ cpu64(wu[e]).T
+        da = D * 2.0 ** -24 * (np.abs(rows) @ np.abs(cpu64(wg[e])).T)
+        db = D * 2.0 ** -24 * (np.abs(rows) @ np.abs(cpu64(wu[e])).T)
+        silu = a / (1.0 + np.exp(-a))
+        n_neg += int((a < -4).sum())
+        bound = (2.0 ** -8 * np.abs(want[e]) + 2.0 ** -11 * np.abs(a * b) + 1.1 * da * np.abs(b)
+                 + np.abs(silu) * db + 1e-30)
+        err = np.abs(yb[e, :u] - want[e])
+        bad = err > bound
+        assert not bad.any(), (e, int(bad.sum()), float((err / bound).max()))
+    assert n_neg > 1000  # the strongly negative range was exercised
