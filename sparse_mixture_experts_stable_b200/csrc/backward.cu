@@ -666,7 +666,8 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     //    GEMM clears the rows past used[e] of an expert's last K block); otherwise from transposed
     //    copies that are zero past used[e].
     if (mn) {
-        auto wgrad = [&](const void* a, int64_t lda, int64_t M, const void* b, int64_t ldb, int64_t N, float* out) {
+        auto wgrad = [&](const void* a, int64_t lda, int64_t M, const void* b, int64_t ldb, int64_t N, float* out,
+                         float* out2 = nullptr, int64_t m_split = 0) {
             TcGemmProblem p{};
             p.a = a;
             p.lda = lda;
@@ -684,15 +685,23 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
             p.K = C;
             p.k_rows = used;
             p.out = out;
+            p.out2 = out2;
+            p.m_split = m_split;
             p.ldo = N;
-            p.out_rows_per_group = M;
+            p.out_rows_per_group = m_split > 0 ? m_split : M;
             p.epilogue = TC_EPI_F32;
             p.status = dev_status;
             return tc_gemm_run(p, stream);
         };
         if ((rc = wgrad(dybuf, H, H, h, F, F, dw_down)) != MOE_OK) return rc;  // dWd[e] (H, F) = dybuf^T h
-        if ((rc = wgrad(dab, F2, F, xb, H, H, dw_gate)) != MOE_OK) return rc;  // dWg[e] (F, H) = da^T x
-        if ((rc = wgrad(dab + F, F2, F, xb, H, H, dw_up)) != MOE_OK) return rc;  // dWu[e] (F, H) = db^T x
+        if (F % 128 == 0) {
+            // [dWg; dWu][e] (2F, H) = [da | db]^T x in one GEMM: each x tile is read from HBM once for
+            // both gradients (the m-tiles of an (expert, n-tile) run back to back); rows >= F go to dWu
+            if ((rc = wgrad(dab, F2, F2, xb, H, H, dw_gate, dw_up, F)) != MOE_OK) return rc;
+        } else {
+            if ((rc = wgrad(dab, F2, F, xb, H, H, dw_gate)) != MOE_OK) return rc;  // dWg[e] (F, H) = da^T x
+            if ((rc = wgrad(dab + F, F2, F, xb, H, H, dw_up)) != MOE_OK) return rc;  // dWu[e] (F, H) = db^T x
+        }
     } else {
         rc = transpose_valid(dybuf, H, C * H, E, C, H, used, Cp, dybufT, Cp, H * Cp, stream);
         if (rc != MOE_OK) return rc;

@@ -53,6 +53,8 @@ struct KParams {
     const int32_t* rows;
     const int32_t* k_rows;
     void* out;
+    void* out2;       // rows m >= m_split of a group (0: none)
+    int64_t m_split;
     int64_t ldo;
     int64_t out_rows_per_group;
     const void* bias;
@@ -137,7 +139,7 @@ template <int EPI, bool AMN, bool BMN>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
-                   const KParams p) {
+                   const __grid_constant__ CUtensorMap tmOut2, const KParams p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_prefix[kMaxGroups + 1];
     // epilogue staging, one 32 x 32 chunk per warp (1024-aligned: the TMA store reads it 128-byte swizzled)
@@ -368,16 +370,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             int64_t rows_g = p.rows ? (int64_t)p.rows[g] : p.M;
             rows_g = rows_g > p.M ? p.M : rows_g;
             const bool row_ok = m < rows_g;
-            const int64_t out_row = (int64_t)g * p.out_rows_per_group + m;
+            // the m-tiles past m_split write the second output (a tile lies wholly on one side)
+            const bool second = p.m_split > 0 && (int64_t)mt * kBM >= p.m_split;
+            void* const outp = second ? p.out2 : p.out;
+            const int64_t out_row = (int64_t)g * p.out_rows_per_group + m - (second ? p.m_split : 0);
             const uint32_t t_row = tmem_base + acc * kBN + ((uint32_t)(q * 32) << 16);
             // this warp's 32 rows for the staged stores
             const int64_t wrow0 = (int64_t)mt * kBM + q * 32;
             const int wrows = (int)(rows_g - wrow0 < 0 ? 0 : (rows_g - wrow0 > 32 ? 32 : rows_g - wrow0));
-            const int64_t out_wrow0 = (int64_t)g * p.out_rows_per_group + wrow0;
+            const int64_t out_wrow0 = (int64_t)g * p.out_rows_per_group + wrow0 - (second ? p.m_split : 0);
             uint32_t* stg = s_stage[q];
 
             if (EPI == TC_EPI_SWIGLU) {
-                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * p.ldo;
+                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(outp) + out_row * p.ldo;
                 const int half = p.n_mma / 2;
                 for (int c = 0; c < half / 32; ++c) {
                     uint32_t rg[32], ru[32];
@@ -395,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
                     if (p.vec_ok && n0 + 32 <= p.N)
                         warp_store_chunk<16>(stg, pk,
-                                             reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                             reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(outp) +
                                                                         out_wrow0 * p.ldo + n0),
                                              p.ldo * 2, wrows, lane);
                     else if (row_ok)
@@ -403,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else if (EPI == TC_EPI_F32_DUAL) {
                 // gate half of the accumulator -> columns [0, N), up half -> [N, 2N)
-                float* orow = reinterpret_cast<float*>(p.out) + out_row * p.ldo;
+                float* orow = reinterpret_cast<float*>(outp) + out_row * p.ldo;
                 const int half = p.n_mma / 2;
                 for (int c = 0; c < p.n_mma / 32; ++c) {
                     uint32_t r[32];
@@ -414,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float* dst = orow + (up ? p.N : 0);
                     if (p.vec_ok && n0 + 32 <= p.N) {
                         warp_store_chunk<32>(stg, r,
-                                             reinterpret_cast<uint8_t*>(reinterpret_cast<float*>(p.out) +
+                                             reinterpret_cast<uint8_t*>(reinterpret_cast<float*>(outp) +
                                                                         out_wrow0 * p.ldo + (up ? p.N : 0) + n0),
                                              p.ldo * 4, wrows, lane);
                     } else if (row_ok) {
@@ -438,13 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tmOut, stg, (int32_t)(nt * p.tile_n_out + c * 32), (int32_t)out_wrow0);
+                        tma_store_2d(second ? &tmOut2 : &tmOut, stg, (int32_t)(nt * p.tile_n_out + c * 32), (int32_t)out_wrow0);
                         bulk_commit();
                     }
                 };
                 pipelined_chunks(t_row, p.n_mma / 32, process);
             } else if (EPI == TC_EPI_F32) {
-                float* orow = reinterpret_cast<float*>(p.out) + out_row * p.ldo;
+                float* orow = reinterpret_cast<float*>(outp) + out_row * p.ldo;
                 const float* bias = reinterpret_cast<const float*>(p.bias);
                 auto process = [&](const int c, const uint32_t (&r)[32]) {
                     const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
@@ -454,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 32; ++i)
                             w[i] = __float_as_uint(__uint_as_float(r[i]) + (bias ? bias[n0 + i] : 0.f));
                         warp_store_chunk<32>(stg, w,
-                                             reinterpret_cast<uint8_t*>(reinterpret_cast<float*>(p.out) +
+                                             reinterpret_cast<uint8_t*>(reinterpret_cast<float*>(outp) +
                                                                         out_wrow0 * p.ldo + n0),
                                              p.ldo * 4, wrows, lane);
                     } else if (row_ok) {
@@ -465,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 };
                 pipelined_chunks(t_row, p.n_mma / 32, process);
             } else {
-                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * p.ldo;
+                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(outp) + out_row * p.ldo;
                 const __nv_bfloat16* bias =
                     reinterpret_cast<const __nv_bfloat16*>(p.bias) + (p.bias ? g * p.bias_group_stride : 0);
                 auto process = [&](const int c, const uint32_t (&r)[32]) {
@@ -488,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (p.vec_ok && n0 + 32 <= p.N)
                         warp_store_chunk<16>(stg, pk,
-                                             reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
+                                             reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(outp) +
                                                                         out_wrow0 * p.ldo + n0),
                                              p.ldo * 2, wrows, lane);
                     else if (row_ok)
@@ -580,7 +585,7 @@ namespace {
 
 template <int EPI, bool AMN = false, bool BMN = false>
 int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const CUtensorMap& out,
-           const KParams& kp, int grid, cudaStream_t stream) {
+           const CUtensorMap& out2, const KParams& kp, int grid, cudaStream_t stream) {
     static bool attr_set[64] = {false};
     int dev = 0;
     MOE_CUDA_TRY(cudaGetDevice(&dev));
@@ -589,7 +594,7 @@ int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, co
                                           (int)kSmemBytes));
         attr_set[dev] = true;
     }
-    tc_gemm_kernel<EPI, AMN, BMN><<<grid, kThreads, kSmemBytes, stream>>>(a, b, b2, out, kp);
+    tc_gemm_kernel<EPI, AMN, BMN><<<grid, kThreads, kSmemBytes, stream>>>(a, b, b2, out, out2, kp);
     return launch_status();
 }
 
@@ -608,6 +613,12 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     if (p.a_mn_major)
         MOE_REQUIRE(p.b_mn_major && p.epilogue == TC_EPI_F32 && p.k_split == 0 && p.rows == nullptr,
                     MOE_ERR_UNSUPPORTED);
+    // the split output: MN-major A only, whole m-tiles on each side
+    MOE_REQUIRE(p.m_split >= 0, MOE_ERR_INVALID_ARG);
+    if (p.m_split > 0)
+        MOE_REQUIRE(p.a_mn_major && p.out2 && p.m_split % kBM == 0 && p.m_split < p.M &&
+                        p.out_rows_per_group >= p.m_split && p.out_rows_per_group >= p.M - p.m_split,
+                    MOE_ERR_INVALID_ARG);
     if (p.b_mn_major) {
         MOE_REQUIRE(p.epilogue == TC_EPI_F32 || p.epilogue == TC_EPI_BF16, MOE_ERR_UNSUPPORTED);
         MOE_REQUIRE(p.k_split % kBK == 0 && p.k_split >= 0 && p.k_split < p.K, MOE_ERR_UNSUPPORTED);
@@ -643,21 +654,24 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     kp.rows = p.rows;
     kp.k_rows = p.k_rows;
     kp.out = p.out;
+    kp.out2 = p.m_split > 0 ? p.out2 : nullptr;
+    kp.m_split = p.m_split;
     kp.ldo = p.ldo;
     kp.out_rows_per_group = p.out_rows_per_group;
     kp.bias = p.bias;
     kp.bias_group_stride = p.bias_group_stride;
     const bool f32_out = p.epilogue == TC_EPI_F32 || p.epilogue == TC_EPI_F32_DUAL;
     const size_t esz = f32_out ? 4 : 2;
-    kp.vec_ok = aligned16(p.out) && (p.ldo * (int64_t)esz) % 16 == 0;
+    kp.vec_ok = aligned16(p.out) && (p.ldo * (int64_t)esz) % 16 == 0 && (p.m_split == 0 || aligned16(p.out2));
     if (p.epilogue == TC_EPI_F32_DUAL) kp.vec_ok = kp.vec_ok && (p.N * 4) % 16 == 0;
     kp.status = p.status;
     // the weight-gradient form writes whole 32 x 32 fp32 boxes through the TMA
     kp.tma_out = p.a_mn_major && p.epilogue == TC_EPI_F32 && p.rows == nullptr && p.bias == nullptr &&
-                 p.M % kBM == 0 && p.N % 32 == 0 && kp.vec_ok && p.out_rows_per_group >= p.M &&
+                 p.M % kBM == 0 && p.N % 32 == 0 && kp.vec_ok &&
+                 (p.m_split > 0 || p.out_rows_per_group >= p.M) &&
                  (int64_t)p.G * p.out_rows_per_group < (int64_t(1) << 31);
 
-    CUtensorMap ma, mb, mb2, mo;
+    CUtensorMap ma, mb, mb2, mo, mo2;
     if (p.a_mn_major)  // (K rows, M columns) with 64 x 64 boxes
         MOE_REQUIRE(make_map(&ma, p.a, p.M, p.a_rows_total, p.lda, kBK), MOE_ERR_CUDA);
     else
@@ -683,17 +697,21 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
         MOE_REQUIRE(make_map_f32(&mo, p.out, p.N, (int64_t)p.G * p.out_rows_per_group, p.ldo, 32), MOE_ERR_CUDA);
     else
         mo = ma;  // unused
-    if (p.a_mn_major) return launch<TC_EPI_F32, true, true>(ma, mb, mb2, mo, kp, grid, stream);
+    if (kp.tma_out && p.m_split > 0)
+        MOE_REQUIRE(make_map_f32(&mo2, p.out2, p.N, (int64_t)p.G * p.out_rows_per_group, p.ldo, 32), MOE_ERR_CUDA);
+    else
+        mo2 = mo;  // unused
+    if (p.a_mn_major) return launch<TC_EPI_F32, true, true>(ma, mb, mb2, mo, mo2, kp, grid, stream);
     if (p.b_mn_major)
-        return p.epilogue == TC_EPI_F32 ? launch<TC_EPI_F32, false, true>(ma, mb, mb2, mo, kp, grid, stream)
-                                        : launch<TC_EPI_BF16, false, true>(ma, mb, mb2, mo, kp, grid, stream);
+        return p.epilogue == TC_EPI_F32 ? launch<TC_EPI_F32, false, true>(ma, mb, mb2, mo, mo2, kp, grid, stream)
+                                        : launch<TC_EPI_BF16, false, true>(ma, mb, mb2, mo, mo2, kp, grid, stream);
     switch (p.epilogue) {
-        case TC_EPI_F32: return launch<TC_EPI_F32>(ma, mb, mb2, mo, kp, grid, stream);
-        case TC_EPI_BF16: return launch<TC_EPI_BF16>(ma, mb, mb2, mo, kp, grid, stream);
-        case TC_EPI_BF16_BIAS: return launch<TC_EPI_BF16_BIAS>(ma, mb, mb2, mo, kp, grid, stream);
-        case TC_EPI_GELU_BIAS: return launch<TC_EPI_GELU_BIAS>(ma, mb, mb2, mo, kp, grid, stream);
-        case TC_EPI_SWIGLU: return launch<TC_EPI_SWIGLU>(ma, mb, mb2, mo, kp, grid, stream);
-        case TC_EPI_F32_DUAL: return launch<TC_EPI_F32_DUAL>(ma, mb, mb2, mo, kp, grid, stream);
+        case TC_EPI_F32: return launch<TC_EPI_F32>(ma, mb, mb2, mo, mo2, kp, grid, stream);
+        case TC_EPI_BF16: return launch<TC_EPI_BF16>(ma, mb, mb2, mo, mo2, kp, grid, stream);
+        case TC_EPI_BF16_BIAS: return launch<TC_EPI_BF16_BIAS>(ma, mb, mb2, mo, mo2, kp, grid, stream);
+        case TC_EPI_GELU_BIAS: return launch<TC_EPI_GELU_BIAS>(ma, mb, mb2, mo, mo2, kp, grid, stream);
+        case TC_EPI_SWIGLU: return launch<TC_EPI_SWIGLU>(ma, mb, mb2, mo, mo2, kp, grid, stream);
+        case TC_EPI_F32_DUAL: return launch<TC_EPI_F32_DUAL>(ma, mb, mb2, mo, mo2, kp, grid, stream);
         default: return MOE_ERR_INVALID_ARG;
     }
 }

@@ -51,6 +51,8 @@ struct TcGemmProblem {
     void* out;                // fp32 or bf16 per epilogue
     int64_t ldo;
     int64_t out_rows_per_group;
+    void* out2;               // with a_mn_major and m_split > 0: rows m >= m_split of each group go to
+    int64_t m_split;          // out2 (row m - m_split, same ldo and out_rows_per_group); a multiple of 128
     const void* bias;         // fp32 (TC_EPI_F32) or bf16, per output column
     int64_t bias_group_stride;
     int epilogue;
