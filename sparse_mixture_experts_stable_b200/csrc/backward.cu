@@ -618,7 +618,9 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     // With H and F multiples of 64 the weights are read in their own layout as MN-major
     // operands; otherwise transposed copies feed the K-major form.
     const bool mn = H % 64 == 0 && F % 64 == 0;
-    // 4. dh = dybuf Wd: B(k = h, n = f) = Wd[e][h][f]
+    // 4. dh = dybuf Wd: B(k = h, n = f) = Wd[e][h][f].  With the forward's bf16 [a | b] at hand the
+    //    GEMM's epilogue also does step 5 (h, da, db from the dh accumulator), so dh never reaches HBM.
+    const bool fused_elem = mn && saved_ab != nullptr;
     if (mn) {
         TcGemmProblem p{};
         p.a = dybuf;
@@ -635,10 +637,18 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
         p.N = F;
         p.K = H;
         p.rows = used;
-        p.out = dh;
-        p.ldo = F;
+        if (fused_elem) {
+            p.out = dab;
+            p.ldo = F2;
+            p.ab = saved_ab;
+            p.h = h;
+            p.epilogue = TC_EPI_SWIGLU_BWD;
+        } else {
+            p.out = dh;
+            p.ldo = F;
+            p.epilogue = TC_EPI_F32;
+        }
         p.out_rows_per_group = C;
-        p.epilogue = TC_EPI_F32;
         p.status = dev_status;
         rc = tc_gemm_run(p, stream);
     } else {
@@ -649,7 +659,7 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
     }
     if (rc != MOE_OK) return rc;
     // 5. h, da, db
-    {
+    if (!fused_elem) {
         const int64_t nb = (C * (F / 8) + 255) / 256;
         const dim3 g2((unsigned)(nb < 1024 ? nb : 1024), (unsigned)E);
         MOE_REQUIRE(E <= 65535, MOE_ERR_UNSUPPORTED);

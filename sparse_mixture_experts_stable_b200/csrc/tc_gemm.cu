@@ -55,6 +55,8 @@ struct KParams {
     void* out;
     void* out2;       // rows m >= m_split of a group (0: none)
     int64_t m_split;
+    const void* ab;   // SwiGLU backward: [a | b] beside the dh accumulator
+    void* h_out;
     int64_t ldo;
     int64_t out_rows_per_group;
     const void* bias;
@@ -406,6 +408,88 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else if (row_ok)
                         store_bf16_32(orow, n0, p.N, pk, p.vec_ok);
                 }
+            } else if (EPI == TC_EPI_SWIGLU_BWD) {
+                // acc = dh.  With s = sigmoid(a): h = a s b, da = dh b (s + a s (1 - s)), db = dh a s.
+                // The warp's 32 rows x 32 columns of [a | b] for a chunk arrive as coalesced loads (one
+                // row's 64 + 64 bytes per 8 lanes), issued two chunks ahead of the math and turned
+                // row-per-lane through the staging buffer; the three bf16 results leave through the
+                // staged coalesced stores.  (An L2 prefetch of the tile by the producer measured slower.)
+                // The sigmoid takes the fast reciprocal (2 ulp): the correctly rounded one cost the
+                // epilogue more than the whole of its loads.
+                const __nv_bfloat16* ab = reinterpret_cast<const __nv_bfloat16*>(p.ab);
+                __nv_bfloat16* hb = reinterpret_cast<__nv_bfloat16*>(p.h_out);
+                __nv_bfloat16* dab = reinterpret_cast<__nv_bfloat16*>(outp);
+                const int nch = p.n_mma / 32;  // even: n_mma is a multiple of 64 with an MN-major B
+                const int lr = lane >> 3, piece = lane & 7;
+                auto load_ab = [&](const int c, uint4 (&v)[8]) {
+                    const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
+                    const int64_t col = (piece < 4 ? n0 : p.N + n0) + 8 * (piece & 3);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = lr + 4 * i;
+                        v[i] = (r < wrows && n0 < p.N)
+                                   ? __ldg(reinterpret_cast<const uint4*>(ab + (out_wrow0 + r) * p.ldo + col))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+                    }
+                };
+                auto chunk = [&](const int c, uint4 (&v)[8]) {
+                    uint32_t r[32];
+                    tmem_ld32(t_row + c * 32, r);
+                    // rows to lanes: row lr + 4i, 16-byte piece `piece` (a: 0-3, b: 4-7)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = lr + 4 * i;
+                        *reinterpret_cast<uint4*>(stg + rr * 32 + 4 * (piece ^ (rr & 7))) = v[i];
+                    }
+                    __syncwarp();
+                    uint32_t aw[16], bw[16];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint4 q4 = *reinterpret_cast<const uint4*>(stg + lane * 32 + 4 * (k ^ (lane & 7)));
+                        uint32_t* d = k < 4 ? aw + 4 * k : bw + 4 * (k - 4);
+                        d[0] = q4.x, d[1] = q4.y, d[2] = q4.z, d[3] = q4.w;
+                    }
+                    __syncwarp();
+                    if (c + 2 < nch) load_ab(c + 2, v);
+                    tmem_ld_wait(r);
+                    const int64_t n0 = (int64_t)nt * p.tile_n_out + c * 32;
+                    if (n0 < p.N) {
+                        uint32_t ph[16], pa[16], pb[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float hv[2], dav[2], dbv[2];
+#pragma unroll
+                            for (int m2 = 0; m2 < 2; ++m2) {
+                                const float a = __uint_as_float(m2 ? (aw[i] & 0xFFFF0000u) : (aw[i] << 16));
+                                const float b = __uint_as_float(m2 ? (bw[i] & 0xFFFF0000u) : (bw[i] << 16));
+                                const float gd = __uint_as_float(r[2 * i + m2]);
+                                const float sg = __fdividef(1.0f, 1.0f + __expf(-a));
+                                const float as = a * sg;
+                                hv[m2] = as * b;
+                                dbv[m2] = gd * as;
+                                dav[m2] = (gd * b) * fmaf(as, 1.0f - sg, sg);
+                            }
+                            ph[i] = pack_bf16x2(hv[0], hv[1]);
+                            pa[i] = pack_bf16x2(dav[0], dav[1]);
+                            pb[i] = pack_bf16x2(dbv[0], dbv[1]);
+                        }
+                        warp_store_chunk<16>(stg, ph, reinterpret_cast<uint8_t*>(hb + out_wrow0 * p.N + n0), p.N * 2,
+                                             wrows, lane);
+                        warp_store_chunk<16>(stg, pa, reinterpret_cast<uint8_t*>(dab + out_wrow0 * p.ldo + n0),
+                                             p.ldo * 2, wrows, lane);
+                        warp_store_chunk<16>(stg, pb,
+                                             reinterpret_cast<uint8_t*>(dab + out_wrow0 * p.ldo + p.N + n0),
+                                             p.ldo * 2, wrows, lane);
+                    }
+                };
+                uint4 v0[8], v1[8];
+                load_ab(0, v0);
+                load_ab(1, v1);
+#pragma unroll 1
+                for (int c = 0; c < nch; c += 2) {
+                    chunk(c, v0);
+                    chunk(c + 1, v1);
+                }
             } else if (EPI == TC_EPI_F32_DUAL) {
                 // gate half of the accumulator -> columns [0, N), up half -> [N, 2N)
                 float* orow = reinterpret_cast<float*>(outp) + out_row * p.ldo;
@@ -620,11 +704,17 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
                         p.out_rows_per_group >= p.m_split && p.out_rows_per_group >= p.M - p.m_split,
                     MOE_ERR_INVALID_ARG);
     if (p.b_mn_major) {
-        MOE_REQUIRE(p.epilogue == TC_EPI_F32 || p.epilogue == TC_EPI_BF16, MOE_ERR_UNSUPPORTED);
+        MOE_REQUIRE(p.epilogue == TC_EPI_F32 || p.epilogue == TC_EPI_BF16 || p.epilogue == TC_EPI_SWIGLU_BWD,
+                    MOE_ERR_UNSUPPORTED);
         MOE_REQUIRE(p.k_split % kBK == 0 && p.k_split >= 0 && p.k_split < p.K, MOE_ERR_UNSUPPORTED);
         MOE_REQUIRE(p.k_split == 0 || (p.b2 && aligned16(p.b2)), MOE_ERR_INVALID_ARG);
         MOE_REQUIRE(p.b_rows_per_group >= (p.k_split > 0 ? p.k_split : p.K), MOE_ERR_INVALID_ARG);
     }
+    // the SwiGLU backward epilogue: MN-major B, whole 32-column chunks, 16-byte aligned rows
+    if (p.epilogue == TC_EPI_SWIGLU_BWD)
+        MOE_REQUIRE(p.b_mn_major && !p.a_mn_major && p.ab && p.h && aligned16(p.ab) && aligned16(p.h) &&
+                        p.N % 32 == 0 && p.ldo >= 2 * p.N && p.m_split == 0,
+                    MOE_ERR_UNSUPPORTED);
     const bool dual = p.epilogue == TC_EPI_SWIGLU || p.epilogue == TC_EPI_F32_DUAL;
     if (dual) MOE_REQUIRE(p.b2 && aligned16(p.b2), MOE_ERR_INVALID_ARG);
     // TMA coordinates are 32-bit.
@@ -656,6 +746,8 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     kp.out = p.out;
     kp.out2 = p.m_split > 0 ? p.out2 : nullptr;
     kp.m_split = p.m_split;
+    kp.ab = p.ab;
+    kp.h_out = p.h;
     kp.ldo = p.ldo;
     kp.out_rows_per_group = p.out_rows_per_group;
     kp.bias = p.bias;
@@ -664,6 +756,7 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     const size_t esz = f32_out ? 4 : 2;
     kp.vec_ok = aligned16(p.out) && (p.ldo * (int64_t)esz) % 16 == 0 && (p.m_split == 0 || aligned16(p.out2));
     if (p.epilogue == TC_EPI_F32_DUAL) kp.vec_ok = kp.vec_ok && (p.N * 4) % 16 == 0;
+    if (p.epilogue == TC_EPI_SWIGLU_BWD) MOE_REQUIRE(kp.vec_ok, MOE_ERR_UNSUPPORTED);
     kp.status = p.status;
     // the weight-gradient form writes whole 32 x 32 fp32 boxes through the TMA
     kp.tma_out = p.a_mn_major && p.epilogue == TC_EPI_F32 && p.rows == nullptr && p.bias == nullptr &&
@@ -702,9 +795,12 @@ int tc_gemm_run(const TcGemmProblem& p, cudaStream_t stream) {
     else
         mo2 = mo;  // unused
     if (p.a_mn_major) return launch<TC_EPI_F32, true, true>(ma, mb, mb2, mo, mo2, kp, grid, stream);
-    if (p.b_mn_major)
+    if (p.b_mn_major) {
+        if (p.epilogue == TC_EPI_SWIGLU_BWD)
+            return launch<TC_EPI_SWIGLU_BWD, false, true>(ma, mb, mb2, mo, mo2, kp, grid, stream);
         return p.epilogue == TC_EPI_F32 ? launch<TC_EPI_F32, false, true>(ma, mb, mb2, mo, mo2, kp, grid, stream)
                                         : launch<TC_EPI_BF16, false, true>(ma, mb, mb2, mo, mo2, kp, grid, stream);
+    }
     switch (p.epilogue) {
         case TC_EPI_F32: return launch<TC_EPI_F32>(ma, mb, mb2, mo, mo2, kp, grid, stream);
         case TC_EPI_BF16: return launch<TC_EPI_BF16>(ma, mb, mb2, mo, mo2, kp, grid, stream);

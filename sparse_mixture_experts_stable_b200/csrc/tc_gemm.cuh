@@ -22,7 +22,9 @@ enum TcEpilogue : int {
     TC_EPI_BF16_BIAS = 2,  // bf16 out, + bf16 bias                       -- GELU MLP fc2
     TC_EPI_GELU_BIAS = 3,  // bf16 gelu(acc + bias)                       -- GELU MLP fc1
     TC_EPI_SWIGLU = 4,     // dual B: bf16 silu(acc_gate) * acc_up        -- SwiGLU gate/up
-    TC_EPI_F32_DUAL = 5    // dual B: fp32 acc_gate -> out[., n], acc_up -> out[., N + n]   -- [a | b] recompute
+    TC_EPI_F32_DUAL = 5,   // dual B: fp32 acc_gate -> out[., n], acc_up -> out[., N + n]   -- [a | b] recompute
+    TC_EPI_SWIGLU_BWD = 6  // acc = dh; with [a | b] = ab (bf16, rows of out): h = silu(a) b -> h,
+                           // [dh b silu'(a) | dh silu(a)] -> out (bf16, 2N wide)  -- SwiGLU backward
 };
 
 struct TcGemmProblem {
@@ -53,6 +55,8 @@ struct TcGemmProblem {
     int64_t out_rows_per_group;
     void* out2;               // with a_mn_major and m_split > 0: rows m >= m_split of each group go to
     int64_t m_split;          // out2 (row m - m_split, same ldo and out_rows_per_group); a multiple of 128
+    const void* ab;           // TC_EPI_SWIGLU_BWD: bf16 [a | b] with the rows and row stride of out
+    void* h;                  // TC_EPI_SWIGLU_BWD: bf16 h = silu(a) b, row stride N
     const void* bias;         // fp32 (TC_EPI_F32) or bf16, per output column
     int64_t bias_group_stride;
     int epilogue;
