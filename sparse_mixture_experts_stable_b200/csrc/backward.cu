@@ -706,7 +706,7 @@ extern "C" int moe_backward_swiglu(moe_dtype dtype, const void* dy, const float*
         if ((rc = wgrad(dybuf, H, H, h, F, F, dw_down)) != MOE_OK) return rc;  // dWd[e] (H, F) = dybuf^T h
         if (F % 128 == 0) {
             // [dWg; dWu][e] (2F, H) = [da | db]^T x in one GEMM: each x tile is read from HBM once for
-            // both gradients (the m-tiles of an (expert, n-tile) run back to back); rows >= F go to dWu
+            // both gradients (the tiles of an expert run back to back, its x stays in L2); rows >= F go to dWu
             if ((rc = wgrad(dab, F2, F2, xb, H, H, dw_gate, dw_up, F)) != MOE_OK) return rc;
         } else {
             if ((rc = wgrad(dab, F2, F, xb, H, H, dw_gate)) != MOE_OK) return rc;  // dWg[e] (F, H) = da^T x

@@ -71,8 +71,10 @@ constexpr bool is_dual(int epi) { return epi == TC_EPI_SWIGLU || epi == TC_EPI_F
 using namespace tc;
 
 // Map a linear tile index to (group, m-tile, n-tile).  prefix[g] is the first
-// tile of group g; tiles of a group run m fastest so that concurrently active
-// CTAs share the group's weight tile.
+// tile of group g; tiles of a group run n fastest, so concurrently active CTAs
+// share an m-tile of A and together write whole output rows (measured on B200:
+// 33 us less per SwiGLU training step than m fastest, the forward unchanged; a
+// group's operands stay in L2 either way).
 __device__ __forceinline__ void decode_tile(int tile, const int* prefix, int G, int n_tiles, int& g,
                                             int& mt, int& nt) {
     int lo = 0, hi = G - 1;
@@ -83,9 +85,8 @@ __device__ __forceinline__ void decode_tile(int tile, const int* prefix, int G, 
     }
     g = lo;
     const int local = tile - prefix[g];
-    const int mtiles = (prefix[g + 1] - prefix[g]) / n_tiles;
-    nt = local / mtiles;
-    mt = local - nt * mtiles;
+    mt = local / n_tiles;
+    nt = local - mt * n_tiles;
 }
 
 // K blocks of group g: all of them, or (k_rows given) those holding its first
