@@ -161,9 +161,10 @@ __device__ __forceinline__ void decode_tile(int tile, const int* prefix, int G, 
     }
     g = lo;
     const int local = tile - prefix[g];
-    const int mtiles = (prefix[g + 1] - prefix[g]) / n_tiles;
-    nt = local / mtiles;
-    mt = local - nt * mtiles;
+    // n fastest: concurrently active CTAs share an m-tile of A and write whole output rows
+    // (measured on B200: the fp32 fwd+bwd step 5 us shorter than with m fastest)
+    mt = local / n_tiles;
+    nt = local - mt * n_tiles;
 }
 
 __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
