@@ -44,10 +44,10 @@ WORKLOAD = dict(workload="full_layer_bf16", T=16384, hidden=2048, experts=256, t
 KERNELS_PER_STEP = 10  # fused router, reduce, scan, gather, 2 routed GEMMs, 2 shared GEMMs, combine, aux
 # DRAM bytes (read + write) per algorithmic byte of the two routed expert-FFN kernels (the SwiGLU
 # gate/up tcw_kernel and the down projection tc_gemm_kernel<BF16>), from one ncu capture of
-# dram__bytes_read.sum + dram__bytes_write.sum on the T=8192, E=128 case (one kernel, a few
-# launches); the bench scales it by its own algorithmic bytes.  None until measured for the
-# current kernels.
-TRAFFIC_PER_ALG_BYTE = None
+# dram__bytes_read.sum + dram__bytes_write.sum on the T=8192, E=128 case (two launches of each;
+# profiles/routed_ffn_dram_traffic_T8192_E128.md); the bench scales it by its own algorithmic
+# bytes.  Set back to None when either kernel changes.
+TRAFFIC_PER_ALG_BYTE = {"gate_up": 1.024, "down": 0.943}
 
 
 def measured_peaks():
