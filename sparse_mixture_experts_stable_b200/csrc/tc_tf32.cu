@@ -127,6 +127,7 @@ struct T3Params {
     int64_t bias_group_stride;
     int epilogue;
     int vec_ok;  // C, ldc (and bias, bias_group_stride) allow 16-byte accesses
+    int tma_out; // plain fp32 out, every tile row valid: 32 x 32 chunks leave through TMA stores (tmC)
     int32_t* status;
 };
 
@@ -170,10 +171,11 @@ __device__ __forceinline__ void decode_tile(int tile, const int* prefix, int G, 
 __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
     tf32x3_kernel(const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CUtensorMap tmAl,
                   const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmBl,
-                  const T3Params p) {
+                  const __grid_constant__ CUtensorMap tmC, const T3Params p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ int s_prefix[kMaxGroups + 1];
-    __shared__ __align__(16) uint32_t s_stage[4][32 * 32];  // epilogue staging, one 32 x 32 chunk per warp
+    // epilogue staging, one 32 x 32 chunk per warp (1024-aligned: a TMA store reads it 128-byte swizzled)
+    __shared__ __align__(1024) uint32_t s_stage[4][32 * 32];
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
 
@@ -402,11 +404,27 @@ __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
             float* crow = p.C + g * p.c_group_stride + m * p.ldc;
             const float* bias = p.bias ? p.bias + g * p.bias_group_stride : nullptr;
             const uint32_t t_row = tmem_base + acc * kAccCols + ((uint32_t)(q * 32) << 16);
-            for (int c = 0; c < p.n_mma / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(t_row + c * 32, r);
-                tmem_ld_wait(r);
+            auto process = [&](const int c, const uint32_t (&r)[32]) {
                 const int64_t n0 = (int64_t)nt * p.n_mma + c * 32;
+                if (p.tma_out) {
+                    // every row valid, whole 32-column chunks: the chunk goes to the warp's staging buffer
+                    // in the map's 128-byte swizzled layout and one lane hands it to the TMA, which streams
+                    // it out while the warp drains the next chunk
+                    uint32_t* stg = s_stage[q];
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+#pragma unroll
+                    for (int m4 = 0; m4 < 8; ++m4)
+                        *reinterpret_cast<uint4*>(stg + lane * 32 + 4 * (m4 ^ (lane & 7))) =
+                            make_uint4(r[4 * m4], r[4 * m4 + 1], r[4 * m4 + 2], r[4 * m4 + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmC, stg, (int32_t)n0, (int32_t)((int64_t)g * p.M + wrow0));
+                        bulk_commit();
+                    }
+                    return;
+                }
                 if (p.epilogue != F32_EPI_SILU_MUL && p.vec_ok && n0 + 32 <= p.N) {
                     // row-contiguous stores through shared memory (see warp_store_chunk)
                     uint32_t w[32];
@@ -418,9 +436,9 @@ __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
                         w[i] = __float_as_uint(v);
                     }
                     warp_store_chunk<32>(s_stage[q], w, reinterpret_cast<uint8_t*>(cw + n0), p.ldc * 4, wrows, lane);
-                    continue;
+                    return;
                 }
-                if (!row_ok) continue;
+                if (!row_ok) return;
                 if (p.vec_ok && n0 + 32 <= p.N) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -462,11 +480,27 @@ __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
                         }
                     }
                 }
+            };
+            // TMEM reads one chunk ahead of the math and stores
+            const int nch = p.n_mma / 32;
+            uint32_t ra[32], rb[32];
+            tmem_ld32(t_row, ra);
+            tmem_ld_wait(ra);
+            for (int c = 0; c < nch; c += 2) {
+                if (c + 1 < nch) tmem_ld32(t_row + (c + 1) * 32, rb);
+                process(c, ra);
+                if (c + 1 < nch) {
+                    tmem_ld_wait(rb);
+                    if (c + 2 < nch) tmem_ld32(t_row + (c + 2) * 32, ra);
+                    process(c + 1, rb);
+                    if (c + 2 < nch) tmem_ld_wait(ra);
+                }
             }
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
             if (s_abort) break;
         }
+        if (p.tma_out && lane == 0) bulk_wait_all();  // the stores are done before the CTA exits
     }
 
     __syncthreads();
@@ -584,6 +618,9 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
     kp.epilogue = g.epilogue;
     kp.vec_ok = aligned16(g.C) && g.ldc % 4 == 0 && g.c_group_stride % 4 == 0 &&
                 (!g.bias || (aligned16(g.bias) && g.bias_group_stride % 4 == 0));
+    // the weight-gradient form: plain fp32 out, all rows of every tile valid, groups back to back
+    kp.tma_out = g.epilogue == F32_EPI_NONE && g.rows_mode != 1 && g.M % kBM == 0 && g.N % 32 == 0 && kp.vec_ok &&
+                 g.c_group_stride == g.M * g.ldc && (int64_t)g.groups * g.M < (int64_t(1) << 31);
     kp.status = status;
 
     CUtensorMap mah, mal, mbh, mbl;
@@ -608,6 +645,10 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
         MOE_REQUIRE(make_map_f32(&mbl, b_lo, l.Kp, (int64_t)g.groups * g.N, l.Kp, kp.n_mma), MOE_ERR_CUDA);
     }
 
+    CUtensorMap mc;
+    if (kp.tma_out) MOE_REQUIRE(make_map_f32(&mc, g.C, g.N, (int64_t)g.groups * g.M, g.ldc, 32), MOE_ERR_CUDA);
+    else mc = mah;  // unused
+
     const int64_t max_tiles = (int64_t)g.groups * ((g.M + kBM - 1) / kBM) * kp.n_tiles;
     MOE_REQUIRE(max_tiles < (int64_t(1) << 30), MOE_ERR_UNSUPPORTED);
     int grid = device_sm_count();
@@ -621,7 +662,7 @@ int tf32x3_gemm_run(const F32Gemm& g, void* workspace, size_t workspace_bytes, i
         MOE_CUDA_TRY(cudaFuncSetAttribute(tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes));
         if (dev < 64) attr_set[dev] = true;
     }
-    tf32x3_kernel<<<grid, kThreads + kConvThreads, kSmemBytes, stream>>>(mah, mal, mbh, mbl, kp);
+    tf32x3_kernel<<<grid, kThreads + kConvThreads, kSmemBytes, stream>>>(mah, mal, mbh, mbl, mc, kp);
     return launch_status();
 }
 
