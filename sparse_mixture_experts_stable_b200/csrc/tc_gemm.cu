@@ -519,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // lane = row) and one lane hands it to the TMA, which streams it out while the warp
                 // drains the next chunk; the buffer is rewritten only once the TMA has read it.
                 auto process = [&](const int c, const uint32_t (&r)[32]) {
+                    if ((int64_t)nt * p.tile_n_out + c * 32 >= p.N) return;  // past N (warp-uniform)
                     if (lane == 0) bulk_wait_read_all();
                     __syncwarp();
 #pragma unroll

@@ -407,6 +407,7 @@ __global__ void __launch_bounds__(kThreads + kConvThreads, 1)
             auto process = [&](const int c, const uint32_t (&r)[32]) {
                 const int64_t n0 = (int64_t)nt * p.n_mma + c * 32;
                 if (p.tma_out) {
+                    if (n0 >= p.N) return;  // the last tile's columns past N (warp-uniform)
                     // every row valid, whole 32-column chunks: the chunk goes to the warp's staging buffer
                     // in the map's 128-byte swizzled layout and one lane hands it to the TMA, which streams
                     // it out while the warp drains the next chunk

@@ -85,6 +85,7 @@ def test_backward_gelu_tiny_layer():
     (517, 72, 40, 5, 3, 0.8, False, 0.2),    # ragged sizes, drops, aux term
     (300, 128, 160, 6, 2, 1.5, True, 0.0),   # several K tiles in every product
     (64, 32, 8, 3, 1, 2.0, True, 0.0),       # top-1, tiny F
+    (300, 160, 256, 4, 2, 1.2, True, 0.0),   # dW1 through TMA stores with a last column tile past D
 ])
 def test_backward_gelu_matches_oracle(T, D, F, E, k, cf, residual, aux):
     g = torch.Generator().manual_seed(T + D + F)

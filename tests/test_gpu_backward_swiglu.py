@@ -31,6 +31,7 @@ def _close(got, want, what):
     (400, 128, 128, 6, 2, 1.0, True, 0.0),   # H, F multiples of 64: weights read MN-major, no transposed copies
     (333, 256, 64, 5, 3, 0.7, False, 0.05),  # the same with drops and the aux term
     (260, 192, 256, 4, 2, 1.2, False, 0.0),  # F a multiple of 128: dW gate and up from one split-output GEMM
+    (300, 320, 128, 4, 2, 1.2, False, 0.0),  # H = 320: the weight gradients' last column tile extends past H
 ])
 @pytest.mark.parametrize("saved", [False, True])
 def test_backward_swiglu_matches_oracle(T, H, F, E, k, cf, residual, aux, saved):
